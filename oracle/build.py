@@ -1,0 +1,32 @@
+"""Compile the C parts of the oracle into oracle/liboracle.so (test infrastructure).
+
+gcc, -O2, OpenMP, no fast-math and no floating-point contraction, so the
+fp32 schedule model performs exactly the IEEE operations it spells out.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCES = ["recurrent_fp64.c", "schedule_fp32.c"]
+LIB = os.path.join(HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    srcs = [os.path.join(HERE, s) for s in SOURCES]
+    if not force and os.path.exists(LIB):
+        lib_m = os.path.getmtime(LIB)
+        if all(os.path.getmtime(s) <= lib_m for s in srcs):
+            return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+           "-fno-fast-math", "-Wall", "-Wno-unknown-pragmas", *srcs, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))
