@@ -1,0 +1,440 @@
+"""Benchmark of the CPR Gated DeltaNet path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step is one CPR forward (prefill / trainer forward: offsets, chunk
+precompute, boundary chain, intra-chunk recurrence, output store) of the
+prefill workload, B=4 sequences x T=4096 tokens, H=16 heads, d_k=d_v=128,
+C=64, bf16 q/k/v, fp32 gates and state.  Inputs are synthetic, from the
+device recipe of gated_deltanet_cpr_delta_b200.synth.  The line also
+reports decode tokens/s for the decode workload: 64 sequences x 32 heads,
+prefilled to 2048 tokens, then 256 decode steps.
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own sequences
+(weak scaling, no data-path collective).  Timing is CUDA events on the
+launching stream, the max over ranks.  L2 is flushed (a 256 MiB write)
+before every timed step.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (fp64 recurrence, OpenMP) on the host
+cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
+
+METRIC = "CPR GDN prefill & decode tokens/s on 1 B200; % of roofline; bitwise parity"
+UNIT = "tokens/s"
+WORKLOAD = dict(name="prefill B=4 H=16 T=4096 d_k=d_v=128 C=64 bf16", seed=1, B=4, H=16, T=4096, D=128, C=64)
+DECODE = dict(name="decode 64 seqs H=32 d=128 C=64: prefill 2048, then 256 steps", seed=2, N=64, H=32, D=128,
+              C=64, Lp=2048, steps=256)
+
+# FP32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (fma) x 1.965 GHz (max SM clock)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# Algorithmic work of one forward, counted from the arithmetic schedule
+# (fma = 2 flops).  Per (token, head): P_tok 7*dk*dv; chunk precompute
+# (C-1)(2dk+dv) per token of a full chunk; boundary chain 4*dk*dv per token
+# of a full chunk.
+def forward_flops(tokens_heads: int, full_tokens_heads: int, dk: int, dv: int, C: int):
+    return dict(tok=7 * dk * dv * tokens_heads,
+                prep=(C - 1) * (2 * dk + dv) * full_tokens_heads,
+                chain=4 * dk * dv * full_tokens_heads)
+
+
+# Algorithmic bytes of one decode step's per-token kernel per (sequence, head):
+# running state read + write (fp32), q, k, v read, o write, token appended to
+# the buffer (k, v, alpha, beta), gates and position.
+def decode_tok_bytes(dk: int, dv: int, esz: int, out_esz: int):
+    return 8 * dk * dv + (2 * dk + dv) * esz + dv * out_esz + (dk + dv) * esz + 8 + 8 + 8
+
+
+# DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
+# dram__bytes_write.sum), keyed by kernel, valid only for the kernel source
+# it was taken from (sha256 of csrc/kernels.cuh + csrc/schedule.cuh).
+NCU_TRAFFIC = {}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("kernels.cuh", "schedule.cuh"):
+        with open(os.path.join(ROOT, "gated_deltanet_cpr_delta_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: str):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"gdn_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.dev, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) == 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+        if not rows:
+            return None
+        sm = sorted(float(r[1]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] != "[N/A]")}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist.get_rank(), world, local
+    return 0, 1, 0
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(seed: int, B: int, H: int, D: int, C: int, T_s: int):
+    """fp64 oracle on the first T_s tokens of every sequence and head of the
+    prefill workload (host recipe inputs).  Returns (seconds, tokens)."""
+    import numpy as np
+    import oracle
+    from gated_deltanet_cpr_delta_b200 import synth
+    b = synth.make_batch(seed, [T_s] * B, H, D, D, "bf16")
+    t0 = time.perf_counter()
+    oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)
+    return time.perf_counter() - t0, B * T_s
+
+
+def cpu_baseline(budget_s: float = 10.0):
+    W = WORKLOAD
+    T_s, secs, toks = 128, 0.0, 0
+    while True:
+        secs, toks = oracle_sample(W["seed"], W["B"], W["H"], W["D"], W["C"], T_s)
+        if secs >= budget_s or T_s >= W["T"]:
+            break
+        T_s = min(W["T"], max(T_s * 2, int(T_s * budget_s / max(secs, 1e-3) * 1.1)))
+    return {"value": toks / secs, "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
+            "sample": f"fp64 recurrence (oracle/recurrent_fp64.c, OpenMP over (sequence, head)) on the first "
+                      f"{T_s} tokens of all {W['B']} sequences x {W['H']} heads of the prefill workload; "
+                      f"{secs:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle._load()
+    W = WORKLOAD
+    # size one step to ~5 s of oracle work
+    T_s = 256
+    secs, _ = oracle_sample(W["seed"], W["B"], W["H"], W["D"], W["C"], T_s)
+    T_s = max(64, min(W["T"], int(T_s * 5.0 / max(secs, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(W["seed"], W["B"], W["H"], W["D"], W["C"], min(T_s, 64))
+    tot_s, tot_tok = 0.0, 0
+    for _ in range(args.steps):
+        s, t = oracle_sample(W["seed"], W["B"], W["H"], W["D"], W["C"], T_s)
+        tot_s += s
+        tot_tok += t
+    v = tot_tok / tot_s
+    sample = (f"fp64 recurrence on the first {T_s} tokens of all {W['B']} sequences x {W['H']} heads "
+              f"of the prefill workload per step")
+    print(json.dumps({
+        "metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": W["name"], "oracle": "cpu fp64"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+    return 0
+
+
+# ---------------------------------------------------------------- native
+def parity_gate(d, o, st, C):
+    """Sequence 0, head 0: bitwise vs the fp32 schedule model, and the max
+    error vs the fp64 oracle (bench refuses to report a speed without it)."""
+    import numpy as np
+    import torch
+    import oracle
+    L = d["cu_host"][1]
+    g = lambda t: t[:L, 0:1].float().cpu().numpy()
+    q, k, v, a, b = g(d["q"]), g(d["k"]), g(d["v"]), g(d["alpha"]), g(d["beta"])
+    cu = np.array([0, L], np.int32)
+    m = oracle.schedule_forward(q, k, v, a, b, cu, C)
+    r = oracle.recurrent(q, k, v, a, b, cu, C)
+    got = o[:L, 0:1].contiguous().cpu()
+    bits_o = np.array_equal(got.view(torch.int16).numpy().view(np.uint16), oracle.to_bf16_bits(m["o"]))
+    ns = L // C + 1
+    bits_s = np.array_equal(st[:ns, 0:1].contiguous().cpu().numpy().view(np.uint32), m["states"].view(np.uint32))
+    err = float(np.max(np.abs(got.float().numpy().astype(np.float64) - r["o"])))
+    rel = err / float(np.max(np.abs(r["o"])))
+    return {"bitwise_vs_schedule_model": bool(bits_o and bits_s), "max_abs_err_vs_fp64": err,
+            "max_err_rel_to_max_o": rel, "tolerance_rel": 2e-2, "ok": bool(bits_o and bits_s and rel <= 2e-2),
+            "sample": "sequence 0, head 0 (4096 tokens)"}
+
+
+def bench_decode(rank: int, world: int, warmup: int):
+    import torch
+    from gated_deltanet_cpr_delta_b200 import gdn, synth
+    Dc = DECODE
+    N, H, D, C, Lp, S = Dc["N"], Dc["H"], Dc["D"], Dc["C"], Dc["Lp"], Dc["steps"]
+    L = Lp + S
+    d = synth.make_batch_device(Dc["seed"], [L] * N, H, D, D, "bf16", seq_ids=range(rank * N, rank * N + N))
+    idx = torch.cat([torch.arange(n * L, n * L + Lp) for n in range(N)]).cuda()
+    cu_p = [n * Lp for n in range(N + 1)]
+    cache = gdn.new_cache(N, H, D, D, C, torch.bfloat16)
+    gdn.gdn_cpr_forward(d["q"][idx], d["k"][idx], d["v"][idx], d["alpha"][idx], d["beta"][idx],
+                        torch.tensor(cu_p, dtype=torch.int32, device="cuda"), C, cu_seqlens_host=cu_p,
+                        cache_out=cache)
+    steps_in = []
+    for s in range(S):
+        t = torch.arange(N, device="cuda") * L + Lp + s
+        steps_in.append([d[n][t].contiguous() for n in ("q", "k", "v", "alpha", "beta")])
+    del d
+    o = torch.empty(N, H, D, dtype=torch.bfloat16, device="cuda")
+    # warm-up on a copy of the cache (the timed steps start at position Lp)
+    wc = {k_: v_.clone() for k_, v_ in cache.items()}
+    for s in range(max(warmup, 3)):
+        gdn.gdn_decode_step(*steps_in[s], wc, C, o=o)
+    del wc
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(S)]
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+    for e in ev:
+        for x in e:
+            x.record()
+    barrier(world)
+    for s in range(S):
+        flush.zero_()
+        outer[s][0].record()
+        gdn.gdn_decode_step(*steps_in[s], cache, C, o=o, events=ev[s])
+        outer[s][1].record()
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in outer]
+    tok_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    res_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    resync_steps = [s for s in range(S) if (Lp + s + 1) % C == 0]
+    plain = [step_ms[s] for s in range(S) if s not in resync_steps]
+    tb = decode_tok_bytes(D, D, 2, 2) * N * H
+    mean_tok = sum(tok_ms) / S
+    peaks, _ = load_peaks()
+    return {"workload": Dc["name"], "value": N * world * S / (total_ms / 1e3), "unit": UNIT,
+            "ms_per_step": total_ms / S, "plain_step_ms_mean": sum(plain) / len(plain),
+            "resync_step_ms_mean": sum(step_ms[s] for s in resync_steps) / max(1, len(resync_steps)),
+            "resync_kernel_ms_max": max(res_ms),
+            "roofline": {"kernel": "k_dec_tok", "bound": "hbm", "achieved": tb / (mean_tok / 1e3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": tb / (mean_tok / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                         "bytes_per_launch": tb}}
+
+
+def run_native(args):
+    import torch
+    from gated_deltanet_cpr_delta_b200 import gdn, synth
+
+    rank, world, local = dist_setup(args.gpus)
+    gdn.load_library()
+    W = WORKLOAD
+    B, H, T, D, C = W["B"], W["H"], W["T"], W["D"], W["C"]
+    d = synth.make_batch_device(W["seed"], [T] * B, H, D, D, "bf16", seq_ids=range(rank * B, rank * B + B))
+    o = torch.empty(B * T, H, D, dtype=torch.bfloat16, device="cuda")
+    st = torch.empty(gdn.gdn_num_chunk_states(d["cu_host"], C), H, D, D, dtype=torch.float32, device="cuda")
+    ws = torch.empty(gdn.gdn_cpr_workspace_size(B * T, B, H, D, D, C), dtype=torch.uint8, device="cuda")
+    fwd = lambda events=None: gdn.gdn_cpr_forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["cu_seqlens"],
+                                                  C, cu_seqlens_host=d["cu_host"], o=o, chunk_states=st,
+                                                  workspace=ws, events=events)
+    fwd()
+    torch.cuda.synchronize()
+    parity = parity_gate(d, o, st, C) if rank == 0 else None
+
+    for _ in range(args.warmup):
+        fwd()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    K = args.steps
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    for e in kev:
+        for x in e:
+            x.record()
+    outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    dev_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local if world > 1 else 0]
+    with ClockSampler(dev_index) as clocks:
+        barrier(world)
+        for s in range(K):
+            flush.zero_()
+            outer[s][0].record()
+            fwd(kev[s])
+            outer[s][1].record()
+        barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in outer]
+    names = ["k_tables", "k_prep", "k_chain", "k_tok", "k_cache_fill"]
+    kern_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in kev) / K for i, n in enumerate(names)}
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_step = total_ms / K
+    tokens = B * T * world
+    value = tokens / (ms_step / 1e3)
+
+    # e2e: host (pinned) inputs -> device, forward, o -> host, every step
+    hin = {n: d[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
+    dev_in = {n: torch.empty_like(d[n]) for n in hin}
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in hin.values()) + 4 * (B + 1)
+    d2h = o.numel() * o.element_size()
+
+    def e2e_step():
+        for n in hin:
+            dev_in[n].copy_(hin[n], non_blocking=True)
+        cu_dev = torch.tensor(d["cu_host"], dtype=torch.int32).pin_memory().cuda(non_blocking=True)
+        gdn.gdn_cpr_forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"], cu_dev, C,
+                            cu_seqlens_host=d["cu_host"], o=o, chunk_states=st, workspace=ws)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        e2e_step()
+    e1.record()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+
+    dec = bench_decode(rank, world, args.warmup) if not args.no_decode else None
+
+    peaks, peak_src = load_peaks()
+    flops = forward_flops(B * T * H, B * (T // C) * C * H, D, D, C)
+    tok_tf = flops["tok"] / (kern_ms["k_tok"] / 1e3) / 1e12
+    sha = kernel_source_sha()
+    traffic = NCU_TRAFFIC.get(("k_tok", sha))
+    kernels = {n: {"ms": kern_ms[n]} for n in names}
+    for n in ("tok", "prep", "chain"):
+        kernels["k_" + n]["tflops"] = flops[n] / (kern_ms["k_" + n] / 1e3) / 1e12 if kern_ms["k_" + n] > 0 else 0
+        kernels["k_" + n]["frac_fp32_peak"] = kernels["k_" + n]["tflops"] / FP32_PEAK_TFLOPS
+    total_flops = sum(flops.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": W["name"], "global_batch": B * world, "seq_len": T, "heads": H, "d_k": D,
+                   "d_v": D, "chunk": C, "io_dtype": "bf16", "state_dtype": "f32",
+                   "parallelism": f"dp{world} (sequences sharded, no collective)",
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": {"kernel": "k_tok (intra-chunk P_tok)", "bound": "alu", "achieved": tok_tf,
+                     "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tok_tf / FP32_PEAK_TFLOPS,
+                     "traffic": traffic, "flops_per_launch": flops["tok"],
+                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"},
+        "forward_roofline": {"flops_per_step": total_flops,
+                             "achieved_tflops": total_flops / (ms_step / 1e3) / 1e12 / world,
+                             "frac": total_flops / (ms_step / 1e3) / 1e12 / world / FP32_PEAK_TFLOPS},
+        "kernels": kernels,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * K,
+        "clocks": clocks.summary(),
+        "parity": parity,
+        "decode": dec,
+        "peaks": {"hbm_gbs": peaks.get("hbm_gbs"), "source": peak_src},
+        "kernel_source_sha": sha,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return run_reference(args) if args.impl == "reference" else run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,65 @@
+"""Build the CUDA library libgdn_cpr.so in-tree for sm_100a with nvcc.
+
+    python -m gated_deltanet_cpr_delta_b200.build [--force] [--verbose]
+
+`--verbose` adds ``-Xptxas -v`` (registers, spills, shared memory per kernel).
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+LIB = os.path.join(PKG, "libgdn_cpr.so")
+SOURCES = ["gdn_cpr.cu"]
+DEPS = ["gdn_cpr.cu", "kernels.cuh", "schedule.cuh"]
+HEADERS = [os.path.join(ROOT, "include", "gdn_cpr.h")]
+
+
+def nvcc_path() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def flags(verbose: bool = False):
+    f = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+         "-Xcompiler", "-fPIC", "-shared",
+         # the schedule's arithmetic is written with explicit _rn intrinsics;
+         # these keep any other fp expression exact too
+         "-fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
+         "-I", os.path.join(ROOT, "include"), "-I", CSRC]
+    if verbose:
+        f += ["-Xptxas", "-v"]
+    return f
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    m = os.path.getmtime(LIB)
+    srcs = [os.path.join(CSRC, s) for s in DEPS] + HEADERS + [os.path.abspath(__file__)]
+    return all(os.path.getmtime(s) <= m for s in srcs)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not verbose and up_to_date():
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), *flags(verbose), *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
+    if verbose:
+        sys.stderr.write(r.stdout + r.stderr)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

@@ -1,0 +1,347 @@
+// gdn_cpr.cu -- host side of the C ABI declared in include/gdn_cpr.h.
+//
+// Validates arguments on the host, carves the caller's workspace and enqueues
+// the kernels of kernels.cuh on the caller's stream.  It allocates no device
+// memory, never synchronises, and keeps no global mutable state.
+#include "gdn_cpr.h"
+#include "kernels.cuh"
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace {
+
+using gdn::ChunkCfg;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported(int32_t dk, int32_t dv, int32_t C)
+{
+    const bool d_ok = dk == dv && (dk == 16 || dk == 32 || dk == 64 || dk == 128);
+    const bool c_ok = C == 16 || C == 32 || C == 64;
+    return d_ok && c_ok;
+}
+
+bool dtype_ok(gdn_dtype_t t) { return t == GDN_F32 || t == GDN_BF16; }
+
+struct SeqTotals {
+    int64_t tasks = 0, full = 0, states = 0;
+};
+
+// Host copy of cu_seqlens -> totals; false if invalid.
+bool seq_totals(const int32_t* cu, int32_t N, int64_t T_total, int32_t C, SeqTotals* out)
+{
+    if (cu == nullptr || N < 0 || C <= 0) return false;
+    if (cu[0] != 0 || (int64_t)cu[N] != T_total) return false;
+    SeqTotals t;
+    for (int32_t n = 0; n < N; ++n) {
+        const int64_t L = (int64_t)cu[n + 1] - cu[n];
+        if (L < 0) return false;
+        t.tasks += (L + C - 1) / C;
+        t.full += L / C;
+        t.states += L / C + 1;
+    }
+    if (t.tasks > INT32_MAX || t.states > INT32_MAX) return false;
+    *out = t;
+    return true;
+}
+
+// Workspace layout: [err | cto | fco | so | w | u0 | dC], each 256-byte aligned.
+struct Workspace {
+    int32_t* err;
+    int32_t* cto;
+    int32_t* fco;
+    int32_t* so;
+    float* w;
+    float* u;
+    float* dC;
+    size_t bytes;
+};
+
+Workspace carve(void* base, int64_t max_full, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C)
+{
+    Workspace ws{};
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        const size_t o = off;
+        off = align_up(off + n);
+        return o;
+    };
+    const size_t o_err = take(16);
+    const size_t o_cto = take(sizeof(int32_t) * (size_t)(N + 1));
+    const size_t o_fco = take(sizeof(int32_t) * (size_t)(N + 1));
+    const size_t o_so = take(sizeof(int32_t) * (size_t)(N + 1));
+    const size_t o_w = take(sizeof(float) * (size_t)max_full * H * C * dk);
+    const size_t o_u = take(sizeof(float) * (size_t)max_full * H * C * dv);
+    const size_t o_dc = take(sizeof(float) * (size_t)max_full * H * (C + 4));
+    ws.bytes = off;
+    char* b = static_cast<char*>(base);
+    if (b != nullptr) {
+        ws.err = reinterpret_cast<int32_t*>(b + o_err);
+        ws.cto = reinterpret_cast<int32_t*>(b + o_cto);
+        ws.fco = reinterpret_cast<int32_t*>(b + o_fco);
+        ws.so = reinterpret_cast<int32_t*>(b + o_so);
+        ws.w = reinterpret_cast<float*>(b + o_w);
+        ws.u = reinterpret_cast<float*>(b + o_u);
+        ws.dC = reinterpret_cast<float*>(b + o_dc);
+    }
+    return ws;
+}
+
+template <typename K>
+cudaError_t set_smem(K* kernel, size_t bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta, *state_in;
+    const int32_t* cu;
+    int32_t N, H;
+    int in_bf16, out_bf16;
+    void* o;
+    float* states;
+    const gdn_cache_t* cache;
+    SeqTotals tot;
+    int64_t T_total;
+    Workspace ws;
+    cudaStream_t stream;
+    void* const* events;  // optional: 6 events around the kernels
+};
+
+inline void mark(void* const* events, int i, cudaStream_t s)
+{
+    if (events != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+}
+
+template <int D, int C>
+gdn_status_t launch_forward(const FwdArgs& a)
+{
+    using Cf = ChunkCfg<D, D, C>;
+    using TC = gdn::TokCfg<D, D, C>;
+    cudaError_t e = cudaSuccess;
+    mark(a.events, 0, a.stream);
+    gdn::k_tables<<<1, 1024, 0, a.stream>>>(a.cu, a.N, C, a.T_total, a.tot.tasks, a.tot.full, a.tot.states,
+                                             a.ws.cto, a.ws.fco, a.ws.so, a.ws.err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
+    mark(a.events, 1, a.stream);
+    if (a.tot.full > 0) {
+        constexpr size_t sm = gdn::PrepSmem<D, D, C>::BYTES;
+        if (set_smem(gdn::k_prep<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
+        gdn::k_prep<D, D, C><<<(unsigned)(a.tot.full * a.H), Cf::THREADS, sm, a.stream>>>(
+            a.k, a.v, a.alpha, a.beta, a.cu, a.ws.fco, a.ws.err, a.N, a.H, a.in_bf16, a.ws.w, a.ws.u, a.ws.dC);
+        if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    mark(a.events, 2, a.stream);
+    if (a.N > 0) {
+        constexpr size_t sm = gdn::ChainSmem<D, D, C>::BYTES;
+        if (set_smem(gdn::k_chain<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
+        gdn::k_chain<D, D, C><<<(unsigned)((int64_t)a.N * a.H * Cf::NTB), Cf::THREADS, sm, a.stream>>>(
+            a.k, a.state_in, a.cu, a.ws.fco, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.ws.w, a.ws.u, a.ws.dC,
+            a.states);
+        if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    mark(a.events, 3, a.stream);
+    if (a.tot.tasks > 0) {
+        constexpr size_t sm = TC::SMEM;
+        if (set_smem(gdn::k_tok<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
+        gdn::k_tok<D, D, C><<<(unsigned)(a.tot.tasks * a.H * TC::NT), TC::THREADS, sm, a.stream>>>(
+            a.q, a.k, a.v, a.alpha, a.beta, a.cu, a.ws.cto, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.out_bf16,
+            a.states, a.o, a.cache ? a.cache->R : nullptr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    mark(a.events, 4, a.stream);
+    if (a.cache != nullptr && a.N > 0) {
+        const gdn_cache_t& c = *a.cache;
+        gdn::k_cache_fill<D, D, C><<<(unsigned)((int64_t)a.N * a.H), 256, 0, a.stream>>>(
+            a.k, a.v, a.alpha, a.beta, a.cu, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.states, c.S_b, c.R, c.kbuf,
+            c.vbuf, c.abuf, c.bbuf, c.pos);
+        if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    mark(a.events, 5, a.stream);
+    (void)e;
+    return GDN_OK;
+}
+
+struct DecArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta;
+    const gdn_cache_t* cache;
+    int32_t N, H;
+    int in_bf16, out_bf16;
+    void* o;
+    cudaStream_t stream;
+    void* const* events;  // optional: 3 events around the kernels
+};
+
+template <int D, int C>
+gdn_status_t launch_decode(const DecArgs& a)
+{
+    const gdn_cache_t& c = *a.cache;
+    const unsigned grid = (unsigned)((int64_t)a.N * a.H);
+    mark(a.events, 0, a.stream);
+    gdn::k_dec_tok<D, D, C><<<grid, gdn::DecCfg<D, D>::THREADS, 0, a.stream>>>(
+        a.q, a.k, a.v, a.alpha, a.beta, a.H, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos,
+        a.o);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    mark(a.events, 1, a.stream);
+    constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
+    if (set_smem(gdn::k_dec_resync<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
+    gdn::k_dec_resync<D, D, C><<<grid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
+        a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    mark(a.events, 2, a.stream);
+    return GDN_OK;
+}
+
+#define GDN_DISPATCH(FN, D_, C_, ARGS)                              \
+    switch (D_ * 1000 + C_) {                                       \
+        case 16016: return FN<16, 16>(ARGS);                        \
+        case 16032: return FN<16, 32>(ARGS);                        \
+        case 16064: return FN<16, 64>(ARGS);                        \
+        case 32016: return FN<32, 16>(ARGS);                        \
+        case 32032: return FN<32, 32>(ARGS);                        \
+        case 32064: return FN<32, 64>(ARGS);                        \
+        case 64016: return FN<64, 16>(ARGS);                        \
+        case 64032: return FN<64, 32>(ARGS);                        \
+        case 64064: return FN<64, 64>(ARGS);                        \
+        case 128016: return FN<128, 16>(ARGS);                      \
+        case 128032: return FN<128, 32>(ARGS);                      \
+        case 128064: return FN<128, 64>(ARGS);                      \
+        default: return GDN_ERR_UNSUPPORTED;                        \
+    }
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v1/NL8"; }
+
+const char* gdn_status_string(gdn_status_t s)
+{
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case GDN_ERR_CUDA: return "CUDA launch failed";
+        case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int64_t gdn_num_chunk_states(const int32_t* cu_seqlens_host, int32_t num_seqs, int32_t C)
+{
+    if (cu_seqlens_host == nullptr || num_seqs < 0 || C <= 0) return -1;
+    SeqTotals t;
+    if (!seq_totals(cu_seqlens_host, num_seqs, cu_seqlens_host[num_seqs], C, &t)) return -1;
+    return t.states;
+}
+
+size_t gdn_cpr_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v,
+                              int32_t C)
+{
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0) return 0;
+    return carve(nullptr, total_tokens / C, num_seqs, H, d_k, d_v, C).bytes;
+}
+
+gdn_status_t gdn_cpr_forward_timed(const void* q, const void* k, const void* v, const float* alpha,
+                                   const float* beta, const float* state_in, const int32_t* cu_seqlens,
+                                   const int32_t* cu_seqlens_host, int32_t num_seqs, int64_t total_tokens,
+                                   int32_t H, int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
+                                   gdn_dtype_t out_dtype, void* o, float* chunk_states,
+                                   const gdn_cache_t* cache_out, void* workspace, size_t workspace_bytes,
+                                   void* stream, void* const* events)
+{
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0)
+        return GDN_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (!supported(d_k, d_v, C)) return GDN_ERR_UNSUPPORTED;
+    SeqTotals tot;
+    if (!seq_totals(cu_seqlens_host, num_seqs, total_tokens, C, &tot)) return GDN_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr || chunk_states == nullptr) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(chunk_states) || (state_in && !aligned16(state_in))) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0) {
+        if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GDN_ERR_INVALID_ARG;
+    }
+    if (cache_out != nullptr) {
+        const gdn_cache_t& c = *cache_out;
+        if (!c.S_b || !c.R || !c.kbuf || !c.vbuf || !c.abuf || !c.bbuf || !c.pos) return GDN_ERR_INVALID_ARG;
+        if (!aligned16(c.S_b) || !aligned16(c.R) || !aligned16(c.kbuf) || !aligned16(c.vbuf))
+            return GDN_ERR_INVALID_ARG;
+        if (total_tokens > 0 && (!k || !v || !alpha || !beta)) return GDN_ERR_INVALID_ARG;
+    }
+    const Workspace need = carve(nullptr, total_tokens / C, num_seqs, H, d_k, d_v, C);
+    if (workspace == nullptr || workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs * H > INT32_MAX || tot.tasks * H * 2 > INT32_MAX) return GDN_ERR_INVALID_ARG;
+
+    FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.state_in = state_in;
+    a.cu = cu_seqlens; a.N = num_seqs; a.H = H;
+    a.in_bf16 = in_dtype == GDN_BF16; a.out_bf16 = out_dtype == GDN_BF16;
+    a.o = o; a.states = chunk_states; a.cache = cache_out; a.tot = tot; a.T_total = total_tokens;
+    a.ws = carve(workspace, total_tokens / C, num_seqs, H, d_k, d_v, C);
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.events = events;
+    if (num_seqs == 0) {
+        for (int i = 0; i < 6; ++i) mark(events, i, a.stream);
+        return GDN_OK;
+    }
+    GDN_DISPATCH(launch_forward, d_k, C, a)
+}
+
+gdn_status_t gdn_cpr_forward(const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                             const float* state_in, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                             int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v,
+                             int32_t C, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* o, float* chunk_states,
+                             const gdn_cache_t* cache_out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    return gdn_cpr_forward_timed(q, k, v, alpha, beta, state_in, cu_seqlens, cu_seqlens_host, num_seqs,
+                                 total_tokens, H, d_k, d_v, C, in_dtype, out_dtype, o, chunk_states, cache_out,
+                                 workspace, workspace_bytes, stream, nullptr);
+}
+
+gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, const float* alpha,
+                                   const float* beta, const gdn_cache_t* cache, int32_t num_seqs, int32_t H,
+                                   int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
+                                   gdn_dtype_t out_dtype, void* o, void* stream, void* const* events)
+{
+    if (num_seqs < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0) return GDN_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
+    if (!supported(d_k, d_v, C)) return GDN_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (cache == nullptr) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) {
+        for (int i = 0; i < 3; ++i) mark(events, i, static_cast<cudaStream_t>(stream));
+        return GDN_OK;
+    }
+    const gdn_cache_t& c = *cache;
+    if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!c.S_b || !c.R || !c.kbuf || !c.vbuf || !c.abuf || !c.bbuf || !c.pos) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(c.S_b) || !aligned16(c.R) ||
+        !aligned16(c.kbuf) || !aligned16(c.vbuf))
+        return GDN_ERR_INVALID_ARG;
+    DecArgs a;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.cache = cache;
+    a.N = num_seqs; a.H = H; a.in_bf16 = in_dtype == GDN_BF16; a.out_bf16 = out_dtype == GDN_BF16;
+    a.o = o; a.stream = static_cast<cudaStream_t>(stream); a.events = events;
+    GDN_DISPATCH(launch_decode, d_k, C, a)
+}
+
+gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                             const gdn_cache_t* cache, int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v,
+                             int32_t C, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* o, void* stream)
+{
+    return gdn_decode_step_timed(q, k, v, alpha, beta, cache, num_seqs, H, d_k, d_v, C, in_dtype, out_dtype, o,
+                                 stream, nullptr);
+}
+
+}  // extern "C"

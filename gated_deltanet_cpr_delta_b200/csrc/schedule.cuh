@@ -1,0 +1,142 @@
+// schedule.cuh -- device primitives of the fp32 CPR arithmetic schedule.
+//
+// Every floating-point operation on the path goes through these helpers.
+// Each is exactly one IEEE binary32 operation, rounded to nearest-even, with
+// no flush-to-zero.  The compiler may not contract them into other operations.
+// The fixed reduction tree over d_k follows the principle on the IsoExec summary
+// page ("Achieving Parallelism Invariance": contiguous K leaves, FP32
+// accumulation inside a leaf, a fixed binary tree over the leaves) and the
+// commentary blog, section 8.  This project fixes NL = 8 leaves.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+constexpr int kLeaves = 8;
+
+__device__ __forceinline__ float fmul(float a, float b) { return __fmul_rn(a, b); }
+__device__ __forceinline__ float fadd(float a, float b) { return __fadd_rn(a, b); }
+__device__ __forceinline__ float fsub(float a, float b) { return __fsub_rn(a, b); }
+__device__ __forceinline__ float ffma(float a, float b, float c) { return __fmaf_rn(a, b, c); }
+
+// Partial results of the 8-leaf tree ((p0+p1)+(p2+p3)) + ((p4+p5)+(p6+p7)),
+// pushed leaf by leaf (l = 0..7, known at compile time after unrolling).
+// t0 holds the final value after leaf 7.
+struct TreeAcc {
+    float t0, t1, t2;
+};
+
+__device__ __forceinline__ void tree_push(TreeAcc& s, int l, float p)
+{
+    switch (l) {
+        case 0: s.t0 = p; break;
+        case 1: s.t0 = fadd(s.t0, p); break;
+        case 2: s.t1 = p; break;
+        case 3: s.t1 = fadd(s.t1, p); s.t0 = fadd(s.t0, s.t1); break;
+        case 4: s.t1 = p; break;
+        case 5: s.t1 = fadd(s.t1, p); break;
+        case 6: s.t2 = p; break;
+        default: s.t2 = fadd(s.t2, p); s.t1 = fadd(s.t1, s.t2); s.t0 = fadd(s.t0, s.t1); break;
+    }
+}
+
+// tree(x, y) over DK elements held by one thread (x, y: any address space).
+template <int DK>
+__device__ __forceinline__ float tree_dot(const float* x, const float* y)
+{
+    constexpr int L = DK / kLeaves;
+    TreeAcc s;
+#pragma unroll
+    for (int l = 0; l < kLeaves; ++l) {
+        float acc = fmul(x[l * L], y[l * L]);
+#pragma unroll
+        for (int m = 1; m < L; ++m) acc = ffma(x[l * L + m], y[l * L + m], acc);
+        tree_push(s, l, acc);
+    }
+    return s.t0;
+}
+
+// One leaf: x[0]*y[0], then ascending fused multiply-adds.
+template <int L>
+__device__ __forceinline__ float leaf_dot(const float* x, const float* y)
+{
+    float acc = fmul(x[0], y[0]);
+#pragma unroll
+    for (int m = 1; m < L; ++m) acc = ffma(x[m], y[m], acc);
+    return acc;
+}
+
+// The tree when 4 consecutive lanes each hold two adjacent leaves (2p, 2p+1):
+// every lane returns the same value, because fp32 addition is commutative bit
+// for bit (lane 1 computes s1+s0, lane 0 computes s0+s1).
+__device__ __forceinline__ float tree_4lanes(float leaf_a, float leaf_b)
+{
+    float s = fadd(leaf_a, leaf_b);                     // (p_{2p} + p_{2p+1})
+    s = fadd(s, __shfl_xor_sync(kFullMask, s, 1));      // ((p0+p1)+(p2+p3)), ((p4+p5)+(p6+p7))
+    s = fadd(s, __shfl_xor_sync(kFullMask, s, 2));      // full tree
+    return s;
+}
+
+// ---------------------------------------------------------------- input/output
+// 8 consecutive elements of a bf16 or fp32 tensor, widened exactly to fp32.
+// `off` is an element offset; the address must be 16-byte aligned.
+__device__ __forceinline__ void load8(const void* base, int64_t off, int bf16, float* o)
+{
+    if (bf16) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + off));
+        o[0] = __uint_as_float(u.x << 16); o[1] = __uint_as_float(u.x & 0xffff0000u);
+        o[2] = __uint_as_float(u.y << 16); o[3] = __uint_as_float(u.y & 0xffff0000u);
+        o[4] = __uint_as_float(u.z << 16); o[5] = __uint_as_float(u.z & 0xffff0000u);
+        o[6] = __uint_as_float(u.w << 16); o[7] = __uint_as_float(u.w & 0xffff0000u);
+    } else {
+        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
+        const float4 a = __ldg(p), b = __ldg(p + 1);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+        o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return a | (b << 16);
+}
+
+// Store 8 consecutive fp32 values as bf16 (nearest-even) or fp32.
+__device__ __forceinline__ void store8(void* base, int64_t off, int bf16, const float* x)
+{
+    if (bf16) {
+        uint4 u;
+        u.x = pack_bf16x2(x[0], x[1]); u.y = pack_bf16x2(x[2], x[3]);
+        u.z = pack_bf16x2(x[4], x[5]); u.w = pack_bf16x2(x[6], x[7]);
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(base) + off) = u;
+    } else {
+        float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + off);
+        p[0] = make_float4(x[0], x[1], x[2], x[3]);
+        p[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+}
+
+__device__ __forceinline__ void store1(void* base, int64_t off, int bf16, float x)
+{
+    if (bf16) reinterpret_cast<__nv_bfloat16*>(base)[off] = __float2bfloat16_rn(x);
+    else reinterpret_cast<float*>(base)[off] = x;
+}
+
+// Largest n in [0, N) with tab[n] <= g (tab non-decreasing, tab[0] = 0 <= g < tab[N]).
+__device__ __forceinline__ int find_seq(const int32_t* tab, int N, int g)
+{
+    int lo = 0, hi = N;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(tab + mid) <= g) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+}  // namespace gdn

@@ -1,0 +1,205 @@
+"""Thin Python binding of the C ABI in include/gdn_cpr.h.
+
+Argument marshalling only.  Torch tensors become device pointers, the current
+torch CUDA stream becomes the stream handle, and output buffers are allocated
+with torch.  Every step of the CPR path runs in the library's CUDA kernels.
+There is no fallback: if libgdn_cpr.so is missing, or no GPU is present, the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn_cpr.so")
+
+GDN_F32, GDN_BF16 = 0, 1
+_STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
+           4: "GDN_ERR_WORKSPACE"}
+
+#: exported symbols of include/gdn_cpr.h
+SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
+           "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [("S_b", ctypes.c_void_p), ("R", ctypes.c_void_p), ("kbuf", ctypes.c_void_p),
+                ("vbuf", ctypes.c_void_p), ("abuf", ctypes.c_void_p), ("bbuf", ctypes.c_void_p),
+                ("pos", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgdn_cpr.so (built by ``python -m gated_deltanet_cpr_delta_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with python -m gated_deltanet_cpr_delta_b200.build")
+    lib = ctypes.CDLL(path)
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.gdn_contract_id.restype = ctypes.c_char_p
+    lib.gdn_contract_id.argtypes = []
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_status_string.argtypes = [ctypes.c_int]
+    lib.gdn_num_chunk_states.restype = i64
+    lib.gdn_num_chunk_states.argtypes = [P, i32, i32]
+    lib.gdn_cpr_workspace_size.restype = sz
+    lib.gdn_cpr_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+    lib.gdn_cpr_forward.restype = ctypes.c_int
+    lib.gdn_cpr_forward.argtypes = [P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
+                                    ctypes.c_int, P, P, ctypes.POINTER(CacheStruct), P, sz, P]
+    lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_decode_step.argtypes = [P, P, P, P, P, ctypes.POINTER(CacheStruct), i32, i32, i32, i32, i32,
+                                    ctypes.c_int, ctypes.c_int, P, P]
+    lib.gdn_cpr_forward_timed.restype = ctypes.c_int
+    lib.gdn_cpr_forward_timed.argtypes = lib.gdn_cpr_forward.argtypes + [P]
+    lib.gdn_decode_step_timed.restype = ctypes.c_int
+    lib.gdn_decode_step_timed.argtypes = lib.gdn_decode_step.argtypes + [P]
+    _lib = lib
+    return lib
+
+
+def _dt(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return GDN_F32
+    if t == torch.bfloat16:
+        return GDN_BF16
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _event_array(events, n: int):
+    """torch.cuda.Event list -> C array of cudaEvent_t handles (events must
+    have been recorded once so that the CUDA event exists)."""
+    if len(events) != n:
+        raise ValueError(f"need {n} events")
+    handles = [e.cuda_event for e in events]
+    if any(h == 0 for h in handles):
+        raise ValueError("record each event once before passing it (creates the CUDA event)")
+    return (ctypes.c_void_p * n)(*handles)
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise GdnError(st, what)
+
+
+def gdn_contract_id() -> str:
+    return load_library().gdn_contract_id().decode()
+
+
+def gdn_num_chunk_states(cu_seqlens_host: Sequence[int], C: int) -> int:
+    arr = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    n = load_library().gdn_num_chunk_states(arr, len(cu_seqlens_host) - 1, C)
+    if n < 0:
+        raise GdnError(1, "gdn_num_chunk_states")
+    return int(n)
+
+
+def gdn_cpr_workspace_size(total_tokens: int, num_seqs: int, H: int, d_k: int, d_v: int, C: int) -> int:
+    return int(load_library().gdn_cpr_workspace_size(total_tokens, num_seqs, H, d_k, d_v, C))
+
+
+def new_cache(N: int, H: int, d_k: int, d_v: int, C: int, dtype: torch.dtype, device="cuda",
+              state: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """Allocate a decode cache (gdn_cache_t layout).  With ``state`` [N,H,d_v,d_k]
+    it starts at a chunk boundary with that state, otherwise at zero."""
+    S = torch.zeros(N, H, d_v, d_k, dtype=torch.float32, device=device) if state is None else state.clone()
+    return dict(S_b=S, R=S.clone(), kbuf=torch.zeros(N, H, C, d_k, dtype=dtype, device=device),
+                vbuf=torch.zeros(N, H, C, d_v, dtype=dtype, device=device),
+                abuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
+                bbuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
+                pos=torch.zeros(N, H, dtype=torch.int32, device=device))
+
+
+def _cache_struct(c: Dict[str, torch.Tensor]) -> CacheStruct:
+    return CacheStruct(*[c[n].data_ptr() for n in ("S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos")])
+
+
+def gdn_cpr_forward(q, k, v, alpha, beta, cu_seqlens, C: int, *, cu_seqlens_host=None, state_in=None,
+                    out_dtype=None, cache_out: Optional[Dict[str, torch.Tensor]] = None, workspace=None,
+                    o=None, chunk_states=None, events=None):
+    """CPR forward (prefill / trainer forward).
+
+    q, k [T,H,d_k], v [T,H,d_v] (bf16 or fp32); alpha, beta [T,H] fp32;
+    cu_seqlens int32 device [N+1] (``cu_seqlens_host``: the same values on the
+    host; read back with a sync when omitted); state_in [N,H,d_v,d_k] fp32 or None.
+    Returns (o [T,H,d_v] in out_dtype (default: q.dtype), chunk_states).
+    ``events``: optional 6 torch.cuda.Events, recorded around the kernels
+    (calls gdn_cpr_forward_timed).
+    """
+    lib = load_library()
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu().tolist()
+    cu_h = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    N = len(cu_seqlens_host) - 1
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    dev = k.device
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=out_dtype, device=dev)
+    if chunk_states is None:
+        ns = lib.gdn_num_chunk_states(cu_h, N, C)
+        if ns < 0:
+            raise GdnError(1, "gdn_num_chunk_states")
+        chunk_states = torch.empty(ns, H, dv, dk, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib.gdn_cpr_workspace_size(T, N, H, dk, dv, C), dtype=torch.uint8, device=dev)
+    cs = _cache_struct(cache_out) if cache_out is not None else None
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in),
+            _ptr(cu_seqlens), cu_h, N, T, H, dk, dv, C, _dt(q.dtype), _dt(out_dtype),
+            _ptr(o), _ptr(chunk_states), ctypes.byref(cs) if cs is not None else None,
+            _ptr(workspace), workspace.numel(), _stream(dev))
+    if events is None:
+        st = lib.gdn_cpr_forward(*args)
+    else:
+        st = lib.gdn_cpr_forward_timed(*args, _event_array(events, 6))
+    _check(st, "gdn_cpr_forward")
+    return o, chunk_states
+
+
+def gdn_decode_step(q, k, v, alpha, beta, cache: Dict[str, torch.Tensor], C: int, *, out_dtype=None, o=None,
+                    events=None):
+    """One decode token per sequence.  q,k [N,H,d_k], v [N,H,d_v]; alpha, beta [N,H].
+    ``cache`` (from :func:`new_cache` or a forward's ``cache_out``) is updated in place.
+    ``events``: optional 3 torch.cuda.Events (calls gdn_decode_step_timed)."""
+    lib = load_library()
+    N, H, dk = k.shape
+    dv = v.shape[2]
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=out_dtype, device=k.device)
+    cs = _cache_struct(cache)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), ctypes.byref(cs), N, H, dk,
+            dv, C, _dt(q.dtype), _dt(out_dtype), _ptr(o), _stream(k.device))
+    if events is None:
+        st = lib.gdn_decode_step(*args)
+    else:
+        st = lib.gdn_decode_step_timed(*args, _event_array(events, 3))
+    _check(st, "gdn_decode_step")
+    return o

@@ -129,3 +129,47 @@ PREFILL = dict(seed=1, B=4, H=16, T=4096, dk=128, dv=128, C=64, dtype="bf16")
 DECODE = dict(seed=2, B=64, H=32, T_prefill=2048, steps=256, dk=128, dv=128, C=64, dtype="bf16")
 VARLEN = dict(seed=3, N=32, H=32, lo=128, hi=8192, dk=128, dv=128, C=64, dtype="bf16")
 TRAIN = dict(seed=4, B=2, H=32, T=8192, dk=128, dv=128, C=64, dtype="bf16")
+
+
+# ---------------------------------------------------------------- device recipe
+# For the full-size workloads (up to ~150k tokens x 32 heads) the same recipe
+# runs with torch on the GPU: sequence n uses a torch Philox generator seeded
+# with seed * 1_000_003 + n, draws fp64 standard normals in the same order,
+# and applies the same transforms.  The values differ from the numpy recipe
+# (different bit generator) but have the same distribution.  Parity checks at
+# these sizes copy the sampled sequences' inputs to the host for the oracle.
+def make_batch_device(seed: int, lengths: Sequence[int], H: int, dk: int, dv: int, dtype: str,
+                      device="cuda", seq_ids: Optional[Sequence[int]] = None):
+    import torch
+
+    seq_ids = list(range(len(lengths))) if seq_ids is None else list(seq_ids)
+    tdt = {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
+    T = int(sum(lengths))
+    q = torch.empty(T, H, dk, dtype=tdt, device=device)
+    k = torch.empty(T, H, dk, dtype=tdt, device=device)
+    v = torch.empty(T, H, dv, dtype=tdt, device=device)
+    alpha = torch.empty(T, H, dtype=torch.float32, device=device)
+    beta = torch.empty(T, H, dtype=torch.float32, device=device)
+    a0 = 0
+    for n, L in zip(seq_ids, lengths):
+        L = int(L)
+        g = torch.Generator(device=device)
+        g.manual_seed(int(seed) * 1_000_003 + int(n))
+        sl = slice(a0, a0 + L)
+        xq = torch.randn(L, H, dk, dtype=torch.float64, device=device, generator=g)
+        q[sl] = (xq / xq.norm(dim=-1, keepdim=True)).float().to(tdt)
+        del xq
+        xk = torch.randn(L, H, dk, dtype=torch.float64, device=device, generator=g)
+        k[sl] = (xk / xk.norm(dim=-1, keepdim=True)).float().to(tdt)
+        del xk
+        v[sl] = torch.randn(L, H, dv, dtype=torch.float64, device=device, generator=g).float().to(tdt)
+        xa = torch.randn(L, H, dtype=torch.float64, device=device, generator=g)
+        xb = torch.randn(L, H, dtype=torch.float64, device=device, generator=g)
+        alpha[sl] = torch.exp(-torch.logaddexp(torch.zeros_like(xa), xa)).float()
+        beta[sl] = torch.sigmoid(xb).float()
+        a0 += L
+    cu_host = [0]
+    for L in lengths:
+        cu_host.append(cu_host[-1] + int(L))
+    cu = torch.tensor(cu_host, dtype=torch.int32, device=device)
+    return dict(q=q, k=k, v=v, alpha=alpha, beta=beta, cu_seqlens=cu, cu_host=cu_host, dtype=dtype)

@@ -1,0 +1,202 @@
+/*
+ * gdn_cpr.h -- C ABI of the CPR Gated DeltaNet library for B200 (sm_100a).
+ *
+ * The layer is the gated delta rule with an fp32 state, per sequence and head
+ * (IsoExec summary page, section "Chunkwise-Parallel Recurrent (CPR) Gated
+ * DeltaNet"; commentary blog, section 10 "Gated DeltaNet"):
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t
+ *
+ * It is evaluated chunkwise-parallel recurrent (CPR).  The recurrence is the
+ * primary computation.  It runs in parallel across chunks of C tokens, each chunk
+ * starting from its boundary state.  Decode re-synchronises its running state
+ * with the boundary state every C tokens (same page and section; daily.dev
+ * digest, "What is chunkwise-parallel recurrent (CPR)").
+ *
+ * Every entry point executes one written-down fp32 arithmetic schedule.  The
+ * schedule fixes an 8-leaf reduction tree over d_k, the operation order and the
+ * rounding (IsoExec summary page, "Achieving Parallelism Invariance";
+ * commentary blog, section 8).  The forward and the decode step therefore give
+ * bit-identical outputs and states.  gdn_contract_id() names the schedule.
+ *
+ * Conventions common to every call:
+ *  - All tensors are caller-owned device memory unless marked "host".
+ *    The library never allocates device memory and keeps no global mutable
+ *    state.  It never synchronises the device.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *    The call returns once the kernels are enqueued.
+ *  - Layouts are row-major and densely packed:
+ *      q, k   [T_total, H, d_k]      v, o [T_total, H, d_v]
+ *      alpha, beta [T_total, H] fp32  (alpha in [0, 1], beta in [0, 1])
+ *      states [.., H, d_v, d_k] fp32  (row i of a state = value channel i)
+ *  - Every device pointer must be 16-byte aligned.
+ *  - Supported shapes: d_k == d_v in {16, 32, 64, 128}; C in {16, 32, 64}.
+ *    Any other shape returns GDN_ERR_UNSUPPORTED.
+ *  - Inputs must be finite.  The results for NaN or Inf inputs are unspecified.
+ *  - Errors are reported by the return code only: no exceptions, no exit,
+ *    and no device trap or assert.  Invalid arguments are caught on the host
+ *    before anything is enqueued.
+ */
+#ifndef GDN_CPR_H
+#define GDN_CPR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* NULL/misaligned pointer, bad size, bad cu_seqlens */
+    GDN_ERR_UNSUPPORTED = 2,   /* (d_k, d_v, C, dtype) not compiled in */
+    GDN_ERR_CUDA = 3,          /* a CUDA launch or attribute call failed */
+    GDN_ERR_WORKSPACE = 4      /* workspace NULL or smaller than gdn_cpr_workspace_size() */
+} gdn_status_t;
+
+typedef enum {
+    GDN_F32 = 0,               /* IEEE binary32 */
+    GDN_BF16 = 1               /* bfloat16; widened exactly to fp32 on load, stored round-to-nearest-even */
+} gdn_dtype_t;
+
+/*
+ * Decode cache of N sequences.  It is the complete resumable state of a CPR
+ * layer at any token position.  All fields are caller-owned device memory.
+ *   S_b  [N, H, d_v, d_k] fp32   the last chunk-boundary state (position floor(p/C)*C)
+ *   R    [N, H, d_v, d_k] fp32   the running per-token state (== S_b when pos == 0)
+ *   kbuf [N, H, C, d_k]  in_dtype  the tokens since the last boundary ...
+ *   vbuf [N, H, C, d_v]  in_dtype
+ *   abuf [N, H, C] fp32, bbuf [N, H, C] fp32   ... their gates
+ *   pos  [N, H] int32            tokens since the last boundary, 0 <= pos < C
+ * A fresh cache for an initial state S_0 is S_b = R = S_0 with pos = 0.  The
+ * buffer contents do not matter while pos == 0.
+ */
+typedef struct {
+    float*   S_b;
+    float*   R;
+    void*    kbuf;
+    void*    vbuf;
+    float*   abuf;
+    float*   bbuf;
+    int32_t* pos;
+} gdn_cache_t;
+
+/* Name of the arithmetic schedule every kernel executes (static string). */
+const char* gdn_contract_id(void);
+
+/* Human-readable text for a status code (static string). */
+const char* gdn_status_string(gdn_status_t status);
+
+/*
+ * Number of chunk states the forward writes.  That is
+ * sum_n (floor(L_n / C) + 1), with L_n = cu_seqlens_host[n+1] - cu_seqlens_host[n].
+ * cu_seqlens_host is host memory with num_seqs + 1 entries.  Returns -1 if
+ * the arguments are invalid (see gdn_cpr_forward).
+ */
+int64_t gdn_num_chunk_states(const int32_t* cu_seqlens_host, int32_t num_seqs, int32_t C);
+
+/*
+ * Device workspace, in bytes, that gdn_cpr_forward needs for a batch of at most
+ * total_tokens tokens in num_seqs sequences.  Returns 0 for invalid sizes.
+ */
+size_t gdn_cpr_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H,
+                              int32_t d_k, int32_t d_v, int32_t C);
+
+/*
+ * CPR forward: rollout prefill and trainer forward are the same call.
+ *
+ * Inputs:
+ *   q, k [T_total,H,d_k], v [T_total,H,d_v] in in_dtype;  alpha, beta [T_total,H] fp32.
+ *   state_in [num_seqs,H,d_v,d_k] fp32 is the state at each sequence's
+ *     position 0, which is a chunk boundary.  NULL means zeros.
+ *   cu_seqlens      device [num_seqs+1] int32, packed sequence offsets
+ *   cu_seqlens_host host   [num_seqs+1] int32, the same values.  It sizes the
+ *     launch grids and is validated on the host: cu[0] == 0, non-decreasing,
+ *     cu[num_seqs] == total_tokens.  The kernels check the device copy against
+ *     the host-derived totals.  If the two copies disagree, the kernels write
+ *     nothing, and the outputs are left unspecified but in bounds.
+ *   Chunks are aligned to each sequence's own token 0, so results do not
+ *   depend on batch composition or packing.
+ * Outputs:
+ *   o [T_total,H,d_v] in out_dtype (fp32, or bf16 with nearest-even rounding)
+ *   chunk_states [gdn_num_chunk_states(),H,d_v,d_k] fp32: for sequence n,
+ *     entries s_n + c (c = 0..floor(L_n/C)) hold the state at position c*C,
+ *     where s_n = sum_{m<n}(floor(L_m/C)+1).  Entry s_n is a copy of state_in.
+ *   cache_out (optional; NULL to skip): filled for a decode continuation of
+ *     every sequence, in the layout of gdn_cache_t with N = num_seqs.  Its
+ *     buffers take in_dtype.
+ *   workspace: at least gdn_cpr_workspace_size(total_tokens, num_seqs, H, d_k,
+ *     d_v, C) bytes of device memory, owned by the caller.  The call may
+ *     overwrite it freely.  It must not be shared with a concurrent call.
+ */
+gdn_status_t gdn_cpr_forward(const void* q, const void* k, const void* v,
+                             const float* alpha, const float* beta,
+                             const float* state_in,
+                             const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                             int32_t num_seqs, int64_t total_tokens, int32_t H,
+                             int32_t d_k, int32_t d_v, int32_t C,
+                             gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                             void* o, float* chunk_states, const gdn_cache_t* cache_out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step: one new token for each of num_seqs sequences.
+ *   q, k [num_seqs,H,d_k], v [num_seqs,H,d_v] in in_dtype; alpha, beta [num_seqs,H] fp32
+ *   cache: updated in place (see gdn_cache_t).  For each (sequence, head):
+ *     the running state R takes one per-token step and gives o.  The token is
+ *     appended to the buffer.  When the buffer then holds C tokens, the
+ *     boundary state is advanced over them (S_b <- P_chunk(S_b, buffer)),
+ *     R <- S_b, and pos wraps to 0 (the resync).
+ *   o [num_seqs,H,d_v] out_dtype.
+ * The call enqueues two kernels: the per-token step, then the resync.  The
+ * resync exits at once for sequences that are not at a boundary.  A prefill
+ * of L tokens followed by m decode steps gives bit-identical o and cache to a
+ * prefill of L + m tokens.
+ * A pos outside [0, C) is not written through.  That (sequence, head) is left
+ * unchanged and its o is unspecified.
+ */
+gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v,
+                             const float* alpha, const float* beta,
+                             const gdn_cache_t* cache,
+                             int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v, int32_t C,
+                             gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                             void* o, void* stream);
+
+/*
+ * Per-kernel timing variants, for benchmarks and profilers.  These are the
+ * same calls with the same launches and the same results.  In addition they
+ * record caller-created CUDA events (cudaEvent_t, created on the current
+ * device) on `stream` between the kernels:
+ *   gdn_cpr_forward_timed: events[0..5] around, in order, the offsets
+ *     kernel, the chunk precompute (w, u0, decays), the boundary-state chain,
+ *     the intra-chunk recurrence and the cache fill.  Kernel i ran between
+ *     events[i] and events[i+1].  A kernel that has no work still gets both
+ *     of its events, so its time is zero.
+ *   gdn_decode_step_timed: events[0..2] around the per-token step and then the
+ *     resync.
+ * events == NULL behaves exactly like the untimed call.
+ */
+gdn_status_t gdn_cpr_forward_timed(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta,
+                                   const float* state_in,
+                                   const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                   int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                   int32_t d_k, int32_t d_v, int32_t C,
+                                   gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                                   void* o, float* chunk_states, const gdn_cache_t* cache_out,
+                                   void* workspace, size_t workspace_bytes, void* stream,
+                                   void* const* events);
+
+gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta,
+                                   const gdn_cache_t* cache,
+                                   int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v, int32_t C,
+                                   gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                                   void* o, void* stream, void* const* events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_CPR_H */
