@@ -31,6 +31,7 @@ bool dtype_ok(gdn_dtype_t t) { return t == GDN_F32 || t == GDN_BF16; }
 
 struct SeqTotals {
     int64_t tasks = 0, full = 0, states = 0;
+    uint64_t hash = 0;  // gdn::cu_entry_hash summed over the host copy
 };
 
 // Host copy of cu_seqlens -> totals; false if invalid.
@@ -45,7 +46,9 @@ bool seq_totals(const int32_t* cu, int32_t N, int64_t T_total, int32_t C, SeqTot
         t.tasks += (L + C - 1) / C;
         t.full += L / C;
         t.states += L / C + 1;
+        t.hash += gdn::cu_entry_hash(n, cu[n]);
     }
+    t.hash += gdn::cu_entry_hash(N, cu[N]);
     if (t.tasks > INT32_MAX || t.states > INT32_MAX) return false;
     *out = t;
     return true;
@@ -128,7 +131,7 @@ gdn_status_t launch_forward(const FwdArgs& a)
     cudaError_t e = cudaSuccess;
     mark(a.events, 0, a.stream);
     gdn::k_tables<<<1, 1024, 0, a.stream>>>(a.cu, a.N, C, a.T_total, a.tot.tasks, a.tot.full, a.tot.states,
-                                             a.ws.cto, a.ws.fco, a.ws.so, a.ws.err);
+                                             a.tot.hash, a.ws.cto, a.ws.fco, a.ws.so, a.ws.err);
     if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     if (a.tot.full > 0) {
@@ -183,18 +186,23 @@ struct DecArgs {
 template <int D, int C>
 gdn_status_t launch_decode(const DecArgs& a)
 {
+    using DC = gdn::DecCfg<D, D>;
     const gdn_cache_t& c = *a.cache;
-    const unsigned grid = (unsigned)((int64_t)a.N * a.H);
+    const int64_t NH = (int64_t)a.N * a.H;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return GDN_ERR_CUDA;
     mark(a.events, 0, a.stream);
-    gdn::k_dec_tok<D, D, C><<<grid, gdn::DecCfg<D, D>::THREADS, 0, a.stream>>>(
-        a.q, a.k, a.v, a.alpha, a.beta, a.H, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos,
-        a.o);
+    gdn::k_dec_tok<D, D, C><<<(unsigned)(NH * DC::NT), DC::THREADS, 0, a.stream>>>(
+        a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, a.o);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
     if (set_smem(gdn::k_dec_resync<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
-    gdn::k_dec_resync<D, D, C><<<grid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
-        a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos);
+    const unsigned rgrid = (unsigned)(NH < sms ? NH : sms);  // persistent: one CTA per SM
+    gdn::k_dec_resync<D, D, C><<<rgrid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
+        (int)NH, a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 2, a.stream);
     return GDN_OK;

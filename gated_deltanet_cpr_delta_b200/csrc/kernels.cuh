@@ -20,25 +20,40 @@
 namespace gdn {
 
 // ------------------------------------------------------------------ tables
+// Position-sensitive hash of cu_seqlens: the wrapping sum over n of
+// mix64((n << 32) | cu[n]) (the splitmix64 finalizer).  The host computes the
+// same sum from its copy; the device recomputes it from the device copy.
+__host__ __device__ inline uint64_t cu_entry_hash(int n, int32_t value)
+{
+    uint64_t z = ((uint64_t)(uint32_t)n << 32) | (uint64_t)(uint32_t)value;
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
 // One CTA.  For every sequence n (L_n = cu[n+1]-cu[n]):
 //   cto[n] = sum_{m<n} ceil(L_m/C)      (chunk tasks of k_tok)
 //   fco[n] = sum_{m<n} floor(L_m/C)     (full chunks: k_prep / k_chain)
 //   so[n]  = sum_{m<n} (floor(L_m/C)+1) (chunk-state slots)
 // and the totals at index N.  err[0] = 1 if the device cu_seqlens is invalid
-// or disagrees with the host-derived totals; every later kernel then exits.
+// or disagrees with the host copy (totals or hash); every later kernel then
+// exits without writing.
 __global__ void k_tables(const int32_t* __restrict__ cu, int N, int C, int64_t T_total,
-                         int64_t want_tasks, int64_t want_full, int64_t want_states,
+                         int64_t want_tasks, int64_t want_full, int64_t want_states, uint64_t want_hash,
                          int32_t* cto, int32_t* fco, int32_t* so, int32_t* err)
 {
     __shared__ long long wsum[3][32];
     __shared__ long long tot[3];
+    __shared__ unsigned long long hsum;
     __shared__ int bad_any;
     const int tid = threadIdx.x, nth = blockDim.x;
-    if (tid == 0) bad_any = 0;
+    if (tid == 0) { bad_any = 0; hsum = 0ull; }
     __syncthreads();
     const int per = (N + nth - 1) / nth;
     const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
     long long a = 0, b = 0, c = 0;
+    unsigned long long hs = 0ull;
     int bad = 0;
     for (int n = n0; n < n1; ++n) {
         const int L = cu[n + 1] - cu[n];
@@ -47,7 +62,10 @@ __global__ void k_tables(const int32_t* __restrict__ cu, int N, int C, int64_t T
         a += (Lc + C - 1) / C;
         b += Lc / C;
         c += Lc / C + 1;
+        hs += cu_entry_hash(n, cu[n]);
     }
+    if (tid == 0) hs += cu_entry_hash(N, cu[N]);
+    atomicAdd(&hsum, hs);
     // block-wide exclusive scan of (a, b, c)
     const int lane = tid & 31, wid = tid >> 5;
     long long va = a, vb = b, vc = c;
@@ -81,67 +99,102 @@ __global__ void k_tables(const int32_t* __restrict__ cu, int N, int C, int64_t T
     if (tid == 0) {
         cto[N] = (int32_t)tot[0]; fco[N] = (int32_t)tot[1]; so[N] = (int32_t)tot[2];
         const bool ok = !bad_any && cu[0] == 0 && (int64_t)cu[N] == T_total &&
-                        tot[0] == want_tasks && tot[1] == want_full && tot[2] == want_states;
+                        tot[0] == want_tasks && tot[1] == want_full && tot[2] == want_states &&
+                        hsum == want_hash;
         err[0] = ok ? 0 : 1;
     }
 }
-
 // ------------------------------------------------------------------ P_tok
 // Per-thread share of one state row in the P_tok kernels: 4 consecutive lanes
-// own a row, lane p holds elements [p*EPT, (p+1)*EPT) = leaves 2p and 2p+1.
+// own a row, lane p holds elements [p*EPT, (p+1)*EPT), which are leaves 2p
+// and 2p+1.  The two leaves' chains are independent, so they run packed:
+// register pair m holds (leaf 2p element m, leaf 2p+1 element m).
 template <int DK>
 struct RowSplit {
     static constexpr int TPR = 4;
-    static constexpr int EPT = DK / TPR;
-    static constexpr int L = DK / kLeaves;
-    // smem row padding: keeps the 4 lanes' 16-byte reads in distinct banks
+    static constexpr int EPT = DK / TPR;      // elements per lane
+    static constexpr int L = DK / kLeaves;    // leaf length = packed pairs per lane
     static constexpr int PAD = EPT >= 16 ? 4 : 0;
-    static constexpr int KS = DK + TPR * PAD;  // padded row stride (floats)
-    __device__ static constexpr int off(int p) { return p * (EPT + PAD); }
-    __device__ static constexpr int smem_index(int j) { return j + (j / EPT) * PAD; }
-};
-
-template <int N>
-__device__ __forceinline__ void lds_vec(float (&r)[N], const float* s)
-{
-    static_assert(N % 4 == 0, "vector load");
-#pragma unroll
-    for (int e = 0; e < N; e += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(s + e);
-        r[e] = x.x; r[e + 1] = x.y; r[e + 2] = x.z; r[e + 3] = x.w;
+    static constexpr int PS = EPT + PAD;      // smem stride between the lanes' slices
+    static constexpr int KS = TPR * PS;       // smem row stride (floats)
+    static_assert(L % 2 == 0, "pairs are read 16 bytes at a time");
+    // smem slot of element j: slices of the 4 lanes, each holding its two
+    // leaves interleaved, so one 16-byte read yields two packed pairs.  PAD
+    // keeps the 4 lanes' reads in distinct banks.
+    __host__ __device__ static constexpr int slot(int j)
+    {
+        return (j / EPT) * PS + ((j % EPT) < L ? 2 * (j % EPT) : 2 * (j % EPT - L) + 1);
     }
-}
-
-// One P_tok step for this thread's share of a row.  kt/qt point at this
-// thread's slice of k_t/q_t (smem).  Returns o_t[row] (same bits in all 4 lanes).
-template <int DK>
-__device__ __forceinline__ float ptok_step(float (&R)[DK / 4], const float* kt, const float* qt,
-                                           float v_i, float a, float b)
-{
-    using RS = RowSplit<DK>;
-    constexpr int L = RS::L;
-    float kr[RS::EPT];
-    lds_vec(kr, kt);
-    const float u = tree_4lanes(leaf_dot<L>(R, kr), leaf_dot<L>(R + L, kr + L));
-    const float d = fmul(b, fsub(v_i, fmul(a, u)));
-#pragma unroll
-    for (int e = 0; e < RS::EPT; ++e) R[e] = ffma(d, kr[e], fmul(a, R[e]));
-    float qr[RS::EPT];
-    lds_vec(qr, qt);
-    return tree_4lanes(leaf_dot<L>(R, qr), leaf_dot<L>(R + L, qr + L));
-}
-
-template <int DK, int DV, int C>
-struct TokCfg {
-    using RS = RowSplit<DK>;
-    static constexpr int RT = DV < 64 ? DV : 64;  // rows per CTA
-    static constexpr int NT = DV / RT;            // row tiles per head
-    static constexpr int THREADS = RT * RS::TPR;
-    static constexpr size_t SMEM = sizeof(float) * (2 * C * RS::KS + 2 * C * RT + 2 * C);
 };
 
-// Stage `len` tokens of a [T,H,D] input (rows tok0.., head h) into smem rows of
-// stride `ld`, widened to fp32; element j goes to column idx(j).
+// One P_tok step on this lane's share of a row.  kt/qt point at this lane's
+// slice of k_t/q_t in smem (slot layout).  Returns o_t[row] (the same bits in
+// all 4 lanes of the row).
+template <int DK>
+__device__ __forceinline__ float ptok_step(f2x (&Rp)[DK / kLeaves], const float* kt, const float* qt, float v_i,
+                                           float a, float b)
+{
+    constexpr int L = DK / kLeaves;
+    f2x kp[L];
+#pragma unroll
+    for (int m = 0; m < L; m += 2) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(kt + 2 * m);
+        kp[m] = x.x;
+        kp[m + 1] = x.y;
+    }
+    f2x acc = fmul2(Rp[0], kp[0]);
+#pragma unroll
+    for (int m = 1; m < L; ++m) acc = ffma2(Rp[m], kp[m], acc);
+    float la, lb;
+    up2(acc, la, lb);
+    const float u = tree_4lanes(la, lb);
+    const float d = fmul(b, fsub(v_i, fmul(a, u)));
+    const f2x aa = pk2(a, a), dd = pk2(d, d);
+#pragma unroll
+    for (int m = 0; m < L; ++m) Rp[m] = ffma2(dd, kp[m], fmul2(aa, Rp[m]));
+    f2x qp[L];
+#pragma unroll
+    for (int m = 0; m < L; m += 2) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(qt + 2 * m);
+        qp[m] = x.x;
+        qp[m + 1] = x.y;
+    }
+    acc = fmul2(Rp[0], qp[0]);
+#pragma unroll
+    for (int m = 1; m < L; ++m) acc = ffma2(Rp[m], qp[m], acc);
+    up2(acc, la, lb);
+    return tree_4lanes(la, lb);
+}
+
+// This lane's slice of a state row (global, EPT contiguous floats) -> packed pairs.
+template <int DK>
+__device__ __forceinline__ void load_row_pairs(f2x (&Rp)[DK / kLeaves], const float* src)
+{
+    using RS = RowSplit<DK>;
+    float t[RS::EPT];
+#pragma unroll
+    for (int e = 0; e < RS::EPT; e += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src + e);
+        t[e] = x.x; t[e + 1] = x.y; t[e + 2] = x.z; t[e + 3] = x.w;
+    }
+#pragma unroll
+    for (int m = 0; m < RS::L; ++m) Rp[m] = pk2(t[m], t[RS::L + m]);
+}
+
+template <int DK>
+__device__ __forceinline__ void store_row_pairs(float* dst, const f2x (&Rp)[DK / kLeaves])
+{
+    using RS = RowSplit<DK>;
+    float t[RS::EPT];
+#pragma unroll
+    for (int m = 0; m < RS::L; ++m) up2(Rp[m], t[m], t[RS::L + m]);
+#pragma unroll
+    for (int e = 0; e < RS::EPT; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
+}
+
+// Stage `len` tokens of a [T,H,D] input (rows tok0.., head h) into smem rows
+// of stride `ld`, widened to fp32; element j goes to column idx(j).
 template <int D, typename IdxFn>
 __device__ __forceinline__ void stage_rows(float* dst, int ld, const void* src, int64_t tok0, int len, int H,
                                            int h, int bf16, IdxFn idx)
@@ -150,9 +203,9 @@ __device__ __forceinline__ void stage_rows(float* dst, int ld, const void* src, 
         const int t = e / (D / 8), j8 = (e % (D / 8)) * 8;
         float x[8];
         load8(src, ((tok0 + t) * H + h) * (int64_t)D + j8, bf16, x);
-        float* d = dst + t * ld + idx(j8);
-        *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<float4*>(d + 4) = make_float4(x[4], x[5], x[6], x[7]);
+        float* d = dst + t * ld;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) d[idx(j8 + m)] = x[m];
     }
 }
 
@@ -160,8 +213,17 @@ struct IdxIdentity {
     __device__ int operator()(int j) const { return j; }
 };
 template <int DK>
-struct IdxRowSplit {
-    __device__ int operator()(int j) const { return RowSplit<DK>::smem_index(j); }
+struct IdxSlot {
+    __device__ int operator()(int j) const { return RowSplit<DK>::slot(j); }
+};
+
+template <int DK, int DV, int C>
+struct TokCfg {
+    using RS = RowSplit<DK>;
+    static constexpr int RT = DV < 64 ? DV : 64;  // rows per CTA
+    static constexpr int NT = DV / RT;            // row tiles per head
+    static constexpr int THREADS = RT * RS::TPR;
+    static constexpr size_t SMEM = sizeof(float) * (2 * C * RS::KS + 2 * C * RT + 2 * C);
 };
 
 // Intra-chunk recurrence: one CTA per (chunk task, head, row tile).
@@ -196,8 +258,8 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
     const int len = min(C, Ln - c * C);
     const int64_t slot = (int64_t)__ldg(so + n) + c;
 
-    stage_rows<DK>(ks, RS::KS, k, tok0, len, H, h, in_bf16, IdxRowSplit<DK>());
-    stage_rows<DK>(qs, RS::KS, q, tok0, len, H, h, in_bf16, IdxRowSplit<DK>());
+    stage_rows<DK>(ks, RS::KS, k, tok0, len, H, h, in_bf16, IdxSlot<DK>());
+    stage_rows<DK>(qs, RS::KS, q, tok0, len, H, h, in_bf16, IdxSlot<DK>());
     for (int e = threadIdx.x; e < len * (Cf::RT / 8); e += blockDim.x) {
         const int t = e / (Cf::RT / 8), i8 = (e % (Cf::RT / 8)) * 8;
         float x[8];
@@ -212,29 +274,19 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
 
     const int row = threadIdx.x / RS::TPR, p = threadIdx.x % RS::TPR;
     const int64_t grow = (int64_t)r * Cf::RT + row;
-    float R[RS::EPT];
-    {
-        const float* src = states + ((slot * H + h) * DV + grow) * DK + p * RS::EPT;
-#pragma unroll
-        for (int e = 0; e < RS::EPT; e += 4) {
-            const float4 x = __ldg(reinterpret_cast<const float4*>(src + e));
-            R[e] = x.x; R[e + 1] = x.y; R[e + 2] = x.z; R[e + 3] = x.w;
-        }
-    }
+    f2x Rp[RS::L];
+    load_row_pairs<DK>(Rp, states + ((slot * H + h) * DV + grow) * DK + p * RS::EPT);
     __syncthreads();
 
+    const float* kt = ks + p * RS::PS;
+    const float* qt = qs + p * RS::PS;
     for (int t = 0; t < len; ++t) {
-        const float ot = ptok_step<DK>(R, ks + t * RS::KS + RS::off(p), qs + t * RS::KS + RS::off(p),
-                                       vs[t * Cf::RT + row], as[t], bs[t]);
+        const float ot = ptok_step<DK>(Rp, kt + t * RS::KS, qt + t * RS::KS, vs[t * Cf::RT + row], as[t], bs[t]);
         if (p == 0) os[t * Cf::RT + row] = ot;
     }
 
-    if (cacheR != nullptr && len < C) {  // last, partial chunk: running state for decode
-        float* dst = cacheR + (((int64_t)n * H + h) * DV + grow) * DK + p * RS::EPT;
-#pragma unroll
-        for (int e = 0; e < RS::EPT; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(R[e], R[e + 1], R[e + 2], R[e + 3]);
-    }
+    if (cacheR != nullptr && len < C)  // last, partial chunk: the running state for decode
+        store_row_pairs<DK>(cacheR + (((int64_t)n * H + h) * DV + grow) * DK + p * RS::EPT, Rp);
     __syncthreads();
     for (int e = threadIdx.x; e < len * (Cf::RT / 8); e += blockDim.x) {
         const int t = e / (Cf::RT / 8), i8 = (e % (Cf::RT / 8)) * 8;
@@ -245,7 +297,7 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
 // ------------------------------------------------------------------ P_chunk
 template <int DK, int DV, int C>
 struct ChunkCfg {
-    static constexpr int KS = DK + 4;      // padded k / w row stride
+    static constexpr int KS = DK + 4;      // padded k / w / S row stride
     static constexpr int C1 = C + 1;       // decay matrix row stride
     static constexpr int CT = C + 4;       // c^T row stride
     static constexpr int DCS = C + 4;      // stride of D[C][.] rows in the workspace
@@ -254,11 +306,85 @@ struct ChunkCfg {
     static constexpr int THREADS = 256;
 };
 
+// VEC consecutive floats from smem (VEC = 4 or 2; 4*VEC-byte aligned).
+template <int VEC>
+__device__ __forceinline__ void lds_n(float (&r)[VEC], const float* s)
+{
+    if constexpr (VEC == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(s);
+        r[0] = x.x; r[1] = x.y; r[2] = x.z; r[3] = x.w;
+    } else {
+        const float2 x = *reinterpret_cast<const float2*>(s);
+        r[0] = x.x; r[1] = x.y;
+    }
+}
+
+// tree(x_a, y_b) for an RA x RB block of row pairs, all rows of stride KS in
+// smem: xa[r] = row r of the first operand, yb[c] = row c of the second.
+// The leaves run in ascending j; VEC elements are read at a time.
+template <int DK, int KS, int RA, int RB>
+__device__ __forceinline__ void tree_block(const float* const (&xa)[RA], const float* const (&yb)[RB],
+                                           float (&out)[RA][RB])
+{
+    constexpr int L = DK / kLeaves;
+    constexpr int VEC = (L % 4 == 0) ? 4 : 2;
+    TreeAcc st[RA][RB];
+#pragma unroll
+    for (int l = 0; l < kLeaves; ++l) {
+        float acc[RA][RB];
+#pragma unroll
+        for (int m = 0; m < L; m += VEC) {
+            float a[RA][VEC], b[RB][VEC];
+#pragma unroll
+            for (int r = 0; r < RA; ++r) lds_n<VEC>(a[r], xa[r] + l * L + m);
+#pragma unroll
+            for (int c = 0; c < RB; ++c) lds_n<VEC>(b[c], yb[c] + l * L + m);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+#pragma unroll
+                for (int r = 0; r < RA; ++r)
+#pragma unroll
+                    for (int c = 0; c < RB; ++c)
+                        acc[r][c] = (m + e == 0) ? fmul(a[r][e], b[c][e]) : ffma(a[r][e], b[c][e], acc[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < RA; ++r)
+#pragma unroll
+            for (int c = 0; c < RB; ++c) tree_push(st[r][c], l, acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < RA; ++r)
+#pragma unroll
+        for (int c = 0; c < RB; ++c) out[r][c] = st[r][c].t0;
+}
+
+// Forward substitution of one column, right-looking and fully unrolled: once
+// token s is final, its term enters every later token's chain.  For each
+// token t the chain still runs over s = 1..t-1 in ascending order.
+// acc[t] holds the chain start on entry and the column's result on exit.
+template <int C, int CT>
+__device__ __forceinline__ void fwd_subst(float (&acc)[C], const float* cT, const float* bs)
+{
+#pragma unroll
+    for (int sig = 0; sig < C; ++sig) {
+        acc[sig] = fmul(bs[sig], acc[sig]);
+        const float x = acc[sig];
+#pragma unroll
+        for (int tg = (sig + 1) / 4; tg < C / 4; ++tg) {
+            const float4 c4 = *reinterpret_cast<const float4*>(cT + sig * CT + 4 * tg);
+            if (4 * tg + 0 > sig) acc[4 * tg + 0] = ffma(-c4.x, x, acc[4 * tg + 0]);
+            if (4 * tg + 1 > sig) acc[4 * tg + 1] = ffma(-c4.y, x, acc[4 * tg + 1]);
+            if (4 * tg + 2 > sig) acc[4 * tg + 2] = ffma(-c4.z, x, acc[4 * tg + 2]);
+            if (4 * tg + 3 > sig) acc[4 * tg + 3] = ffma(-c4.w, x, acc[4 * tg + 3]);
+        }
+    }
+}
+
 // P_chunk part 1 for one chunk, by one CTA.  ks [C][KS], vs [C][DV], as/bs [C]
 // in smem.  Dm [(C+1)^2] and cT [C][CT] are smem scratch.  Writes
 //   w_t  -> wout[(t-1)*ldw + j],   u0_t -> uout[(t-1)*ldu + i],   D[C][s] -> dCout[s]
-// (any address space).  uout may alias vs: each column of vs is read by the
-// same thread that later writes that column of uout, and only before it does.
+// (any address space).  uout may alias vs: each column of vs is read only by
+// the thread that later writes that column of uout, and only before it does.
 template <int DK, int DV, int C>
 __device__ __forceinline__ void chunk_prep(const float* ks, const float* vs, const float* as, const float* bs,
                                            float* Dm, float* cT, float* wout, int ldw, float* uout, int ldu,
@@ -276,38 +402,46 @@ __device__ __forceinline__ void chunk_prep(const float* ks, const float* vs, con
         }
     }
     __syncthreads();
-    // c[t][s] = D[t][s] * tree(k_s, k_t), stored transposed: cT[s-1][t-1]
-    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-        const int tau = e / C, sig = e % C;  // 0-based tokens, need sig < tau
-        if (sig < tau) {
-            const float G = tree_dot<DK>(ks + sig * KS, ks + tau * KS);
-            cT[sig * CT + tau] = fmul(Dm[(tau + 1) * C1 + (sig + 1)], G);
-        }
+    // c[t][s] = D[t][s] * tree(k_s, k_t), stored transposed: cT[s-1][t-1];
+    // 4x4 blocks of the strictly lower triangle, one block per thread
+    constexpr int NB = C / 4, NBLK = NB * (NB + 1) / 2;
+    for (int blk = threadIdx.x; blk < NBLK; blk += blockDim.x) {
+        int bt = 0;
+        while ((bt + 1) * (bt + 2) / 2 <= blk) ++bt;
+        const int bsg = blk - bt * (bt + 1) / 2;
+        const float* const xa[4] = {ks + (4 * bt) * KS, ks + (4 * bt + 1) * KS, ks + (4 * bt + 2) * KS,
+                                    ks + (4 * bt + 3) * KS};
+        const float* const yb[4] = {ks + (4 * bsg) * KS, ks + (4 * bsg + 1) * KS, ks + (4 * bsg + 2) * KS,
+                                    ks + (4 * bsg + 3) * KS};
+        float G[4][4];
+        tree_block<DK, KS, 4, 4>(xa, yb, G);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int tau = 4 * bt + r, sig = 4 * bsg + c;
+                if (sig < tau) cT[sig * CT + tau] = fmul(Dm[(tau + 1) * C1 + (sig + 1)], G[r][c]);
+            }
     }
     if (dCout != nullptr)
         for (int s = threadIdx.x; s <= C; s += blockDim.x) dCout[s] = Dm[C * C1 + s];
     __syncthreads();
-    // forward substitution, one column per thread, right-looking: after token
-    // s is final, its term enters every later token's chain.  For each token t
-    // the chain still runs over s = 1..t-1 in ascending order.
+    // forward substitution, one column per thread
     for (int col = threadIdx.x; col < DV + DK; col += blockDim.x) {
         float acc[C];
-        const bool is_u = col < DV;
-        const int j = is_u ? 0 : col - DV;
-        if (is_u) {
+        if (col < DV) {
 #pragma unroll
             for (int tau = 0; tau < C; ++tau) acc[tau] = vs[tau * DV + col];
+            fwd_subst<C, CT>(acc, cT, bs);
+#pragma unroll
+            for (int tau = 0; tau < C; ++tau) uout[tau * ldu + col] = acc[tau];
         } else {
+            const int j = col - DV;
 #pragma unroll
             for (int tau = 0; tau < C; ++tau) acc[tau] = fmul(Dm[(tau + 1) * C1], ks[tau * KS + j]);
-        }
+            fwd_subst<C, CT>(acc, cT, bs);
 #pragma unroll
-        for (int sig = 0; sig < C; ++sig) {
-            const float x = fmul(bs[sig], acc[sig]);
-            if (is_u) uout[sig * ldu + col] = x;
-            else wout[sig * ldw + j] = x;
-#pragma unroll
-            for (int tau = sig + 1; tau < C; ++tau) acc[tau] = ffma(-cT[sig * CT + tau], x, acc[tau]);
+            for (int tau = 0; tau < C; ++tau) wout[tau * ldw + j] = acc[tau];
         }
     }
     __syncthreads();
@@ -315,26 +449,63 @@ __device__ __forceinline__ void chunk_prep(const float* ks, const float* vs, con
 
 // P_chunk part 2 on a tile of RTB boundary-state rows, by one CTA:
 //   e_t[i] = D[C][t] * (u0_t[i] - tree(S_i, w_t)),
-//   S_i,j <- chain_t fma(e_t[i], k_t[j], .) from D[C][0] * S_ij.
-// Ss [RTB][KS], ws [C][KS], ks [C][KS], us [C][ldu], dCs [C+1], es [C][RTB] (scratch).
+//   S_ij <- chain_t fma(e_t[i], k_t[j], .) from D[C][0] * S_ij.
+// Ss [RTB][KS], ws [C][KS], ks [C][KS], us [C][ldu], dCs [C+1], es [C][RTB]
+// (scratch), all smem.  The new rows also go to dst1 / dst2 (global, row
+// stride DK) when non-null.
 template <int DK, int RTB, int C>
 __device__ __forceinline__ void chunk_advance(float* Ss, const float* ws, const float* us, int ldu,
-                                              const float* ks, const float* dCs, float* es)
+                                              const float* ks, const float* dCs, float* es, float* dst1,
+                                              float* dst2)
 {
     constexpr int KS = DK + 4;
-    for (int e = threadIdx.x; e < C * RTB; e += blockDim.x) {
-        const int i = e % RTB, tau = e / RTB;
-        const float sw = tree_dot<DK>(Ss + i * KS, ws + tau * KS);
-        es[tau * RTB + i] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], sw));
+    // phase 1: tiles of 4 tokens x 2 rows (rows ig and ig + RTB/2)
+    constexpr int IG = RTB / 2, TG = C / 4;
+    for (int tile = threadIdx.x; tile < TG * IG; tile += blockDim.x) {
+        const int ig = tile % IG, tg = tile / IG;
+        const float* const xa[4] = {ws + (4 * tg) * KS, ws + (4 * tg + 1) * KS, ws + (4 * tg + 2) * KS,
+                                    ws + (4 * tg + 3) * KS};
+        const float* const yb[2] = {Ss + ig * KS, Ss + (ig + IG) * KS};
+        float sw[4][2];
+        tree_block<DK, KS, 4, 2>(xa, yb, sw);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int tau = 4 * tg + r, i = ig + c * IG;
+                es[tau * RTB + i] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], sw[r][c]));
+            }
     }
     __syncthreads();
+    // phase 2: tiles of 4 rows x 4 columns
+    constexpr int JG = DK / 4, IG2 = RTB / 4;
     const float d0 = dCs[0];
-    for (int e = threadIdx.x; e < RTB * DK; e += blockDim.x) {
-        const int i = e / DK, j = e % DK;
-        float acc = fmul(d0, Ss[i * KS + j]);
-#pragma unroll 8
-        for (int tau = 0; tau < C; ++tau) acc = ffma(es[tau * RTB + i], ks[tau * KS + j], acc);
-        Ss[i * KS + j] = acc;  // only this thread reads or writes element (i, j) in this phase
+    for (int tile = threadIdx.x; tile < IG2 * JG; tile += blockDim.x) {
+        const int jg = tile % JG, ig = tile / JG;
+        float acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float4 s = *reinterpret_cast<const float4*>(Ss + (4 * ig + r) * KS + 4 * jg);
+            acc[r][0] = fmul(d0, s.x); acc[r][1] = fmul(d0, s.y);
+            acc[r][2] = fmul(d0, s.z); acc[r][3] = fmul(d0, s.w);
+        }
+#pragma unroll 4
+        for (int tau = 0; tau < C; ++tau) {
+            const float4 e4 = *reinterpret_cast<const float4*>(es + tau * RTB + 4 * ig);
+            const float4 k4 = *reinterpret_cast<const float4*>(ks + tau * KS + 4 * jg);
+            const float ev[4] = {e4.x, e4.y, e4.z, e4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = ffma(ev[r], kv[c], acc[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float4 x = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            *reinterpret_cast<float4*>(Ss + (4 * ig + r) * KS + 4 * jg) = x;  // element owned by this thread
+            if (dst1 != nullptr) *reinterpret_cast<float4*>(dst1 + (int64_t)(4 * ig + r) * DK + 4 * jg) = x;
+            if (dst2 != nullptr) *reinterpret_cast<float4*>(dst2 + (int64_t)(4 * ig + r) * DK + 4 * jg) = x;
+        }
     }
     __syncthreads();
 }
@@ -446,18 +617,14 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
         }
         stage_rows<DK>(ks, KS, k, (int64_t)seq0 + (int64_t)c * C, C, H, h, in_bf16, IdxIdentity());
         const float* usrc = u_ws + task * C * DV + row0;
-        for (int e = threadIdx.x; e < C * RTB; e += blockDim.x) {
-            const int t = e / RTB, i = e % RTB;
-            us[t * RTB + i] = __ldg(usrc + t * DV + i);
+        for (int e = threadIdx.x; e < C * (RTB / 4); e += blockDim.x) {
+            const int t = e / (RTB / 4), i4 = (e % (RTB / 4)) * 4;
+            *reinterpret_cast<float4*>(us + t * RTB + i4) = __ldg(reinterpret_cast<const float4*>(usrc + t * DV + i4));
         }
         for (int s = threadIdx.x; s <= C; s += blockDim.x) dCs[s] = __ldg(dC_ws + task * Cf::DCS + s);
         __syncthreads();
-        chunk_advance<DK, RTB, C>(Ss, ws, us, RTB, ks, dCs, es);
-        float* dst = states + (((slot0 + c + 1) * H + h) * DV + row0) * DK;
-        for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-            const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-            *reinterpret_cast<float4*>(dst + (int64_t)i * DK + j4) = *reinterpret_cast<const float4*>(Ss + i * KS + j4);
-        }
+        chunk_advance<DK, RTB, C>(Ss, ws, us, RTB, ks, dCs, es,
+                                  states + (((slot0 + c + 1) * H + h) * DV + row0) * DK, nullptr);
     }
 }
 
@@ -510,56 +677,59 @@ k_cache_fill(const void* __restrict__ k, const void* __restrict__ v, const float
 template <int DK, int DV>
 struct DecCfg {
     using RS = RowSplit<DK>;
-    static constexpr int THREADS = DV * RS::TPR;
+    static constexpr int RT = DV < 32 ? DV : 32;  // rows per CTA
+    static constexpr int NT = DV / RT;
+    static constexpr int THREADS = RT * RS::TPR;
 };
 
-// One decode token per (sequence, head): P_tok on the running state R, append
-// the token to the buffer, pos += 1 (pos == C marks a pending resync).
+// One decode token per (sequence, head), one CTA per row tile: P_tok on the
+// running state R; tile 0 also appends the token to the buffer at slot pos.
+// pos itself is advanced by k_dec_resync, which runs next.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(DecCfg<DK, DV>::THREADS)
 k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
-          const float* __restrict__ alpha, const float* __restrict__ beta, int H, int in_bf16, int out_bf16,
-          float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, int32_t* pos, void* __restrict__ o)
+          const float* __restrict__ alpha, const float* __restrict__ beta, int in_bf16, int out_bf16,
+          float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos, void* __restrict__ o)
 {
-    using RS = RowSplit<DK>;
+    using Cf = DecCfg<DK, DV>;
+    using RS = typename Cf::RS;
     __shared__ __align__(16) float ks[RS::KS];
     __shared__ __align__(16) float qs[RS::KS];
-    __shared__ __align__(16) float vs[DV];
-    const int nh = blockIdx.x;
+    __shared__ __align__(16) float vs[Cf::RT];
+    const int nh = blockIdx.x / Cf::NT, r = blockIdx.x % Cf::NT;
     const int p = pos[nh];
     if (p < 0 || p >= C) return;
-    stage_rows<DK>(ks, RS::KS, k, nh, 1, 1, 0, in_bf16, IdxRowSplit<DK>());
-    stage_rows<DK>(qs, RS::KS, q, nh, 1, 1, 0, in_bf16, IdxRowSplit<DK>());
-    stage_rows<DV>(vs, DV, v, nh, 1, 1, 0, in_bf16, IdxIdentity());
+    stage_rows<DK>(ks, RS::KS, k, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
+    stage_rows<DK>(qs, RS::KS, q, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
+    for (int e = threadIdx.x; e < Cf::RT / 8; e += blockDim.x) {
+        float x[8];
+        load8(v, (int64_t)nh * DV + r * Cf::RT + e * 8, in_bf16, x);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) vs[e * 8 + m] = x[m];
+    }
     const float a = __ldg(alpha + nh), b = __ldg(beta + nh);
     const int row = threadIdx.x / RS::TPR, part = threadIdx.x % RS::TPR;
-    float* Rrow = R + ((int64_t)nh * DV + row) * DK + part * RS::EPT;
-    float Rr[RS::EPT];
-#pragma unroll
-    for (int e = 0; e < RS::EPT; e += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(Rrow + e);
-        Rr[e] = x.x; Rr[e + 1] = x.y; Rr[e + 2] = x.z; Rr[e + 3] = x.w;
-    }
+    const int grow = r * Cf::RT + row;
+    float* Rrow = R + ((int64_t)nh * DV + grow) * DK + part * RS::EPT;
+    f2x Rp[RS::L];
+    load_row_pairs<DK>(Rp, Rrow);
     __syncthreads();
-    const float ot = ptok_step<DK>(Rr, ks + RS::off(part), qs + RS::off(part), vs[row], a, b);
-#pragma unroll
-    for (int e = 0; e < RS::EPT; e += 4)
-        *reinterpret_cast<float4*>(Rrow + e) = make_float4(Rr[e], Rr[e + 1], Rr[e + 2], Rr[e + 3]);
-    if (part == 0) store1(o, (int64_t)nh * DV + row, out_bf16, ot);
-    // append the raw token to the buffer at slot p
-    const int esz = in_bf16 ? 2 : 4;
-    for (int e = threadIdx.x; e < DK * esz / 16; e += blockDim.x)
-        reinterpret_cast<uint4*>(kbuf)[((int64_t)nh * C + p) * (DK * esz / 16) + e] =
-            __ldg(reinterpret_cast<const uint4*>(k) + (int64_t)nh * (DK * esz / 16) + e);
-    for (int e = threadIdx.x; e < DV * esz / 16; e += blockDim.x)
-        reinterpret_cast<uint4*>(vbuf)[((int64_t)nh * C + p) * (DV * esz / 16) + e] =
-            __ldg(reinterpret_cast<const uint4*>(v) + (int64_t)nh * (DV * esz / 16) + e);
-    if (threadIdx.x == 0) {
-        abuf[(int64_t)nh * C + p] = a;
-        bbuf[(int64_t)nh * C + p] = b;
+    const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
+    store_row_pairs<DK>(Rrow, Rp);
+    if (part == 0) store1(o, (int64_t)nh * DV + grow, out_bf16, ot);
+    if (r == 0) {  // append the raw token to the buffer at slot p
+        const int esz = in_bf16 ? 2 : 4;
+        for (int e = threadIdx.x; e < DK * esz / 16; e += blockDim.x)
+            reinterpret_cast<uint4*>(kbuf)[((int64_t)nh * C + p) * (DK * esz / 16) + e] =
+                __ldg(reinterpret_cast<const uint4*>(k) + (int64_t)nh * (DK * esz / 16) + e);
+        for (int e = threadIdx.x; e < DV * esz / 16; e += blockDim.x)
+            reinterpret_cast<uint4*>(vbuf)[((int64_t)nh * C + p) * (DV * esz / 16) + e] =
+                __ldg(reinterpret_cast<const uint4*>(v) + (int64_t)nh * (DV * esz / 16) + e);
+        if (threadIdx.x == 0) {
+            abuf[(int64_t)nh * C + p] = a;
+            bbuf[(int64_t)nh * C + p] = b;
+        }
     }
-    __syncthreads();  // every thread has read pos before it moves
-    if (threadIdx.x == 0) pos[nh] = p + 1;
 }
 
 template <int DK, int DV, int C>
@@ -577,18 +747,18 @@ struct ResyncSmem {
     static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
 };
 
-// Resync: for every (sequence, head) whose buffer holds C tokens (pos == C),
-// S_b <- P_chunk(S_b, buffer), R <- S_b, pos <- 0.  Other CTAs exit at once.
+// Advances pos after k_dec_tok appended a token at slot pos, and resyncs
+// where that token completed a chunk: S_b <- P_chunk(S_b, buffer), R <- S_b,
+// pos <- 0.  Persistent: CTA b handles (sequence, head) pairs b, b + grid, ...
+// A pos outside [0, C) is left unchanged.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256)
-k_dec_resync(int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
+k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
              const float* bbuf, int32_t* pos)
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ResyncSmem<DK, DV, C>;
     constexpr int KS = Cf::KS, RTB = Cf::RTB;
-    const int nh = blockIdx.x;
-    if (pos[nh] != C) return;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
     float* ks = sm + Sm::KS_OFF;
@@ -602,33 +772,35 @@ k_dec_resync(int in_bf16, float* S_b, float* R, const void* kbuf, const void* vb
     float* bs = as + C;
     float* dCs = sm + Sm::DC_OFF;
 
-    // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
-    stage_rows<DK>(ks, KS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
-    stage_rows<DV>(vs, DV, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
-    for (int t = threadIdx.x; t < C; t += blockDim.x) {
-        as[t] = abuf[(int64_t)nh * C + t];
-        bs[t] = bbuf[(int64_t)nh * C + t];
-    }
-    __syncthreads();
-    chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, ws, KS, vs, DV, dCs);  // u0 overwrites v in place
-    for (int r = 0; r < Cf::NTB; ++r) {
-        float* Sg = S_b + ((int64_t)nh * DV + r * RTB) * DK;
-        float* Rg = R + ((int64_t)nh * DV + r * RTB) * DK;
-        for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-            const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-            *reinterpret_cast<float4*>(Ss + i * KS + j4) = *reinterpret_cast<const float4*>(Sg + (int64_t)i * DK + j4);
+    for (int nh = blockIdx.x; nh < NH; nh += gridDim.x) {
+        const int p = pos[nh];
+        __syncthreads();  // every thread has read pos (and the previous pair's smem) before anything moves
+        if (p < 0 || p >= C) continue;
+        if (p + 1 < C) {
+            if (threadIdx.x == 0) pos[nh] = p + 1;
+            continue;
+        }
+        // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
+        stage_rows<DK>(ks, KS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        stage_rows<DV>(vs, DV, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        for (int t = threadIdx.x; t < C; t += blockDim.x) {
+            as[t] = abuf[(int64_t)nh * C + t];
+            bs[t] = bbuf[(int64_t)nh * C + t];
         }
         __syncthreads();
-        chunk_advance<DK, RTB, C>(Ss, ws, vs + r * RTB, DV, ks, dCs, es);
-        for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-            const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-            const float4 x = *reinterpret_cast<const float4*>(Ss + i * KS + j4);
-            *reinterpret_cast<float4*>(Sg + (int64_t)i * DK + j4) = x;
-            *reinterpret_cast<float4*>(Rg + (int64_t)i * DK + j4) = x;
+        chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, ws, KS, vs, DV, dCs);  // u0 overwrites v in place
+        for (int r = 0; r < Cf::NTB; ++r) {
+            float* Sg = S_b + ((int64_t)nh * DV + r * RTB) * DK;
+            float* Rg = R + ((int64_t)nh * DV + r * RTB) * DK;
+            for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
+                const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
+                *reinterpret_cast<float4*>(Ss + i * KS + j4) = *reinterpret_cast<const float4*>(Sg + (int64_t)i * DK + j4);
+            }
+            __syncthreads();
+            chunk_advance<DK, RTB, C>(Ss, ws, vs + r * RTB, DV, ks, dCs, es, Sg, Rg);
         }
-        __syncthreads();
+        if (threadIdx.x == 0) pos[nh] = 0;
     }
-    if (threadIdx.x == 0) pos[nh] = 0;
 }
 
 }  // namespace gdn

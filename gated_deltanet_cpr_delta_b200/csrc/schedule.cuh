@@ -23,6 +23,38 @@ __device__ __forceinline__ float fadd(float a, float b) { return __fadd_rn(a, b)
 __device__ __forceinline__ float fsub(float a, float b) { return __fsub_rn(a, b); }
 __device__ __forceinline__ float ffma(float a, float b, float c) { return __fmaf_rn(a, b, c); }
 
+// Two fp32 lanes in one 64-bit register, for the sm_100 packed instructions
+// fma.rn.f32x2 / mul.rn.f32x2.  Each lane is rounded exactly like the scalar
+// fma.rn.f32 / mul.rn.f32 (no flush-to-zero), so packing two independent
+// chains changes no bit of either; it halves the issue slots they take.
+typedef unsigned long long f2x;
+
+__device__ __forceinline__ f2x pk2(float lo, float hi)
+{
+    f2x r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void up2(f2x x, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+
+__device__ __forceinline__ f2x ffma2(f2x a, f2x b, f2x c)
+{
+    f2x d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ f2x fmul2(f2x a, f2x b)
+{
+    f2x d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // Partial results of the 8-leaf tree ((p0+p1)+(p2+p3)) + ((p4+p5)+(p6+p7)),
 // pushed leaf by leaf (l = 0..7, known at compile time after unrolling).
 // t0 holds the final value after leaf 7.

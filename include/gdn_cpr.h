@@ -114,8 +114,9 @@ size_t gdn_cpr_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H,
  *   cu_seqlens_host host   [num_seqs+1] int32, the same values.  It sizes the
  *     launch grids and is validated on the host: cu[0] == 0, non-decreasing,
  *     cu[num_seqs] == total_tokens.  The kernels check the device copy against
- *     the host-derived totals.  If the two copies disagree, the kernels write
- *     nothing, and the outputs are left unspecified but in bounds.
+ *     the host copy: chunk totals and a 64-bit position-sensitive hash of
+ *     the values.  If the two copies disagree, the kernels write nothing, and
+ *     the outputs keep their previous contents.
  *   Chunks are aligned to each sequence's own token 0, so results do not
  *   depend on batch composition or packing.
  * Outputs:
