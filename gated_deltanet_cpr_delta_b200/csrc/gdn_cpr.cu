@@ -2,13 +2,15 @@
 //
 // Validates arguments on the host, carves the caller's workspace and enqueues
 // the kernels of kernels.cuh on the caller's stream.  It allocates no device
-// memory, never synchronises, and keeps no global mutable state.
+// memory and never synchronises.  Its only global mutable state is the
+// per-device address cache of gdn_cpr_forward_noalloc (end of file).
 #include "gdn_cpr.h"
 #include "kernels.cuh"
 
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 namespace {
 
@@ -353,3 +355,58 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation forward
+// Workspace for gdn_cpr_forward_noalloc: a fixed device array that lives in this
+// library's module, so callers that cannot allocate device memory still get
+// a CPR forward.  Every device that loads the library holds these bytes until
+// the process exits.  All calls on a device share them.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = (size_t)GDN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address must come
+// from cudaGetSymbolAddress, called once per device with that device current.
+gdn_status_t noalloc_scratch(void** out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" gdn_status_t gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
+                                                const float* beta, const float* state_in,
+                                                const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                                int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                                                int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
+                                                gdn_dtype_t out_dtype, void* o, float* chunk_states,
+                                                const gdn_cache_t* cache_out, void* stream)
+{
+    if (num_seqs < 0 || total_tokens < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0)
+        return GDN_ERR_INVALID_ARG;
+    if (carve(nullptr, total_tokens / C, num_seqs, H, d_k, d_v, C).bytes > kNoallocScratchBytes)
+        return GDN_ERR_WORKSPACE;  // the batch needs more than the fixed scratch holds
+    void* ws = nullptr;
+    const gdn_status_t st = noalloc_scratch(&ws);
+    if (st != GDN_OK) return st;
+    // Nothing in the workspace has to start at zero: every kernel writes its
+    // part of it (offset tables, error word, w, u0, decays) before any read.
+    return gdn_cpr_forward(q, k, v, alpha, beta, state_in, cu_seqlens, cu_seqlens_host, num_seqs, total_tokens,
+                           H, d_k, d_v, C, in_dtype, out_dtype, o, chunk_states, cache_out, ws,
+                           kNoallocScratchBytes, stream);
+}

@@ -23,7 +23,11 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 
 #: exported symbols of include/gdn_cpr.h
 SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
-           "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed")
+           "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed",
+           "gdn_cpr_forward_noalloc")
+
+#: size of the fixed device array behind gdn_cpr_forward_noalloc (GDN_NOALLOC_SCRATCH_BYTES)
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class GdnError(RuntimeError):
@@ -68,6 +72,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_cpr_forward_timed.argtypes = lib.gdn_cpr_forward.argtypes + [P]
     lib.gdn_decode_step_timed.restype = ctypes.c_int
     lib.gdn_decode_step_timed.argtypes = lib.gdn_decode_step.argtypes + [P]
+    lib.gdn_cpr_forward_noalloc.restype = ctypes.c_int
+    lib.gdn_cpr_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
+                                            ctypes.c_int, P, P, ctypes.POINTER(CacheStruct), P]
     _lib = lib
     return lib
 
@@ -203,3 +210,35 @@ def gdn_decode_step(q, k, v, alpha, beta, cache: Dict[str, torch.Tensor], C: int
         st = lib.gdn_decode_step_timed(*args, _event_array(events, 3))
     _check(st, "gdn_decode_step")
     return o
+
+
+def gdn_cpr_forward_noalloc(q, k, v, alpha, beta, cu_seqlens, C: int, *, cu_seqlens_host=None, state_in=None,
+                            out_dtype=None, cache_out: Optional[Dict[str, torch.Tensor]] = None, o=None,
+                            chunk_states=None):
+    """CPR forward whose workspace is the library's fixed device array (see
+    gdn_cpr_forward_noalloc in include/gdn_cpr.h): for callers that cannot
+    allocate device memory when they call.  Same arguments and results as
+    :func:`gdn_cpr_forward` without ``workspace``; ``o`` and ``chunk_states``
+    should be passed in by such callers (they are allocated here only when
+    omitted).  Calls that overlap on the GPU race on the shared array."""
+    lib = load_library()
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu().tolist()
+    cu_h = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    N = len(cu_seqlens_host) - 1
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    dev = k.device
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=out_dtype, device=dev)
+    if chunk_states is None:
+        chunk_states = torch.empty(gdn_num_chunk_states(cu_seqlens_host, C), H, dv, dk, dtype=torch.float32,
+                                   device=dev)
+    cs = _cache_struct(cache_out) if cache_out is not None else None
+    st = lib.gdn_cpr_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state_in),
+                                     _ptr(cu_seqlens), cu_h, N, T, H, dk, dv, C, _dt(q.dtype), _dt(out_dtype),
+                                     _ptr(o), _ptr(chunk_states), ctypes.byref(cs) if cs is not None else None,
+                                     _stream(dev))
+    _check(st, "gdn_cpr_forward_noalloc")
+    return o, chunk_states

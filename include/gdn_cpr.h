@@ -22,7 +22,9 @@
  * Conventions common to every call:
  *  - All tensors are caller-owned device memory unless marked "host".
  *    The library never allocates device memory and keeps no global mutable
- *    state.  It never synchronises the device.
+ *    state.  It never synchronises the device.  The one exception is
+ *    gdn_cpr_forward_noalloc (end of this file): it uses a fixed device array
+ *    inside the library and caches that array's address per device.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
  *    The call returns once the kernels are enqueued.
  *  - Layouts are row-major and densely packed:
@@ -195,6 +197,45 @@ gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v,
                                    int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v, int32_t C,
                                    gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
                                    void* o, void* stream, void* const* events);
+
+/*
+ * Forward without any device allocation, for callers that cannot allocate
+ * device memory at the point of the call.  Examples: a plugin whose host
+ * framework owns all device memory and forbids allocation inside its execute
+ * callback; a process that has already reserved the whole device for its own
+ * memory pool; a latency-critical loop that cannot take the implicit device
+ * synchronisation of cudaMalloc.  The pages have no counterpart to this call;
+ * it exists for such integrations only.
+ *
+ * It is gdn_cpr_forward, with the same arguments, results and errors, except
+ * that its workspace is a fixed array of GDN_NOALLOC_SCRATCH_BYTES inside the
+ * library.  The caller still passes every input and output.
+ *  - Limit: the batch must fit the fixed array, i.e.
+ *    gdn_cpr_workspace_size(total_tokens, num_seqs, H, d_k, d_v, C) <=
+ *    GDN_NOALLOC_SCRATCH_BYTES.  At d_k = d_v = 128 and C = 64 that is about
+ *    65,000 (token, head) pairs, for example 4,000 tokens with 16 heads.  Larger
+ *    batches return GDN_ERR_WORKSPACE before anything is enqueued.
+ *  - Every device that loads the library holds the array until the process exits.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it.  Make
+ *    that first call before any stream capture begins.
+ *  - All calls on a device share the one array, and it keeps the last call's
+ *    contents; no part of it needs to start at zero.  Calls whose work
+ *    overlaps on the GPU (different streams, or different host threads)
+ *    race on the array and give wrong results; serialise them.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+gdn_status_t gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v,
+                                     const float* alpha, const float* beta,
+                                     const float* state_in,
+                                     const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                     int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                     int32_t d_k, int32_t d_v, int32_t C,
+                                     gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                                     void* o, float* chunk_states, const gdn_cache_t* cache_out,
+                                     void* stream);
 
 #ifdef __cplusplus
 }
