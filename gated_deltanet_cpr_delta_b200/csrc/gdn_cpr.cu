@@ -156,7 +156,7 @@ gdn_status_t launch_forward(const FwdArgs& a)
     if (a.tot.tasks > 0) {
         constexpr size_t sm = TC::SMEM;
         if (set_smem(gdn::k_tok<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
-        gdn::k_tok<D, D, C><<<(unsigned)(a.tot.tasks * a.H * TC::NT), TC::THREADS, sm, a.stream>>>(
+        gdn::k_tok<D, D, C><<<(unsigned)(a.tot.tasks * a.H), TC::THREADS, sm, a.stream>>>(
             a.q, a.k, a.v, a.alpha, a.beta, a.cu, a.ws.cto, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.out_bf16,
             a.states, a.o, a.cache ? a.cache->R : nullptr);
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;

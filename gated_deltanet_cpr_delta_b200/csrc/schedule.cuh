@@ -160,6 +160,23 @@ __device__ __forceinline__ void store1(void* base, int64_t off, int bf16, float 
     else reinterpret_cast<float*>(base)[off] = x;
 }
 
+// Asynchronous global -> shared copies (cp.async; 16 bytes bypass L1, 4 bytes go through it).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
 // Largest n in [0, N) with tab[n] <= g (tab non-decreasing, tab[0] = 0 <= g < tab[N]).
 __device__ __forceinline__ int find_seq(const int32_t* tab, int N, int g)
 {
