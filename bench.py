@@ -70,13 +70,13 @@ def decode_tok_bytes(dk: int, dv: int, esz: int, out_esz: int):
 
 # DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
 # dram__bytes_write.sum), keyed by kernel, valid only for the kernel source
-# it was taken from (sha256 of csrc/kernels.cuh + csrc/schedule.cuh).
+# it was taken from (sha256 of the csrc/*.cuh kernel sources).
 NCU_TRAFFIC = {}
 
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("kernels.cuh", "schedule.cuh"):
+    for f in ("kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_pchunk.cuh", "k_decode.cuh"):
         with open(os.path.join(ROOT, "gated_deltanet_cpr_delta_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgdn_cpr.so")
 SOURCES = ["gdn_cpr.cu"]
-DEPS = ["gdn_cpr.cu", "kernels.cuh", "schedule.cuh"]
+DEPS = ["gdn_cpr.cu", "kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_pchunk.cuh", "k_decode.cuh"]
 HEADERS = [os.path.join(ROOT, "include", "gdn_cpr.h")]
 
 

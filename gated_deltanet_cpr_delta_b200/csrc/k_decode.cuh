@@ -1,0 +1,139 @@
+// k_decode.cuh -- decode step: k_dec_tok and k_dec_resync (sm_100a).
+#pragma once
+
+#include "k_ptok.cuh"
+#include "k_pchunk.cuh"
+
+namespace gdn {
+
+// ------------------------------------------------------------------ decode
+template <int DK, int DV>
+struct DecCfg {
+    using RS = RowSplit<DK>;
+    static constexpr int RT = DV < 32 ? DV : 32;  // rows per CTA
+    static constexpr int NT = DV / RT;
+    static constexpr int THREADS = RT * RS::TPR;
+};
+
+// One decode token per (sequence, head), one CTA per row tile: P_tok on the
+// running state R; tile 0 also appends the token to the buffer at slot pos.
+// pos itself is advanced by k_dec_resync, which runs next.
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(DecCfg<DK, DV>::THREADS)
+k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+          const float* __restrict__ alpha, const float* __restrict__ beta, int in_bf16, int out_bf16,
+          float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos, void* __restrict__ o)
+{
+    using Cf = DecCfg<DK, DV>;
+    using RS = typename Cf::RS;
+    __shared__ __align__(16) float ks[RS::KS];
+    __shared__ __align__(16) float qs[RS::KS];
+    __shared__ __align__(16) float vs[Cf::RT];
+    const int nh = blockIdx.x / Cf::NT, r = blockIdx.x % Cf::NT;
+    const int p = pos[nh];
+    if (p < 0 || p >= C) return;
+    stage_rows<DK>(ks, RS::KS, k, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
+    stage_rows<DK>(qs, RS::KS, q, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
+    for (int e = threadIdx.x; e < Cf::RT / 8; e += blockDim.x) {
+        float x[8];
+        load8(v, (int64_t)nh * DV + r * Cf::RT + e * 8, in_bf16, x);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) vs[e * 8 + m] = x[m];
+    }
+    const float a = __ldg(alpha + nh), b = __ldg(beta + nh);
+    const int row = threadIdx.x / RS::TPR, part = threadIdx.x % RS::TPR;
+    const int grow = r * Cf::RT + row;
+    float* Rrow = R + ((int64_t)nh * DV + grow) * DK + part * RS::EPT;
+    f2x Rp[RS::L];
+    load_row_pairs<DK>(Rp, Rrow);
+    __syncthreads();
+    const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
+    store_row_pairs<DK>(Rrow, Rp);
+    if (part == 0) store1(o, (int64_t)nh * DV + grow, out_bf16, ot);
+    if (r == 0) {  // append the raw token to the buffer at slot p
+        const int esz = in_bf16 ? 2 : 4;
+        for (int e = threadIdx.x; e < DK * esz / 16; e += blockDim.x)
+            reinterpret_cast<uint4*>(kbuf)[((int64_t)nh * C + p) * (DK * esz / 16) + e] =
+                __ldg(reinterpret_cast<const uint4*>(k) + (int64_t)nh * (DK * esz / 16) + e);
+        for (int e = threadIdx.x; e < DV * esz / 16; e += blockDim.x)
+            reinterpret_cast<uint4*>(vbuf)[((int64_t)nh * C + p) * (DV * esz / 16) + e] =
+                __ldg(reinterpret_cast<const uint4*>(v) + (int64_t)nh * (DV * esz / 16) + e);
+        if (threadIdx.x == 0) {
+            abuf[(int64_t)nh * C + p] = a;
+            bbuf[(int64_t)nh * C + p] = b;
+        }
+    }
+}
+
+template <int DK, int DV, int C>
+struct ResyncSmem {
+    using Cf = ChunkCfg<DK, DV, C>;
+    static constexpr int KS_OFF = 0;
+    static constexpr int VS_OFF = KS_OFF + C * Cf::KS;
+    static constexpr int WS_OFF = VS_OFF + C * DV;
+    static constexpr int DM_OFF = WS_OFF + C * Cf::KS;
+    static constexpr int CT_OFF = DM_OFF + ((Cf::C1 * Cf::C1 + 3) / 4) * 4;
+    static constexpr int SS_OFF = CT_OFF + C * Cf::CT;
+    static constexpr int ES_OFF = SS_OFF + Cf::RTB * Cf::KS;
+    static constexpr int AB_OFF = ES_OFF + C * Cf::RTB;
+    static constexpr int DC_OFF = AB_OFF + 2 * C;
+    static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
+};
+
+// Advances pos after k_dec_tok appended a token at slot pos, and resyncs
+// where that token completed a chunk: S_b <- P_chunk(S_b, buffer), R <- S_b,
+// pos <- 0.  Persistent: CTA b handles (sequence, head) pairs b, b + grid, ...
+// A pos outside [0, C) is left unchanged.
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256)
+k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
+             const float* bbuf, int32_t* pos)
+{
+    using Cf = ChunkCfg<DK, DV, C>;
+    using Sm = ResyncSmem<DK, DV, C>;
+    constexpr int KS = Cf::KS, RTB = Cf::RTB;
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    float* ks = sm + Sm::KS_OFF;
+    float* vs = sm + Sm::VS_OFF;
+    float* ws = sm + Sm::WS_OFF;
+    float* Dm = sm + Sm::DM_OFF;
+    float* cT = sm + Sm::CT_OFF;
+    float* Ss = sm + Sm::SS_OFF;
+    float* es = sm + Sm::ES_OFF;
+    float* as = sm + Sm::AB_OFF;
+    float* bs = as + C;
+    float* dCs = sm + Sm::DC_OFF;
+
+    for (int nh = blockIdx.x; nh < NH; nh += gridDim.x) {
+        const int p = pos[nh];
+        __syncthreads();  // every thread has read pos (and the previous pair's smem) before anything moves
+        if (p < 0 || p >= C) continue;
+        if (p + 1 < C) {
+            if (threadIdx.x == 0) pos[nh] = p + 1;
+            continue;
+        }
+        // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
+        stage_rows<DK>(ks, KS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        stage_rows<DV>(vs, DV, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        for (int t = threadIdx.x; t < C; t += blockDim.x) {
+            as[t] = abuf[(int64_t)nh * C + t];
+            bs[t] = bbuf[(int64_t)nh * C + t];
+        }
+        __syncthreads();
+        chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, ws, KS, vs, DV, dCs);  // u0 overwrites v in place
+        for (int r = 0; r < Cf::NTB; ++r) {
+            float* Sg = S_b + ((int64_t)nh * DV + r * RTB) * DK;
+            float* Rg = R + ((int64_t)nh * DV + r * RTB) * DK;
+            for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
+                const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
+                *reinterpret_cast<float4*>(Ss + i * KS + j4) = *reinterpret_cast<const float4*>(Sg + (int64_t)i * DK + j4);
+            }
+            __syncthreads();
+            chunk_advance<DK, RTB, C>(Ss, ws, vs + r * RTB, DV, ks, dCs, es, Sg, Rg);
+        }
+        if (threadIdx.x == 0) pos[nh] = 0;
+    }
+}
+
+}  // namespace gdn

@@ -1,0 +1,387 @@
+// k_pchunk.cuh -- chunk-boundary update P_chunk: k_prep, k_chain, k_cache_fill (sm_100a).
+#pragma once
+
+#include "k_ptok.cuh"
+
+namespace gdn {
+
+// ------------------------------------------------------------------ P_chunk
+template <int DK, int DV, int C>
+struct ChunkCfg {
+    static constexpr int KS = DK + 4;      // padded k / w / S row stride
+    static constexpr int C1 = C + 1;       // decay matrix row stride
+    static constexpr int CT = C + 4;       // c^T row stride
+    static constexpr int DCS = C + 4;      // stride of D[C][.] rows in the workspace
+    static constexpr int RTB = DV < 32 ? DV : 32;  // boundary-state rows per tile
+    static constexpr int NTB = DV / RTB;
+    static constexpr int THREADS = 256;
+};
+
+// VEC consecutive floats from smem (VEC = 4 or 2; 4*VEC-byte aligned).
+template <int VEC>
+__device__ __forceinline__ void lds_n(float (&r)[VEC], const float* s)
+{
+    if constexpr (VEC == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(s);
+        r[0] = x.x; r[1] = x.y; r[2] = x.z; r[3] = x.w;
+    } else {
+        const float2 x = *reinterpret_cast<const float2*>(s);
+        r[0] = x.x; r[1] = x.y;
+    }
+}
+
+// tree(x_a, y_b) for an RA x RB block of row pairs, all rows of stride KS in
+// smem: xa[r] = row r of the first operand, yb[c] = row c of the second.
+// The leaves run in ascending j; VEC elements are read at a time.
+template <int DK, int KS, int RA, int RB>
+__device__ __forceinline__ void tree_block(const float* const (&xa)[RA], const float* const (&yb)[RB],
+                                           float (&out)[RA][RB])
+{
+    constexpr int L = DK / kLeaves;
+    constexpr int VEC = (L % 4 == 0) ? 4 : 2;
+    TreeAcc st[RA][RB];
+#pragma unroll
+    for (int l = 0; l < kLeaves; ++l) {
+        float acc[RA][RB];
+#pragma unroll
+        for (int m = 0; m < L; m += VEC) {
+            float a[RA][VEC], b[RB][VEC];
+#pragma unroll
+            for (int r = 0; r < RA; ++r) lds_n<VEC>(a[r], xa[r] + l * L + m);
+#pragma unroll
+            for (int c = 0; c < RB; ++c) lds_n<VEC>(b[c], yb[c] + l * L + m);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+#pragma unroll
+                for (int r = 0; r < RA; ++r)
+#pragma unroll
+                    for (int c = 0; c < RB; ++c)
+                        acc[r][c] = (m + e == 0) ? fmul(a[r][e], b[c][e]) : ffma(a[r][e], b[c][e], acc[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < RA; ++r)
+#pragma unroll
+            for (int c = 0; c < RB; ++c) tree_push(st[r][c], l, acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < RA; ++r)
+#pragma unroll
+        for (int c = 0; c < RB; ++c) out[r][c] = st[r][c].t0;
+}
+
+// Forward substitution of one column, right-looking and fully unrolled: once
+// token s is final, its term enters every later token's chain.  For each
+// token t the chain still runs over s = 1..t-1 in ascending order.
+// acc[t] holds the chain start on entry and the column's result on exit.
+template <int C, int CT>
+__device__ __forceinline__ void fwd_subst(float (&acc)[C], const float* cT, const float* bs)
+{
+#pragma unroll
+    for (int sig = 0; sig < C; ++sig) {
+        acc[sig] = fmul(bs[sig], acc[sig]);
+        const float x = acc[sig];
+#pragma unroll
+        for (int tg = (sig + 1) / 4; tg < C / 4; ++tg) {
+            const float4 c4 = *reinterpret_cast<const float4*>(cT + sig * CT + 4 * tg);
+            if (4 * tg + 0 > sig) acc[4 * tg + 0] = ffma(-c4.x, x, acc[4 * tg + 0]);
+            if (4 * tg + 1 > sig) acc[4 * tg + 1] = ffma(-c4.y, x, acc[4 * tg + 1]);
+            if (4 * tg + 2 > sig) acc[4 * tg + 2] = ffma(-c4.z, x, acc[4 * tg + 2]);
+            if (4 * tg + 3 > sig) acc[4 * tg + 3] = ffma(-c4.w, x, acc[4 * tg + 3]);
+        }
+    }
+}
+
+// P_chunk part 1 for one chunk, by one CTA.  ks [C][KS], vs [C][DV], as/bs [C]
+// in smem.  Dm [(C+1)^2] and cT [C][CT] are smem scratch.  Writes
+//   w_t  -> wout[(t-1)*ldw + j],   u0_t -> uout[(t-1)*ldu + i],   D[C][s] -> dCout[s]
+// (any address space).  uout may alias vs: each column of vs is read only by
+// the thread that later writes that column of uout, and only before it does.
+template <int DK, int DV, int C>
+__device__ __forceinline__ void chunk_prep(const float* ks, const float* vs, const float* as, const float* bs,
+                                           float* Dm, float* cT, float* wout, int ldw, float* uout, int ldu,
+                                           float* dCout)
+{
+    using Cf = ChunkCfg<DK, DV, C>;
+    constexpr int KS = Cf::KS, C1 = Cf::C1, CT = Cf::CT;
+    // decay products D[t][s] = D[t-1][s] * alpha_t, D[s][s] = 1  (tokens 1..C)
+    for (int s = threadIdx.x; s <= C; s += blockDim.x) {
+        float d = 1.0f;
+        Dm[s * C1 + s] = d;
+        for (int t = s + 1; t <= C; ++t) {
+            d = fmul(d, as[t - 1]);
+            Dm[t * C1 + s] = d;
+        }
+    }
+    __syncthreads();
+    // c[t][s] = D[t][s] * tree(k_s, k_t), stored transposed: cT[s-1][t-1];
+    // 4x4 blocks of the strictly lower triangle, one block per thread
+    constexpr int NB = C / 4, NBLK = NB * (NB + 1) / 2;
+    for (int blk = threadIdx.x; blk < NBLK; blk += blockDim.x) {
+        int bt = 0;
+        while ((bt + 1) * (bt + 2) / 2 <= blk) ++bt;
+        const int bsg = blk - bt * (bt + 1) / 2;
+        const float* const xa[4] = {ks + (4 * bt) * KS, ks + (4 * bt + 1) * KS, ks + (4 * bt + 2) * KS,
+                                    ks + (4 * bt + 3) * KS};
+        const float* const yb[4] = {ks + (4 * bsg) * KS, ks + (4 * bsg + 1) * KS, ks + (4 * bsg + 2) * KS,
+                                    ks + (4 * bsg + 3) * KS};
+        float G[4][4];
+        tree_block<DK, KS, 4, 4>(xa, yb, G);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int tau = 4 * bt + r, sig = 4 * bsg + c;
+                if (sig < tau) cT[sig * CT + tau] = fmul(Dm[(tau + 1) * C1 + (sig + 1)], G[r][c]);
+            }
+    }
+    if (dCout != nullptr)
+        for (int s = threadIdx.x; s <= C; s += blockDim.x) dCout[s] = Dm[C * C1 + s];
+    __syncthreads();
+    // forward substitution, one column per thread
+    for (int col = threadIdx.x; col < DV + DK; col += blockDim.x) {
+        float acc[C];
+        if (col < DV) {
+#pragma unroll
+            for (int tau = 0; tau < C; ++tau) acc[tau] = vs[tau * DV + col];
+            fwd_subst<C, CT>(acc, cT, bs);
+#pragma unroll
+            for (int tau = 0; tau < C; ++tau) uout[tau * ldu + col] = acc[tau];
+        } else {
+            const int j = col - DV;
+#pragma unroll
+            for (int tau = 0; tau < C; ++tau) acc[tau] = fmul(Dm[(tau + 1) * C1], ks[tau * KS + j]);
+            fwd_subst<C, CT>(acc, cT, bs);
+#pragma unroll
+            for (int tau = 0; tau < C; ++tau) wout[tau * ldw + j] = acc[tau];
+        }
+    }
+    __syncthreads();
+}
+
+// P_chunk part 2 on a tile of RTB boundary-state rows, by one CTA:
+//   e_t[i] = D[C][t] * (u0_t[i] - tree(S_i, w_t)),
+//   S_ij <- chain_t fma(e_t[i], k_t[j], .) from D[C][0] * S_ij.
+// Ss [RTB][KS], ws [C][KS], ks [C][KS], us [C][ldu], dCs [C+1], es [C][RTB]
+// (scratch), all smem.  The new rows also go to dst1 / dst2 (global, row
+// stride DK) when non-null.
+template <int DK, int RTB, int C>
+__device__ __forceinline__ void chunk_advance(float* Ss, const float* ws, const float* us, int ldu,
+                                              const float* ks, const float* dCs, float* es, float* dst1,
+                                              float* dst2)
+{
+    constexpr int KS = DK + 4;
+    // phase 1: tiles of 4 tokens x 2 rows (rows ig and ig + RTB/2)
+    constexpr int IG = RTB / 2, TG = C / 4;
+    for (int tile = threadIdx.x; tile < TG * IG; tile += blockDim.x) {
+        const int ig = tile % IG, tg = tile / IG;
+        const float* const xa[4] = {ws + (4 * tg) * KS, ws + (4 * tg + 1) * KS, ws + (4 * tg + 2) * KS,
+                                    ws + (4 * tg + 3) * KS};
+        const float* const yb[2] = {Ss + ig * KS, Ss + (ig + IG) * KS};
+        float sw[4][2];
+        tree_block<DK, KS, 4, 2>(xa, yb, sw);
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int tau = 4 * tg + r, i = ig + c * IG;
+                es[tau * RTB + i] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], sw[r][c]));
+            }
+    }
+    __syncthreads();
+    // phase 2: tiles of 4 rows x 4 columns
+    constexpr int JG = DK / 4, IG2 = RTB / 4;
+    const float d0 = dCs[0];
+    for (int tile = threadIdx.x; tile < IG2 * JG; tile += blockDim.x) {
+        const int jg = tile % JG, ig = tile / JG;
+        float acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float4 s = *reinterpret_cast<const float4*>(Ss + (4 * ig + r) * KS + 4 * jg);
+            acc[r][0] = fmul(d0, s.x); acc[r][1] = fmul(d0, s.y);
+            acc[r][2] = fmul(d0, s.z); acc[r][3] = fmul(d0, s.w);
+        }
+#pragma unroll 4
+        for (int tau = 0; tau < C; ++tau) {
+            const float4 e4 = *reinterpret_cast<const float4*>(es + tau * RTB + 4 * ig);
+            const float4 k4 = *reinterpret_cast<const float4*>(ks + tau * KS + 4 * jg);
+            const float ev[4] = {e4.x, e4.y, e4.z, e4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = ffma(ev[r], kv[c], acc[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float4 x = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+            *reinterpret_cast<float4*>(Ss + (4 * ig + r) * KS + 4 * jg) = x;  // element owned by this thread
+            if (dst1 != nullptr) *reinterpret_cast<float4*>(dst1 + (int64_t)(4 * ig + r) * DK + 4 * jg) = x;
+            if (dst2 != nullptr) *reinterpret_cast<float4*>(dst2 + (int64_t)(4 * ig + r) * DK + 4 * jg) = x;
+        }
+    }
+    __syncthreads();
+}
+
+template <int DK, int DV, int C>
+struct PrepSmem {
+    using Cf = ChunkCfg<DK, DV, C>;
+    static constexpr int KS_OFF = 0;
+    static constexpr int VS_OFF = KS_OFF + C * Cf::KS;
+    static constexpr int DM_OFF = VS_OFF + C * DV;
+    static constexpr int CT_OFF = DM_OFF + ((Cf::C1 * Cf::C1 + 3) / 4) * 4;
+    static constexpr int AB_OFF = CT_OFF + C * Cf::CT;
+    static constexpr size_t BYTES = sizeof(float) * (AB_OFF + 2 * C);
+};
+
+// P_chunk part 1 for every full chunk: one CTA per (full chunk, head).
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256)
+k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
+       const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ fco,
+       const int32_t* __restrict__ err, int N, int H, int in_bf16,
+       float* __restrict__ w_ws, float* __restrict__ u_ws, float* __restrict__ dC_ws)
+{
+    using Cf = ChunkCfg<DK, DV, C>;
+    using Sm = PrepSmem<DK, DV, C>;
+    if (__ldg(err)) return;
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    float* ks = sm + Sm::KS_OFF;
+    float* vs = sm + Sm::VS_OFF;
+    float* Dm = sm + Sm::DM_OFF;
+    float* cT = sm + Sm::CT_OFF;
+    float* as = sm + Sm::AB_OFF;
+    float* bs = as + C;
+
+    const int task = blockIdx.x;
+    const int h = task % H, g = task / H;
+    const int n = find_seq(fco, N, g);
+    const int64_t tok0 = (int64_t)__ldg(cu + n) + (int64_t)(g - __ldg(fco + n)) * C;
+    stage_rows<DK>(ks, Cf::KS, k, tok0, C, H, h, in_bf16, IdxIdentity());
+    stage_rows<DV>(vs, DV, v, tok0, C, H, h, in_bf16, IdxIdentity());
+    for (int t = threadIdx.x; t < C; t += blockDim.x) {
+        as[t] = __ldg(alpha + (tok0 + t) * H + h);
+        bs[t] = __ldg(beta + (tok0 + t) * H + h);
+    }
+    __syncthreads();
+    chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, w_ws + (int64_t)task * C * DK, DK,
+                          u_ws + (int64_t)task * C * DV, DV, dC_ws + (int64_t)task * Cf::DCS);
+}
+
+template <int DK, int DV, int C>
+struct ChainSmem {
+    using Cf = ChunkCfg<DK, DV, C>;
+    static constexpr int SS_OFF = 0;
+    static constexpr int WS_OFF = SS_OFF + Cf::RTB * Cf::KS;
+    static constexpr int KS_OFF = WS_OFF + C * Cf::KS;
+    static constexpr int US_OFF = KS_OFF + C * Cf::KS;
+    static constexpr int ES_OFF = US_OFF + C * Cf::RTB;
+    static constexpr int DC_OFF = ES_OFF + C * Cf::RTB;
+    static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
+};
+
+// Boundary states: one CTA per (sequence, head, row tile), serial over the
+// sequence's full chunks.  Writes chunk_states[so[n] + c] for c = 0..floor(L/C).
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256)
+k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const int32_t* __restrict__ cu,
+        const int32_t* __restrict__ fco, const int32_t* __restrict__ so, const int32_t* __restrict__ err,
+        int N, int H, int in_bf16, const float* __restrict__ w_ws, const float* __restrict__ u_ws,
+        const float* __restrict__ dC_ws, float* __restrict__ states)
+{
+    using Cf = ChunkCfg<DK, DV, C>;
+    using Sm = ChainSmem<DK, DV, C>;
+    constexpr int KS = Cf::KS, RTB = Cf::RTB;
+    if (__ldg(err)) return;
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    float* Ss = sm + Sm::SS_OFF;
+    float* ws = sm + Sm::WS_OFF;
+    float* ks = sm + Sm::KS_OFF;
+    float* us = sm + Sm::US_OFF;
+    float* es = sm + Sm::ES_OFF;
+    float* dCs = sm + Sm::DC_OFF;
+
+    const int r = blockIdx.x % Cf::NTB;
+    const int nh = blockIdx.x / Cf::NTB;
+    const int h = nh % H, n = nh / H;
+    const int seq0 = __ldg(cu + n);
+    const int nfull = (__ldg(cu + n + 1) - seq0) / C;
+    const int64_t slot0 = __ldg(so + n);
+    const int64_t g0 = __ldg(fco + n);
+    const int64_t row0 = (int64_t)r * RTB;
+
+    for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
+        const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (state_in != nullptr)
+            x = __ldg(reinterpret_cast<const float4*>(state_in + (((int64_t)n * H + h) * DV + row0 + i) * DK + j4));
+        *reinterpret_cast<float4*>(Ss + i * KS + j4) = x;
+        *reinterpret_cast<float4*>(states + ((slot0 * H + h) * DV + row0 + i) * DK + j4) = x;
+    }
+    for (int c = 0; c < nfull; ++c) {
+        __syncthreads();
+        const int64_t task = (g0 + c) * H + h;
+        const float* wsrc = w_ws + task * C * DK;
+        for (int e = threadIdx.x; e < C * (DK / 4); e += blockDim.x) {
+            const int t = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
+            *reinterpret_cast<float4*>(ws + t * KS + j4) = __ldg(reinterpret_cast<const float4*>(wsrc + t * DK + j4));
+        }
+        stage_rows<DK>(ks, KS, k, (int64_t)seq0 + (int64_t)c * C, C, H, h, in_bf16, IdxIdentity());
+        const float* usrc = u_ws + task * C * DV + row0;
+        for (int e = threadIdx.x; e < C * (RTB / 4); e += blockDim.x) {
+            const int t = e / (RTB / 4), i4 = (e % (RTB / 4)) * 4;
+            *reinterpret_cast<float4*>(us + t * RTB + i4) = __ldg(reinterpret_cast<const float4*>(usrc + t * DV + i4));
+        }
+        for (int s = threadIdx.x; s <= C; s += blockDim.x) dCs[s] = __ldg(dC_ws + task * Cf::DCS + s);
+        __syncthreads();
+        chunk_advance<DK, RTB, C>(Ss, ws, us, RTB, ks, dCs, es,
+                                  states + (((slot0 + c + 1) * H + h) * DV + row0) * DK, nullptr);
+    }
+}
+
+// Decode cache for a continuation: one CTA per (sequence, head).
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256)
+k_cache_fill(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
+             const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ so,
+             const int32_t* __restrict__ err, int N, int H, int in_bf16, const float* __restrict__ states,
+             float* S_b, float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, int32_t* pos)
+{
+    if (__ldg(err)) return;
+    const int nh = blockIdx.x;
+    const int n = nh / H, h = nh % H;
+    const int seq0 = __ldg(cu + n);
+    const int Ln = __ldg(cu + n + 1) - seq0;
+    const int p = Ln % C;
+    const int64_t last = (int64_t)__ldg(so + n) + Ln / C;
+    const float4* src = reinterpret_cast<const float4*>(states + (last * H + h) * (int64_t)DV * DK);
+    float4* sb = reinterpret_cast<float4*>(S_b + (int64_t)nh * DV * DK);
+    float4* rr = reinterpret_cast<float4*>(R + (int64_t)nh * DV * DK);
+    for (int e = threadIdx.x; e < DV * DK / 4; e += blockDim.x) {
+        const float4 x = src[e];
+        sb[e] = x;
+        if (p == 0) rr[e] = x;  // at a boundary the running state is the boundary state
+    }
+    const int esz = in_bf16 ? 2 : 4;
+    // the p tokens of the open chunk, raw copies in the input dtype
+    for (int e = threadIdx.x; e < p * (DK * esz / 16); e += blockDim.x) {
+        const int s = e / (DK * esz / 16), b16 = e % (DK * esz / 16);
+        const int64_t tok = (int64_t)seq0 + Ln - p + s;
+        reinterpret_cast<uint4*>(kbuf)[((int64_t)nh * C + s) * (DK * esz / 16) + b16] =
+            __ldg(reinterpret_cast<const uint4*>(k) + (tok * H + h) * (DK * esz / 16) + b16);
+    }
+    for (int e = threadIdx.x; e < p * (DV * esz / 16); e += blockDim.x) {
+        const int s = e / (DV * esz / 16), b16 = e % (DV * esz / 16);
+        const int64_t tok = (int64_t)seq0 + Ln - p + s;
+        reinterpret_cast<uint4*>(vbuf)[((int64_t)nh * C + s) * (DV * esz / 16) + b16] =
+            __ldg(reinterpret_cast<const uint4*>(v) + (tok * H + h) * (DV * esz / 16) + b16);
+    }
+    for (int s = threadIdx.x; s < p; s += blockDim.x) {
+        const int64_t tok = (int64_t)seq0 + Ln - p + s;
+        abuf[(int64_t)nh * C + s] = __ldg(alpha + tok * H + h);
+        bbuf[(int64_t)nh * C + s] = __ldg(beta + tok * H + h);
+    }
+    if (threadIdx.x == 0) pos[nh] = p;
+}
+
+}  // namespace gdn
