@@ -146,14 +146,27 @@ def dist_setup(n_gpus: int):
     return 0, 1, 0
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank timing over all ranks (the job's time is the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_sequence_ids(rank: int, per_rank: int):
+    """Weak scaling: rank r runs its own sequences r*per_rank .. (r+1)*per_rank-1
+    of the seeded workload, so no rank repeats another's data and no data-path
+    collective is needed."""
+    return range(rank * per_rank, (rank + 1) * per_rank)
+
+
+def job_throughput(tokens_per_rank: int, world: int, max_ms: float, steps: int) -> float:
+    """Whole-job tokens/s: the tokens all ranks processed / the slowest rank's time."""
+    return tokens_per_rank * world * steps / (max_ms / 1e3)
 
 
 def barrier(world: int):
@@ -253,7 +266,7 @@ def bench_decode(rank: int, world: int, warmup: int):
     Dc = DECODE
     N, H, D, C, Lp, S = Dc["N"], Dc["H"], Dc["D"], Dc["C"], Dc["Lp"], Dc["steps"]
     L = Lp + S
-    d = synth.make_batch_device(Dc["seed"], [L] * N, H, D, D, "bf16", seq_ids=range(rank * N, rank * N + N))
+    d = synth.make_batch_device(Dc["seed"], [L] * N, H, D, D, "bf16", seq_ids=rank_sequence_ids(rank, N))
     idx = torch.cat([torch.arange(n * L, n * L + Lp) for n in range(N)]).cuda()
     cu_p = [n * Lp for n in range(N + 1)]
     cache = gdn.new_cache(N, H, D, D, C, torch.bfloat16)
@@ -311,7 +324,7 @@ def run_native(args):
     gdn.load_library()
     W = WORKLOAD
     B, H, T, D, C = W["B"], W["H"], W["T"], W["D"], W["C"]
-    d = synth.make_batch_device(W["seed"], [T] * B, H, D, D, "bf16", seq_ids=range(rank * B, rank * B + B))
+    d = synth.make_batch_device(W["seed"], [T] * B, H, D, D, "bf16", seq_ids=rank_sequence_ids(rank, B))
     o = torch.empty(B * T, H, D, dtype=torch.bfloat16, device="cuda")
     st = torch.empty(gdn.gdn_num_chunk_states(d["cu_host"], C), H, D, D, dtype=torch.float32, device="cuda")
     ws = torch.empty(gdn.gdn_cpr_workspace_size(B * T, B, H, D, D, C), dtype=torch.uint8, device="cuda")
@@ -346,7 +359,7 @@ def run_native(args):
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_step = total_ms / K
     tokens = B * T * world
-    value = tokens / (ms_step / 1e3)
+    value = job_throughput(B * T, world, total_ms, K)
 
     # e2e: host (pinned) inputs -> device, forward, o -> host, every step
     hin = {n: d[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
