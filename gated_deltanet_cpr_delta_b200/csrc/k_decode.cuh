@@ -68,22 +68,25 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
 template <int DK, int DV, int C>
 struct ResyncSmem {
     using Cf = ChunkCfg<DK, DV, C>;
-    static constexpr int KS_OFF = 0;
-    static constexpr int VS_OFF = KS_OFF + C * Cf::KS;
-    static constexpr int WS_OFF = VS_OFF + C * DV;
-    static constexpr int DM_OFF = WS_OFF + C * Cf::KS;
+    using M = MmaAdv<DK, Cf::RTB, C>;
+    static constexpr int KS_OFF = 0;                                 // [C][KS] k
+    static constexpr int VS_OFF = KS_OFF + C * Cf::KS;               // [C][DV] v, then u0
+    static constexpr int WS_OFF = VS_OFF + C * DV;                   // [C][KS] w
+    static constexpr int DM_OFF = WS_OFF + C * Cf::KS;               // decays
     static constexpr int CT_OFF = DM_OFF + ((Cf::C1 * Cf::C1 + 3) / 4) * 4;
-    static constexpr int SS_OFF = CT_OFF + C * Cf::CT;
-    static constexpr int ES_OFF = SS_OFF + Cf::RTB * Cf::KS;
-    static constexpr int AB_OFF = ES_OFF + C * Cf::RTB;
+    static constexpr int SS_OFF = CT_OFF + C * Cf::CT;               // [RTB][KS] S tile
+    static constexpr int ES_OFF = SS_OFF + Cf::RTB * M::KS;          // [RTB][ES] e
+    static constexpr int KT_OFF = ES_OFF + Cf::RTB * M::ES;          // [DK][ES] k^T
+    static constexpr int AB_OFF = KT_OFF + DK * M::ES;
     static constexpr int DC_OFF = AB_OFF + 2 * C;
     static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
 };
 
 // Advances pos after k_dec_tok appended a token at slot pos, and resyncs
 // where that token completed a chunk: S_b <- P_chunk(S_b, buffer), R <- S_b,
-// pos <- 0.  Persistent: CTA b handles (sequence, head) pairs b, b + grid, ...
-// A pos outside [0, C) is left unchanged.
+// pos <- 0.  P_chunk runs the same device functions as the prefill (chunk_prep,
+// then the tensor-core phases per row tile).  Persistent: CTA b handles
+// (sequence, head) pairs b, b + grid, ...  A pos outside [0, C) is left unchanged.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256)
 k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
@@ -91,6 +94,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ResyncSmem<DK, DV, C>;
+    using M = MmaAdv<DK, Cf::RTB, C>;
     constexpr int KS = Cf::KS, RTB = Cf::RTB;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
@@ -101,6 +105,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
     float* cT = sm + Sm::CT_OFF;
     float* Ss = sm + Sm::SS_OFF;
     float* es = sm + Sm::ES_OFF;
+    float* kT = sm + Sm::KT_OFF;
     float* as = sm + Sm::AB_OFF;
     float* bs = as + C;
     float* dCs = sm + Sm::DC_OFF;
@@ -116,21 +121,22 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
         // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
         stage_rows<DK>(ks, KS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
         stage_rows<DV>(vs, DV, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        stage_kT<DK, C>(kT, kbuf, (int64_t)nh * C, 1, 0, in_bf16);
         for (int t = threadIdx.x; t < C; t += blockDim.x) {
             as[t] = abuf[(int64_t)nh * C + t];
             bs[t] = bbuf[(int64_t)nh * C + t];
         }
         __syncthreads();
         chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, ws, KS, vs, DV, dCs);  // u0 overwrites v in place
+        float Sreg[M::P2][4];
         for (int r = 0; r < Cf::NTB; ++r) {
             float* Sg = S_b + ((int64_t)nh * DV + r * RTB) * DK;
             float* Rg = R + ((int64_t)nh * DV + r * RTB) * DK;
-            for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-                const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-                *reinterpret_cast<float4*>(Ss + i * KS + j4) = *reinterpret_cast<const float4*>(Sg + (int64_t)i * DK + j4);
-            }
+            mma_load_state<DK, RTB, C>(Sreg, Ss, Sg);
+            mma_phase1<DK, RTB, C>(Ss, ws, vs + r * RTB, DV, dCs, es);
             __syncthreads();
-            chunk_advance<DK, RTB, C>(Ss, ws, vs + r * RTB, DV, ks, dCs, es, Sg, Rg);
+            mma_phase2<DK, RTB, C>(Sreg, Ss, es, kT, dCs[0], in_bf16, Sg, Rg);
+            __syncthreads();
         }
         if (threadIdx.x == 0) pos[nh] = 0;
     }

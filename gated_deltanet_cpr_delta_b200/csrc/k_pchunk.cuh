@@ -158,67 +158,183 @@ __device__ __forceinline__ void chunk_prep(const float* ks, const float* vs, con
     __syncthreads();
 }
 
-// P_chunk part 2 on a tile of RTB boundary-state rows, by one CTA:
-//   e_t[i] = D[C][t] * (u0_t[i] - tree(S_i, w_t)),
-//   S_ij <- chain_t fma(e_t[i], k_t[j], .) from D[C][0] * S_ij.
-// Ss [RTB][KS], ws [C][KS], ks [C][KS], us [C][ldu], dCs [C+1], es [C][RTB]
-// (scratch), all smem.  The new rows also go to dst1 / dst2 (global, row
-// stride DK) when non-null.
+// ---------------------------------------------------------------- tensor-core P_chunk part 2
+// The two contractions of the boundary update on the tensor cores
+// (mma.sync m16n8k8, tf32 operands, fp32 accumulate), with every fp32
+// operand x split into hi = tf32(x) and lo = tf32(x - hi):
+//   phase 1: E[i][t] = sum_j S[i][j] w_t[j]; per 8-wide block of j, in
+//            ascending order: E += S_lo*w_hi, E += S_hi*w_lo, E += S_hi*w_hi;
+//            then e_t[i] = D[C][t] * (u0_t[i] - E[i][t]).
+//   phase 2: S'[i][j] = D[C][0]*S[i][j] + sum_t e_t[i] k_t[j]; accumulator
+//            starts at D[C][0]*S[i][j], then per 8-token block, ascending:
+//            S' += e_lo*k_hi, S' += e_hi*k_lo, S' += e_hi*k_hi.  When k is
+//            exactly tf32 (bf16 inputs), k_lo = 0 and that product is skipped.
+// The prefill chain and the decode resync run these same functions, so the
+// same operands give the same bits.  A CTA has 4 warps on a tile of RTB rows
+// (RTB = 16 or 32): warp w owns m16 tile w % MT and every WG-th n8 tile.
 template <int DK, int RTB, int C>
-__device__ __forceinline__ void chunk_advance(float* Ss, const float* ws, const float* us, int ldu,
-                                              const float* ks, const float* dCs, float* es, float* dst1,
-                                              float* dst2)
+struct MmaAdv {
+    static constexpr int MT = RTB / 16;             // m16 row tiles
+    static constexpr int WG = 4 / MT;               // warps sharing a row tile
+    static constexpr int NT1 = C / 8, NT2 = DK / 8;
+    static constexpr int P1 = (NT1 + WG - 1) / WG;  // phase-1 n8 tiles per warp
+    static constexpr int P2 = (NT2 + WG - 1) / WG;  // phase-2 n8 tiles per warp
+    static constexpr int KS = DK + 4;               // S and w row stride (floats)
+    static constexpr int ES = C + 4;                // e and k^T row stride (floats)
+    static constexpr int THREADS = 128;
+    static_assert(RTB == 16 || RTB == 32, "row tile");
+};
+
+// Phase 1 (warps 0..3): es[i*ES + t] = e_t[i] for the RTB rows of the tile.
+template <int DK, int RTB, int C>
+__device__ __forceinline__ void mma_phase1(const float* Ss, const float* ws, const float* us, int ldu,
+                                           const float* dCs, float* es)
 {
-    constexpr int KS = DK + 4;
-    // phase 1: tiles of 4 tokens x 2 rows (rows ig and ig + RTB/2)
-    constexpr int IG = RTB / 2, TG = C / 4;
-    for (int tile = threadIdx.x; tile < TG * IG; tile += blockDim.x) {
-        const int ig = tile % IG, tg = tile / IG;
-        const float* const xa[4] = {ws + (4 * tg) * KS, ws + (4 * tg + 1) * KS, ws + (4 * tg + 2) * KS,
-                                    ws + (4 * tg + 3) * KS};
-        const float* const yb[2] = {Ss + ig * KS, Ss + (ig + IG) * KS};
-        float sw[4][2];
-        tree_block<DK, KS, 4, 2>(xa, yb, sw);
+    using M = MmaAdv<DK, RTB, C>;
+    constexpr int KS = M::KS, ES = M::ES;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    if (warp >= 4) return;
+    const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
+    float acc[M::P1][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+    for (int q = 0; q < M::P1; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+#pragma unroll 2
+    for (int kb = 0; kb < DK / 8; ++kb) {
+        const int k0 = kb * 8;
+        uint32_t ah[4], al[4];
+        tf32_split(Ss[(r0 + g) * KS + k0 + t], ah[0], al[0]);
+        tf32_split(Ss[(r0 + g + 8) * KS + k0 + t], ah[1], al[1]);
+        tf32_split(Ss[(r0 + g) * KS + k0 + t + 4], ah[2], al[2]);
+        tf32_split(Ss[(r0 + g + 8) * KS + k0 + t + 4], ah[3], al[3]);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int tau = 4 * tg + r, i = ig + c * IG;
-                es[tau * RTB + i] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], sw[r][c]));
+        for (int q = 0; q < M::P1; ++q) {
+            const int nt = wg + M::WG * q;
+            if (nt < M::NT1) {
+                uint32_t bh[2], bl[2];
+                tf32_split(ws[(nt * 8 + g) * KS + k0 + t], bh[0], bl[0]);
+                tf32_split(ws[(nt * 8 + g) * KS + k0 + t + 4], bh[1], bl[1]);
+                mma_tf32(acc[q], al, bh);
+                mma_tf32(acc[q], ah, bl);
+                mma_tf32(acc[q], ah, bh);
             }
-    }
-    __syncthreads();
-    // phase 2: tiles of 4 rows x 4 columns
-    constexpr int JG = DK / 4, IG2 = RTB / 4;
-    const float d0 = dCs[0];
-    for (int tile = threadIdx.x; tile < IG2 * JG; tile += blockDim.x) {
-        const int jg = tile % JG, ig = tile / JG;
-        float acc[4][4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const float4 s = *reinterpret_cast<const float4*>(Ss + (4 * ig + r) * KS + 4 * jg);
-            acc[r][0] = fmul(d0, s.x); acc[r][1] = fmul(d0, s.y);
-            acc[r][2] = fmul(d0, s.z); acc[r][3] = fmul(d0, s.w);
-        }
-#pragma unroll 4
-        for (int tau = 0; tau < C; ++tau) {
-            const float4 e4 = *reinterpret_cast<const float4*>(es + tau * RTB + 4 * ig);
-            const float4 k4 = *reinterpret_cast<const float4*>(ks + tau * KS + 4 * jg);
-            const float ev[4] = {e4.x, e4.y, e4.z, e4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = ffma(ev[r], kv[c], acc[r][c]);
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const float4 x = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-            *reinterpret_cast<float4*>(Ss + (4 * ig + r) * KS + 4 * jg) = x;  // element owned by this thread
-            if (dst1 != nullptr) *reinterpret_cast<float4*>(dst1 + (int64_t)(4 * ig + r) * DK + 4 * jg) = x;
-            if (dst2 != nullptr) *reinterpret_cast<float4*>(dst2 + (int64_t)(4 * ig + r) * DK + 4 * jg) = x;
         }
     }
+#pragma unroll
+    for (int q = 0; q < M::P1; ++q) {
+        const int nt = wg + M::WG * q;
+        if (nt < M::NT1) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int i = r0 + g + (c >> 1) * 8, tau = nt * 8 + 2 * t + (c & 1);
+                es[i * ES + tau] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], acc[q][c]));
+            }
+        }
+    }
+}
+
+// Phase 2 (warps 0..3): Sreg (this lane's entries of the tile in the phase-2
+// accumulator layout) <- S'.  The new rows also go to Ss and, when non-null,
+// to dst1 / dst2 (global, row stride DK).  k_exact: k values are exact tf32.
+template <int DK, int RTB, int C>
+__device__ __forceinline__ void mma_phase2(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* es,
+                                           const float* kT, float d0, int k_exact, float* dst1, float* dst2)
+{
+    using M = MmaAdv<DK, RTB, C>;
+    constexpr int KS = M::KS, ES = M::ES;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    if (warp >= 4) return;
+    const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
+    float acc[M::P2][4];
+#pragma unroll
+    for (int q = 0; q < M::P2; ++q)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[q][c] = fmul(d0, Sreg[q][c]);
+#pragma unroll 2
+    for (int kb = 0; kb < C / 8; ++kb) {
+        const int k0 = kb * 8;
+        uint32_t ah[4], al[4];
+        tf32_split(es[(r0 + g) * ES + k0 + t], ah[0], al[0]);
+        tf32_split(es[(r0 + g + 8) * ES + k0 + t], ah[1], al[1]);
+        tf32_split(es[(r0 + g) * ES + k0 + t + 4], ah[2], al[2]);
+        tf32_split(es[(r0 + g + 8) * ES + k0 + t + 4], ah[3], al[3]);
+#pragma unroll
+        for (int q = 0; q < M::P2; ++q) {
+            const int nt = wg + M::WG * q;
+            if (nt < M::NT2) {
+                const float b0 = kT[(nt * 8 + g) * ES + k0 + t], b1 = kT[(nt * 8 + g) * ES + k0 + t + 4];
+                if (k_exact) {
+                    const uint32_t b[2] = {__float_as_uint(b0), __float_as_uint(b1)};
+                    mma_tf32(acc[q], al, b);
+                    mma_tf32(acc[q], ah, b);
+                } else {
+                    uint32_t bh[2], bl[2];
+                    tf32_split(b0, bh[0], bl[0]);
+                    tf32_split(b1, bh[1], bl[1]);
+                    mma_tf32(acc[q], al, bh);
+                    mma_tf32(acc[q], ah, bl);
+                    mma_tf32(acc[q], ah, bh);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < M::P2; ++q) {
+        const int nt = wg + M::WG * q;
+        if (nt < M::NT2) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) Sreg[q][c] = acc[q][c];
+#pragma unroll
+            for (int hrow = 0; hrow < 2; ++hrow) {
+                const int i = r0 + g + hrow * 8, j = nt * 8 + 2 * t;
+                const float2 x = make_float2(acc[q][2 * hrow], acc[q][2 * hrow + 1]);
+                *reinterpret_cast<float2*>(Ss + i * KS + j) = x;
+                if (dst1 != nullptr) *reinterpret_cast<float2*>(dst1 + (int64_t)i * DK + j) = x;
+                if (dst2 != nullptr) *reinterpret_cast<float2*>(dst2 + (int64_t)i * DK + j) = x;
+            }
+        }
+    }
+}
+
+// Load the RTB rows at src (global, row stride DK) into Ss and this lane's
+// phase-2 registers (warps 0..3).  Ends with a barrier.
+template <int DK, int RTB, int C>
+__device__ __forceinline__ void mma_load_state(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* src)
+{
+    using M = MmaAdv<DK, RTB, C>;
+    for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
+        const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (src != nullptr) x = *reinterpret_cast<const float4*>(src + (int64_t)i * DK + j4);
+        *reinterpret_cast<float4*>(Ss + i * M::KS + j4) = x;
+    }
     __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    if (warp < 4) {
+        const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
+#pragma unroll
+        for (int q = 0; q < M::P2; ++q) {
+            const int nt = wg + M::WG * q;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                Sreg[q][c] = nt < M::NT2 ? Ss[(r0 + g + (c >> 1) * 8) * M::KS + nt * 8 + 2 * t + (c & 1)] : 0.f;
+        }
+    }
+}
+
+// k of C tokens (rows of a [T, H, DK] input from token tok0, head h) -> kT
+// [DK][ES] fp32 (transposed; token index fastest across threads, so the
+// scattered stores hit consecutive banks).
+template <int DK, int C>
+__device__ __forceinline__ void stage_kT(float* kT, const void* k, int64_t tok0, int H, int h, int bf16)
+{
+    constexpr int ES = C + 4;
+    for (int e = threadIdx.x; e < C * (DK / 8); e += blockDim.x) {
+        const int tau = e % C, j8 = (e / C) * 8;
+        float x[8];
+        load8(k, ((tok0 + tau) * H + h) * (int64_t)DK + j8, bf16, x);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) kT[(j8 + m) * ES + tau] = x[m];
+    }
 }
 
 template <int DK, int DV, int C>
@@ -270,19 +386,22 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
 template <int DK, int DV, int C>
 struct ChainSmem {
     using Cf = ChunkCfg<DK, DV, C>;
-    static constexpr int SS_OFF = 0;
-    static constexpr int WS_OFF = SS_OFF + Cf::RTB * Cf::KS;
-    static constexpr int KS_OFF = WS_OFF + C * Cf::KS;
-    static constexpr int US_OFF = KS_OFF + C * Cf::KS;
-    static constexpr int ES_OFF = US_OFF + C * Cf::RTB;
-    static constexpr int DC_OFF = ES_OFF + C * Cf::RTB;
+    using M = MmaAdv<DK, Cf::RTB, C>;
+    static constexpr int SS_OFF = 0;                              // [RTB][KS] fp32 S
+    static constexpr int WS_OFF = SS_OFF + Cf::RTB * M::KS;       // [C][KS] w
+    static constexpr int ES_OFF = WS_OFF + C * M::KS;             // [RTB][ES] e
+    static constexpr int KT_OFF = ES_OFF + Cf::RTB * M::ES;       // [DK][ES] k^T
+    static constexpr int US_OFF = KT_OFF + DK * M::ES;            // [C][RTB] u0 rows of the tile
+    static constexpr int DC_OFF = US_OFF + C * Cf::RTB;           // [C+4] D[C][.]
     static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
 };
 
-// Boundary states: one CTA per (sequence, head, row tile), serial over the
-// sequence's full chunks.  Writes chunk_states[so[n] + c] for c = 0..floor(L/C).
+// Boundary states: one CTA (4 warps) per (sequence, head, row tile), serial
+// over the sequence's full chunks; the tile's state stays in registers.
+// Writes chunk_states[so[n] + c] for c = 0..floor(L/C).  The next chunk's w,
+// u0 and decays arrive by cp.async during phase 2.
 template <int DK, int DV, int C>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const int32_t* __restrict__ cu,
         const int32_t* __restrict__ fco, const int32_t* __restrict__ so, const int32_t* __restrict__ err,
         int N, int H, int in_bf16, const float* __restrict__ w_ws, const float* __restrict__ u_ws,
@@ -290,15 +409,16 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ChainSmem<DK, DV, C>;
-    constexpr int KS = Cf::KS, RTB = Cf::RTB;
+    using M = MmaAdv<DK, Cf::RTB, C>;
+    constexpr int KS = M::KS, RTB = Cf::RTB;
     if (__ldg(err)) return;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
     float* Ss = sm + Sm::SS_OFF;
     float* ws = sm + Sm::WS_OFF;
-    float* ks = sm + Sm::KS_OFF;
-    float* us = sm + Sm::US_OFF;
     float* es = sm + Sm::ES_OFF;
+    float* kT = sm + Sm::KT_OFF;
+    float* us = sm + Sm::US_OFF;
     float* dCs = sm + Sm::DC_OFF;
 
     const int r = blockIdx.x % Cf::NTB;
@@ -310,32 +430,48 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
     const int64_t g0 = __ldg(fco + n);
     const int64_t row0 = (int64_t)r * RTB;
 
-    for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-        const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (state_in != nullptr)
-            x = __ldg(reinterpret_cast<const float4*>(state_in + (((int64_t)n * H + h) * DV + row0 + i) * DK + j4));
-        *reinterpret_cast<float4*>(Ss + i * KS + j4) = x;
-        *reinterpret_cast<float4*>(states + ((slot0 * H + h) * DV + row0 + i) * DK + j4) = x;
-    }
-    for (int c = 0; c < nfull; ++c) {
-        __syncthreads();
+    auto fetch = [&](int c) {
         const int64_t task = (g0 + c) * H + h;
         const float* wsrc = w_ws + task * C * DK;
         for (int e = threadIdx.x; e < C * (DK / 4); e += blockDim.x) {
             const int t = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-            *reinterpret_cast<float4*>(ws + t * KS + j4) = __ldg(reinterpret_cast<const float4*>(wsrc + t * DK + j4));
+            cp_async16(ws + t * KS + j4, wsrc + t * DK + j4);
         }
-        stage_rows<DK>(ks, KS, k, (int64_t)seq0 + (int64_t)c * C, C, H, h, in_bf16, IdxIdentity());
         const float* usrc = u_ws + task * C * DV + row0;
         for (int e = threadIdx.x; e < C * (RTB / 4); e += blockDim.x) {
             const int t = e / (RTB / 4), i4 = (e % (RTB / 4)) * 4;
-            *reinterpret_cast<float4*>(us + t * RTB + i4) = __ldg(reinterpret_cast<const float4*>(usrc + t * DV + i4));
+            cp_async16(us + t * RTB + i4, usrc + t * DV + i4);
         }
-        for (int s = threadIdx.x; s <= C; s += blockDim.x) dCs[s] = __ldg(dC_ws + task * Cf::DCS + s);
-        __syncthreads();
-        chunk_advance<DK, RTB, C>(Ss, ws, us, RTB, ks, dCs, es,
-                                  states + (((slot0 + c + 1) * H + h) * DV + row0) * DK, nullptr);
+        for (int e = threadIdx.x; e < Cf::DCS / 4; e += blockDim.x)
+            cp_async16(dCs + 4 * e, dC_ws + task * Cf::DCS + 4 * e);
+        cp_async_commit();
+    };
+
+    float Sreg[M::P2][4];
+    mma_load_state<DK, RTB, C>(Sreg, Ss,
+                               state_in != nullptr ? state_in + (((int64_t)n * H + h) * DV + row0) * DK : nullptr);
+    for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
+        const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
+        *reinterpret_cast<float4*>(states + ((slot0 * H + h) * DV + row0 + i) * DK + j4) =
+            *reinterpret_cast<const float4*>(Ss + i * KS + j4);
+    }
+    if (nfull > 0) {
+        fetch(0);
+        stage_kT<DK, C>(kT, k, (int64_t)seq0, H, h, in_bf16);
+    }
+    for (int c = 0; c < nfull; ++c) {
+        cp_async_wait_all();
+        __syncthreads();  // w/u0/D and k of chunk c are in smem; Ss is current
+        mma_phase1<DK, RTB, C>(Ss, ws, us, RTB, dCs, es);
+        const float d0 = dCs[0];
+        __syncthreads();  // e complete; w, u0 and D may be overwritten
+        if (c + 1 < nfull) fetch(c + 1);
+        mma_phase2<DK, RTB, C>(Sreg, Ss, es, kT, d0, in_bf16,
+                               states + (((slot0 + c + 1) * H + h) * DV + row0) * DK, nullptr);
+        if (c + 1 < nfull) {
+            __syncthreads();  // phase 2 is done with k
+            stage_kT<DK, C>(kT, k, (int64_t)seq0 + (int64_t)(c + 1) * C, H, h, in_bf16);
+        }
     }
 }
 

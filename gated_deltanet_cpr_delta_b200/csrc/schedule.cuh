@@ -177,6 +177,35 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
+
+// ---------------------------------------------------------------- tensor-core tiles
+// fp32 -> tf32 (round to nearest, ties away; low 13 bits zero) and the split
+// x = hi + lo with hi = tf32(x), lo = tf32(x - hi).
+__device__ __forceinline__ uint32_t tf32_of(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo)
+{
+    hi = tf32_of(x);
+    lo = tf32_of(__fsub_rn(x, __uint_as_float(hi)));
+}
+
+// d += a * b on one 16x8x8 tf32 tile (warp-wide, fp32 accumulate).  Fragment
+// layouts (g = lane / 4, t = lane % 4):
+//   a[0] = A[g][t], a[1] = A[g+8][t], a[2] = A[g][t+4], a[3] = A[g+8][t+4]
+//   b[0] = B[t][g], b[1] = B[t+4][g]                      (B is K x N)
+//   d[0] = D[g][2t], d[1] = D[g][2t+1], d[2] = D[g+8][2t], d[3] = D[g+8][2t+1]
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // Largest n in [0, N) with tab[n] <= g (tab non-decreasing, tab[0] = 0 <= g < tab[N]).
 __device__ __forceinline__ int find_seq(const int32_t* tab, int N, int g)
 {

@@ -143,3 +143,29 @@ def to_bf16_bits(x):
     y = np.zeros(x.shape, np.uint16)
     lib.sched_f32_to_bf16(_p(x), _p(y), x.size)
     return y
+
+
+def schedule_tok_from_states(q, k, v, alpha, beta, states, cu_seqlens, C):
+    """fp32 schedule model of P_tok, started from the given boundary states
+    (chunk_states layout).  Returns (o [T,H,dv] fp32 before the output cast,
+    R_final [N,H,dv,dk])."""
+    lib = _load()
+    if not hasattr(lib, "_tok_states_ready"):
+        P, i32 = ctypes.c_void_p, ctypes.c_int32
+        lib.sched_tok_from_states.restype = ctypes.c_int
+        lib.sched_tok_from_states.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P]
+        lib._tok_states_ready = True
+    q, k, v = _c(q, np.float32), _c(k, np.float32), _c(v, np.float32)
+    alpha, beta = _c(alpha, np.float32), _c(beta, np.float32)
+    states = _c(states, np.float32)
+    cu = _c(cu_seqlens, np.int32)
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    N = cu.shape[0] - 1
+    o = np.zeros((T, H, dv), np.float32)
+    Rf = np.zeros((N, H, dv, dk), np.float32)
+    rc = lib.sched_tok_from_states(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(states), _p(cu),
+                                   N, H, dk, dv, C, _p(o), _p(Rf))
+    if rc:
+        raise RuntimeError(f"sched_tok_from_states failed ({rc})")
+    return o, Rf

@@ -263,3 +263,55 @@ int sched_decode_step(const float* q, const float* k, const float* v,
     }
     return bad ? 2 : 0;
 }
+
+/*
+ * P_tok over every chunk, started from GIVEN boundary states (layout of the
+ * forward's chunk_states).  o [T,H,dv] fp32 before the output cast; R_final
+ * [N,H,dv,dk]: the running state after each sequence's last token (the
+ * boundary state itself when L % C == 0).  This isolates the per-token
+ * schedule from how the boundary states were produced.
+ */
+int sched_tok_from_states(const float* q, const float* k, const float* v,
+                          const float* alpha, const float* beta, const float* states,
+                          const int32_t* cu_seqlens, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C,
+                          float* o, float* R_final)
+{
+    if (N < 0 || H <= 0 || dk <= 0 || dk % NL || dv <= 0 || C <= 0) return 1;
+    int64_t* soff = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N + 1));
+    if (!soff) return 2;
+    soff[0] = 0;
+    for (int32_t n = 0; n < N; ++n) {
+        const int32_t L = cu_seqlens[n + 1] - cu_seqlens[n];
+        if (L < 0) { free(soff); return 1; }
+        soff[n + 1] = soff[n] + L / C + 1;
+    }
+    const int64_t SZ = (int64_t)dv * dk;
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int32_t n = 0; n < N; ++n) {
+        for (int32_t h = 0; h < H; ++h) {
+            float* R = (float*)malloc(sizeof(float) * (size_t)SZ);
+            if (!R) { bad = 1; continue; }
+            const int32_t t0 = cu_seqlens[n], L = cu_seqlens[n + 1] - t0;
+            memcpy(R, states + (soff[n] * H + h) * SZ, sizeof(float) * (size_t)SZ);
+            for (int32_t c0 = 0; c0 < L; c0 += C) {
+                memcpy(R, states + ((soff[n] + c0 / C) * H + h) * SZ, sizeof(float) * (size_t)SZ);
+                const int32_t len = (L - c0 < C) ? (L - c0) : C;
+                for (int32_t t = 0; t < len; ++t) {
+                    const int64_t tok = (int64_t)(t0 + c0 + t) * H + h;
+                    p_tok(R, k + tok * dk, v + tok * dv, q + tok * dk, alpha[tok], beta[tok], dk, dv, o + tok * dv);
+                }
+            }
+            if (R_final) {
+                const int64_t nh = (int64_t)n * H + h;
+                if (L % C == 0)
+                    memcpy(R_final + nh * SZ, states + ((soff[n] + L / C) * H + h) * SZ, sizeof(float) * (size_t)SZ);
+                else
+                    memcpy(R_final + nh * SZ, R, sizeof(float) * (size_t)SZ);
+            }
+            free(R);
+        }
+    }
+    free(soff);
+    return bad ? 2 : 0;
+}

@@ -32,13 +32,13 @@ def check_pair(d, o, st, n, h, C, state_base, bf16_out=True):
     got_s = st[state_base:state_base + ns, h:h + 1].cpu().numpy().astype(np.float64)
     assert np.max(np.abs(got_o - r["o"])) <= 2e-2 * np.max(np.abs(r["o"]))
     assert np.max(np.abs(got_s - r["states"])) <= 2e-2 * np.max(np.abs(r["states"]))
-    # bit-exact against the fp32 schedule model
-    m = oracle.schedule_forward(q, k, v, a, b, cu, C)
-    assert np.array_equal(bits(st[state_base:state_base + ns, h:h + 1].contiguous()), bits(m["states"]))
+    # per-token schedule bit-exact against the fp32 model, started from the GPU's boundary states
+    mo, _ = oracle.schedule_tok_from_states(q, k, v, a, b, st[state_base:state_base + ns, h:h + 1].cpu().numpy(),
+                                            cu, C)
     if bf16_out:
-        assert np.array_equal(bits(o[a0:a1, h:h + 1].contiguous()), oracle.to_bf16_bits(m["o"]))
+        assert np.array_equal(bits(o[a0:a1, h:h + 1].contiguous()), oracle.to_bf16_bits(mo))
     else:
-        assert np.array_equal(bits(o[a0:a1, h:h + 1].contiguous()), bits(m["o"]))
+        assert np.array_equal(bits(o[a0:a1, h:h + 1].contiguous()), bits(mo))
 
 
 def test_prefill_workload_sampled():

@@ -1,7 +1,10 @@
 """GPU parity of the CUDA path through the C ABI (small and ragged shapes).
 
-* Bitwise against the fp32 schedule model (oracle/schedule_fp32.c): o in fp32
-  and bf16, chunk states, and the decode cache.
+* Bitwise against the fp32 schedule model (oracle/schedule_fp32.c) for the
+  per-token schedule: o in fp32 and bf16 and the running cache state, with the
+  model's P_tok started from the GPU's boundary states.  Those boundary states
+  come from the tensor-core P_chunk; they are checked against the fp64 oracle
+  within tolerance, and bit for bit across GPU paths.
 * Within tolerance of the fp64 oracle: max|o - o*| <= 1e-4 for fp32 inputs,
   <= 2e-2 * ||o*||_inf for bf16 inputs; the same bounds for states.
 * CPR self-consistency on the GPU, bit for bit: prefill == decode, split at a
@@ -47,9 +50,8 @@ def test_tiny_workload_bitwise_prefill_vs_decode_and_oracle():
     b = synth.make_batch(cfg["seed"], [cfg["T"]] * cfg["B"], cfg["H"], cfg["dk"], cfg["dv"], cfg["dtype"])
     C = cfg["C"]
     o, st, _ = fwd(b, C)
-    m = oracle.schedule_forward(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)
-    assert np.array_equal(bits(o), bits(m["o"]))
-    assert np.array_equal(bits(st), bits(m["states"]))
+    mo, _ = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st.cpu().numpy(), b.cu_seqlens, C)
+    assert np.array_equal(bits(o), bits(mo))
     r = oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)
     tol_check("f32", o.cpu().numpy(), r["o"], "o")
     tol_check("f32", st.cpu().numpy(), r["states"], "states")
@@ -71,18 +73,24 @@ SHAPES = [(d, C) for d in (16, 32, 64, 128) for C in (16, 32, 64)]
 
 @pytest.mark.parametrize("d,C", SHAPES)
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_forward_bitwise_vs_schedule_model(d, C, dtype):
+def test_forward_vs_schedule_model_and_oracle(d, C, dtype):
     lens = [1, C - 1, C, 0, C + 1, 3 * C + 5] if d <= 64 else [C - 1, 2 * C + 3, 0, C]
     H = 3 if d <= 64 else 2
     b = synth.make_batch(100 + d + C, lens, H, d, d, dtype)
     rng = np.random.default_rng(d * C)
     S0 = (rng.standard_normal((len(lens), H, d, d)) * 0.2).astype(np.float32)
     o, st, cache = fwd(b, C, torch.float32, torch.from_numpy(S0).to(DEV), cache=True)
+    st_h = st.cpu().numpy()
+    # P_tok bit for bit: the model's per-token schedule, started from the GPU's boundary states
+    mo, mR = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st_h, b.cu_seqlens, C)
+    assert np.array_equal(bits(o), bits(mo))
+    assert np.array_equal(bits(cache["R"]), bits(mR))
+    # the first state of every sequence is state_in itself; S_b is the last boundary state
+    first = np.concatenate([[0], np.cumsum([L // C + 1 for L in lens])])
+    last = first[1:] - 1
+    assert np.array_equal(bits(st_h[first[:-1]]), bits(S0))
+    assert np.array_equal(bits(cache["S_b"]), bits(st_h[last]))
     m = oracle.schedule_forward(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C, S0, with_cache=True)
-    assert np.array_equal(bits(o), bits(m["o"]))
-    assert np.array_equal(bits(st), bits(m["states"]))
-    for key in ("S_b", "R"):
-        assert np.array_equal(bits(cache[key]), bits(m[key])), key
     pos = cache["pos"].cpu().numpy()
     assert np.array_equal(pos, m["pos"])
     for n in range(len(lens)):
@@ -93,7 +101,7 @@ def test_forward_bitwise_vs_schedule_model(d, C, dtype):
         assert np.array_equal(cache["bbuf"][n, :, :p].cpu().numpy(), m["bbuf"][n, :, :p])
     # bf16 output = nearest-even rounding of the same fp32 values
     o16, st16, _ = fwd(b, C, torch.bfloat16, torch.from_numpy(S0).to(DEV))
-    assert np.array_equal(bits(o16), oracle.to_bf16_bits(m["o"]))
+    assert np.array_equal(bits(o16), oracle.to_bf16_bits(mo))
     assert np.array_equal(bits(st16), bits(st))
     # fp64 oracle
     r = oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C, S0)

@@ -144,6 +144,21 @@ def test_prefill_equals_decode_bitwise(Lp, steps, C):
     assert np.array_equal(m["S_b"], full["states"][last])
 
 
+def test_tok_from_states_reproduces_the_model_forward():
+    """Driving the model's P_tok from given boundary states (its own here)
+    reproduces its forward outputs and running states bit for bit."""
+    C = 16
+    bat = synth.make_batch(10, [40, 16, 5, 0, 33], 2, 16, 16, "bf16")
+    m = oracle.schedule_forward(bat.q, bat.k, bat.v, bat.alpha, bat.beta, bat.cu_seqlens, C, with_cache=True)
+    o, Rf = oracle.schedule_tok_from_states(bat.q, bat.k, bat.v, bat.alpha, bat.beta, m["states"],
+                                            bat.cu_seqlens, C)
+    assert np.array_equal(o, m["o"]) and np.array_equal(Rf, m["R"])
+    # and it really uses the states it is given: other states change the outputs
+    o2, _ = oracle.schedule_tok_from_states(bat.q, bat.k, bat.v, bat.alpha, bat.beta, m["states"] * 2,
+                                            bat.cu_seqlens, C)
+    assert not np.array_equal(o2, m["o"])
+
+
 def test_split_at_chunk_boundary_equals_unsplit():
     C, L = 16, 100
     bat = synth.make_batch(6, [L], 2, 16, 16, "bf16")
