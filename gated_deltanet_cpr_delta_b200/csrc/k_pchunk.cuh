@@ -466,11 +466,44 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
         const float d0 = dCs[0];
         __syncthreads();  // e complete; w, u0 and D may be overwritten
         if (c + 1 < nfull) fetch(c + 1);
+        // bf16 inputs: the next chunk's k (raw 16-byte pieces) is loaded into
+        // registers now and written to smem after phase 2, so the load latency
+        // overlaps the tensor-core work
+        constexpr int ITEMS = C * (DK / 8), NPRE = (ITEMS + M::THREADS - 1) / M::THREADS;
+        uint4 kpre[NPRE];
+        const int64_t tok1 = (int64_t)seq0 + (int64_t)(c + 1) * C;
+        if (c + 1 < nfull && in_bf16) {
+#pragma unroll
+            for (int i = 0; i < NPRE; ++i) {
+                const int e = threadIdx.x + i * M::THREADS;
+                if (e < ITEMS) {
+                    const int tau = e % C, j8 = (e / C) * 8;
+                    kpre[i] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(k) +
+                                                                   ((tok1 + tau) * H + h) * (int64_t)DK + j8));
+                }
+            }
+        }
         mma_phase2<DK, RTB, C>(Sreg, Ss, es, kT, d0, in_bf16,
                                states + (((slot0 + c + 1) * H + h) * DV + row0) * DK, nullptr);
         if (c + 1 < nfull) {
             __syncthreads();  // phase 2 is done with k
-            stage_kT<DK, C>(kT, k, (int64_t)seq0 + (int64_t)(c + 1) * C, H, h, in_bf16);
+            if (in_bf16) {
+#pragma unroll
+                for (int i = 0; i < NPRE; ++i) {
+                    const int e = threadIdx.x + i * M::THREADS;
+                    if (e < ITEMS) {
+                        const int tau = e % C, j8 = (e / C) * 8;
+                        const uint32_t w4[4] = {kpre[i].x, kpre[i].y, kpre[i].z, kpre[i].w};
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            kT[(j8 + 2 * m) * M::ES + tau] = __uint_as_float(w4[m] << 16);
+                            kT[(j8 + 2 * m + 1) * M::ES + tau] = __uint_as_float(w4[m] & 0xffff0000u);
+                        }
+                    }
+                }
+            } else {
+                stage_kT<DK, C>(kT, k, tok1, H, h, in_bf16);
+            }
         }
     }
 }
