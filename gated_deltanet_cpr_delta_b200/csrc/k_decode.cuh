@@ -69,12 +69,14 @@ template <int DK, int DV, int C>
 struct ResyncSmem {
     using Cf = ChunkCfg<DK, DV, C>;
     using M = MmaAdv<DK, Cf::RTB, C>;
-    static constexpr int KS_OFF = 0;                                 // [C][KS] k
-    static constexpr int VS_OFF = KS_OFF + C * Cf::KS;               // [C][DV] v, then u0
-    static constexpr int WS_OFF = VS_OFF + C * DV;                   // [C][KS] w
-    static constexpr int DM_OFF = WS_OFF + C * Cf::KS;               // decays
-    static constexpr int CT_OFF = DM_OFF + ((Cf::C1 * Cf::C1 + 3) / 4) * 4;
-    static constexpr int SS_OFF = CT_OFF + C * Cf::CT;               // [RTB][KS] S tile
+    using PL = PrepLayout<DK, DV, C>;
+    static constexpr int KX_OFF = 0;                                 // [C][KXS] k, then w
+    static constexpr int VX_OFF = KX_OFF + C * PL::KXS;              // [C][VXS] v, then u0
+    static constexpr int CC_OFF = VX_OFF + C * PL::VXS;              // [C][CCS] c
+    static constexpr int DM_OFF = CC_OFF + C * PL::CCS;              // decays / staging
+    static constexpr int D0_OFF = DM_OFF + ((PL::DM + 3) / 4) * 4;   // D[t][0]
+    static constexpr int WS_OFF = D0_OFF + C + 4;                    // [C][KS] w for the tensor-core phases
+    static constexpr int SS_OFF = WS_OFF + C * M::KS;                // [RTB][KS] S tile
     static constexpr int ES_OFF = SS_OFF + Cf::RTB * M::KS;          // [RTB][ES] e
     static constexpr int KT_OFF = ES_OFF + Cf::RTB * M::ES;          // [DK][ES] k^T
     static constexpr int AB_OFF = KT_OFF + DK * M::ES;
@@ -95,14 +97,16 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ResyncSmem<DK, DV, C>;
     using M = MmaAdv<DK, Cf::RTB, C>;
-    constexpr int KS = Cf::KS, RTB = Cf::RTB;
+    using PL = PrepLayout<DK, DV, C>;
+    constexpr int RTB = Cf::RTB;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
-    float* ks = sm + Sm::KS_OFF;
-    float* vs = sm + Sm::VS_OFF;
+    float* kx = sm + Sm::KX_OFF;
+    float* vx = sm + Sm::VX_OFF;
+    float* cc = sm + Sm::CC_OFF;
+    float* dm = sm + Sm::DM_OFF;
+    float* d0 = sm + Sm::D0_OFF;
     float* ws = sm + Sm::WS_OFF;
-    float* Dm = sm + Sm::DM_OFF;
-    float* cT = sm + Sm::CT_OFF;
     float* Ss = sm + Sm::SS_OFF;
     float* es = sm + Sm::ES_OFF;
     float* kT = sm + Sm::KT_OFF;
@@ -119,21 +123,21 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
             continue;
         }
         // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
-        stage_rows<DK>(ks, KS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
-        stage_rows<DV>(vs, DV, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        stage_rows<DK>(kx, PL::KXS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
+        stage_rows<DV>(vx, PL::VXS, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
         stage_kT<DK, C>(kT, kbuf, (int64_t)nh * C, 1, 0, in_bf16);
         for (int t = threadIdx.x; t < C; t += blockDim.x) {
             as[t] = abuf[(int64_t)nh * C + t];
             bs[t] = bbuf[(int64_t)nh * C + t];
         }
         __syncthreads();
-        chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, ws, KS, vs, DV, dCs);  // u0 overwrites v in place
+        chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, ws, M::KS, vx, PL::VXS, dCs);
         float Sreg[M::P2][4];
         for (int r = 0; r < Cf::NTB; ++r) {
             float* Sg = S_b + ((int64_t)nh * DV + r * RTB) * DK;
             float* Rg = R + ((int64_t)nh * DV + r * RTB) * DK;
             mma_load_state<DK, RTB, C>(Sreg, Ss, Sg);
-            mma_phase1<DK, RTB, C>(Ss, ws, vs + r * RTB, DV, dCs, es);
+            mma_phase1<DK, RTB, C>(Ss, ws, vx + r * RTB, PL::VXS, dCs, es);
             __syncthreads();
             mma_phase2<DK, RTB, C>(Sreg, Ss, es, kT, dCs[0], in_bf16, Sg, Rg);
             __syncthreads();

@@ -91,72 +91,174 @@ __device__ __forceinline__ void fwd_subst(float (&acc)[C], const float* cT, cons
     }
 }
 
-// P_chunk part 1 for one chunk, by one CTA.  ks [C][KS], vs [C][DV], as/bs [C]
-// in smem.  Dm [(C+1)^2] and cT [C][CT] are smem scratch.  Writes
-//   w_t  -> wout[(t-1)*ldw + j],   u0_t -> uout[(t-1)*ldu + i],   D[C][s] -> dCout[s]
-// (any address space).  uout may alias vs: each column of vs is read only by
-// the thread that later writes that column of uout, and only before it does.
+// P_chunk part 1 for one chunk, by one CTA (>= 128 threads), on the tensor
+// cores where the work is a dense contraction:
+//   D[s][s] = 1, D[t][s] = D[t-1][s] * alpha_t                     (fp32 chains)
+//   G[t][s] = k_t . k_s for s < t: mma tf32 over 8-wide blocks of d_k,
+//             ascending, k = k_hi + k_lo (k_lo = 0 and skipped when every k
+//             is exactly tf32, i.e. bf16 inputs):  G += k_lo*k_hi, k_hi*k_lo, k_hi*k_hi
+//   c[t][s] = D[t][s] * G[t][s]
+//   forward substitution for the columns x = u0 (init v_t) and w (init
+//   D[t][0] * k_t), in blocks of 16 tokens: for block b, acc_t = init_t;
+//   acc_t += sum over 8-token blocks of s < 16b (ascending) of the mma
+//   products (-c)_lo*x_hi, (-c)_hi*x_lo, (-c)_hi*x_hi; then, for s in
+//   [16b, t) ascending, acc_t = fma(-c[t][s], x_s, acc_t); x_t = beta_t * acc_t.
+// kx [C][DK+8] holds k on entry and w on exit; vx [C][DV+8] holds v on entry
+// and u0 on exit (row strides chosen so the mma fragment reads are
+// conflict-free); as, bs [C] gates; cc [C][C+4], dm, d0 are smem scratch.
+// Also writes w -> wout[t*ldw + j], u0 -> uout[t*ldu + i], D[C][s] -> dCout[s]
+// (any address space; uout may be vx itself).
 template <int DK, int DV, int C>
-__device__ __forceinline__ void chunk_prep(const float* ks, const float* vs, const float* as, const float* bs,
-                                           float* Dm, float* cT, float* wout, int ldw, float* uout, int ldu,
+struct PrepLayout {
+    static constexpr int KXS = DK + 8, VXS = DV + 8, CCS = C + 4;
+    static constexpr int NCOL = DV + DK;
+    static constexpr int DM = ((C + 1) * (C + 1) > 16 * NCOL ? (C + 1) * (C + 1) : 16 * NCOL);
+};
+
+template <int DK, int DV, int C>
+__device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as, const float* bs, float* cc, float* dm,
+                                           float* d0, int k_exact, float* wout, int ldw, float* uout, int ldu,
                                            float* dCout)
 {
-    using Cf = ChunkCfg<DK, DV, C>;
-    constexpr int KS = Cf::KS, C1 = Cf::C1, CT = Cf::CT;
-    // decay products D[t][s] = D[t-1][s] * alpha_t, D[s][s] = 1  (tokens 1..C)
+    using PL = PrepLayout<DK, DV, C>;
+    constexpr int KXS = PL::KXS, VXS = PL::VXS, CCS = PL::CCS, C1 = C + 1, NCOL = PL::NCOL;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
+    // decay products
     for (int s = threadIdx.x; s <= C; s += blockDim.x) {
         float d = 1.0f;
-        Dm[s * C1 + s] = d;
+        dm[s * C1 + s] = d;
         for (int t = s + 1; t <= C; ++t) {
             d = fmul(d, as[t - 1]);
-            Dm[t * C1 + s] = d;
+            dm[t * C1 + s] = d;
         }
     }
     __syncthreads();
-    // c[t][s] = D[t][s] * tree(k_s, k_t), stored transposed: cT[s-1][t-1];
-    // 4x4 blocks of the strictly lower triangle, one block per thread
-    constexpr int NB = C / 4, NBLK = NB * (NB + 1) / 2;
-    for (int blk = threadIdx.x; blk < NBLK; blk += blockDim.x) {
-        int bt = 0;
-        while ((bt + 1) * (bt + 2) / 2 <= blk) ++bt;
-        const int bsg = blk - bt * (bt + 1) / 2;
-        const float* const xa[4] = {ks + (4 * bt) * KS, ks + (4 * bt + 1) * KS, ks + (4 * bt + 2) * KS,
-                                    ks + (4 * bt + 3) * KS};
-        const float* const yb[4] = {ks + (4 * bsg) * KS, ks + (4 * bsg + 1) * KS, ks + (4 * bsg + 2) * KS,
-                                    ks + (4 * bsg + 3) * KS};
-        float G[4][4];
-        tree_block<DK, KS, 4, 4>(xa, yb, G);
+    // Gram on the tensor cores: warp w owns rows 16w..16w+15 (w < C/16) and the
+    // n8 tiles of columns below them
+    if (warp < C / 16) {
+        const int r0 = warp * 16;
+        const int ntiles = 2 * warp + 2;
+        float acc[2 * (C / 16)][4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int q = 0; q < 2 * (C / 16); ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+#pragma unroll 2
+        for (int kb = 0; kb < DK / 8; ++kb) {
+            const int k0 = kb * 8;
+            uint32_t ah[4], al[4];
+            tf32_split(kx[(r0 + g) * KXS + k0 + t4], ah[0], al[0]);
+            tf32_split(kx[(r0 + g + 8) * KXS + k0 + t4], ah[1], al[1]);
+            tf32_split(kx[(r0 + g) * KXS + k0 + t4 + 4], ah[2], al[2]);
+            tf32_split(kx[(r0 + g + 8) * KXS + k0 + t4 + 4], ah[3], al[3]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int tau = 4 * bt + r, sig = 4 * bsg + c;
-                if (sig < tau) cT[sig * CT + tau] = fmul(Dm[(tau + 1) * C1 + (sig + 1)], G[r][c]);
+            for (int q = 0; q < 2 * (C / 16); ++q) {
+                if (q < ntiles) {
+                    uint32_t bh[2], bl[2];
+                    tf32_split(kx[(q * 8 + g) * KXS + k0 + t4], bh[0], bl[0]);
+                    tf32_split(kx[(q * 8 + g) * KXS + k0 + t4 + 4], bh[1], bl[1]);
+                    if (!k_exact) {
+                        mma_tf32(acc[q], al, bh);
+                        mma_tf32(acc[q], ah, bl);
+                    }
+                    mma_tf32(acc[q], ah, bh);
+                }
             }
-    }
-    if (dCout != nullptr)
-        for (int s = threadIdx.x; s <= C; s += blockDim.x) dCout[s] = Dm[C * C1 + s];
-    __syncthreads();
-    // forward substitution, one column per thread
-    for (int col = threadIdx.x; col < DV + DK; col += blockDim.x) {
-        float acc[C];
-        if (col < DV) {
+        }
 #pragma unroll
-            for (int tau = 0; tau < C; ++tau) acc[tau] = vs[tau * DV + col];
-            fwd_subst<C, CT>(acc, cT, bs);
+        for (int q = 0; q < 2 * (C / 16); ++q) {
+            if (q < ntiles) {
 #pragma unroll
-            for (int tau = 0; tau < C; ++tau) uout[tau * ldu + col] = acc[tau];
-        } else {
-            const int j = col - DV;
-#pragma unroll
-            for (int tau = 0; tau < C; ++tau) acc[tau] = fmul(Dm[(tau + 1) * C1], ks[tau * KS + j]);
-            fwd_subst<C, CT>(acc, cT, bs);
-#pragma unroll
-            for (int tau = 0; tau < C; ++tau) wout[tau * ldw + j] = acc[tau];
+                for (int c = 0; c < 4; ++c) {
+                    const int tau = r0 + g + (c >> 1) * 8, sig = q * 8 + 2 * t4 + (c & 1);
+                    if (sig < tau) cc[tau * CCS + sig] = fmul(dm[(tau + 1) * C1 + (sig + 1)], acc[q][c]);
+                }
+            }
         }
     }
+    for (int t = threadIdx.x; t < C; t += blockDim.x) d0[t] = dm[(t + 1) * C1];  // D[t][0], t = 1..C
+    if (dCout != nullptr)
+        for (int s = threadIdx.x; s <= C; s += blockDim.x) dCout[s] = dm[C * C1 + s];
     __syncthreads();
+    float* stage = dm;  // [16][NCOL]: the block's accumulators, column-major per thread afterwards
+    for (int b = 0; b < C / 16; ++b) {
+        const int t0 = 16 * b;
+        // init + tensor-core part (warps 0..3, 8 column tiles of 8 each per warp)
+        if (warp < 4) {
+            constexpr int NTW = NCOL / 8 / 4;  // n8 column tiles per warp
+            float acc[NTW][4];
+#pragma unroll
+            for (int q = 0; q < NTW; ++q) {
+                const int n0 = (warp * NTW + q) * 8;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int tau = t0 + g + (c >> 1) * 8, col = n0 + 2 * t4 + (c & 1);
+                    acc[q][c] = col < DV ? vx[tau * VXS + col] : fmul(d0[tau], kx[tau * KXS + (col - DV)]);
+                }
+            }
+            for (int kb = 0; kb < 2 * b; ++kb) {
+                const int s0 = kb * 8;
+                uint32_t ah[4], al[4];
+                tf32_split(-cc[(t0 + g) * CCS + s0 + t4], ah[0], al[0]);
+                tf32_split(-cc[(t0 + g + 8) * CCS + s0 + t4], ah[1], al[1]);
+                tf32_split(-cc[(t0 + g) * CCS + s0 + t4 + 4], ah[2], al[2]);
+                tf32_split(-cc[(t0 + g + 8) * CCS + s0 + t4 + 4], ah[3], al[3]);
+#pragma unroll
+                for (int q = 0; q < NTW; ++q) {
+                    const int col = (warp * NTW + q) * 8 + g;
+                    const float x0 = col < DV ? vx[(s0 + t4) * VXS + col] : kx[(s0 + t4) * KXS + (col - DV)];
+                    const float x1 = col < DV ? vx[(s0 + t4 + 4) * VXS + col] : kx[(s0 + t4 + 4) * KXS + (col - DV)];
+                    uint32_t bh[2], bl[2];
+                    tf32_split(x0, bh[0], bl[0]);
+                    tf32_split(x1, bh[1], bl[1]);
+                    mma_tf32(acc[q], al, bh);
+                    mma_tf32(acc[q], ah, bl);
+                    mma_tf32(acc[q], ah, bh);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < NTW; ++q) {
+                const int n0 = (warp * NTW + q) * 8;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) stage[(g + (c >> 1) * 8) * NCOL + n0 + 2 * t4 + (c & 1)] = acc[q][c];
+            }
+        }
+        __syncthreads();
+        // in-block part: one column per thread, sequential over the block's 16 tokens
+        for (int col = threadIdx.x; col < NCOL; col += blockDim.x) {
+            float xb[16];
+#pragma unroll
+            for (int tr = 0; tr < 16; ++tr) {
+                float acc = stage[tr * NCOL + col];
+#pragma unroll
+                for (int sr = 0; sr < tr; ++sr) acc = ffma(-cc[(t0 + tr) * CCS + t0 + sr], xb[sr], acc);
+                xb[tr] = fmul(bs[t0 + tr], acc);
+            }
+#pragma unroll
+            for (int tr = 0; tr < 16; ++tr) {
+                const int tau = t0 + tr;
+                if (col < DV) {
+                    vx[tau * VXS + col] = xb[tr];
+                    uout[tau * ldu + col] = xb[tr];
+                } else {
+                    kx[tau * KXS + (col - DV)] = xb[tr];
+                    wout[tau * ldw + (col - DV)] = xb[tr];
+                }
+            }
+        }
+        __syncthreads();
+    }
 }
+
+template <int DK, int DV, int C>
+struct PrepSmem {
+    using PL = PrepLayout<DK, DV, C>;
+    static constexpr int KX_OFF = 0;
+    static constexpr int VX_OFF = KX_OFF + C * PL::KXS;
+    static constexpr int CC_OFF = VX_OFF + C * PL::VXS;
+    static constexpr int DM_OFF = CC_OFF + C * PL::CCS;
+    static constexpr int D0_OFF = DM_OFF + ((PL::DM + 3) / 4) * 4;
+    static constexpr int AB_OFF = D0_OFF + C + 4;
+    static constexpr size_t BYTES = sizeof(float) * (AB_OFF + 2 * C);
+};
 
 // ---------------------------------------------------------------- tensor-core P_chunk part 2
 // The two contractions of the boundary update on the tensor cores
@@ -337,17 +439,6 @@ __device__ __forceinline__ void stage_kT(float* kT, const void* k, int64_t tok0,
     }
 }
 
-template <int DK, int DV, int C>
-struct PrepSmem {
-    using Cf = ChunkCfg<DK, DV, C>;
-    static constexpr int KS_OFF = 0;
-    static constexpr int VS_OFF = KS_OFF + C * Cf::KS;
-    static constexpr int DM_OFF = VS_OFF + C * DV;
-    static constexpr int CT_OFF = DM_OFF + ((Cf::C1 * Cf::C1 + 3) / 4) * 4;
-    static constexpr int AB_OFF = CT_OFF + C * Cf::CT;
-    static constexpr size_t BYTES = sizeof(float) * (AB_OFF + 2 * C);
-};
-
 // P_chunk part 1 for every full chunk: one CTA per (full chunk, head).
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256)
@@ -358,13 +449,15 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = PrepSmem<DK, DV, C>;
+    using PL = PrepLayout<DK, DV, C>;
     if (__ldg(err)) return;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
-    float* ks = sm + Sm::KS_OFF;
-    float* vs = sm + Sm::VS_OFF;
-    float* Dm = sm + Sm::DM_OFF;
-    float* cT = sm + Sm::CT_OFF;
+    float* kx = sm + Sm::KX_OFF;
+    float* vx = sm + Sm::VX_OFF;
+    float* cc = sm + Sm::CC_OFF;
+    float* dm = sm + Sm::DM_OFF;
+    float* d0 = sm + Sm::D0_OFF;
     float* as = sm + Sm::AB_OFF;
     float* bs = as + C;
 
@@ -372,14 +465,14 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
     const int h = task % H, g = task / H;
     const int n = find_seq(fco, N, g);
     const int64_t tok0 = (int64_t)__ldg(cu + n) + (int64_t)(g - __ldg(fco + n)) * C;
-    stage_rows<DK>(ks, Cf::KS, k, tok0, C, H, h, in_bf16, IdxIdentity());
-    stage_rows<DV>(vs, DV, v, tok0, C, H, h, in_bf16, IdxIdentity());
+    stage_rows<DK>(kx, PL::KXS, k, tok0, C, H, h, in_bf16, IdxIdentity());
+    stage_rows<DV>(vx, PL::VXS, v, tok0, C, H, h, in_bf16, IdxIdentity());
     for (int t = threadIdx.x; t < C; t += blockDim.x) {
         as[t] = __ldg(alpha + (tok0 + t) * H + h);
         bs[t] = __ldg(beta + (tok0 + t) * H + h);
     }
     __syncthreads();
-    chunk_prep<DK, DV, C>(ks, vs, as, bs, Dm, cT, w_ws + (int64_t)task * C * DK, DK,
+    chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, w_ws + (int64_t)task * C * DK, DK,
                           u_ws + (int64_t)task * C * DV, DV, dC_ws + (int64_t)task * Cf::DCS);
 }
 
