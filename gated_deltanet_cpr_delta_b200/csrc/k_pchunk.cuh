@@ -112,7 +112,8 @@ template <int DK, int DV, int C>
 struct PrepLayout {
     static constexpr int KXS = DK + 8, VXS = DV + 8, CCS = C + 4;
     static constexpr int NCOL = DV + DK;
-    static constexpr int DM = ((C + 1) * (C + 1) > 16 * NCOL ? (C + 1) * (C + 1) : 16 * NCOL);
+    static constexpr int STS = NCOL + 8;  // staging row stride: conflict-free fragment stores
+    static constexpr int DM = ((C + 1) * (C + 1) > 16 * STS ? (C + 1) * (C + 1) : 16 * STS);
 };
 
 template <int DK, int DV, int C>
@@ -121,77 +122,91 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
                                            float* dCout)
 {
     using PL = PrepLayout<DK, DV, C>;
-    constexpr int KXS = PL::KXS, VXS = PL::VXS, CCS = PL::CCS, C1 = C + 1, NCOL = PL::NCOL;
+    constexpr int KXS = PL::KXS, VXS = PL::VXS, CCS = PL::CCS, C1 = C + 1, NCOL = PL::NCOL, STS = PL::STS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
-    // decay products
+    const int nwarps = blockDim.x >> 5;
+    // decay products: column s is the chain D[t][s] = D[t-1][s] * alpha_t, t = s+1..C
     for (int s = threadIdx.x; s <= C; s += blockDim.x) {
         float d = 1.0f;
         dm[s * C1 + s] = d;
-        for (int t = s + 1; t <= C; ++t) {
-            d = fmul(d, as[t - 1]);
-            dm[t * C1 + s] = d;
+#pragma unroll
+        for (int t4i = 0; t4i < C; t4i += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(as + t4i);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = t4i + e + 1;
+                if (t > s) {
+                    d = fmul(d, av[e]);
+                    dm[t * C1 + s] = d;
+                }
+            }
         }
     }
     __syncthreads();
-    // Gram on the tensor cores: warp w owns rows 16w..16w+15 (w < C/16) and the
-    // n8 tiles of columns below them
-    if (warp < C / 16) {
-        const int r0 = warp * 16;
-        const int ntiles = 2 * warp + 2;
-        float acc[2 * (C / 16)][4];
-#pragma unroll
-        for (int q = 0; q < 2 * (C / 16); ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
-#pragma unroll 2
+    // Gram on the tensor cores: the (m16, n8) tiles of the lower triangle,
+    // spread over the warps; each tile's chain runs over d_k in 8-wide blocks
+    constexpr int MT = C / 16, NTILE = MT * (MT + 1);  // tile (m, q) with q <= 2m+1
+    for (int tile = warp; tile < NTILE; tile += nwarps) {
+        int m = 0;
+        while ((m + 1) * (m + 2) <= tile) ++m;
+        const int q = tile - m * (m + 1);
+        const int r0 = m * 16, n0 = q * 8;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
         for (int kb = 0; kb < DK / 8; ++kb) {
             const int k0 = kb * 8;
-            uint32_t ah[4], al[4];
-            tf32_split(kx[(r0 + g) * KXS + k0 + t4], ah[0], al[0]);
-            tf32_split(kx[(r0 + g + 8) * KXS + k0 + t4], ah[1], al[1]);
-            tf32_split(kx[(r0 + g) * KXS + k0 + t4 + 4], ah[2], al[2]);
-            tf32_split(kx[(r0 + g + 8) * KXS + k0 + t4 + 4], ah[3], al[3]);
-#pragma unroll
-            for (int q = 0; q < 2 * (C / 16); ++q) {
-                if (q < ntiles) {
-                    uint32_t bh[2], bl[2];
-                    tf32_split(kx[(q * 8 + g) * KXS + k0 + t4], bh[0], bl[0]);
-                    tf32_split(kx[(q * 8 + g) * KXS + k0 + t4 + 4], bh[1], bl[1]);
-                    if (!k_exact) {
-                        mma_tf32(acc[q], al, bh);
-                        mma_tf32(acc[q], ah, bl);
-                    }
-                    mma_tf32(acc[q], ah, bh);
-                }
+            const float a0 = kx[(r0 + g) * KXS + k0 + t4], a1 = kx[(r0 + g + 8) * KXS + k0 + t4];
+            const float a2 = kx[(r0 + g) * KXS + k0 + t4 + 4], a3 = kx[(r0 + g + 8) * KXS + k0 + t4 + 4];
+            const float b0 = kx[(n0 + g) * KXS + k0 + t4], b1 = kx[(n0 + g) * KXS + k0 + t4 + 4];
+            if (k_exact) {
+                const uint32_t ah[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
+                                        __float_as_uint(a3)};
+                const uint32_t bh[2] = {__float_as_uint(b0), __float_as_uint(b1)};
+                mma_tf32(acc, ah, bh);
+            } else {
+                uint32_t ah[4], al[4], bh[2], bl[2];
+                tf32_split(a0, ah[0], al[0]); tf32_split(a1, ah[1], al[1]);
+                tf32_split(a2, ah[2], al[2]); tf32_split(a3, ah[3], al[3]);
+                tf32_split(b0, bh[0], bl[0]); tf32_split(b1, bh[1], bl[1]);
+                mma_tf32(acc, al, bh);
+                mma_tf32(acc, ah, bl);
+                mma_tf32(acc, ah, bh);
             }
         }
 #pragma unroll
-        for (int q = 0; q < 2 * (C / 16); ++q) {
-            if (q < ntiles) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int tau = r0 + g + (c >> 1) * 8, sig = q * 8 + 2 * t4 + (c & 1);
-                    if (sig < tau) cc[tau * CCS + sig] = fmul(dm[(tau + 1) * C1 + (sig + 1)], acc[q][c]);
-                }
-            }
+        for (int c = 0; c < 4; ++c) {
+            const int tau = r0 + g + (c >> 1) * 8, sig = n0 + 2 * t4 + (c & 1);
+            if (sig < tau) cc[tau * CCS + sig] = fmul(dm[(tau + 1) * C1 + (sig + 1)], acc[c]);
         }
     }
     for (int t = threadIdx.x; t < C; t += blockDim.x) d0[t] = dm[(t + 1) * C1];  // D[t][0], t = 1..C
     if (dCout != nullptr)
         for (int s = threadIdx.x; s <= C; s += blockDim.x) dCout[s] = dm[C * C1 + s];
     __syncthreads();
-    float* stage = dm;  // [16][NCOL]: the block's accumulators, column-major per thread afterwards
+    float* stage = dm;  // [16][STS]: the block's accumulators
     for (int b = 0; b < C / 16; ++b) {
         const int t0 = 16 * b;
-        // init + tensor-core part (warps 0..3, 8 column tiles of 8 each per warp)
-        if (warp < 4) {
-            constexpr int NTW = NCOL / 8 / 4;  // n8 column tiles per warp
+        // init + tensor-core part: warp w owns column tiles w, w + nw, ... (each
+        // tile all u0 or all w columns); its tiles share the split c fragment
+        {
+            constexpr int NTW = (NCOL / 8 + 7) / 8;  // tiles per warp with 8 warps
             float acc[NTW][4];
+            const float* xb[NTW];
+            int xs[NTW];
 #pragma unroll
             for (int q = 0; q < NTW; ++q) {
-                const int n0 = (warp * NTW + q) * 8;
+                const int nt = warp + nwarps * q;
+                const int n0 = nt * 8;
+                const bool is_u = n0 < DV;
+                xb[q] = is_u ? vx + n0 : kx + (n0 - DV);
+                xs[q] = is_u ? VXS : KXS;
+                if (nt < NCOL / 8) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int tau = t0 + g + (c >> 1) * 8, col = n0 + 2 * t4 + (c & 1);
-                    acc[q][c] = col < DV ? vx[tau * VXS + col] : fmul(d0[tau], kx[tau * KXS + (col - DV)]);
+                    for (int c = 0; c < 4; ++c) {
+                        const int tau = t0 + g + (c >> 1) * 8, cl = 2 * t4 + (c & 1);
+                        acc[q][c] = is_u ? xb[q][tau * xs[q] + cl] : fmul(d0[tau], xb[q][tau * xs[q] + cl]);
+                    }
                 }
             }
             for (int kb = 0; kb < 2 * b; ++kb) {
@@ -203,22 +218,24 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
                 tf32_split(-cc[(t0 + g + 8) * CCS + s0 + t4 + 4], ah[3], al[3]);
 #pragma unroll
                 for (int q = 0; q < NTW; ++q) {
-                    const int col = (warp * NTW + q) * 8 + g;
-                    const float x0 = col < DV ? vx[(s0 + t4) * VXS + col] : kx[(s0 + t4) * KXS + (col - DV)];
-                    const float x1 = col < DV ? vx[(s0 + t4 + 4) * VXS + col] : kx[(s0 + t4 + 4) * KXS + (col - DV)];
-                    uint32_t bh[2], bl[2];
-                    tf32_split(x0, bh[0], bl[0]);
-                    tf32_split(x1, bh[1], bl[1]);
-                    mma_tf32(acc[q], al, bh);
-                    mma_tf32(acc[q], ah, bl);
-                    mma_tf32(acc[q], ah, bh);
+                    if (warp + nwarps * q < NCOL / 8) {
+                        uint32_t bh[2], bl[2];
+                        tf32_split(xb[q][(s0 + t4) * xs[q] + g], bh[0], bl[0]);
+                        tf32_split(xb[q][(s0 + t4 + 4) * xs[q] + g], bh[1], bl[1]);
+                        mma_tf32(acc[q], al, bh);
+                        mma_tf32(acc[q], ah, bl);
+                        mma_tf32(acc[q], ah, bh);
+                    }
                 }
             }
 #pragma unroll
             for (int q = 0; q < NTW; ++q) {
-                const int n0 = (warp * NTW + q) * 8;
+                const int nt = warp + nwarps * q;
+                if (nt < NCOL / 8) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) stage[(g + (c >> 1) * 8) * NCOL + n0 + 2 * t4 + (c & 1)] = acc[q][c];
+                    for (int c = 0; c < 4; ++c)
+                        stage[(g + (c >> 1) * 8) * STS + nt * 8 + 2 * t4 + (c & 1)] = acc[q][c];
+                }
             }
         }
         __syncthreads();
@@ -227,7 +244,7 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
             float xb[16];
 #pragma unroll
             for (int tr = 0; tr < 16; ++tr) {
-                float acc = stage[tr * NCOL + col];
+                float acc = stage[tr * STS + col];
 #pragma unroll
                 for (int sr = 0; sr < tr; ++sr) acc = ffma(-cc[(t0 + tr) * CCS + t0 + sr], xb[sr], acc);
                 xb[tr] = fmul(bs[t0 + tr], acc);
@@ -465,11 +482,39 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
     const int h = task % H, g = task / H;
     const int n = find_seq(fco, N, g);
     const int64_t tok0 = (int64_t)__ldg(cu + n) + (int64_t)(g - __ldg(fco + n)) * C;
-    stage_rows<DK>(kx, PL::KXS, k, tok0, C, H, h, in_bf16, IdxIdentity());
-    stage_rows<DV>(vx, PL::VXS, v, tok0, C, H, h, in_bf16, IdxIdentity());
     for (int t = threadIdx.x; t < C; t += blockDim.x) {
-        as[t] = __ldg(alpha + (tok0 + t) * H + h);
-        bs[t] = __ldg(beta + (tok0 + t) * H + h);
+        cp_async4(as + t, alpha + (tok0 + t) * H + h);
+        cp_async4(bs + t, beta + (tok0 + t) * H + h);
+    }
+    if (in_bf16) {
+        // raw bf16 rows [k | v] of the chunk land in the c / decay buffers
+        // (unused until the Gram), all copies in flight at once; then widen
+        static_assert(Sm::DM_OFF + ((PL::DM + 3) / 4) * 4 - Sm::CC_OFF >= C * (DK + DV) / 2, "raw staging fits");
+        unsigned char* raw = reinterpret_cast<unsigned char*>(cc);
+        constexpr int PK = DK / 8, PV = DV / 8;  // 16-byte pieces per row
+        for (int e = threadIdx.x; e < C * (PK + PV); e += blockDim.x) {
+            const int t = e / (PK + PV), pc = e % (PK + PV);
+            const int64_t row = (tok0 + t) * H + h;
+            const uint16_t* src = pc < PK ? reinterpret_cast<const uint16_t*>(k) + row * DK + pc * 8
+                                          : reinterpret_cast<const uint16_t*>(v) + row * DV + (pc - PK) * 8;
+            cp_async16(raw + (size_t)e * 16, src);
+        }
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncthreads();
+        for (int e = threadIdx.x; e < C * (PK + PV); e += blockDim.x) {
+            const int t = e / (PK + PV), pc = e % (PK + PV);
+            float x[8];
+            lds8_raw(raw + (size_t)e * 16, 0, 1, x);
+            float* d = pc < PK ? kx + t * PL::KXS + pc * 8 : vx + t * PL::VXS + (pc - PK) * 8;
+            *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
+            *reinterpret_cast<float4*>(d + 4) = make_float4(x[4], x[5], x[6], x[7]);
+        }
+    } else {
+        stage_rows<DK>(kx, PL::KXS, k, tok0, C, H, h, in_bf16, IdxIdentity());
+        stage_rows<DV>(vx, PL::VXS, v, tok0, C, H, h, in_bf16, IdxIdentity());
+        cp_async_commit();
+        cp_async_wait_all();
     }
     __syncthreads();
     chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, w_ws + (int64_t)task * C * DK, DK,
