@@ -152,7 +152,9 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
         while ((m + 1) * (m + 2) <= tile) ++m;
         const int q = tile - m * (m + 1);
         const int r0 = m * 16, n0 = q * 8;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
 #pragma unroll 4
         for (int kb = 0; kb < DK / 8; ++kb) {
             const int k0 = kb * 8;
@@ -163,21 +165,23 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
                 const uint32_t ah[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
                                         __float_as_uint(a3)};
                 const uint32_t bh[2] = {__float_as_uint(b0), __float_as_uint(b1)};
-                mma_tf32(acc, ah, bh);
+                mma_tf32(acc[kb & 3], ah, bh);
             } else {
                 uint32_t ah[4], al[4], bh[2], bl[2];
                 tf32_split(a0, ah[0], al[0]); tf32_split(a1, ah[1], al[1]);
                 tf32_split(a2, ah[2], al[2]); tf32_split(a3, ah[3], al[3]);
                 tf32_split(b0, bh[0], bl[0]); tf32_split(b1, bh[1], bl[1]);
-                mma_tf32(acc, al, bh);
-                mma_tf32(acc, ah, bl);
-                mma_tf32(acc, ah, bh);
+                mma_tf32(acc[0], al, bh);
+                mma_tf32(acc[1], ah, bl);
+                mma_tf32(acc[2], ah, bh);
             }
         }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int tau = r0 + g + (c >> 1) * 8, sig = n0 + 2 * t4 + (c & 1);
-            if (sig < tau) cc[tau * CCS + sig] = fmul(dm[(tau + 1) * C1 + (sig + 1)], acc[c]);
+            const float G = k_exact ? fadd(fadd(acc[0][c], acc[1][c]), fadd(acc[2][c], acc[3][c]))
+                                    : fadd(fadd(acc[0][c], acc[1][c]), acc[2][c]);
+            if (sig < tau) cc[tau * CCS + sig] = fmul(dm[(tau + 1) * C1 + (sig + 1)], G);
         }
     }
     for (int t = threadIdx.x; t < C; t += blockDim.x) d0[t] = dm[(t + 1) * C1];  // D[t][0], t = 1..C
@@ -191,7 +195,7 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
         // tile all u0 or all w columns); its tiles share the split c fragment
         {
             constexpr int NTW = (NCOL / 8 + 7) / 8;  // tiles per warp with 8 warps
-            float acc[NTW][4];
+            float init[NTW][4], plh[NTW][4], phl[NTW][4], phh[NTW][4];
             const float* xb[NTW];
             int xs[NTW];
 #pragma unroll
@@ -201,12 +205,12 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
                 const bool is_u = n0 < DV;
                 xb[q] = is_u ? vx + n0 : kx + (n0 - DV);
                 xs[q] = is_u ? VXS : KXS;
-                if (nt < NCOL / 8) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int tau = t0 + g + (c >> 1) * 8, cl = 2 * t4 + (c & 1);
-                        acc[q][c] = is_u ? xb[q][tau * xs[q] + cl] : fmul(d0[tau], xb[q][tau * xs[q] + cl]);
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    plh[q][c] = phl[q][c] = phh[q][c] = 0.f;
+                    const int tau = t0 + g + (c >> 1) * 8, cl = 2 * t4 + (c & 1);
+                    init[q][c] = nt >= NCOL / 8 ? 0.f
+                                 : is_u ? xb[q][tau * xs[q] + cl] : fmul(d0[tau], xb[q][tau * xs[q] + cl]);
                 }
             }
             for (int kb = 0; kb < 2 * b; ++kb) {
@@ -222,9 +226,9 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
                         uint32_t bh[2], bl[2];
                         tf32_split(xb[q][(s0 + t4) * xs[q] + g], bh[0], bl[0]);
                         tf32_split(xb[q][(s0 + t4 + 4) * xs[q] + g], bh[1], bl[1]);
-                        mma_tf32(acc[q], al, bh);
-                        mma_tf32(acc[q], ah, bl);
-                        mma_tf32(acc[q], ah, bh);
+                        mma_tf32(plh[q], al, bh);
+                        mma_tf32(phl[q], ah, bl);
+                        mma_tf32(phh[q], ah, bh);
                     }
                 }
             }
@@ -233,8 +237,11 @@ __device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as
                 const int nt = warp + nwarps * q;
                 if (nt < NCOL / 8) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        stage[(g + (c >> 1) * 8) * STS + nt * 8 + 2 * t4 + (c & 1)] = acc[q][c];
+                    for (int c = 0; c < 4; ++c) {
+                        const float acc = b == 0 ? init[q][c]
+                                                 : fadd(init[q][c], fadd(fadd(plh[q][c], phl[q][c]), phh[q][c]));
+                        stage[(g + (c >> 1) * 8) * STS + nt * 8 + 2 * t4 + (c & 1)] = acc;
+                    }
                 }
             }
         }
@@ -314,9 +321,12 @@ __device__ __forceinline__ void mma_phase1(const float* Ss, const float* ws, con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     if (warp >= 4) return;
     const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
-    float acc[M::P1][4];
+    // one accumulator per split product (independent tensor-core chains)
+    float alh[M::P1][4], ahl[M::P1][4], ahh[M::P1][4];
 #pragma unroll
-    for (int q = 0; q < M::P1; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+    for (int q = 0; q < M::P1; ++q)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) alh[q][c] = ahl[q][c] = ahh[q][c] = 0.f;
 #pragma unroll 2
     for (int kb = 0; kb < DK / 8; ++kb) {
         const int k0 = kb * 8;
@@ -332,9 +342,9 @@ __device__ __forceinline__ void mma_phase1(const float* Ss, const float* ws, con
                 uint32_t bh[2], bl[2];
                 tf32_split(ws[(nt * 8 + g) * KS + k0 + t], bh[0], bl[0]);
                 tf32_split(ws[(nt * 8 + g) * KS + k0 + t + 4], bh[1], bl[1]);
-                mma_tf32(acc[q], al, bh);
-                mma_tf32(acc[q], ah, bl);
-                mma_tf32(acc[q], ah, bh);
+                mma_tf32(alh[q], al, bh);
+                mma_tf32(ahl[q], ah, bl);
+                mma_tf32(ahh[q], ah, bh);
             }
         }
     }
@@ -345,7 +355,8 @@ __device__ __forceinline__ void mma_phase1(const float* Ss, const float* ws, con
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int i = r0 + g + (c >> 1) * 8, tau = nt * 8 + 2 * t + (c & 1);
-                es[i * ES + tau] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], acc[q][c]));
+                const float E = fadd(fadd(alh[q][c], ahl[q][c]), ahh[q][c]);
+                es[i * ES + tau] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], E));
             }
         }
     }
@@ -354,21 +365,26 @@ __device__ __forceinline__ void mma_phase1(const float* Ss, const float* ws, con
 // Phase 2 (warps 0..3): Sreg (this lane's entries of the tile in the phase-2
 // accumulator layout) <- S'.  The new rows also go to Ss and, when non-null,
 // to dst1 / dst2 (global, row stride DK).  k_exact: k values are exact tf32.
-template <int DK, int RTB, int C>
-__device__ __forceinline__ void mma_phase2(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* es,
-                                           const float* kT, float d0, int k_exact, float* dst1, float* dst2)
+template <int DK, int RTB, int C, bool K_EXACT>
+__device__ __forceinline__ void mma_phase2_t(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* es,
+                                             const float* kT, float d0, float* dst1, float* dst2)
 {
     using M = MmaAdv<DK, RTB, C>;
     constexpr int KS = M::KS, ES = M::ES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     if (warp >= 4) return;
     const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
-    float acc[M::P2][4];
+    constexpr int NHL = K_EXACT ? 1 : M::P2;  // the k_lo product is absent when k is exact tf32
+    float alh[M::P2][4], ahl[NHL][4], ahh[M::P2][4];
 #pragma unroll
     for (int q = 0; q < M::P2; ++q)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[q][c] = fmul(d0, Sreg[q][c]);
-#pragma unroll 2
+        for (int c = 0; c < 4; ++c) alh[q][c] = ahh[q][c] = 0.f;
+#pragma unroll
+    for (int q = 0; q < NHL; ++q)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ahl[q][c] = 0.f;
+#pragma unroll 1
     for (int kb = 0; kb < C / 8; ++kb) {
         const int k0 = kb * 8;
         uint32_t ah[4], al[4];
@@ -381,17 +397,17 @@ __device__ __forceinline__ void mma_phase2(float (&Sreg)[MmaAdv<DK, RTB, C>::P2]
             const int nt = wg + M::WG * q;
             if (nt < M::NT2) {
                 const float b0 = kT[(nt * 8 + g) * ES + k0 + t], b1 = kT[(nt * 8 + g) * ES + k0 + t + 4];
-                if (k_exact) {
+                if constexpr (K_EXACT) {
                     const uint32_t b[2] = {__float_as_uint(b0), __float_as_uint(b1)};
-                    mma_tf32(acc[q], al, b);
-                    mma_tf32(acc[q], ah, b);
+                    mma_tf32(alh[q], al, b);
+                    mma_tf32(ahh[q], ah, b);
                 } else {
                     uint32_t bh[2], bl[2];
                     tf32_split(b0, bh[0], bl[0]);
                     tf32_split(b1, bh[1], bl[1]);
-                    mma_tf32(acc[q], al, bh);
-                    mma_tf32(acc[q], ah, bl);
-                    mma_tf32(acc[q], ah, bh);
+                    mma_tf32(alh[q], al, bh);
+                    mma_tf32(ahl[q], ah, bl);
+                    mma_tf32(ahh[q], ah, bh);
                 }
             }
         }
@@ -401,17 +417,29 @@ __device__ __forceinline__ void mma_phase2(float (&Sreg)[MmaAdv<DK, RTB, C>::P2]
         const int nt = wg + M::WG * q;
         if (nt < M::NT2) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) Sreg[q][c] = acc[q][c];
+            for (int c = 0; c < 4; ++c) {
+                float x = fadd(fmul(d0, Sreg[q][c]), alh[q][c]);
+                if constexpr (!K_EXACT) x = fadd(x, ahl[q][c]);
+                Sreg[q][c] = fadd(x, ahh[q][c]);
+            }
 #pragma unroll
             for (int hrow = 0; hrow < 2; ++hrow) {
                 const int i = r0 + g + hrow * 8, j = nt * 8 + 2 * t;
-                const float2 x = make_float2(acc[q][2 * hrow], acc[q][2 * hrow + 1]);
+                const float2 x = make_float2(Sreg[q][2 * hrow], Sreg[q][2 * hrow + 1]);
                 *reinterpret_cast<float2*>(Ss + i * KS + j) = x;
                 if (dst1 != nullptr) *reinterpret_cast<float2*>(dst1 + (int64_t)i * DK + j) = x;
                 if (dst2 != nullptr) *reinterpret_cast<float2*>(dst2 + (int64_t)i * DK + j) = x;
             }
         }
     }
+}
+
+template <int DK, int RTB, int C>
+__device__ __forceinline__ void mma_phase2(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* es,
+                                           const float* kT, float d0, int k_exact, float* dst1, float* dst2)
+{
+    if (k_exact) mma_phase2_t<DK, RTB, C, true>(Sreg, Ss, es, kT, d0, dst1, dst2);
+    else mma_phase2_t<DK, RTB, C, false>(Sreg, Ss, es, kT, d0, dst1, dst2);
 }
 
 // Load the RTB rows at src (global, row stride DK) into Ss and this lane's
