@@ -9,6 +9,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -203,7 +204,9 @@ gdn_status_t launch_decode(const DecArgs& a)
     mark(a.events, 1, a.stream);
     constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
     if (set_smem(gdn::k_dec_resync<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
-    const unsigned rgrid = (unsigned)(NH < sms ? NH : sms);  // persistent: one CTA per SM
+    // persistent: one CTA per SM, and at most 1024 (sequence, head) pairs per CTA
+    const int64_t min_grid = (NH + 1023) / 1024;
+    const unsigned rgrid = (unsigned)std::max<int64_t>(std::min<int64_t>(NH, sms), min_grid);
     gdn::k_dec_resync<D, D, C><<<rgrid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
         (int)NH, a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;

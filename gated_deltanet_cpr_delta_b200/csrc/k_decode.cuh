@@ -32,6 +32,12 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
     const int nh = blockIdx.x / Cf::NT, r = blockIdx.x % Cf::NT;
     const int p = pos[nh];
     if (p < 0 || p >= C) return;
+    // the state rows are the bulk of the traffic: issue their loads before staging the token
+    const int row = threadIdx.x / RS::TPR, part = threadIdx.x % RS::TPR;
+    const int grow = r * Cf::RT + row;
+    float* Rrow = R + ((int64_t)nh * DV + grow) * DK + part * RS::EPT;
+    f2x Rp[RS::L];
+    load_row_pairs<DK>(Rp, Rrow);
     stage_rows<DK>(ks, RS::KS, k, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
     stage_rows<DK>(qs, RS::KS, q, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
     for (int e = threadIdx.x; e < Cf::RT / 8; e += blockDim.x) {
@@ -41,11 +47,6 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
         for (int m = 0; m < 8; ++m) vs[e * 8 + m] = x[m];
     }
     const float a = __ldg(alpha + nh), b = __ldg(beta + nh);
-    const int row = threadIdx.x / RS::TPR, part = threadIdx.x % RS::TPR;
-    const int grow = r * Cf::RT + row;
-    float* Rrow = R + ((int64_t)nh * DV + grow) * DK + part * RS::EPT;
-    f2x Rp[RS::L];
-    load_row_pairs<DK>(Rp, Rrow);
     __syncthreads();
     const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
     store_row_pairs<DK>(Rrow, Rp);
@@ -114,14 +115,27 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
     float* bs = as + C;
     float* dCs = sm + Sm::DC_OFF;
 
-    for (int nh = blockIdx.x; nh < NH; nh += gridDim.x) {
+    // this CTA's pairs are blockIdx.x + i*gridDim.x: read all their positions
+    // at once, advance the ones inside a chunk, and list the ones at a boundary
+    __shared__ int todo[1024];
+    __shared__ int ntodo;
+    if (threadIdx.x == 0) ntodo = 0;
+    __syncthreads();
+    for (int nh = blockIdx.x + threadIdx.x * gridDim.x; nh < NH; nh += blockDim.x * gridDim.x) {
         const int p = pos[nh];
-        __syncthreads();  // every thread has read pos (and the previous pair's smem) before anything moves
-        if (p < 0 || p >= C) continue;
+        if (p < 0 || p >= C) continue;          // invalid: left unchanged
         if (p + 1 < C) {
-            if (threadIdx.x == 0) pos[nh] = p + 1;
-            continue;
+            pos[nh] = p + 1;
+        } else {
+            const int slot = atomicAdd(&ntodo, 1);
+            if (slot < 1024) todo[slot] = nh;   // the host sizes the grid so that a CTA has <= 1024 pairs
         }
+    }
+    __syncthreads();
+    const int nt = min(ntodo, 1024);
+    for (int it = 0; it < nt; ++it) {
+        const int nh = todo[it];
+        __syncthreads();  // the previous pair's smem reads are done
         // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
         stage_rows<DK>(kx, PL::KXS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
         stage_rows<DV>(vx, PL::VXS, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
