@@ -69,14 +69,24 @@ def decode_tok_bytes(dk: int, dv: int, esz: int, out_esz: int):
 
 
 # DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
-# dram__bytes_write.sum), keyed by kernel, valid only for the kernel source
-# it was taken from (sha256 of the csrc/*.cuh kernel sources).
-NCU_TRAFFIC = {}
+# dram__bytes_write.sum), keyed by kernel and by the sha256 of the sources that
+# kernel is compiled from; a changed source drops the figure (reported null).
+NCU_TRAFFIC = {
+    # profiles/k_tok_prefill_B4_H16_T4096_d128_C64.md: 472,237,312 read + 57,675,520 written
+    ("k_tok", "92818b084eaef9b3"): 529912832,
+    # profiles/k_dec_tok_decode_N64_H32_d128_C64.md: 135,855,104 read + 82,424,320 written
+    ("k_dec_tok", "929039235fd7a689"): 218279424,
+}
+
+KERNEL_SOURCES = {
+    "k_tok": ("schedule.cuh", "k_ptok.cuh"),
+    "k_dec_tok": ("schedule.cuh", "k_ptok.cuh", "k_decode.cuh"),
+}
 
 
-def kernel_source_sha():
+def kernel_source_sha(kernel: str = "k_tok"):
     h = hashlib.sha256()
-    for f in ("kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_pchunk.cuh", "k_decode.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "gated_deltanet_cpr_delta_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -279,6 +289,7 @@ def bench_decode(rank: int, world: int, warmup: int):
         t = torch.arange(N, device="cuda") * L + Lp + s
         steps_in.append([d[n][t].contiguous() for n in ("q", "k", "v", "alpha", "beta")])
     del d
+    torch.cuda.empty_cache()   # only the cache and the step inputs stay on the device
     o = torch.empty(N, H, D, dtype=torch.bfloat16, device="cuda")
     # warm-up on a copy of the cache (the timed steps start at position Lp)
     wc = {k_: v_.clone() for k_, v_ in cache.items()}
@@ -313,7 +324,8 @@ def bench_decode(rank: int, world: int, warmup: int):
             "resync_kernel_ms_max": max(res_ms),
             "roofline": {"kernel": "k_dec_tok", "bound": "hbm", "achieved": tb / (mean_tok / 1e3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": tb / (mean_tok / 1e3) / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                         "frac": tb / (mean_tok / 1e3) / 1e9 / peaks["hbm_gbs"],
+                         "traffic": NCU_TRAFFIC.get(("k_dec_tok", kernel_source_sha("k_dec_tok"))),
                          "bytes_per_launch": tb}}
 
 
