@@ -148,8 +148,7 @@ gdn_status_t launch_forward(const FwdArgs& a)
     if (a.N > 0) {
         constexpr size_t sm = gdn::ChainSmem<D, D, C>::BYTES;
         if (set_smem(gdn::k_chain<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
-        gdn::k_chain<D, D, C><<<(unsigned)((int64_t)a.N * a.H * Cf::NTB), gdn::MmaAdv<D, Cf::RTB, C>::THREADS, sm,
-                                a.stream>>>(
+        gdn::k_chain<D, D, C><<<(unsigned)((int64_t)a.N * a.H), gdn::TcCfg<D, D, C>::THREADS, sm, a.stream>>>(
             a.k, a.state_in, a.cu, a.ws.fco, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.ws.w, a.ws.u, a.ws.dC,
             a.states);
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;

@@ -69,37 +69,42 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
 template <int DK, int DV, int C>
 struct ResyncSmem {
     using Cf = ChunkCfg<DK, DV, C>;
-    using M = MmaAdv<DK, Cf::RTB, C>;
     using PL = PrepLayout<DK, DV, C>;
+    using T = TcCfg<DK, DV, C>;
     static constexpr int KX_OFF = 0;                                 // [C][KXS] k, then w
     static constexpr int VX_OFF = KX_OFF + C * PL::KXS;              // [C][VXS] v, then u0
-    static constexpr int CC_OFF = VX_OFF + C * PL::VXS;              // [C][CCS] c
+    static constexpr int WLO_OFF = VX_OFF + C * PL::VXS;             // canonical w lo, then w hi ...
+    static constexpr int CC_OFF = WLO_OFF + T::W_FLOATS;             // ... in the [C][CCS] c of chunk_prep
     static constexpr int DM_OFF = CC_OFF + C * PL::CCS;              // decays / staging
     static constexpr int D0_OFF = DM_OFF + ((PL::DM + 3) / 4) * 4;   // D[t][0]
-    static constexpr int WS_OFF = D0_OFF + C + 4;                    // [C][KS] w for the tensor-core phases
-    static constexpr int SS_OFF = WS_OFF + C * M::KS;                // [RTB][KS] S tile
-    static constexpr int ES_OFF = SS_OFF + Cf::RTB * M::KS;          // [RTB][ES] e
-    static constexpr int KT_OFF = ES_OFF + Cf::RTB * M::ES;          // [DK][ES] k^T
-    static constexpr int AB_OFF = KT_OFF + DK * M::ES;
+    static constexpr int AB_OFF = D0_OFF + C + 4;
     static constexpr int DC_OFF = AB_OFF + 2 * C;
-    static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
+    static constexpr int KLO_OFF = DC_OFF + Cf::DCS;                 // canonical k^T lo | hi, then S' staging
+    static constexpr int KHI_OFF = KLO_OFF + T::K_FLOATS;
+    static constexpr int BAR_OFF = KLO_OFF + T::K_REGION;            // mbarrier (8 bytes) + TMEM base
+    // at least 120 KB, so that one CTA fits per SM: each allocates all 512 TMEM columns
+    static constexpr size_t USED = sizeof(float) * (BAR_OFF + 4);
+    static constexpr size_t BYTES = USED > 120 * 1024 ? USED : 120 * 1024;
+    static_assert(BYTES <= 232448, "fits the 227 KB of shared memory a CTA can have");
+    static_assert(D0_OFF - CC_OFF >= T::W_FLOATS, "w hi fits in the c / decay scratch");
+    static_assert(BAR_OFF % 2 == 0 && DC_OFF % 4 == 0 && KLO_OFF % 4 == 0, "alignment");
 };
 
 // Advances pos after k_dec_tok appended a token at slot pos, and resyncs
 // where that token completed a chunk: S_b <- P_chunk(S_b, buffer), R <- S_b,
-// pos <- 0.  P_chunk runs the same device functions as the prefill (chunk_prep,
-// then the tensor-core phases per row tile).  Persistent: CTA b handles
-// (sequence, head) pairs b, b + grid, ...  A pos outside [0, C) is left unchanged.
+// pos <- 0.  P_chunk runs the same device functions as the prefill
+// (chunk_prep, then the tcgen05 boundary step).  Persistent: CTA b handles
+// (sequence, head) pairs b, b + grid, ...  A pos outside [0, C) is left
+// unchanged.  If an MMA completion wait times out, the pairs this CTA had
+// still to resync get pos = -1 and are not written.
 template <int DK, int DV, int C>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 1)
 k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
              const float* bbuf, int32_t* pos)
 {
-    using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ResyncSmem<DK, DV, C>;
-    using M = MmaAdv<DK, Cf::RTB, C>;
     using PL = PrepLayout<DK, DV, C>;
-    constexpr int RTB = Cf::RTB;
+    using T = TcCfg<DK, DV, C>;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
     float* kx = sm + Sm::KX_OFF;
@@ -107,13 +112,15 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
     float* cc = sm + Sm::CC_OFF;
     float* dm = sm + Sm::DM_OFF;
     float* d0 = sm + Sm::D0_OFF;
-    float* ws = sm + Sm::WS_OFF;
-    float* Ss = sm + Sm::SS_OFF;
-    float* es = sm + Sm::ES_OFF;
-    float* kT = sm + Sm::KT_OFF;
     float* as = sm + Sm::AB_OFF;
     float* bs = as + C;
     float* dCs = sm + Sm::DC_OFF;
+    float* Wlo = sm + Sm::WLO_OFF;
+    float* Whi = cc;  // == Wlo + C * DK
+    float* Khi = sm + Sm::KHI_OFF;
+    float* Klo = sm + Sm::KLO_OFF;
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Sm::BAR_OFF);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Sm::BAR_OFF + 2);
 
     // this CTA's pairs are blockIdx.x + i*gridDim.x: read all their positions
     // at once, advance the ones inside a chunk, and list the ones at a boundary
@@ -133,31 +140,49 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
     }
     __syncthreads();
     const int nt = min(ntodo, 1024);
-    for (int it = 0; it < nt; ++it) {
+    if (nt == 0) return;
+
+    if (threadIdx.x == 0) mbar_init(mbar, 1);
+    if (threadIdx.x < 32) tmem_alloc(tslot, T::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tslot;
+    const TcThread<DK> th(tbase);
+    uint32_t parity = 0;
+    float SR[DK / 2];
+    int it = 0;
+    for (; it < nt; ++it) {
         const int nh = todo[it];
-        __syncthreads();  // the previous pair's smem reads are done
         // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
         stage_rows<DK>(kx, PL::KXS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
         stage_rows<DV>(vx, PL::VXS, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
-        stage_kT<DK, C>(kT, kbuf, (int64_t)nh * C, 1, 0, in_bf16);
+        tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
         for (int t = threadIdx.x; t < C; t += blockDim.x) {
             as[t] = abuf[(int64_t)nh * C + t];
             bs[t] = bbuf[(int64_t)nh * C + t];
         }
         __syncthreads();
-        chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, ws, M::KS, vx, PL::VXS, dCs);
-        float Sreg[M::P2][4];
-        for (int r = 0; r < Cf::NTB; ++r) {
-            float* Sg = S_b + ((int64_t)nh * DV + r * RTB) * DK;
-            float* Rg = R + ((int64_t)nh * DV + r * RTB) * DK;
-            mma_load_state<DK, RTB, C>(Sreg, Ss, Sg);
-            mma_phase1<DK, RTB, C>(Ss, ws, vx + r * RTB, PL::VXS, dCs, es);
-            __syncthreads();
-            mma_phase2<DK, RTB, C>(Sreg, Ss, es, kT, dCs[0], in_bf16, Sg, Rg);
-            __syncthreads();
-        }
+        chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, kx, PL::KXS, vx, PL::VXS, dCs);
+        tc_stage_w<DK, DV, C>(kx, PL::KXS, Whi, Wlo, threadIdx.x, blockDim.x);
+        float* Sg = S_b + (int64_t)nh * DV * DK;
+        tc_load_state<DK, DV, C>(SR, th, Sg, nullptr);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (!tc_step<DK, DV, C>(SR, th, tbase, mbar, parity, Wlo, Klo, vx, PL::VXS, dCs, in_bf16, Sg,
+                                R + (int64_t)nh * DV * DK))
+            break;
         if (threadIdx.x == 0) pos[nh] = 0;
     }
+    for (int r = it + threadIdx.x; r < nt; r += blockDim.x) pos[todo[r]] = -1;  // after a timeout
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        tc_fence_after();
+        tmem_dealloc(tbase, T::TMEM_COLS);
+    }
 }
+
 
 }  // namespace gdn

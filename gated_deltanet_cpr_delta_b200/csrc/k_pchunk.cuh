@@ -2,6 +2,7 @@
 #pragma once
 
 #include "k_ptok.cuh"
+#include "k_tc.cuh"
 
 namespace gdn {
 
@@ -16,80 +17,6 @@ struct ChunkCfg {
     static constexpr int NTB = DV / RTB;
     static constexpr int THREADS = 256;
 };
-
-// VEC consecutive floats from smem (VEC = 4 or 2; 4*VEC-byte aligned).
-template <int VEC>
-__device__ __forceinline__ void lds_n(float (&r)[VEC], const float* s)
-{
-    if constexpr (VEC == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(s);
-        r[0] = x.x; r[1] = x.y; r[2] = x.z; r[3] = x.w;
-    } else {
-        const float2 x = *reinterpret_cast<const float2*>(s);
-        r[0] = x.x; r[1] = x.y;
-    }
-}
-
-// tree(x_a, y_b) for an RA x RB block of row pairs, all rows of stride KS in
-// smem: xa[r] = row r of the first operand, yb[c] = row c of the second.
-// The leaves run in ascending j; VEC elements are read at a time.
-template <int DK, int KS, int RA, int RB>
-__device__ __forceinline__ void tree_block(const float* const (&xa)[RA], const float* const (&yb)[RB],
-                                           float (&out)[RA][RB])
-{
-    constexpr int L = DK / kLeaves;
-    constexpr int VEC = (L % 4 == 0) ? 4 : 2;
-    TreeAcc st[RA][RB];
-#pragma unroll
-    for (int l = 0; l < kLeaves; ++l) {
-        float acc[RA][RB];
-#pragma unroll
-        for (int m = 0; m < L; m += VEC) {
-            float a[RA][VEC], b[RB][VEC];
-#pragma unroll
-            for (int r = 0; r < RA; ++r) lds_n<VEC>(a[r], xa[r] + l * L + m);
-#pragma unroll
-            for (int c = 0; c < RB; ++c) lds_n<VEC>(b[c], yb[c] + l * L + m);
-#pragma unroll
-            for (int e = 0; e < VEC; ++e)
-#pragma unroll
-                for (int r = 0; r < RA; ++r)
-#pragma unroll
-                    for (int c = 0; c < RB; ++c)
-                        acc[r][c] = (m + e == 0) ? fmul(a[r][e], b[c][e]) : ffma(a[r][e], b[c][e], acc[r][c]);
-        }
-#pragma unroll
-        for (int r = 0; r < RA; ++r)
-#pragma unroll
-            for (int c = 0; c < RB; ++c) tree_push(st[r][c], l, acc[r][c]);
-    }
-#pragma unroll
-    for (int r = 0; r < RA; ++r)
-#pragma unroll
-        for (int c = 0; c < RB; ++c) out[r][c] = st[r][c].t0;
-}
-
-// Forward substitution of one column, right-looking and fully unrolled: once
-// token s is final, its term enters every later token's chain.  For each
-// token t the chain still runs over s = 1..t-1 in ascending order.
-// acc[t] holds the chain start on entry and the column's result on exit.
-template <int C, int CT>
-__device__ __forceinline__ void fwd_subst(float (&acc)[C], const float* cT, const float* bs)
-{
-#pragma unroll
-    for (int sig = 0; sig < C; ++sig) {
-        acc[sig] = fmul(bs[sig], acc[sig]);
-        const float x = acc[sig];
-#pragma unroll
-        for (int tg = (sig + 1) / 4; tg < C / 4; ++tg) {
-            const float4 c4 = *reinterpret_cast<const float4*>(cT + sig * CT + 4 * tg);
-            if (4 * tg + 0 > sig) acc[4 * tg + 0] = ffma(-c4.x, x, acc[4 * tg + 0]);
-            if (4 * tg + 1 > sig) acc[4 * tg + 1] = ffma(-c4.y, x, acc[4 * tg + 1]);
-            if (4 * tg + 2 > sig) acc[4 * tg + 2] = ffma(-c4.z, x, acc[4 * tg + 2]);
-            if (4 * tg + 3 > sig) acc[4 * tg + 3] = ffma(-c4.w, x, acc[4 * tg + 3]);
-        }
-    }
-}
 
 // P_chunk part 1 for one chunk, by one CTA (>= 128 threads), on the tensor
 // cores where the work is a dense contraction:
@@ -284,206 +211,6 @@ struct PrepSmem {
     static constexpr size_t BYTES = sizeof(float) * (AB_OFF + 2 * C);
 };
 
-// ---------------------------------------------------------------- tensor-core P_chunk part 2
-// The two contractions of the boundary update on the tensor cores
-// (mma.sync m16n8k8, tf32 operands, fp32 accumulate), with every fp32
-// operand x split into hi = tf32(x) and lo = tf32(x - hi):
-//   phase 1: E[i][t] = sum_j S[i][j] w_t[j]; per 8-wide block of j, in
-//            ascending order: E += S_lo*w_hi, E += S_hi*w_lo, E += S_hi*w_hi;
-//            then e_t[i] = D[C][t] * (u0_t[i] - E[i][t]).
-//   phase 2: S'[i][j] = D[C][0]*S[i][j] + sum_t e_t[i] k_t[j]; accumulator
-//            starts at D[C][0]*S[i][j], then per 8-token block, ascending:
-//            S' += e_lo*k_hi, S' += e_hi*k_lo, S' += e_hi*k_hi.  When k is
-//            exactly tf32 (bf16 inputs), k_lo = 0 and that product is skipped.
-// The prefill chain and the decode resync run these same functions, so the
-// same operands give the same bits.  A CTA has 4 warps on a tile of RTB rows
-// (RTB = 16 or 32): warp w owns m16 tile w % MT and every WG-th n8 tile.
-template <int DK, int RTB, int C>
-struct MmaAdv {
-    static constexpr int MT = RTB / 16;             // m16 row tiles
-    static constexpr int WG = 4 / MT;               // warps sharing a row tile
-    static constexpr int NT1 = C / 8, NT2 = DK / 8;
-    static constexpr int P1 = (NT1 + WG - 1) / WG;  // phase-1 n8 tiles per warp
-    static constexpr int P2 = (NT2 + WG - 1) / WG;  // phase-2 n8 tiles per warp
-    static constexpr int KS = DK + 4;               // S and w row stride (floats)
-    static constexpr int ES = C + 4;                // e and k^T row stride (floats)
-    static constexpr int THREADS = 128;
-    static_assert(RTB == 16 || RTB == 32, "row tile");
-};
-
-// Phase 1 (warps 0..3): es[i*ES + t] = e_t[i] for the RTB rows of the tile.
-template <int DK, int RTB, int C>
-__device__ __forceinline__ void mma_phase1(const float* Ss, const float* ws, const float* us, int ldu,
-                                           const float* dCs, float* es)
-{
-    using M = MmaAdv<DK, RTB, C>;
-    constexpr int KS = M::KS, ES = M::ES;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    if (warp >= 4) return;
-    const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
-    // one accumulator per split product (independent tensor-core chains)
-    float alh[M::P1][4], ahl[M::P1][4], ahh[M::P1][4];
-#pragma unroll
-    for (int q = 0; q < M::P1; ++q)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) alh[q][c] = ahl[q][c] = ahh[q][c] = 0.f;
-#pragma unroll 2
-    for (int kb = 0; kb < DK / 8; ++kb) {
-        const int k0 = kb * 8;
-        uint32_t ah[4], al[4];
-        tf32_split(Ss[(r0 + g) * KS + k0 + t], ah[0], al[0]);
-        tf32_split(Ss[(r0 + g + 8) * KS + k0 + t], ah[1], al[1]);
-        tf32_split(Ss[(r0 + g) * KS + k0 + t + 4], ah[2], al[2]);
-        tf32_split(Ss[(r0 + g + 8) * KS + k0 + t + 4], ah[3], al[3]);
-#pragma unroll
-        for (int q = 0; q < M::P1; ++q) {
-            const int nt = wg + M::WG * q;
-            if (nt < M::NT1) {
-                uint32_t bh[2], bl[2];
-                tf32_split(ws[(nt * 8 + g) * KS + k0 + t], bh[0], bl[0]);
-                tf32_split(ws[(nt * 8 + g) * KS + k0 + t + 4], bh[1], bl[1]);
-                mma_tf32(alh[q], al, bh);
-                mma_tf32(ahl[q], ah, bl);
-                mma_tf32(ahh[q], ah, bh);
-            }
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < M::P1; ++q) {
-        const int nt = wg + M::WG * q;
-        if (nt < M::NT1) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int i = r0 + g + (c >> 1) * 8, tau = nt * 8 + 2 * t + (c & 1);
-                const float E = fadd(fadd(alh[q][c], ahl[q][c]), ahh[q][c]);
-                es[i * ES + tau] = fmul(dCs[tau + 1], fsub(us[tau * ldu + i], E));
-            }
-        }
-    }
-}
-
-// Phase 2 (warps 0..3): Sreg (this lane's entries of the tile in the phase-2
-// accumulator layout) <- S'.  The new rows also go to Ss and, when non-null,
-// to dst1 / dst2 (global, row stride DK).  k_exact: k values are exact tf32.
-template <int DK, int RTB, int C, bool K_EXACT>
-__device__ __forceinline__ void mma_phase2_t(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* es,
-                                             const float* kT, float d0, float* dst1, float* dst2)
-{
-    using M = MmaAdv<DK, RTB, C>;
-    constexpr int KS = M::KS, ES = M::ES;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    if (warp >= 4) return;
-    const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
-    constexpr int NHL = K_EXACT ? 1 : M::P2;  // the k_lo product is absent when k is exact tf32
-    float alh[M::P2][4], ahl[NHL][4], ahh[M::P2][4];
-#pragma unroll
-    for (int q = 0; q < M::P2; ++q)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) alh[q][c] = ahh[q][c] = 0.f;
-#pragma unroll
-    for (int q = 0; q < NHL; ++q)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ahl[q][c] = 0.f;
-#pragma unroll 1
-    for (int kb = 0; kb < C / 8; ++kb) {
-        const int k0 = kb * 8;
-        uint32_t ah[4], al[4];
-        tf32_split(es[(r0 + g) * ES + k0 + t], ah[0], al[0]);
-        tf32_split(es[(r0 + g + 8) * ES + k0 + t], ah[1], al[1]);
-        tf32_split(es[(r0 + g) * ES + k0 + t + 4], ah[2], al[2]);
-        tf32_split(es[(r0 + g + 8) * ES + k0 + t + 4], ah[3], al[3]);
-#pragma unroll
-        for (int q = 0; q < M::P2; ++q) {
-            const int nt = wg + M::WG * q;
-            if (nt < M::NT2) {
-                const float b0 = kT[(nt * 8 + g) * ES + k0 + t], b1 = kT[(nt * 8 + g) * ES + k0 + t + 4];
-                if constexpr (K_EXACT) {
-                    const uint32_t b[2] = {__float_as_uint(b0), __float_as_uint(b1)};
-                    mma_tf32(alh[q], al, b);
-                    mma_tf32(ahh[q], ah, b);
-                } else {
-                    uint32_t bh[2], bl[2];
-                    tf32_split(b0, bh[0], bl[0]);
-                    tf32_split(b1, bh[1], bl[1]);
-                    mma_tf32(alh[q], al, bh);
-                    mma_tf32(ahl[q], ah, bl);
-                    mma_tf32(ahh[q], ah, bh);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < M::P2; ++q) {
-        const int nt = wg + M::WG * q;
-        if (nt < M::NT2) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float x = fadd(fmul(d0, Sreg[q][c]), alh[q][c]);
-                if constexpr (!K_EXACT) x = fadd(x, ahl[q][c]);
-                Sreg[q][c] = fadd(x, ahh[q][c]);
-            }
-#pragma unroll
-            for (int hrow = 0; hrow < 2; ++hrow) {
-                const int i = r0 + g + hrow * 8, j = nt * 8 + 2 * t;
-                const float2 x = make_float2(Sreg[q][2 * hrow], Sreg[q][2 * hrow + 1]);
-                *reinterpret_cast<float2*>(Ss + i * KS + j) = x;
-                if (dst1 != nullptr) *reinterpret_cast<float2*>(dst1 + (int64_t)i * DK + j) = x;
-                if (dst2 != nullptr) *reinterpret_cast<float2*>(dst2 + (int64_t)i * DK + j) = x;
-            }
-        }
-    }
-}
-
-template <int DK, int RTB, int C>
-__device__ __forceinline__ void mma_phase2(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* es,
-                                           const float* kT, float d0, int k_exact, float* dst1, float* dst2)
-{
-    if (k_exact) mma_phase2_t<DK, RTB, C, true>(Sreg, Ss, es, kT, d0, dst1, dst2);
-    else mma_phase2_t<DK, RTB, C, false>(Sreg, Ss, es, kT, d0, dst1, dst2);
-}
-
-// Load the RTB rows at src (global, row stride DK) into Ss and this lane's
-// phase-2 registers (warps 0..3).  Ends with a barrier.
-template <int DK, int RTB, int C>
-__device__ __forceinline__ void mma_load_state(float (&Sreg)[MmaAdv<DK, RTB, C>::P2][4], float* Ss, const float* src)
-{
-    using M = MmaAdv<DK, RTB, C>;
-    for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-        const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (src != nullptr) x = *reinterpret_cast<const float4*>(src + (int64_t)i * DK + j4);
-        *reinterpret_cast<float4*>(Ss + i * M::KS + j4) = x;
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    if (warp < 4) {
-        const int mt = warp % M::MT, wg = warp / M::MT, r0 = mt * 16;
-#pragma unroll
-        for (int q = 0; q < M::P2; ++q) {
-            const int nt = wg + M::WG * q;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                Sreg[q][c] = nt < M::NT2 ? Ss[(r0 + g + (c >> 1) * 8) * M::KS + nt * 8 + 2 * t + (c & 1)] : 0.f;
-        }
-    }
-}
-
-// k of C tokens (rows of a [T, H, DK] input from token tok0, head h) -> kT
-// [DK][ES] fp32 (transposed; token index fastest across threads, so the
-// scattered stores hit consecutive banks).
-template <int DK, int C>
-__device__ __forceinline__ void stage_kT(float* kT, const void* k, int64_t tok0, int H, int h, int bf16)
-{
-    constexpr int ES = C + 4;
-    for (int e = threadIdx.x; e < C * (DK / 8); e += blockDim.x) {
-        const int tau = e % C, j8 = (e / C) * 8;
-        float x[8];
-        load8(k, ((tok0 + tau) * H + h) * (int64_t)DK + j8, bf16, x);
-#pragma unroll
-        for (int m = 0; m < 8; ++m) kT[(j8 + m) * ES + tau] = x[m];
-    }
-}
-
 // P_chunk part 1 for every full chunk: one CTA per (full chunk, head).
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256)
@@ -551,126 +278,151 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
 
 template <int DK, int DV, int C>
 struct ChainSmem {
-    using Cf = ChunkCfg<DK, DV, C>;
-    using M = MmaAdv<DK, Cf::RTB, C>;
-    static constexpr int SS_OFF = 0;                              // [RTB][KS] fp32 S
-    static constexpr int WS_OFF = SS_OFF + Cf::RTB * M::KS;       // [C][KS] w
-    static constexpr int ES_OFF = WS_OFF + C * M::KS;             // [RTB][ES] e
-    static constexpr int KT_OFF = ES_OFF + Cf::RTB * M::ES;       // [DK][ES] k^T
-    static constexpr int US_OFF = KT_OFF + DK * M::ES;            // [C][RTB] u0 rows of the tile
-    static constexpr int DC_OFF = US_OFF + C * Cf::RTB;           // [C+4] D[C][.]
-    static constexpr size_t BYTES = sizeof(float) * (DC_OFF + Cf::DCS);
+    using T = TcCfg<DK, DV, C>;
+    static constexpr int WRS = DK + 4;                       // raw w row stride (conflict-free conversion reads)
+    static constexpr int WLO_OFF = 0;                        // canonical w lo | hi (adjacent)
+    static constexpr int WHI_OFF = WLO_OFF + T::W_FLOATS;
+    static constexpr int KLO_OFF = WHI_OFF + T::W_FLOATS;    // canonical k^T lo | hi (adjacent), then S' staging
+    static constexpr int KHI_OFF = KLO_OFF + T::K_FLOATS;
+    static constexpr int WRAW_OFF = KLO_OFF + T::K_REGION;   // [C][WRS] the next chunk's w, in flight
+    static constexpr int US_OFF = WRAW_OFF + C * WRS;        // [C][DV] u0
+    static constexpr int DC_OFF = US_OFF + C * DV;           // [C+4] D[C][.]
+    static constexpr int BAR_OFF = DC_OFF + ChunkCfg<DK, DV, C>::DCS;  // mbarrier (8 bytes) + TMEM base
+    // at least 120 KB, so that one CTA fits per SM: each allocates all 512 TMEM columns
+    static constexpr size_t USED = sizeof(float) * (BAR_OFF + 4);
+    static constexpr size_t BYTES = USED > 120 * 1024 ? USED : 120 * 1024;
+    static_assert(BYTES <= 232448, "fits the 227 KB of shared memory a CTA can have");
+    static_assert(BAR_OFF % 2 == 0 && WRAW_OFF % 4 == 0 && US_OFF % 4 == 0, "alignment");
 };
 
-// Boundary states: one CTA (4 warps) per (sequence, head, row tile), serial
-// over the sequence's full chunks; the tile's state stays in registers.
-// Writes chunk_states[so[n] + c] for c = 0..floor(L/C).  The next chunk's w,
-// u0 and decays arrive by cp.async during phase 2.
+// Boundary states: one CTA per (sequence, head), serial over the sequence's
+// full chunks, on the tensor cores (tcgen05; the state stays in TMEM and in
+// registers between chunks).  Writes chunk_states[so[n] + c] for
+// c = 0..floor(L/C).  Thread 0 issues the MMAs; while they run, warps 1..7
+// move data: during phase 1 they store the previous chunk's S' rows, write this
+// chunk's k^T (loaded into registers one chunk ahead) and start the next
+// chunk's w and k loads; during phase 2 they convert the next chunk's w into
+// the split operands and start its u0 and decay copies.  An MMA completion
+// wait that times out sets *err = 2 and ends the CTA; the kernels after it
+// then write nothing.
 template <int DK, int DV, int C>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256, 1)
 k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const int32_t* __restrict__ cu,
-        const int32_t* __restrict__ fco, const int32_t* __restrict__ so, const int32_t* __restrict__ err,
-        int N, int H, int in_bf16, const float* __restrict__ w_ws, const float* __restrict__ u_ws,
-        const float* __restrict__ dC_ws, float* __restrict__ states)
+        const int32_t* __restrict__ fco, const int32_t* __restrict__ so, int32_t* err, int N, int H, int in_bf16,
+        const float* __restrict__ w_ws, const float* __restrict__ u_ws, const float* __restrict__ dC_ws,
+        float* __restrict__ states)
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ChainSmem<DK, DV, C>;
-    using M = MmaAdv<DK, Cf::RTB, C>;
-    constexpr int KS = M::KS, RTB = Cf::RTB;
-    if (__ldg(err)) return;
+    using T = TcCfg<DK, DV, C>;
+    constexpr int NP = T::THREADS - 32;  // data-moving threads: warps 1..7
+    if (*reinterpret_cast<volatile int32_t*>(err)) return;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
-    float* Ss = sm + Sm::SS_OFF;
-    float* ws = sm + Sm::WS_OFF;
-    float* es = sm + Sm::ES_OFF;
-    float* kT = sm + Sm::KT_OFF;
+    float* Whi = sm + Sm::WHI_OFF;
+    float* Wlo = sm + Sm::WLO_OFF;
+    float* Khi = sm + Sm::KHI_OFF;
+    float* Klo = sm + Sm::KLO_OFF;
+    float* wraw = sm + Sm::WRAW_OFF;
     float* us = sm + Sm::US_OFF;
     float* dCs = sm + Sm::DC_OFF;
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Sm::BAR_OFF);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Sm::BAR_OFF + 2);
 
-    const int r = blockIdx.x % Cf::NTB;
-    const int nh = blockIdx.x / Cf::NTB;
+    const int nh = blockIdx.x;
     const int h = nh % H, n = nh / H;
     const int seq0 = __ldg(cu + n);
     const int nfull = (__ldg(cu + n + 1) - seq0) / C;
     const int64_t slot0 = __ldg(so + n);
     const int64_t g0 = __ldg(fco + n);
-    const int64_t row0 = (int64_t)r * RTB;
+    const bool mover = threadIdx.x >= 32;
+    const int pt = threadIdx.x - 32;  // index among the data-moving threads
+    auto state_dst = [&](int c) { return states + ((slot0 + c) * H + h) * (int64_t)DV * DK; };
+    auto movers_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NP) : "memory"); };
 
-    auto fetch = [&](int c) {
-        const int64_t task = (g0 + c) * H + h;
-        const float* wsrc = w_ws + task * C * DK;
-        for (int e = threadIdx.x; e < C * (DK / 4); e += blockDim.x) {
+    auto fetch_w = [&](int c, int tid, int nthr) {  // raw w of chunk c -> wraw
+        const float* src = w_ws + ((g0 + c) * H + h) * (int64_t)C * DK;
+        for (int e = tid; e < C * DK / 4; e += nthr) {
             const int t = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-            cp_async16(ws + t * KS + j4, wsrc + t * DK + j4);
+            cp_async16(wraw + t * Sm::WRS + j4, src + t * DK + j4);
         }
-        const float* usrc = u_ws + task * C * DV + row0;
-        for (int e = threadIdx.x; e < C * (RTB / 4); e += blockDim.x) {
-            const int t = e / (RTB / 4), i4 = (e % (RTB / 4)) * 4;
-            cp_async16(us + t * RTB + i4, usrc + t * DV + i4);
-        }
-        for (int e = threadIdx.x; e < Cf::DCS / 4; e += blockDim.x)
-            cp_async16(dCs + 4 * e, dC_ws + task * Cf::DCS + 4 * e);
+        cp_async_commit();
+    };
+    auto fetch_u = [&](int c, int tid, int nthr) {  // u0 and D[C][.] of chunk c
+        const int64_t task = (g0 + c) * H + h;
+        const float* usrc = u_ws + task * C * DV;
+        for (int e = tid; e < C * DV / 4; e += nthr) cp_async16(us + 4 * e, usrc + 4 * e);
+        for (int e = tid; e < Cf::DCS / 4; e += nthr) cp_async16(dCs + 4 * e, dC_ws + task * Cf::DCS + 4 * e);
         cp_async_commit();
     };
 
-    float Sreg[M::P2][4];
-    mma_load_state<DK, RTB, C>(Sreg, Ss,
-                               state_in != nullptr ? state_in + (((int64_t)n * H + h) * DV + row0) * DK : nullptr);
-    for (int e = threadIdx.x; e < RTB * (DK / 4); e += blockDim.x) {
-        const int i = e / (DK / 4), j4 = (e % (DK / 4)) * 4;
-        *reinterpret_cast<float4*>(states + ((slot0 * H + h) * DV + row0 + i) * DK + j4) =
-            *reinterpret_cast<const float4*>(Ss + i * KS + j4);
-    }
-    if (nfull > 0) {
-        fetch(0);
-        stage_kT<DK, C>(kT, k, (int64_t)seq0, H, h, in_bf16);
-    }
-    for (int c = 0; c < nfull; ++c) {
+    if (threadIdx.x == 0) mbar_init(mbar, 1);
+    if (threadIdx.x < 32) tmem_alloc(tslot, T::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tslot;
+    const TcThread<DK> th(tbase);
+
+    float SR[DK / 2];
+    tc_load_state<DK, DV, C>(SR, th, state_in != nullptr ? state_in + ((int64_t)n * H + h) * DV * DK : nullptr,
+                             state_dst(0));
+    if (nfull > 0) {  // chunk 0's operands, by every thread
+        fetch_w(0, threadIdx.x, T::THREADS);
+        fetch_u(0, threadIdx.x, T::THREADS);
+        tc_stage_kT<DK, DV, C>(k, (int64_t)seq0, H, h, in_bf16, Khi, Klo);
         cp_async_wait_all();
-        __syncthreads();  // w/u0/D and k of chunk c are in smem; Ss is current
-        mma_phase1<DK, RTB, C>(Ss, ws, us, RTB, dCs, es);
-        const float d0 = dCs[0];
-        __syncthreads();  // e complete; w, u0 and D may be overwritten
-        if (c + 1 < nfull) fetch(c + 1);
-        // bf16 inputs: the next chunk's k (raw 16-byte pieces) is loaded into
-        // registers now and written to smem after phase 2, so the load latency
-        // overlaps the tensor-core work
-        constexpr int ITEMS = C * (DK / 8), NPRE = (ITEMS + M::THREADS - 1) / M::THREADS;
-        uint4 kpre[NPRE];
-        const int64_t tok1 = (int64_t)seq0 + (int64_t)(c + 1) * C;
-        if (c + 1 < nfull && in_bf16) {
-#pragma unroll
-            for (int i = 0; i < NPRE; ++i) {
-                const int e = threadIdx.x + i * M::THREADS;
-                if (e < ITEMS) {
-                    const int tau = e % C, j8 = (e / C) * 8;
-                    kpre[i] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(k) +
-                                                                   ((tok1 + tau) * H + h) * (int64_t)DK + j8));
-                }
+        __syncthreads();
+        tc_stage_w<DK, DV, C>(wraw, Sm::WRS, Whi, Wlo, threadIdx.x, T::THREADS);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    KPrefetch<DK, DV, C, NP> kpre;
+    uint32_t parity = 0;
+    bool ok = true;
+    for (int c = 0; c < nfull; ++c) {
+        const bool more = c + 1 < nfull;
+        if (threadIdx.x == 0) tc_issue_phase1<DK, DV, C>(tbase, Wlo, mbar);
+        if (mover) {
+            if (c > 0) {
+                tc_store_rows<DK, DV>(Klo, state_dst(c), nullptr, pt, NP);  // S' of chunk c-1, staged in Klo
+                movers_sync();
+                kpre.store(Khi, Klo, in_bf16, pt);                            // k^T of chunk c
+                fence_async_smem();
             }
-        }
-        mma_phase2<DK, RTB, C>(Sreg, Ss, es, kT, d0, in_bf16,
-                               states + (((slot0 + c + 1) * H + h) * DV + row0) * DK, nullptr);
-        if (c + 1 < nfull) {
-            __syncthreads();  // phase 2 is done with k
-            if (in_bf16) {
-#pragma unroll
-                for (int i = 0; i < NPRE; ++i) {
-                    const int e = threadIdx.x + i * M::THREADS;
-                    if (e < ITEMS) {
-                        const int tau = e % C, j8 = (e / C) * 8;
-                        const uint32_t w4[4] = {kpre[i].x, kpre[i].y, kpre[i].z, kpre[i].w};
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            kT[(j8 + 2 * m) * M::ES + tau] = __uint_as_float(w4[m] << 16);
-                            kT[(j8 + 2 * m + 1) * M::ES + tau] = __uint_as_float(w4[m] & 0xffff0000u);
-                        }
-                    }
-                }
+            if (more) {
+                fetch_w(c + 1, pt, NP);
+                kpre.load(k, (int64_t)seq0 + (int64_t)(c + 1) * C, H, h, in_bf16, pt);
+                cp_async_wait_1();  // u0 and decays of chunk c (w of chunk c+1 may still be in flight)
             } else {
-                stage_kT<DK, C>(kT, k, tok1, H, h, in_bf16);
+                cp_async_wait_all();
             }
         }
+        ok = tc_wait(mbar, parity);
+        if (!ok) break;
+        const float d0 = tc_epilogue_e<DK, DV, C>(th, us, DV, dCs);
+        if (threadIdx.x == 0) tc_issue_phase2<DK, DV, C>(tbase, Klo, in_bf16, mbar);
+        if (mover && more) {  // phase 1 is done with w: the next chunk's w goes in while phase 2 runs
+            cp_async_wait_all();
+            movers_sync();
+            tc_stage_w<DK, DV, C>(wraw, Sm::WRS, Whi, Wlo, pt, NP);
+            fence_async_smem();
+            fetch_u(c + 1, pt, NP);
+        }
+        ok = tc_wait(mbar, parity);
+        if (!ok) break;
+        tc_epilogue_S<DK, DV, C>(SR, th, d0, in_bf16, Klo);
+    }
+    if (ok && nfull > 0 && mover) tc_store_rows<DK, DV>(Klo, state_dst(nfull), nullptr, pt, NP);
+    if (!ok && threadIdx.x == 0) atomicExch(err, 2);
+    cp_async_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        tc_fence_after();
+        tmem_dealloc(tbase, T::TMEM_COLS);
     }
 }
 
