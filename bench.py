@@ -436,6 +436,11 @@ def run_native(args):
         "decode": dec,
         "peaks": {"hbm_gbs": peaks.get("hbm_gbs"), "source": peak_src},
         "kernel_source_sha": sha,
+        "contract": {"id": gdn.gdn_contract_id(),
+                     "numerical_policy": gdn.gdn_contract_identity(gdn.ID_NUMERICAL_POLICY, D, D, C, gdn.GDN_BF16,
+                                                                   gdn.GDN_BF16),
+                     "deployment": gdn.gdn_contract_identity(gdn.ID_DEPLOYMENT, D, D, C, gdn.GDN_BF16,
+                                                             gdn.GDN_BF16)},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

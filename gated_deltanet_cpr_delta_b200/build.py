@@ -6,6 +6,7 @@
 """
 from __future__ import annotations
 
+import hashlib
 import os
 import shutil
 import subprocess
@@ -15,9 +16,21 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgdn_cpr.so")
-SOURCES = ["gdn_cpr.cu"]
-DEPS = ["gdn_cpr.cu", "kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_pchunk.cuh", "k_decode.cuh"]
+SOURCES = ["gdn_cpr.cu", "identity.cu"]
+DEPS = ["gdn_cpr.cu", "identity.cu", "kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_tc.cuh",
+        "k_pchunk.cuh", "k_decode.cuh"]
 HEADERS = [os.path.join(ROOT, "include", "gdn_cpr.h")]
+
+
+def sources_sha256() -> str:
+    """SHA-256 over the library's sources (file name, NUL, contents, in DEPS
+    order, then the public header): the deployment identity names it."""
+    h = hashlib.sha256()
+    for path in [os.path.join(CSRC, s) for s in DEPS] + HEADERS:
+        h.update(os.path.basename(path).encode() + b"\0")
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def nvcc_path() -> str:
@@ -33,7 +46,8 @@ def flags(verbose: bool = False):
          # the schedule's arithmetic is written with explicit _rn intrinsics;
          # these keep any other fp expression exact too
          "-fmad=false", "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
-         "-I", os.path.join(ROOT, "include"), "-I", CSRC]
+         "-I", os.path.join(ROOT, "include"), "-I", CSRC,
+         f'-DGDN_SOURCES_SHA256="{sources_sha256()}"']
     if verbose:
         f += ["-Xptxas", "-v"]
     return f

@@ -234,7 +234,7 @@ gdn_status_t launch_decode(const DecArgs& a)
 
 extern "C" {
 
-const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v2/NL8/chain-mma-tf32x3"; }
+const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v3/NL8/prep-mma-tf32x3/chain-tcgen05-tf32x3"; }
 
 const char* gdn_status_string(gdn_status_t s)
 {

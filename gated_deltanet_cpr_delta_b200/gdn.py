@@ -24,7 +24,10 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 #: exported symbols of include/gdn_cpr.h
 SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
            "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed",
-           "gdn_cpr_forward_noalloc")
+           "gdn_cpr_forward_noalloc", "gdn_contract_text", "gdn_contract_identity", "gdn_sha256_hex")
+
+#: gdn_identity_kind_t
+ID_SEMANTIC, ID_NUMERICAL_POLICY, ID_DEPLOYMENT = 0, 1, 2
 
 #: size of the fixed device array behind gdn_cpr_forward_noalloc (GDN_NOALLOC_SCRATCH_BYTES)
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -56,6 +59,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     lib.gdn_contract_id.restype = ctypes.c_char_p
     lib.gdn_contract_id.argtypes = []
+    lib.gdn_contract_text.restype = i64
+    lib.gdn_contract_text.argtypes = [ctypes.c_int, i32, i32, i32, ctypes.c_int, ctypes.c_int, ctypes.c_char_p, sz]
+    lib.gdn_contract_identity.restype = ctypes.c_int
+    lib.gdn_contract_identity.argtypes = [ctypes.c_int, i32, i32, i32, ctypes.c_int, ctypes.c_int, ctypes.c_char_p]
+    lib.gdn_sha256_hex.restype = ctypes.c_int
+    lib.gdn_sha256_hex.argtypes = [ctypes.c_void_p, sz, ctypes.c_char_p]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_status_string.argtypes = [ctypes.c_int]
     lib.gdn_num_chunk_states.restype = i64
@@ -117,6 +126,29 @@ def _check(st: int, what: str):
 
 def gdn_contract_id() -> str:
     return load_library().gdn_contract_id().decode()
+
+
+def gdn_contract_text(kind: int, d_k: int, d_v: int, C: int, in_dtype: int, out_dtype: int) -> str:
+    lib = load_library()
+    n = lib.gdn_contract_text(kind, d_k, d_v, C, in_dtype, out_dtype, None, 0)
+    if n < 0:
+        raise GdnError(1, "gdn_contract_text")
+    buf = ctypes.create_string_buffer(n + 1)
+    lib.gdn_contract_text(kind, d_k, d_v, C, in_dtype, out_dtype, buf, n + 1)
+    return buf.value.decode()
+
+
+def gdn_contract_identity(kind: int, d_k: int, d_v: int, C: int, in_dtype: int, out_dtype: int) -> str:
+    out = ctypes.create_string_buffer(65)
+    _check(load_library().gdn_contract_identity(kind, d_k, d_v, C, in_dtype, out_dtype, out), "gdn_contract_identity")
+    return out.value.decode()
+
+
+def gdn_sha256_hex(data: bytes) -> str:
+    out = ctypes.create_string_buffer(65)
+    buf = ctypes.create_string_buffer(bytes(data), len(data))
+    _check(load_library().gdn_sha256_hex(buf, len(data), out), "gdn_sha256_hex")
+    return out.value.decode()
 
 
 def gdn_num_chunk_states(cu_seqlens_host: Sequence[int], C: int) -> int:

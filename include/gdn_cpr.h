@@ -87,6 +87,48 @@ typedef struct {
 /* Name of the arithmetic schedule every kernel executes (static string). */
 const char* gdn_contract_id(void);
 
+/*
+ * Contract identities.  Runtimes that must give the same bits compare SHA-256
+ * identities of the contract they execute, in three parts (IsoExec summary
+ * page, "Contract Structure and Enforcement", Identities; commentary blog,
+ * section 6):
+ *   GDN_ID_SEMANTIC          what the layer computes: the recurrence, the CPR
+ *                            composition, layouts, shapes and dtypes;
+ *   GDN_ID_NUMERICAL_POLICY  how: the fp32 rules, the reduction tree, the
+ *                            operation order, the split products and the
+ *                            instruction shapes of every step (it names
+ *                            gdn_contract_id());
+ *   GDN_ID_DEPLOYMENT        which build: target, a SHA-256 of the kernel
+ *                            sources, the compiler version.
+ * Two runtimes with equal semantic and numerical-policy identities for the
+ * same (d_k, d_v, C, dtypes) produce bit-identical results.
+ */
+typedef enum {
+    GDN_ID_SEMANTIC = 0,
+    GDN_ID_NUMERICAL_POLICY = 1,
+    GDN_ID_DEPLOYMENT = 2
+} gdn_identity_kind_t;
+
+/*
+ * The canonical text an identity digests.  Writes at most cap bytes
+ * (NUL-terminated, truncated if cap is too small) and returns the full length
+ * without the NUL, or -1 for an unsupported shape, a bad kind, or buf == NULL
+ * with cap != 0.  gdn_contract_text(kind, ..., NULL, 0) returns the length.
+ */
+int64_t gdn_contract_text(gdn_identity_kind_t kind, int32_t d_k, int32_t d_v, int32_t C,
+                          gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, char* buf, size_t cap);
+
+/*
+ * SHA-256 of gdn_contract_text as 64 lowercase hex digits plus NUL into
+ * out_hex (65 bytes, host memory).  GDN_ERR_UNSUPPORTED for a shape or dtype
+ * that is not compiled in; GDN_ERR_INVALID_ARG for out_hex == NULL or a bad kind.
+ */
+gdn_status_t gdn_contract_identity(gdn_identity_kind_t kind, int32_t d_k, int32_t d_v, int32_t C,
+                                   gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, char* out_hex);
+
+/* SHA-256 (FIPS 180-4) of n bytes of host memory as 64 hex digits plus NUL. */
+gdn_status_t gdn_sha256_hex(const void* data, size_t n, char* out_hex);
+
 /* Human-readable text for a status code (static string). */
 const char* gdn_status_string(gdn_status_t status);
 
