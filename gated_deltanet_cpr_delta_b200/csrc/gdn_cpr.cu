@@ -33,7 +33,7 @@ bool supported(int32_t dk, int32_t dv, int32_t C)
 bool dtype_ok(gdn_dtype_t t) { return t == GDN_F32 || t == GDN_BF16; }
 
 struct SeqTotals {
-    int64_t tasks = 0, full = 0, states = 0;
+    int64_t tasks = 0, full = 0, states = 0, maxc = 0;  // maxc: most chunk tasks of one sequence
     uint64_t hash = 0;  // gdn::cu_entry_hash summed over the host copy
 };
 
@@ -49,6 +49,7 @@ bool seq_totals(const int32_t* cu, int32_t N, int64_t T_total, int32_t C, SeqTot
         t.tasks += (L + C - 1) / C;
         t.full += L / C;
         t.states += L / C + 1;
+        t.maxc = std::max<int64_t>(t.maxc, (L + C - 1) / C);
         t.hash += gdn::cu_entry_hash(n, cu[n]);
     }
     t.hash += gdn::cu_entry_hash(N, cu[N]);
@@ -57,12 +58,18 @@ bool seq_totals(const int32_t* cu, int32_t N, int64_t T_total, int32_t C, SeqTot
     return true;
 }
 
-// Workspace layout: [err | cto | fco | so | w | u0 | dC], each 256-byte aligned.
+// Workspace layout: [err | cto | fco | so | order | cumc | progress | w | u0 | dC],
+// each 256-byte aligned (order, cumc and progress serve the fused chain + P_tok
+// kernel; tok_next shares the error word's 16 bytes).
 struct Workspace {
     int32_t* err;
+    int32_t* tok_next;
     int32_t* cto;
     int32_t* fco;
     int32_t* so;
+    int32_t* order;
+    int32_t* cumc;
+    int32_t* progress;
     float* w;
     float* u;
     float* dC;
@@ -82,6 +89,9 @@ Workspace carve(void* base, int64_t max_full, int32_t N, int32_t H, int32_t dk, 
     const size_t o_cto = take(sizeof(int32_t) * (size_t)(N + 1));
     const size_t o_fco = take(sizeof(int32_t) * (size_t)(N + 1));
     const size_t o_so = take(sizeof(int32_t) * (size_t)(N + 1));
+    const size_t o_ord = take(sizeof(int32_t) * (size_t)(N + 1));
+    const size_t o_cumc = take(sizeof(int32_t) * (size_t)(max_full + 2));  // maxc <= ceil(T / C)
+    const size_t o_prog = take(sizeof(int32_t) * (size_t)N * H);
     const size_t o_w = take(sizeof(float) * (size_t)max_full * H * C * dk);
     const size_t o_u = take(sizeof(float) * (size_t)max_full * H * C * dv);
     const size_t o_dc = take(sizeof(float) * (size_t)max_full * H * (C + 4));
@@ -92,6 +102,10 @@ Workspace carve(void* base, int64_t max_full, int32_t N, int32_t H, int32_t dk, 
         ws.cto = reinterpret_cast<int32_t*>(b + o_cto);
         ws.fco = reinterpret_cast<int32_t*>(b + o_fco);
         ws.so = reinterpret_cast<int32_t*>(b + o_so);
+        ws.tok_next = reinterpret_cast<int32_t*>(b + o_err + 4);
+        ws.order = reinterpret_cast<int32_t*>(b + o_ord);
+        ws.cumc = reinterpret_cast<int32_t*>(b + o_cumc);
+        ws.progress = reinterpret_cast<int32_t*>(b + o_prog);
         ws.w = reinterpret_cast<float*>(b + o_w);
         ws.u = reinterpret_cast<float*>(b + o_u);
         ws.dC = reinterpret_cast<float*>(b + o_dc);
@@ -132,9 +146,27 @@ gdn_status_t launch_forward(const FwdArgs& a)
     using Cf = ChunkCfg<D, D, C>;
     using TC = gdn::TokCfg<D, D, C>;
     cudaError_t e = cudaSuccess;
+    // Few (sequence, head) pairs leave most SMs idle during the serial chain:
+    // then the chain and P_tok run as one cooperative kernel (one CTA per SM),
+    // the P_tok tasks filling the SMs the chains do not use.
+    const int npairs = a.N * a.H;
+    int dev = 0, sms = 0, per_sm = 0;
+    constexpr size_t fsm = gdn::FusedSmem<D, D, C>::BYTES;
+    bool fused = false;
+    if constexpr (gdn::FusedSmem<D, D, C>::OK) {
+        if (a.tot.tasks > 0 && cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            npairs + 16 <= sms && set_smem(gdn::k_chain_tok<D, D, C>, fsm) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gdn::k_chain_tok<D, D, C>, 256, fsm) ==
+                cudaSuccess &&
+            per_sm >= 1)
+            fused = true;
+    }
     mark(a.events, 0, a.stream);
     gdn::k_tables<<<1, 1024, 0, a.stream>>>(a.cu, a.N, C, a.T_total, a.tot.tasks, a.tot.full, a.tot.states,
-                                             a.tot.hash, a.ws.cto, a.ws.fco, a.ws.so, a.ws.err);
+                                             a.tot.hash, a.ws.cto, a.ws.fco, a.ws.so, a.ws.err,
+                                             fused ? a.ws.order : nullptr, a.ws.cumc, (int)a.tot.maxc,
+                                             a.ws.progress, a.ws.tok_next, npairs);
     if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     if (a.tot.full > 0) {
@@ -145,7 +177,25 @@ gdn_status_t launch_forward(const FwdArgs& a)
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 2, a.stream);
-    if (a.N > 0) {
+    if constexpr (gdn::FusedSmem<D, D, C>::OK) if (fused) {
+        mark(a.events, 3, a.stream);  // the chain has no separate time: it runs inside the next kernel
+        const void *q = a.q, *k = a.k, *v = a.v;
+        const float *alpha = a.alpha, *beta = a.beta, *state_in = a.state_in;
+        const int32_t *cu = a.cu, *fco = a.ws.fco, *so = a.ws.so, *order = a.ws.order, *cumc = a.ws.cumc;
+        int32_t *err = a.ws.err, *progress = a.ws.progress, *tok_next = a.ws.tok_next;
+        int N = a.N, H = a.H, in_bf16 = a.in_bf16, out_bf16 = a.out_bf16, maxc = (int)a.tot.maxc;
+        const float *w = a.ws.w, *u = a.ws.u, *dC = a.ws.dC;
+        float* states = a.states;
+        void* o = a.o;
+        float* cacheR = a.cache ? a.cache->R : nullptr;
+        void* args[] = {&q, &k, &v, &alpha, &beta, &state_in, &cu, &fco, &so, &err, &N, &H, &in_bf16, &out_bf16,
+                        &w, &u, &dC, &states, &o, &cacheR, &progress, &tok_next, &order, &cumc, &maxc};
+        if (cudaLaunchCooperativeKernel((const void*)gdn::k_chain_tok<D, D, C>, dim3((unsigned)sms), dim3(256), args,
+                                        fsm, a.stream) != cudaSuccess ||
+            cudaGetLastError() != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    if (!fused && a.N > 0) {
         constexpr size_t sm = gdn::ChainSmem<D, D, C>::BYTES;
         if (set_smem(gdn::k_chain<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
         gdn::k_chain<D, D, C><<<(unsigned)((int64_t)a.N * a.H), gdn::TcCfg<D, D, C>::THREADS, sm, a.stream>>>(
@@ -153,8 +203,8 @@ gdn_status_t launch_forward(const FwdArgs& a)
             a.states);
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     }
-    mark(a.events, 3, a.stream);
-    if (a.tot.tasks > 0) {
+    if (!fused) mark(a.events, 3, a.stream);
+    if (!fused && a.tot.tasks > 0) {
         constexpr size_t sm = TC::SMEM;
         if (set_smem(gdn::k_tok<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
         gdn::k_tok<D, D, C><<<(unsigned)(a.tot.tasks * a.H), TC::THREADS, sm, a.stream>>>(

@@ -305,20 +305,22 @@ struct ChainSmem {
 // the split operands and start its u0 and decay copies.  An MMA completion
 // wait that times out sets *err = 2 and ends the CTA; the kernels after it
 // then write nothing.
+//
+// progress (when non-null) publishes, for the pair, how many of its chunk
+// states are in global memory: after state c is written (and fenced),
+// progress[nh] = c + 1, with release semantics.
 template <int DK, int DV, int C>
-__global__ void __launch_bounds__(256, 1)
-k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const int32_t* __restrict__ cu,
-        const int32_t* __restrict__ fco, const int32_t* __restrict__ so, int32_t* err, int N, int H, int in_bf16,
-        const float* __restrict__ w_ws, const float* __restrict__ u_ws, const float* __restrict__ dC_ws,
-        float* __restrict__ states)
+__device__ __forceinline__ void chain_run(const void* __restrict__ k, const float* __restrict__ state_in,
+                                          const int32_t* __restrict__ cu, const int32_t* __restrict__ fco,
+                                          const int32_t* __restrict__ so, int32_t* err, int H, int in_bf16,
+                                          const float* __restrict__ w_ws, const float* __restrict__ u_ws,
+                                          const float* __restrict__ dC_ws, float* states, int nh,
+                                          int32_t* progress, float* sm)
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ChainSmem<DK, DV, C>;
     using T = TcCfg<DK, DV, C>;
     constexpr int NP = T::THREADS - 32;  // data-moving threads: warps 1..7
-    if (*reinterpret_cast<volatile int32_t*>(err)) return;
-    extern __shared__ float4 smem_f4[];
-    float* sm = reinterpret_cast<float*>(smem_f4);
     float* Whi = sm + Sm::WHI_OFF;
     float* Wlo = sm + Sm::WLO_OFF;
     float* Khi = sm + Sm::KHI_OFF;
@@ -329,7 +331,6 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
     uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Sm::BAR_OFF);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Sm::BAR_OFF + 2);
 
-    const int nh = blockIdx.x;
     const int h = nh % H, n = nh / H;
     const int seq0 = __ldg(cu + n);
     const int nfull = (__ldg(cu + n + 1) - seq0) / C;
@@ -339,6 +340,9 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
     const int pt = threadIdx.x - 32;  // index among the data-moving threads
     auto state_dst = [&](int c) { return states + ((slot0 + c) * H + h) * (int64_t)DV * DK; };
     auto movers_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NP) : "memory"); };
+    auto publish = [&](int count) {  // after a fence and a barrier over the writers
+        if (progress != nullptr) st_release_gpu(progress + nh, count);
+    };
 
     auto fetch_w = [&](int c, int tid, int nthr) {  // raw w of chunk c -> wraw
         const float* src = w_ws + ((g0 + c) * H + h) * (int64_t)C * DK;
@@ -375,9 +379,11 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
         __syncthreads();
         tc_stage_w<DK, DV, C>(wraw, Sm::WRS, Whi, Wlo, threadIdx.x, T::THREADS);
     }
+    __threadfence();  // state 0 (written by every thread above) is visible ...
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) publish(1);  // ... before it is published
 
     KPrefetch<DK, DV, C, NP> kpre;
     uint32_t parity = 0;
@@ -388,7 +394,9 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
         if (mover) {
             if (c > 0) {
                 tc_store_rows<DK, DV>(Klo, state_dst(c), nullptr, pt, NP);  // S' of chunk c-1, staged in Klo
+                __threadfence();
                 movers_sync();
+                if (pt == 0) publish(c + 1);
                 kpre.store(Khi, Klo, in_bf16, pt);                            // k^T of chunk c
                 fence_async_smem();
             }
@@ -415,14 +423,100 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
         if (!ok) break;
         tc_epilogue_S<DK, DV, C>(SR, th, d0, in_bf16, Klo);
     }
-    if (ok && nfull > 0 && mover) tc_store_rows<DK, DV>(Klo, state_dst(nfull), nullptr, pt, NP);
+    if (ok && nfull > 0 && mover) {
+        tc_store_rows<DK, DV>(Klo, state_dst(nfull), nullptr, pt, NP);
+        __threadfence();
+    }
     if (!ok && threadIdx.x == 0) atomicExch(err, 2);
     cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
+    if (ok && nfull > 0 && threadIdx.x == 0) publish(nfull + 1);
     if (threadIdx.x < 32) {
         tc_fence_after();
         tmem_dealloc(tbase, T::TMEM_COLS);
+    }
+}
+
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256, 1)
+k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const int32_t* __restrict__ cu,
+        const int32_t* __restrict__ fco, const int32_t* __restrict__ so, int32_t* err, int N, int H, int in_bf16,
+        const float* __restrict__ w_ws, const float* __restrict__ u_ws, const float* __restrict__ dC_ws,
+        float* __restrict__ states)
+{
+    if (*reinterpret_cast<volatile int32_t*>(err)) return;
+    extern __shared__ float4 smem_f4[];
+    chain_run<DK, DV, C>(k, state_in, cu, fco, so, err, H, in_bf16, w_ws, u_ws, dC_ws, states, blockIdx.x, nullptr,
+                         reinterpret_cast<float*>(smem_f4));
+}
+
+// ------------------------------------------------------------------ fused chain + P_tok
+template <int DK, int DV, int C>
+struct FusedSmem {
+    static constexpr size_t TOK = ((TokCfg<DK, DV, C>::SMEM + 15) / 16) * 16;  // one P_tok task
+    static constexpr size_t BYTES = ChainSmem<DK, DV, C>::BYTES > 2 * TOK ? ChainSmem<DK, DV, C>::BYTES : 2 * TOK;
+    static constexpr bool OK = TokCfg<DK, DV, C>::THREADS == 128;  // two P_tok tasks per 256-thread CTA
+};
+
+// Boundary chain and intra-chunk recurrence in one cooperative launch, for
+// batches with fewer (sequence, head) pairs than SMs.  CTA b < N*H runs the
+// chain of pair b (publishing progress[b] as its states land), then joins the
+// others as a P_tok worker.  Workers take P_tok tasks from one queue in
+// chunk-major order (task t -> chunk c with cumc[c] <= t < cumc[c+1],
+// sequence order[t - cumc[c]], the sequences sorted by chunk count), two
+// tasks per CTA at a time (one per 128-thread half), each after its boundary
+// state is published.  Every CTA is resident (cooperative launch), and chains
+// wait on nothing, so every wait ends; a wait that exceeds ~1 s sets *err = 3.
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256, 1)
+k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+            const float* __restrict__ alpha, const float* __restrict__ beta, const float* __restrict__ state_in,
+            const int32_t* __restrict__ cu, const int32_t* __restrict__ fco, const int32_t* __restrict__ so,
+            int32_t* err, int N, int H, int in_bf16, int out_bf16, const float* __restrict__ w_ws,
+            const float* __restrict__ u_ws, const float* __restrict__ dC_ws, float* states, void* __restrict__ o,
+            float* __restrict__ cacheR, int32_t* progress, int32_t* tok_next, const int32_t* __restrict__ order,
+            const int32_t* __restrict__ cumc, int maxc)
+{
+    using Fs = FusedSmem<DK, DV, C>;
+    static_assert(Fs::OK, "d_v = 128: two 128-thread P_tok tasks per CTA");
+    volatile int32_t* verr = err;
+    if (*verr) return;
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    if ((int)blockIdx.x < N * H) {
+        chain_run<DK, DV, C>(k, state_in, cu, fco, so, err, H, in_bf16, w_ws, u_ws, dC_ws, states, blockIdx.x,
+                             progress, sm);
+        __syncthreads();
+    }
+    const int half = threadIdx.x >> 7, tid = threadIdx.x & 127;
+    float* tsm = sm + half * (Fs::TOK / 4);
+    const HalfSync hs{2 + half};
+    __shared__ int qslot[2], go[2];
+    const int ntask = __ldg(cumc + maxc);
+    for (;;) {
+        if (tid == 0) qslot[half] = atomicAdd(tok_next, 1);
+        hs();
+        const int qi = qslot[half];
+        if (qi >= ntask * H) break;
+        const int t = qi / H, h = qi % H;
+        int lo = 0, hi = maxc;  // cumc[0] = 0 <= t < cumc[maxc]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(cumc + mid) <= t) lo = mid; else hi = mid;
+        }
+        const int c = lo, n = __ldg(order + t - __ldg(cumc + c));
+        if (tid == 0) {  // one thread waits and decides for the half
+            const bool ready = wait_at_least(progress + (int64_t)n * H + h, c + 1);
+            if (!ready) atomicExch(err, 3);
+            __threadfence();
+            go[half] = ready && *verr == 0;
+        }
+        hs();
+        if (!go[half]) break;
+        const int seq0 = __ldg(cu + n);
+        tok_task<DK, DV, C, true>(q, k, v, alpha, beta, n, c, h, H, seq0, __ldg(cu + n + 1) - seq0,
+                                  (int64_t)__ldg(so + n) + c, in_bf16, out_bf16, states, o, cacheR, tsm, tid, hs);
     }
 }
 

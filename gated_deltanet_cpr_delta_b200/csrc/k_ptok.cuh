@@ -212,21 +212,31 @@ __device__ __forceinline__ void lds8_raw(const unsigned char* base, int el, int 
     }
 }
 
-// Intra-chunk recurrence: one CTA per (chunk task, head).
-template <int DK, int DV, int C>
-__global__ void __launch_bounds__(TokCfg<DK, DV, C>::THREADS)
-k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
-      const float* __restrict__ alpha, const float* __restrict__ beta,
-      const int32_t* __restrict__ cu, const int32_t* __restrict__ cto, const int32_t* __restrict__ so,
-      const int32_t* __restrict__ err, int N, int H, int in_bf16, int out_bf16,
-      const float* __restrict__ states, void* __restrict__ o, float* __restrict__ cacheR)
+// Barriers for a P_tok task: the whole CTA, or one 128-thread half of a
+// larger CTA (named barrier `id`).
+struct CtaSync {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct HalfSync {
+    int id;
+    __device__ __forceinline__ void operator()() const { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+};
+
+// Intra-chunk recurrence for chunk c of sequence n (tokens seq0 + cC ..), head
+// h, by TokCfg::THREADS threads (tid = 0..THREADS-1) with smem `sm` of
+// TokCfg::SMEM bytes.  The chunk starts from states[slot] (COHERENT: read
+// through L2, for states written earlier in the same launch).
+template <int DK, int DV, int C, bool COHERENT, typename Sync>
+__device__ __forceinline__ void tok_task(const void* __restrict__ q, const void* __restrict__ k,
+                                         const void* __restrict__ v, const float* __restrict__ alpha,
+                                         const float* __restrict__ beta, int n, int c, int h, int H, int seq0, int Ln,
+                                         int64_t slot, int in_bf16, int out_bf16, const float* states,
+                                         void* __restrict__ o, float* __restrict__ cacheR, float* sm, int tid,
+                                         Sync sync)
 {
     using Cf = TokCfg<DK, DV, C>;
     using RS = typename Cf::RS;
-    constexpr int RHO = Cf::RHO, SC = Cf::SC, L = RS::L, KS = RS::KS;
-    if (__ldg(err)) return;
-    extern __shared__ float4 smem_f4[];
-    float* sm = reinterpret_cast<float*>(smem_f4);
+    constexpr int RHO = Cf::RHO, SC = Cf::SC, L = RS::L, KS = RS::KS, NT = Cf::THREADS;
     float* kq = sm + Cf::KQ_OFF;
     float* vs = sm + Cf::VS_OFF;
     float* os = sm + Cf::OS_OFF;
@@ -234,22 +244,15 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
     float* rab = sm + Cf::RAB_OFF;
     unsigned char* raw = reinterpret_cast<unsigned char*>(sm + Cf::RAW_OFF);
 
-    const int h = blockIdx.x % H;
-    const int g = blockIdx.x / H;
-    const int n = find_seq(cto, N, g);
-    const int c = g - __ldg(cto + n);
-    const int seq0 = __ldg(cu + n);
-    const int Ln = __ldg(cu + n + 1) - seq0;
     const int64_t tok0 = (int64_t)seq0 + (int64_t)c * C;
     const int len = min(C, Ln - c * C);
-    const int64_t slot = (int64_t)__ldg(so + n) + c;
     const int esz = in_bf16 ? 2 : 4;
     const int kb = DK * esz, vb = DV * esz, tb = 2 * kb + vb;  // bytes per k/q row, v row, token
 
     // async copies of sub-chunk s: raw token rows [k | q | v] and the gates
     auto fetch = [&](int s) {
         const int t0 = s * SC, ls = min(SC, len - t0), pieces = tb / 16;
-        for (int e = threadIdx.x; e < ls * pieces; e += blockDim.x) {
+        for (int e = tid; e < ls * pieces; e += NT) {
             const int t = e / pieces, off = (e % pieces) * 16;
             const int64_t row = (tok0 + t0 + t) * H + h;
             const char* src = off < kb ? reinterpret_cast<const char*>(k) + row * kb + off
@@ -257,7 +260,7 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
                                            : reinterpret_cast<const char*>(v) + row * vb + (off - 2 * kb);
             cp_async16(raw + t * Cf::RAW_TOK + off, src);
         }
-        for (int t = threadIdx.x; t < ls; t += blockDim.x) {
+        for (int t = tid; t < ls; t += NT) {
             cp_async4(rab + t, alpha + (tok0 + t0 + t) * H + h);
             cp_async4(rab + SC + t, beta + (tok0 + t0 + t) * H + h);
         }
@@ -266,7 +269,7 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
     // raw sub-chunk -> fp32: k, q in the slot layout, v by row, gates
     auto widen = [&](int ls) {
         constexpr int G8 = (2 * DK + DV) / 8;
-        for (int e = threadIdx.x; e < ls * G8; e += blockDim.x) {
+        for (int e = tid; e < ls * G8; e += NT) {
             const int t = e / G8, el = (e % G8) * 8;
             float x[8];
             lds8_raw(raw + t * Cf::RAW_TOK, el, in_bf16, x);
@@ -280,27 +283,40 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
                 for (int m = 0; m < 8; ++m) vs[t * DV + (el - 2 * DK) + m] = x[m];
             }
         }
-        for (int t = threadIdx.x; t < ls; t += blockDim.x) {
+        for (int t = tid; t < ls; t += NT) {
             ab[t] = rab[t];
             ab[SC + t] = rab[SC + t];
         }
     };
 
-    const int gi = threadIdx.x / RS::TPR, p = threadIdx.x % RS::TPR;
+    const int gi = tid / RS::TPR, p = tid % RS::TPR;
     const int row0 = gi * RHO;
     f2x Rp[RHO][L];
 #pragma unroll
-    for (int r = 0; r < RHO; ++r)
-        load_row_pairs<DK>(Rp[r], states + ((slot * H + h) * DV + row0 + r) * DK + p * RS::EPT);
+    for (int r = 0; r < RHO; ++r) {
+        const float* src = states + ((slot * H + h) * DV + row0 + r) * DK + p * RS::EPT;
+        if (COHERENT) {
+            float t[RS::EPT];
+#pragma unroll
+            for (int e = 0; e < RS::EPT; e += 4) {
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(src + e));
+                t[e] = x.x; t[e + 1] = x.y; t[e + 2] = x.z; t[e + 3] = x.w;
+            }
+#pragma unroll
+            for (int m = 0; m < L; ++m) Rp[r][m] = pk2(t[m], t[L + m]);
+        } else {
+            load_row_pairs<DK>(Rp[r], src);
+        }
+    }
 
     const int nsub = (len + SC - 1) / SC;
     fetch(0);
     for (int s = 0; s < nsub; ++s) {
         const int ls = min(SC, len - s * SC);
         cp_async_wait_all();
-        __syncthreads();  // raw(s) landed; the previous sub-chunk's outputs are stored
+        sync();  // raw(s) landed; the previous sub-chunk's outputs are stored
         widen(ls);
-        __syncthreads();  // fp32 buffers ready; raw is free again
+        sync();  // fp32 buffers ready; raw is free again
         if (s + 1 < nsub) fetch(s + 1);
         for (int t = 0; t < ls; ++t) {
             float vv[RHO], oo[RHO];
@@ -313,8 +329,8 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
                 for (int r = 0; r < RHO; ++r) os[t * DV + row0 + r] = oo[r];
             }
         }
-        __syncthreads();
-        for (int e = threadIdx.x; e < ls * (DV / 8); e += blockDim.x) {
+        sync();
+        for (int e = tid; e < ls * (DV / 8); e += NT) {
             const int t = e / (DV / 8), i8 = (e % (DV / 8)) * 8;
             store8(o, ((tok0 + s * SC + t) * H + h) * (int64_t)DV + i8, out_bf16, os + t * DV + i8);
         }
@@ -325,6 +341,28 @@ k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __rest
         for (int r = 0; r < RHO; ++r)
             store_row_pairs<DK>(cacheR + (((int64_t)n * H + h) * DV + row0 + r) * DK + p * RS::EPT, Rp[r]);
     }
+    sync();  // smem free for the next task
+}
+
+// Intra-chunk recurrence: one CTA per (chunk task, head).
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(TokCfg<DK, DV, C>::THREADS)
+k_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+      const float* __restrict__ alpha, const float* __restrict__ beta,
+      const int32_t* __restrict__ cu, const int32_t* __restrict__ cto, const int32_t* __restrict__ so,
+      const int32_t* __restrict__ err, int N, int H, int in_bf16, int out_bf16,
+      const float* __restrict__ states, void* __restrict__ o, float* __restrict__ cacheR)
+{
+    if (__ldg(err)) return;
+    extern __shared__ float4 smem_f4[];
+    const int h = blockIdx.x % H;
+    const int g = blockIdx.x / H;
+    const int n = find_seq(cto, N, g);
+    const int c = g - __ldg(cto + n);
+    const int seq0 = __ldg(cu + n);
+    tok_task<DK, DV, C, false>(q, k, v, alpha, beta, n, c, h, H, seq0, __ldg(cu + n + 1) - seq0,
+                               (int64_t)__ldg(so + n) + c, in_bf16, out_bf16, states, o, cacheR,
+                               reinterpret_cast<float*>(smem_f4), threadIdx.x, CtaSync{});
 }
 
 }  // namespace gdn

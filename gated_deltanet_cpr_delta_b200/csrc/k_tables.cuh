@@ -25,9 +25,15 @@ __host__ __device__ inline uint64_t cu_entry_hash(int n, int32_t value)
 // and the totals at index N.  err[0] = 1 if the device cu_seqlens is invalid
 // or disagrees with the host copy (totals or hash); every later kernel then
 // exits without writing.
+// With order != NULL, also the tables of the fused chain + P_tok kernel
+// (nt_n = ceil(L_n/C) chunk tasks of sequence n, maxc = max nt_n):
+//   order[r]  sequences by nt_n descending (ties by n)
+//   cumc[c]   = sum_n min(nt_n, c), c = 0..maxc (the chunk-major task offsets)
+//   progress[0..npairs) = 0 and *tok_next = 0.
 __global__ void k_tables(const int32_t* __restrict__ cu, int N, int C, int64_t T_total,
                          int64_t want_tasks, int64_t want_full, int64_t want_states, uint64_t want_hash,
-                         int32_t* cto, int32_t* fco, int32_t* so, int32_t* err)
+                         int32_t* cto, int32_t* fco, int32_t* so, int32_t* err, int32_t* order, int32_t* cumc,
+                         int maxc, int32_t* progress, int32_t* tok_next, int npairs)
 {
     __shared__ long long wsum[3][32];
     __shared__ long long tot[3];
@@ -88,6 +94,25 @@ __global__ void k_tables(const int32_t* __restrict__ cu, int N, int C, int64_t T
                         tot[0] == want_tasks && tot[1] == want_full && tot[2] == want_states &&
                         hsum == want_hash;
         err[0] = ok ? 0 : 1;
+    }
+    if (order != nullptr) {
+        auto nt = [&](int m) { return (max(0, cu[m + 1] - cu[m]) + C - 1) / C; };
+        for (int n = tid; n < N; n += nth) {
+            const int a = nt(n);
+            int rank = 0;
+            for (int m = 0; m < N; ++m) {
+                const int b = nt(m);
+                rank += (b > a || (b == a && m < n)) ? 1 : 0;
+            }
+            order[rank] = n;
+        }
+        for (int c = tid; c <= maxc; c += nth) {
+            int sum = 0;
+            for (int m = 0; m < N; ++m) sum += min(nt(m), c);
+            cumc[c] = sum;
+        }
+        for (int i = tid; i < npairs; i += nth) progress[i] = 0;
+        if (tid == 0) *tok_next = 0;
     }
 }
 

@@ -176,6 +176,28 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+// Release store / bounded acquire wait on a global int (cross-CTA progress).
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v)
+{
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p)
+{
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Waits until *p >= v; false after ~2^31 clocks (about a second).
+__device__ __forceinline__ bool wait_at_least(const int32_t* p, int32_t v)
+{
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(p) < v) {
+        if (clock64() - t0 > (1ll << 31)) return false;
+        __nanosleep(256);
+    }
+    return true;
+}
+
 // All but the most recently committed group have landed.
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
