@@ -246,9 +246,18 @@ gdn_status_t launch_decode(const DecArgs& a)
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         return GDN_ERR_CUDA;
+    int per_sm = 0;
+    if (set_smem(gdn::k_dec_tok<D, D, C>, DC::SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gdn::k_dec_tok<D, D, C>, DC::THREADS, DC::SMEM) !=
+            cudaSuccess ||
+        per_sm <= 0)
+        return GDN_ERR_CUDA;
+    const int64_t items = NH * DC::NT;
+    const unsigned tgrid = (unsigned)std::min<int64_t>(items, (int64_t)sms * per_sm);
     mark(a.events, 0, a.stream);
-    gdn::k_dec_tok<D, D, C><<<(unsigned)(NH * DC::NT), DC::THREADS, 0, a.stream>>>(
-        a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, a.o);
+    gdn::k_dec_tok<D, D, C><<<tgrid, DC::THREADS, DC::SMEM, a.stream>>>(
+        a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, a.o,
+        (int)items);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;

@@ -7,63 +7,144 @@
 namespace gdn {
 
 // ------------------------------------------------------------------ decode
+// One decode token per (sequence, head): P_tok on the running state R, and
+// the token appended to the buffer at slot pos (pos itself is advanced by
+// k_dec_resync, which runs next).  Work item = (sequence-head, row tile).
+// Persistent: CTA b takes items b, b + grid, ...  Each item's state rows and
+// raw token stream into shared memory by cp.async, DecCfg::S - 1 items ahead
+// of the one being computed, so several items' loads are in flight per CTA
+// without holding registers.  Each lane's slice of a row (EPT contiguous
+// floats) sits in its own padded slot, so the lane reads it conflict-free;
+// the tile moves between global and shared memory a row per warp access
+// (coalesced), in both directions.
 template <int DK, int DV>
 struct DecCfg {
     using RS = RowSplit<DK>;
-    static constexpr int RT = DV < 32 ? DV : 32;  // rows per CTA
+    static constexpr int RT = DV < 32 ? DV : 32;  // rows per item
     static constexpr int NT = DV / RT;
     static constexpr int THREADS = RT * RS::TPR;
+    static constexpr int S = 3;                   // pipeline stages
+    static constexpr int SLOT = RS::EPT + 4;      // floats per lane slice, padded
+    static constexpr int RSTAGE = THREADS * SLOT; // state floats per stage
+    static constexpr int RAWB = (2 * DK + RT) * 4 + 16;  // raw token bytes per stage (fp32 worst case) + gates, pos
+    static constexpr int STAGE = RSTAGE + RAWB / 4;      // floats per stage
+    static constexpr int TOKF = 2 * RS::KS + RT;         // widened token
+    static constexpr size_t SMEM = sizeof(float) * ((size_t)S * STAGE + TOKF);
 };
 
-// One decode token per (sequence, head), one CTA per row tile: P_tok on the
-// running state R; tile 0 also appends the token to the buffer at slot pos.
-// pos itself is advanced by k_dec_resync, which runs next.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(DecCfg<DK, DV>::THREADS)
 k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
           const float* __restrict__ alpha, const float* __restrict__ beta, int in_bf16, int out_bf16,
-          float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos, void* __restrict__ o)
+          float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos, void* __restrict__ o,
+          int nitems)
 {
     using Cf = DecCfg<DK, DV>;
     using RS = typename Cf::RS;
-    __shared__ __align__(16) float ks[RS::KS];
-    __shared__ __align__(16) float qs[RS::KS];
-    __shared__ __align__(16) float vs[Cf::RT];
-    const int nh = blockIdx.x / Cf::NT, r = blockIdx.x % Cf::NT;
-    const int p = pos[nh];
-    if (p < 0 || p >= C) return;
-    // the state rows are the bulk of the traffic: issue their loads before staging the token
-    const int row = threadIdx.x / RS::TPR, part = threadIdx.x % RS::TPR;
-    const int grow = r * Cf::RT + row;
-    float* Rrow = R + ((int64_t)nh * DV + grow) * DK + part * RS::EPT;
-    f2x Rp[RS::L];
-    load_row_pairs<DK>(Rp, Rrow);
-    stage_rows<DK>(ks, RS::KS, k, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
-    stage_rows<DK>(qs, RS::KS, q, nh, 1, 1, 0, in_bf16, IdxSlot<DK>());
-    for (int e = threadIdx.x; e < Cf::RT / 8; e += blockDim.x) {
-        float x[8];
-        load8(v, (int64_t)nh * DV + r * Cf::RT + e * 8, in_bf16, x);
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    float* ks = sm + Cf::S * Cf::STAGE;
+    float* qs = ks + RS::KS;
+    float* vs = qs + RS::KS;
+    const int t = threadIdx.x;
+    const int row = t / RS::TPR, part = t % RS::TPR;
+    const int esz = in_bf16 ? 2 : 4;
+    const int kp = DK * esz / 16, vp = Cf::RT * esz / 16;  // 16-byte pieces of k (= of q) and of the v rows
+    const int el = 16 / esz;                               // elements per piece
+    const int G = gridDim.x;
+    auto rslot = [&](int st) { return sm + st * Cf::STAGE + t * Cf::SLOT; };
+    // 16-byte chunk f of the tile (row-major) <-> its place in the lane slots
+    constexpr int CPR = DK / 4, CPS = RS::EPT / 4;  // chunks per row, per lane slice
+    auto chunk_slot = [&](int st, int f) {
+        const int rr = f / CPR, c = f % CPR;
+        return sm + st * Cf::STAGE + (rr * RS::TPR + c / CPS) * Cf::SLOT + 4 * (c % CPS);
+    };
+    auto raw = [&](int st) { return reinterpret_cast<unsigned char*>(sm + st * Cf::STAGE + Cf::RSTAGE); };
+
+    auto fetch = [&](int it, int st) {  // item it -> stage st; always commits a group
+        if (it < nitems) {
+            const int nh = it / Cf::NT, r = it % Cf::NT;
+            const float* src = R + ((int64_t)nh * DV + r * Cf::RT) * DK;
+            for (int f = t; f < Cf::RT * CPR; f += Cf::THREADS) cp_async16(chunk_slot(st, f), src + 4 * f);
+            unsigned char* rw = raw(st);
+            if (t < kp) cp_async16(rw + 16 * t, reinterpret_cast<const uint4*>(k) + (int64_t)nh * kp + t);
+            else if (t < 2 * kp) cp_async16(rw + 16 * t, reinterpret_cast<const uint4*>(q) + (int64_t)nh * kp + (t - kp));
+            else if (t < 2 * kp + vp)
+                cp_async16(rw + 16 * t, reinterpret_cast<const uint4*>(v) + ((int64_t)nh * DV + r * Cf::RT) * esz / 16 +
+                                            (t - 2 * kp));
+            float* gates = reinterpret_cast<float*>(rw + 16 * (2 * kp + vp));
+            if (t == 0) cp_async4(gates, alpha + nh);
+            if (t == 1) cp_async4(gates + 1, beta + nh);
+            if (t == 2) cp_async4(gates + 2, pos + nh);
+        }
+        cp_async_commit();
+    };
+
+    int it = blockIdx.x;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) vs[e * 8 + m] = x[m];
-    }
-    const float a = __ldg(alpha + nh), b = __ldg(beta + nh);
-    __syncthreads();
-    const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
-    store_row_pairs<DK>(Rrow, Rp);
-    if (part == 0) store1(o, (int64_t)nh * DV + grow, out_bf16, ot);
-    if (r == 0) {  // append the raw token to the buffer at slot p
-        const int esz = in_bf16 ? 2 : 4;
-        for (int e = threadIdx.x; e < DK * esz / 16; e += blockDim.x)
-            reinterpret_cast<uint4*>(kbuf)[((int64_t)nh * C + p) * (DK * esz / 16) + e] =
-                __ldg(reinterpret_cast<const uint4*>(k) + (int64_t)nh * (DK * esz / 16) + e);
-        for (int e = threadIdx.x; e < DV * esz / 16; e += blockDim.x)
-            reinterpret_cast<uint4*>(vbuf)[((int64_t)nh * C + p) * (DV * esz / 16) + e] =
-                __ldg(reinterpret_cast<const uint4*>(v) + (int64_t)nh * (DV * esz / 16) + e);
-        if (threadIdx.x == 0) {
+    for (int s = 0; s < Cf::S - 1; ++s) fetch(it + s * G, s);
+    for (int i = 0; it < nitems; ++i, it += G) {
+        const int st = i % Cf::S;
+        fetch(it + (Cf::S - 1) * G, (i + Cf::S - 1) % Cf::S);
+        cp_async_wait_n<Cf::S - 1>();  // this item's copies (each thread's own) have landed
+        __syncthreads();
+        const int nh = it / Cf::NT, r = it % Cf::NT;
+        const unsigned char* rw = raw(st);
+        const float* gates = reinterpret_cast<const float*>(rw + 16 * (2 * kp + vp));
+        const float a = gates[0], b = gates[1];
+        const int p = __float_as_int(gates[2]);
+        if (t < 2 * kp + vp) {  // widen the raw token
+            const uint4 pc = *reinterpret_cast<const uint4*>(rw + 16 * t);
+            const uint32_t w[4] = {pc.x, pc.y, pc.z, pc.w};
+            float x[8];
+            if (in_bf16) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    x[2 * m] = __uint_as_float(w[m] << 16);
+                    x[2 * m + 1] = __uint_as_float(w[m] & 0xffff0000u);
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) x[m] = __uint_as_float(w[m]);
+            }
+            if (t < 2 * kp) {
+                float* d = t < kp ? ks : qs;
+                const int j0 = (t < kp ? t : t - kp) * el;
+                for (int m = 0; m < el; ++m) d[RS::slot(j0 + m)] = x[m];
+            } else {
+                const int i0 = (t - 2 * kp) * el;
+                for (int m = 0; m < el; ++m) vs[i0 + m] = x[m];
+            }
+            // append the raw token at slot p: k by tile 0, each tile its v rows
+            if (p >= 0 && p < C) {
+                if (t < kp && r == 0) reinterpret_cast<uint4*>(kbuf)[((int64_t)nh * C + p) * kp + t] = pc;
+                if (t >= 2 * kp)
+                    reinterpret_cast<uint4*>(vbuf)[(((int64_t)nh * C + p) * DV + r * Cf::RT) * esz / 16 +
+                                                   (t - 2 * kp)] = pc;
+            }
+        }
+        if (r == 0 && t == 0 && p >= 0 && p < C) {
             abuf[(int64_t)nh * C + p] = a;
             bbuf[(int64_t)nh * C + p] = b;
         }
+        f2x Rp[RS::L];
+        load_row_pairs<DK>(Rp, rslot(st));
+        __syncthreads();  // the widened token is complete
+        const bool valid = p >= 0 && p < C;  // an invalid position writes nothing
+        if (valid) {
+            const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
+            store_row_pairs<DK>(rslot(st), Rp);
+            if (part == 0) store1(o, (int64_t)nh * DV + r * Cf::RT + row, out_bf16, ot);
+        }
+        __syncthreads();  // the new rows are in the slots
+        if (valid) {
+            float* dst = R + ((int64_t)nh * DV + r * Cf::RT) * DK;
+            for (int f = t; f < Cf::RT * CPR; f += Cf::THREADS)
+                *reinterpret_cast<float4*>(dst + 4 * f) = *reinterpret_cast<const float4*>(chunk_slot(st, f));
+        }
+        __syncthreads();  // ks / qs / vs and this stage are free again
     }
+    cp_async_wait_all();
 }
 
 template <int DK, int DV, int C>

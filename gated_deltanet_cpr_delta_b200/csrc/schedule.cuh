@@ -198,6 +198,10 @@ __device__ __forceinline__ bool wait_at_least(const int32_t* p, int32_t v)
     return true;
 }
 
+// All but the N most recently committed groups have landed.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_n() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 // All but the most recently committed group have landed.
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
