@@ -217,7 +217,10 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v,
  *     kernel, the chunk precompute (w, u0, decays), the boundary-state chain,
  *     the intra-chunk recurrence and the cache fill.  Kernel i ran between
  *     events[i] and events[i+1].  A kernel that has no work still gets both
- *     of its events, so its time is zero.
+ *     of its events, so its time is zero.  When the chain and the
+ *     intra-chunk recurrence run as one kernel (batches with d_v = 128 and
+ *     fewer (sequence, head) pairs than SMs), events[2] and events[3] are
+ *     recorded back to back and events[3..4] span that kernel.
  *   gdn_decode_step_timed: events[0..2] around the per-token step and then the
  *     resync.
  * events == NULL behaves exactly like the untimed call.

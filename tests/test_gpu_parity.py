@@ -161,6 +161,32 @@ def test_batch_composition_and_packing_invariance():
     assert np.array_equal(bits(ho), bits(o[:, [2, 0]].contiguous()))
 
 
+def test_fused_chain_tok_path_equals_separate_kernels():
+    """With d_v = 128 and fewer (sequence, head) pairs than SMs the library runs
+    the boundary chain and P_tok as one cooperative kernel; with more pairs it
+    runs them as separate kernels.  The same sequences give the same bits
+    either way (ragged lengths, a partial last chunk, the decode cache)."""
+    C, d, H = 64, 128, 4
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    lens = [300, 64, 1, 129, 0, 191]                       # 24 pairs: the fused kernel
+    n_more = (sms + 64) // H                                # enough pairs for the separate kernels
+    more = lens + [37 + 11 * i for i in range(n_more)]
+    b = synth.make_batch(350, more, H, d, d, "bf16")
+    o_big, st_big, c_big = fwd(b, C, torch.bfloat16, cache=True)
+    small = b.subset(range(len(lens)))
+    o, st, c = fwd(small, C, torch.bfloat16, cache=True)
+    T = int(small.cu_seqlens[-1])
+    ns = sum(L // C + 1 for L in lens)
+    assert np.array_equal(bits(o), bits(o_big[:T]))
+    assert np.array_equal(bits(st), bits(st_big[:ns]))
+    for key in ("S_b", "R", "pos"):
+        assert torch.equal(c[key], c_big[key][:len(lens)]), key
+    # and the fused result is the model's P_tok from the GPU's states, bit for bit
+    mo, _ = oracle.schedule_tok_from_states(small.q, small.k, small.v, small.alpha, small.beta, st.cpu().numpy(),
+                                            small.cu_seqlens, C)
+    assert np.array_equal(bits(o), oracle.to_bf16_bits(mo))
+
+
 def test_split_at_chunk_boundary_equals_unsplit():
     C, d, H, L = 16, 32, 2, 150
     b = synth.make_batch(400, [L], H, d, d, "bf16")
