@@ -375,30 +375,65 @@ def run_native(args):
     tokens = B * T * world
     value = job_throughput(B * T, world, total_ms, K)
 
-    # e2e: host (pinned) inputs -> device, forward, o -> host, every step
+    # e2e: every step copies its inputs host (pinned) -> device, runs the
+    # forward through the public API and copies o device -> host.  Steps are
+    # pipelined the way a serving loop would run them: step i+1's inputs
+    # upload on a copy stream while step i computes, and step i's o downloads
+    # on a second copy stream (two device buffer sets alternate).
     hin = {n: d[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
-    dev_in = {n: torch.empty_like(d[n]) for n in hin}
-    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in hin.values()) + 4 * (B + 1)
+    cu_pin = torch.tensor(d["cu_host"], dtype=torch.int32).pin_memory()
+    dev_in = [{n: torch.empty_like(d[n]) for n in hin} for _ in range(2)]
+    cu_dev = [torch.empty_like(d["cu_seqlens"]) for _ in range(2)]
+    o_dev = [torch.empty_like(o) for _ in range(2)]
+    o_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in hin.values()) + cu_pin.numel() * 4
     d2h = o.numel() * o.element_size()
+    compute = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for n in hin:
-            dev_in[n].copy_(hin[n], non_blocking=True)
-        cu_dev = torch.tensor(d["cu_host"], dtype=torch.int32).pin_memory().cuda(non_blocking=True)
-        gdn.gdn_cpr_forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"], cu_dev, C,
-                            cu_seqlens_host=d["cu_host"], o=o, chunk_states=st, workspace=ws)
-        o_host.copy_(o, non_blocking=True)
+    def upload(i):
+        j = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(done[j])           # the forward two steps back is done with buffer set j
+            for n in hin:
+                dev_in[j][n].copy_(hin[n], non_blocking=True)
+            cu_dev[j].copy_(cu_pin, non_blocking=True)
+            in_ready[j].record(s_in)
 
-    for _ in range(2):
-        e2e_step()
+    def run_steps(nsteps):
+        for j in range(2):
+            done[j].record(compute)
+            out_done[j].record(compute)
+        upload(0)
+        for i in range(nsteps):
+            j = i % 2
+            if i + 1 < nsteps:
+                upload(i + 1)
+            compute.wait_event(in_ready[j])
+            compute.wait_event(out_done[j])   # o buffer j has been downloaded
+            gdn.gdn_cpr_forward(dev_in[j]["q"], dev_in[j]["k"], dev_in[j]["v"], dev_in[j]["alpha"],
+                                dev_in[j]["beta"], cu_dev[j], C, cu_seqlens_host=d["cu_host"], o=o_dev[j],
+                                chunk_states=st, workspace=ws)
+            done[j].record(compute)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[j])
+                o_host[j].copy_(o_dev[j], non_blocking=True)
+                out_done[j].record(s_out)
+        for j in range(2):
+            compute.wait_event(out_done[j])
+            compute.wait_event(in_ready[j])
+
+    run_steps(2)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(K):
-        e2e_step()
+    run_steps(K)
     e1.record()
     barrier(world)
+    assert torch.equal(o_dev[(K - 1) % 2].cpu(), o_host[(K - 1) % 2])
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / K
 
     dec = bench_decode(rank, world, args.warmup) if not args.no_decode else None
@@ -442,7 +477,9 @@ def run_native(args):
                              "frac": total_flops / (ms_step / 1e3) / 1e12 / world / FP32_PEAK_TFLOPS},
         "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "pipelining": "step i+1's upload and step i-1's download overlap step i's forward "
+                              "(two device buffer sets, two copy streams)"},
         "gpu_launches": (3 if fused else 4) * K,
         "clocks": clocks.summary(),
         "parity": parity,
