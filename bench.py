@@ -323,6 +323,8 @@ def bench_decode(rank: int, world: int, warmup: int):
             "ms_per_step": total_ms / S, "plain_step_ms_mean": sum(plain) / len(plain),
             "resync_step_ms_mean": sum(step_ms[s] for s in resync_steps) / max(1, len(resync_steps)),
             "resync_kernel_ms_max": max(res_ms),
+            "step_kernel_ms_mean": sum(tok_ms) / S,
+            "resync_kernel_plain_ms_mean": sum(res_ms[s] for s in range(S) if s not in resync_steps) / len(plain),
             "roofline": {"kernel": "k_dec_tok", "bound": "hbm", "achieved": tb / (mean_tok / 1e3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": tb / (mean_tok / 1e3) / 1e9 / peaks["hbm_gbs"],

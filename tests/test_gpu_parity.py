@@ -187,6 +187,56 @@ def test_fused_chain_tok_path_equals_separate_kernels():
     assert np.array_equal(bits(o), oracle.to_bf16_bits(mo))
 
 
+def test_forward_and_decode_replay_from_cuda_graphs():
+    """Both calls enqueue only stream work, so they can be captured into CUDA
+    graphs (the fused cooperative kernel included); a replay gives the same
+    bits as the eager calls."""
+    C, d, H, N, L0, steps = 64, 128, 2, 3, 62, 4   # the decode steps cross a chunk boundary (a resync)
+    b = synth.make_batch(360, [L0 + steps] * N, H, d, d, "bf16")
+    dev = to_device(b)
+    idx = torch.cat([torch.arange(n * (L0 + steps), n * (L0 + steps) + L0) for n in range(N)]).to(DEV)
+    pre = {n: dev[n][idx].contiguous() for n in ("q", "k", "v", "alpha", "beta")}
+    cu = [n * L0 for n in range(N + 1)]
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device=DEV)
+    ws = torch.empty(gdn.gdn_cpr_workspace_size(N * L0, N, H, d, d, C), dtype=torch.uint8, device=DEV)
+    o_e = torch.empty(N * L0, H, d, dtype=torch.bfloat16, device=DEV)
+    st_e = torch.empty(gdn.gdn_num_chunk_states(cu, C), H, d, d, dtype=torch.float32, device=DEV)
+    cache = gdn.new_cache(N, H, d, d, C, torch.bfloat16, DEV)
+    fwd = lambda o, st, c: gdn.gdn_cpr_forward(pre["q"], pre["k"], pre["v"], pre["alpha"], pre["beta"], cu_dev, C,
+                                               cu_seqlens_host=cu, o=o, chunk_states=st, workspace=ws, cache_out=c)
+    fwd(o_e, st_e, cache)
+    torch.cuda.synchronize()
+    o_g, st_g = torch.zeros_like(o_e), torch.zeros_like(st_e)
+    cache_g = {n: torch.zeros_like(t) for n, t in cache.items()}
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fwd(o_g, st_g, cache_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o_g.view(torch.int16), o_e.view(torch.int16)) and torch.equal(st_g, st_e)
+    for n in cache:
+        assert torch.equal(cache_g[n], cache[n]), n
+    # decode: eager steps on one copy of the cache, graph replay on another
+    step_in = []
+    for s in range(steps):
+        t = torch.arange(N, device=DEV) * (L0 + steps) + L0 + s
+        step_in.append([dev[n][t].contiguous() for n in ("q", "k", "v", "alpha", "beta")])
+    c_e = {n: t.clone() for n, t in cache.items()}
+    outs_e = [gdn.gdn_decode_step(*step_in[s], c_e, C) for s in range(steps)]
+    c_g = {n: t.clone() for n, t in cache.items()}
+    outs_g = [torch.empty_like(outs_e[0]) for _ in range(steps)]
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2):
+        for s in range(steps):
+            gdn.gdn_decode_step(*step_in[s], c_g, C, o=outs_g[s])
+    g2.replay()
+    torch.cuda.synchronize()
+    for s in range(steps):
+        assert torch.equal(outs_g[s].view(torch.int16), outs_e[s].view(torch.int16)), s
+    for n in c_e:
+        assert torch.equal(c_g[n], c_e[n]), n
+
+
 def test_split_at_chunk_boundary_equals_unsplit():
     C, d, H, L = 16, 32, 2, 150
     b = synth.make_batch(400, [L], H, d, d, "bf16")
