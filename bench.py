@@ -215,8 +215,18 @@ def cpu_baseline(budget_s: float = 10.0):
                       f"{secs:.1f} s"}
 
 
+def workload_config(world: int) -> dict:
+    """The bench workload's config, shared by both arms of the benchmark."""
+    W = WORKLOAD
+    return {"workload": W["name"], "global_batch": W["B"] * world, "seq_len": W["T"], "heads": W["H"],
+            "d_k": W["D"], "d_v": W["D"], "chunk": W["C"], "io_dtype": "bf16", "state_dtype": "f32",
+            "parallelism": f"dp{world} (sequences sharded, no collective)",
+            "l2": "flushed before every timed step (256 MiB write)"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     import oracle
@@ -240,7 +250,7 @@ def run_reference(args):
         "metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": W["name"], "oracle": "cpu fp64"},
+        "config": workload_config(world),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
@@ -464,10 +474,7 @@ def run_native(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": W["name"], "global_batch": B * world, "seq_len": T, "heads": H, "d_k": D,
-                   "d_v": D, "chunk": C, "io_dtype": "bf16", "state_dtype": "f32",
-                   "parallelism": f"dp{world} (sequences sharded, no collective)",
-                   "l2": "flushed before every timed step (256 MiB write)"},
+        "config": workload_config(world),
         "roofline": {"kernel": ("k_chain_tok (boundary chain on tcgen05 + intra-chunk P_tok, one cooperative "
                                 "launch)") if fused else "k_tok (intra-chunk P_tok)",
                      "bound": "alu", "achieved": tok_tf,
