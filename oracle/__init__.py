@@ -36,6 +36,8 @@ def _load():
         i32 = ctypes.c_int32
         lib.oracle_recurrent_fp64.restype = ctypes.c_int
         lib.oracle_recurrent_fp64.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P]
+        lib.oracle_adjoint_fp64.restype = ctypes.c_int
+        lib.oracle_adjoint_fp64.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
         lib.sched_forward.restype = ctypes.c_int
         lib.sched_forward.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
                                       P, P, P, P, P, P, P, P, P]
@@ -82,6 +84,28 @@ def recurrent(q, k, v, alpha, beta, cu_seqlens, C, state_in=None):
     if rc:
         raise RuntimeError(f"oracle_recurrent_fp64 failed ({rc})")
     return dict(o=o, states=states, final=final)
+
+
+def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None):
+    """fp64 gradient of L = sum_t dO_t . o_t through the recurrence
+    (oracle/adjoint_fp64.c).  Returns dict(dq, dk, dv, dalpha, dbeta,
+    dstate_in [N,H,dv,dk])."""
+    lib = _load()
+    q, k, v = _c(q, np.float64), _c(k, np.float64), _c(v, np.float64)
+    alpha, beta, dO = _c(alpha, np.float64), _c(beta, np.float64), _c(dO, np.float64)
+    cu = _c(cu_seqlens, np.int32)
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    N = cu.shape[0] - 1
+    s_in = _c(state_in, np.float64)
+    out = dict(dq=np.zeros((T, H, dk)), dk=np.zeros((T, H, dk)), dv=np.zeros((T, H, dv)),
+               dalpha=np.zeros((T, H)), dbeta=np.zeros((T, H)), dstate_in=np.zeros((N, H, dv, dk)))
+    rc = lib.oracle_adjoint_fp64(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s_in), _p(dO), _p(cu), N, H, dk, dv, C,
+                                 _p(out["dq"]), _p(out["dk"]), _p(out["dv"]), _p(out["dalpha"]), _p(out["dbeta"]),
+                                 _p(out["dstate_in"]))
+    if rc:
+        raise RuntimeError(f"oracle_adjoint_fp64 failed ({rc})")
+    return out
 
 
 def chunkwise(q, k, v, alpha, beta, cu_seqlens, C, state_in=None):

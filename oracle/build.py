@@ -10,7 +10,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SOURCES = ["recurrent_fp64.c", "schedule_fp32.c"]
+SOURCES = ["recurrent_fp64.c", "schedule_fp32.c", "adjoint_fp64.c"]
 LIB = os.path.join(HERE, "liboracle.so")
 
 

@@ -1,0 +1,79 @@
+"""Pins of the fp64 adjoint oracle (oracle/adjoint_fp64.c), the gradient of
+L = sum_t dO_t . o_t through the gated delta rule.
+
+* Complex-step derivatives: the recurrence is a polynomial in every input, so
+  Im(L(x + i h e_j)) / h is the exact derivative up to rounding (no
+  cancellation).  A complex128 forward written independently here, with the
+  literal matrix (I - beta k k^T), gives every partial derivative on small
+  inputs; the adjoint must match them all.
+* A closed form: with alpha = 1 and beta = 0 the state never changes, so
+  dq_t = S_0^T dO_t, dS_0 = sum_t dO_t q_t^T, dv = dk = 0 and
+  dalpha_t = <sum_{t' >= t} dO_t' q_t'^T, S_0>.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gated_deltanet_cpr_delta_b200 import synth
+
+
+def _loss_complex(q, k, v, alpha, beta, S0, dO, cu):
+    """sum_t dO_t . o_t with the recurrence S_t = a S (I - b k k^T) + b v k^T, complex128."""
+    L = 0.0 + 0.0j
+    H = k.shape[1]
+    for n in range(len(cu) - 1):
+        for h in range(H):
+            S = S0[n, h].astype(np.complex128).copy()
+            for t in range(cu[n], cu[n + 1]):
+                kt, qt, vt = k[t, h], q[t, h], v[t, h]
+                M = np.eye(len(kt), dtype=np.complex128) - beta[t, h] * np.outer(kt, kt)
+                S = alpha[t, h] * (S @ M) + beta[t, h] * np.outer(vt, kt)
+                L += dO[t, h] @ (S @ qt)
+    return L
+
+
+@pytest.mark.parametrize("C", [2, 4])
+def test_adjoint_matches_complex_step_derivatives(C):
+    rng = np.random.default_rng(5)
+    lens, H, dk, dv = [7, 4], 1, 3, 2
+    b = synth.make_batch(21, lens, H, dk, dv, "f32")
+    T = int(b.cu_seqlens[-1])
+    S0 = rng.standard_normal((2, H, dv, dk))
+    dO = rng.standard_normal((T, H, dv))
+    ins = dict(q=b.q.astype(np.float64), k=b.k.astype(np.float64), v=b.v.astype(np.float64),
+               alpha=b.alpha.astype(np.float64), beta=b.beta.astype(np.float64), S0=S0)
+    g = oracle.adjoint(ins["q"], ins["k"], ins["v"], ins["alpha"], ins["beta"], dO, b.cu_seqlens, C, state_in=S0)
+    grads = dict(q=g["dq"], k=g["dk"], v=g["dv"], alpha=g["dalpha"], beta=g["dbeta"], S0=g["dstate_in"])
+    h = 1e-30
+    for name, base in ins.items():
+        for idx in np.ndindex(base.shape):
+            x = {k_: v_.astype(np.complex128) for k_, v_ in ins.items()}
+            x[name][idx] += 1j * h
+            d = _loss_complex(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], dO, b.cu_seqlens).imag / h
+            assert abs(d - grads[name][idx]) <= 1e-12 * max(1.0, abs(d)), (name, idx, d, grads[name][idx])
+
+
+def test_adjoint_closed_form_with_a_frozen_state():
+    rng = np.random.default_rng(6)
+    T, H, dk, dv = 9, 2, 4, 3
+    q, k, v = (rng.standard_normal((T, H, d)) for d in (dk, dk, dv))
+    alpha, beta = np.ones((T, H)), np.zeros((T, H))
+    S0 = rng.standard_normal((1, H, dv, dk))
+    dO = rng.standard_normal((T, H, dv))
+    g = oracle.adjoint(q, k, v, alpha, beta, dO, np.array([0, T], np.int32), 4, state_in=S0)
+    for h in range(H):
+        assert np.allclose(g["dq"][:, h], dO[:, h] @ S0[0, h], rtol=0, atol=1e-12)
+        assert np.allclose(g["dstate_in"][0, h], dO[:, h].T @ q[:, h], rtol=0, atol=1e-12)
+        for t in range(T):
+            Gt = dO[t:, h].T @ q[t:, h]
+            assert abs(g["dalpha"][t, h] - np.sum(Gt * S0[0, h])) <= 1e-12 * max(1, abs(np.sum(Gt * S0[0, h])))
+    assert np.all(g["dv"] == 0) and np.allclose(g["dk"], 0, atol=1e-14)
+
+
+def test_adjoint_is_independent_of_the_checkpoint_span():
+    b = synth.make_batch(22, [37, 1, 20], 2, 8, 4, "bf16")
+    dO = np.random.default_rng(7).standard_normal((58, 2, 4))
+    a = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, 4)
+    c = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, 16)
+    for key in a:
+        assert np.allclose(a[key], c[key], rtol=1e-12, atol=1e-12), key
