@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgdn_cpr.so")
 SOURCES = ["gdn_cpr.cu", "identity.cu"]
 DEPS = ["gdn_cpr.cu", "identity.cu", "kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_tc.cuh",
-        "k_pchunk.cuh", "k_decode.cuh"]
+        "k_pchunk.cuh", "k_decode.cuh", "k_bwd.cuh"]
 HEADERS = [os.path.join(ROOT, "include", "gdn_cpr.h")]
 
 

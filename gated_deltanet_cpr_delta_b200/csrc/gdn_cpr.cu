@@ -272,6 +272,80 @@ gdn_status_t launch_decode(const DecArgs& a)
     return GDN_OK;
 }
 
+// Backward workspace: [err | cto | fco | so | ...] as the forward's tables,
+// then the checkpoints of every (sequence, head, row tile) CTA and the
+// per-tile partial sums of dq, dk (fp32 [NT][T][H][d_k]) and dalpha, dbeta.
+struct BwdWorkspace {
+    Workspace t;  // tables only (err, tok_next, cto, fco, so, ...)
+    float *scratch, *pq, *pk, *pa, *pb;
+    size_t bytes;
+};
+
+BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C)
+{
+    BwdWorkspace w{};
+    const int32_t RT = dv < 32 ? dv : 32, NT = dv / RT, SUB = C < 8 ? C : 8;
+    const Workspace tables = carve(nullptr, 0, N, H, dk, dv, C);  // the tables part alone
+    size_t off = tables.bytes;
+    auto take = [&](size_t n) {
+        const size_t o = off;
+        off = align_up(off + n);
+        return o;
+    };
+    const size_t o_sc = take(sizeof(float) * (size_t)N * H * NT * (C / SUB) * RT * dk);
+    const size_t o_pq = take(sizeof(float) * (size_t)NT * T * H * dk);
+    const size_t o_pk = take(sizeof(float) * (size_t)NT * T * H * dk);
+    const size_t o_pa = take(sizeof(float) * (size_t)NT * T * H);
+    const size_t o_pb = take(sizeof(float) * (size_t)NT * T * H);
+    w.bytes = off;
+    char* b = static_cast<char*>(base);
+    if (b != nullptr) {
+        w.t = carve(base, 0, N, H, dk, dv, C);
+        w.scratch = reinterpret_cast<float*>(b + o_sc);
+        w.pq = reinterpret_cast<float*>(b + o_pq);
+        w.pk = reinterpret_cast<float*>(b + o_pk);
+        w.pa = reinterpret_cast<float*>(b + o_pa);
+        w.pb = reinterpret_cast<float*>(b + o_pb);
+    }
+    return w;
+}
+
+struct BwdArgs {
+    const void *q, *k, *v, *dO;
+    const float *alpha, *beta, *states;
+    const int32_t* cu;
+    int32_t N, H;
+    int in_bf16;
+    float *dq, *dk, *dv, *dalpha, *dbeta, *dstate;
+    SeqTotals tot;
+    int64_t T_total;
+    BwdWorkspace ws;
+    cudaStream_t stream;
+};
+
+template <int D, int C>
+gdn_status_t launch_backward(const BwdArgs& a)
+{
+    using BC = gdn::BwdCfg<D, D, C>;
+    gdn::k_tables<<<1, 1024, 0, a.stream>>>(a.cu, a.N, C, a.T_total, a.tot.tasks, a.tot.full, a.tot.states,
+                                             a.tot.hash, a.ws.t.cto, a.ws.t.fco, a.ws.t.so, a.ws.t.err, nullptr,
+                                             nullptr, 0, nullptr, nullptr, 0);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    if (set_smem(gdn::k_bwd_rows<D, D, C>, BC::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
+    gdn::k_bwd_rows<D, D, C><<<(unsigned)((int64_t)a.N * a.H * BC::NT), BC::THREADS, BC::SMEM, a.stream>>>(
+        a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.cu, a.ws.t.so, a.ws.t.err, a.N, a.H, a.T_total,
+        a.in_bf16, a.dv, a.dstate, a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.scratch);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    const int64_t TH = a.T_total * a.H;
+    if (TH > 0) {
+        const unsigned grid = (unsigned)std::min<int64_t>((TH * (D + 1) + 255) / 256, 148 * 16);
+        gdn::k_bwd_reduce<D, BC::NT><<<grid, 256, 0, a.stream>>>(a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.t.err, TH,
+                                                               a.dq, a.dk, a.dalpha, a.dbeta);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
+}
+
 #define GDN_DISPATCH(FN, D_, C_, ARGS)                              \
     switch (D_ * 1000 + C_) {                                       \
         case 16016: return FN<16, 16>(ARGS);                        \
@@ -379,6 +453,49 @@ gdn_status_t gdn_cpr_forward(const void* q, const void* k, const void* v, const 
     return gdn_cpr_forward_timed(q, k, v, alpha, beta, state_in, cu_seqlens, cu_seqlens_host, num_seqs,
                                  total_tokens, H, d_k, d_v, C, in_dtype, out_dtype, o, chunk_states, cache_out,
                                  workspace, workspace_bytes, stream, nullptr);
+}
+
+size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v,
+                                       int32_t C)
+{
+    if (total_tokens < 0 || num_seqs < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0) return 0;
+    return carve_bwd(nullptr, total_tokens, num_seqs, H, d_k, d_v, C).bytes;
+}
+
+gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                              const void* dO, const float* chunk_states, const int32_t* cu_seqlens,
+                              const int32_t* cu_seqlens_host, int32_t num_seqs, int64_t total_tokens, int32_t H,
+                              int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype, float* dq, float* dk,
+                              float* dv, float* dalpha, float* dbeta, float* dstate_in, void* workspace,
+                              size_t workspace_bytes, void* stream)
+{
+    if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0)
+        return GDN_ERR_INVALID_ARG;
+    if (!dtype_ok(in_dtype)) return GDN_ERR_INVALID_ARG;
+    if (!supported(d_k, d_v, C)) return GDN_ERR_UNSUPPORTED;
+    SeqTotals tot;
+    if (!seq_totals(cu_seqlens_host, num_seqs, total_tokens, C, &tot)) return GDN_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr || chunk_states == nullptr || dstate_in == nullptr) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(chunk_states) || !aligned16(dstate_in)) return GDN_ERR_INVALID_ARG;
+    if (total_tokens > 0) {
+        if (!q || !k || !v || !alpha || !beta || !dO || !dq || !dk || !dv || !dalpha || !dbeta)
+            return GDN_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+            !aligned16(dv))
+            return GDN_ERR_INVALID_ARG;
+    }
+    const BwdWorkspace need = carve_bwd(nullptr, total_tokens, num_seqs, H, d_k, d_v, C);
+    if (workspace == nullptr || workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.dO = dO; a.alpha = alpha; a.beta = beta; a.states = chunk_states;
+    a.cu = cu_seqlens; a.N = num_seqs; a.H = H; a.in_bf16 = in_dtype == GDN_BF16;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dalpha = dalpha; a.dbeta = dbeta; a.dstate = dstate_in;
+    a.tot = tot; a.T_total = total_tokens;
+    a.ws = carve_bwd(workspace, total_tokens, num_seqs, H, d_k, d_v, C);
+    a.stream = static_cast<cudaStream_t>(stream);
+    GDN_DISPATCH(launch_backward, d_k, C, a)
 }
 
 gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, const float* alpha,

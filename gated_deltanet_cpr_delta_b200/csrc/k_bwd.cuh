@@ -1,0 +1,298 @@
+// k_bwd.cuh -- CPR backward: gradients of L = sum_t dO_t . o_t (sm_100a).
+//
+// Reverse-mode differentiation of the token recurrence of the gated delta rule
+// (IsoExec summary page, section "Chunkwise-Parallel Recurrent (CPR) Gated
+// DeltaNet"; commentary blog, section 10).  With u = S_{t-1} k_t,
+// delta = beta_t (v_t - alpha_t u), S_t = alpha_t S_{t-1} + delta k_t^T and
+// G = dL/dS_t, one token backward is
+//
+//     G       += dO_t q_t^T
+//     dq_t     = S_t^T dO_t                       ddelta = G k_t
+//     dv_t     = beta_t ddelta                    dbeta_t = ddelta . (v_t - alpha_t u)
+//     dalpha_t = <G, S_{t-1}> - beta_t ddelta . u
+//     dk_t     = G^T delta - alpha_t beta_t S_{t-1}^T ddelta
+//     G       <- alpha_t G - alpha_t beta_t ddelta k_t^T      (= dL/dS_{t-1})
+//
+// Every row i of S and G evolves on its own; only dq, dk, dalpha and dbeta sum
+// over rows.  k_bwd_rows runs one (sequence, head, tile of RT rows) per CTA,
+// serial over the sequence from its last token back: per chunk (from the
+// forward's boundary state) it recomputes the states with the forward's P_tok
+// arithmetic, keeping one checkpoint per SUB tokens (global scratch, L2
+// resident), and for each token recomputes S_{t-1} from the nearest
+// checkpoint.  The tile's row sums of the dq / dk / dalpha / dbeta terms go to
+// per-tile partial buffers; k_bwd_reduce adds the tiles in a fixed order, so
+// the gradients are deterministic.  Everything is fp32.
+#pragma once
+
+#include "k_ptok.cuh"
+
+namespace gdn {
+
+template <int DK, int DV, int C>
+struct BwdCfg {
+    using RS = RowSplit<DK>;
+    static constexpr int RT = DV < 32 ? DV : 32;  // rows per CTA
+    static constexpr int NT = DV / RT;            // row tiles per head
+    static constexpr int THREADS = RT * RS::TPR;
+    static constexpr int SUB = C < 8 ? C : 8;     // tokens per checkpoint
+    static constexpr int NCK = C / SUB;           // checkpoints per chunk
+    // staged floats per token: k, q (slots), v, dO rows, gates; a multiple of 4 (16-byte rows)
+    static constexpr int TOKF = ((2 * RS::KS + 2 * RT + 2) + 3) / 4 * 4;
+    static constexpr int RED = DK + 4;            // reduction buffer row stride
+    // smem: SUB staged tokens | dq rows | dk rows | [RT][2] scalars
+    static constexpr int TOK_OFF = 0;
+    static constexpr int RQ_OFF = TOK_OFF + SUB * TOKF;
+    static constexpr int RK_OFF = RQ_OFF + RT * RED;
+    static constexpr int RS_OFF = RK_OFF + RT * RED;
+    static constexpr size_t SMEM = sizeof(float) * (size_t)(RS_OFF + 2 * RT);
+    static constexpr int64_t SCRATCH = (int64_t)NCK * RT * DK;  // floats of checkpoints per CTA
+};
+
+// One forward P_tok step on this lane's share of a row: the u tree, delta and
+// the update, with exactly the forward's operations (ptok_step without the
+// output tree).  Returns u; *d_out = delta.
+template <int DK>
+__device__ __forceinline__ float ptok_advance(f2x (&Rp)[DK / kLeaves], const float* kt, float v_i, float a, float b,
+                                              float* d_out)
+{
+    constexpr int L = DK / kLeaves;
+    f2x kp[L];
+#pragma unroll
+    for (int m = 0; m < L; m += 2) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(kt + 2 * m);
+        kp[m] = x.x;
+        kp[m + 1] = x.y;
+    }
+    f2x acc = fmul2(Rp[0], kp[0]);
+#pragma unroll
+    for (int m = 1; m < L; ++m) acc = ffma2(Rp[m], kp[m], acc);
+    float la, lb;
+    up2(acc, la, lb);
+    const float u = tree_4lanes(la, lb);
+    const float d = fmul(b, fsub(v_i, fmul(a, u)));
+    const f2x aa = pk2(a, a), dd = pk2(d, d);
+#pragma unroll
+    for (int m = 0; m < L; ++m) Rp[m] = ffma2(dd, kp[m], fmul2(aa, Rp[m]));
+    *d_out = d;
+    return u;
+}
+
+// Dot product of two lane shares of rows over all DK columns (leaf chains,
+// then the 4-lane tree), every lane of the row getting the sum.
+template <int DK>
+__device__ __forceinline__ float row_dot(const f2x (&x)[DK / kLeaves], const f2x (&y)[DK / kLeaves])
+{
+    constexpr int L = DK / kLeaves;
+    f2x acc = fmul2(x[0], y[0]);
+#pragma unroll
+    for (int m = 1; m < L; ++m) acc = ffma2(x[m], y[m], acc);
+    float la, lb;
+    up2(acc, la, lb);
+    return tree_4lanes(la, lb);
+}
+
+template <int DK>
+__device__ __forceinline__ void load_pairs_slot(f2x (&p)[DK / kLeaves], const float* s)
+{
+    constexpr int L = DK / kLeaves;
+#pragma unroll
+    for (int m = 0; m < L; m += 2) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(s + 2 * m);
+        p[m] = x.x;
+        p[m + 1] = x.y;
+    }
+}
+
+// Backward of one (sequence, head, row tile).  Outputs: dv rows (direct),
+// dstate_in rows (direct), and the tile's partial sums of dq, dk (per token,
+// [NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(BwdCfg<DK, DV, C>::THREADS)
+k_bwd_rows(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+           const float* __restrict__ alpha, const float* __restrict__ beta, const void* __restrict__ dO,
+           const float* __restrict__ states, const int32_t* __restrict__ cu, const int32_t* __restrict__ so,
+           const int32_t* __restrict__ err, int N, int H, int64_t T_total, int in_bf16,
+           float* __restrict__ dv, float* __restrict__ dstate, float* __restrict__ pq, float* __restrict__ pk,
+           float* __restrict__ pa, float* __restrict__ pb, float* __restrict__ scratch)
+{
+    using Cf = BwdCfg<DK, DV, C>;
+    using RS = typename Cf::RS;
+    constexpr int L = RS::L, KS = RS::KS, RT = Cf::RT, SUB = Cf::SUB, TOKF = Cf::TOKF, NT = Cf::NT;
+    if (__ldg(err)) return;
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    float* tok = sm + Cf::TOK_OFF;
+    float* redq = sm + Cf::RQ_OFF;
+    float* redk = sm + Cf::RK_OFF;
+    float* reds = sm + Cf::RS_OFF;
+
+    const int r = blockIdx.x % NT;
+    const int nh = blockIdx.x / NT;
+    const int h = nh % H, n = nh / H;
+    const int tid = threadIdx.x;
+    const int row = tid / RS::TPR, part = tid % RS::TPR;
+    const int grow = r * RT + row;
+    const int seq0 = __ldg(cu + n);
+    const int Ln = __ldg(cu + n + 1) - seq0;
+    const int64_t slot0 = __ldg(so + n);
+    float* ck = scratch + (int64_t)blockIdx.x * Cf::SCRATCH;  // this CTA's checkpoints
+
+    // stage tokens [t0, t0 + len) of the sequence: k, q into the slot layout,
+    // this tile's v and dO rows, the gates
+    auto stage = [&](int t0, int len) {
+        constexpr int G8 = (2 * DK) / 8;
+        for (int e = tid; e < len * G8; e += blockDim.x) {
+            const int t = e / G8, el = (e % G8) * 8;
+            float x[8];
+            const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+            load8(el < DK ? k : q, trow * DK + (el % DK), in_bf16, x);
+            float* d = tok + t * TOKF + (el >= DK ? KS : 0);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) d[RS::slot((el % DK) + m)] = x[m];
+        }
+        for (int e = tid; e < len * (2 * RT / 8); e += blockDim.x) {
+            const int t = e / (2 * RT / 8), el = (e % (2 * RT / 8)) * 8;
+            float x[8];
+            const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+            load8(el < RT ? v : dO, trow * DV + r * RT + (el % RT), in_bf16, x);
+            float* d = tok + t * TOKF + 2 * KS + (el >= RT ? RT : 0) + (el % RT);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) d[m] = x[m];
+        }
+        for (int t = tid; t < len; t += blockDim.x) {
+            const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+            tok[t * TOKF + 2 * KS + 2 * RT] = __ldg(alpha + trow);
+            tok[t * TOKF + 2 * KS + 2 * RT + 1] = __ldg(beta + trow);
+        }
+    };
+    auto step = [&](f2x (&Sp)[L], int t) {  // forward step with staged token t
+        const float* tt = tok + t * TOKF;
+        float d;
+        ptok_advance<DK>(Sp, tt + part * RS::PS, tt[2 * KS + row], tt[2 * KS + 2 * RT], tt[2 * KS + 2 * RT + 1], &d);
+    };
+
+    f2x G[L];
+#pragma unroll
+    for (int m = 0; m < L; ++m) G[m] = pk2(0.f, 0.f);
+    const int nchunks = (Ln + C - 1) / C;
+    for (int c = nchunks - 1; c >= 0; --c) {
+        const int cb = c * C, clen = min(C, Ln - cb);
+        const int nsub = (clen + SUB - 1) / SUB;
+        // checkpoints: the state at cb + j*SUB, j = 1..nsub-1 (j = 0 is the chunk state)
+        f2x Sp[L];
+        load_row_pairs<DK>(Sp, states + (((slot0 + c) * H + h) * DV + grow) * DK + part * RS::EPT);
+        for (int j = 1; j < nsub; ++j) {
+            __syncthreads();
+            stage(cb + (j - 1) * SUB, SUB);
+            __syncthreads();
+            for (int t = 0; t < SUB; ++t) step(Sp, t);
+            store_row_pairs<DK>(ck + ((int64_t)(j - 1) * RT + row) * DK + part * RS::EPT, Sp);
+        }
+        // backward over the sub-chunks, last first
+        for (int j = nsub - 1; j >= 0; --j) {
+            const int sb = cb + j * SUB, slen = min(SUB, clen - j * SUB);
+            __syncthreads();
+            stage(sb, slen);
+            __syncthreads();
+            for (int t = slen - 1; t >= 0; --t) {
+                // S_{t-1}: from the sub-chunk's checkpoint, forward over its first t tokens
+                if (j == 0) load_row_pairs<DK>(Sp, states + (((slot0 + c) * H + h) * DV + grow) * DK + part * RS::EPT);
+                else load_row_pairs<DK>(Sp, ck + ((int64_t)(j - 1) * RT + row) * DK + part * RS::EPT);
+                for (int m = 0; m < t; ++m) step(Sp, m);
+                const float* tt = tok + t * TOKF;
+                const float a = tt[2 * KS + 2 * RT], b = tt[2 * KS + 2 * RT + 1];
+                const float vi = tt[2 * KS + row], doi = tt[2 * KS + RT + row];
+                f2x kp[L], qp[L];
+                load_pairs_slot<DK>(kp, tt + part * RS::PS);
+                load_pairs_slot<DK>(qp, tt + KS + part * RS::PS);
+                const float u = row_dot<DK>(Sp, kp);
+                const float de = fmul(b, fsub(vi, fmul(a, u)));
+                const f2x aa = pk2(a, a), dd = pk2(de, de), oo = pk2(doi, doi);
+                // G += dO_i q ; the dq and dk row terms ; dot products
+#pragma unroll
+                for (int m = 0; m < L; ++m) G[m] = ffma2(oo, qp[m], G[m]);
+                const float dlt = row_dot<DK>(G, kp);   // ddelta_i
+                const float gs = row_dot<DK>(G, Sp);    // <G_i, S_{t-1,i}>
+                const float ab = fmul(a, b);
+                const f2x ng = pk2(-fmul(ab, dlt), -fmul(ab, dlt));
+                float xq[RS::EPT], xk[RS::EPT];
+#pragma unroll
+                for (int m = 0; m < L; ++m) {
+                    const f2x st = ffma2(dd, kp[m], fmul2(aa, Sp[m]));                 // S_t
+                    const f2x gq = fmul2(oo, st);                                      // dO_i S_t
+                    const f2x gk = ffma2(ng, Sp[m], fmul2(dd, G[m]));                  // G delta - ab ddelta S_{t-1}
+                    up2(gq, xq[m], xq[L + m]);
+                    up2(gk, xk[m], xk[L + m]);
+                }
+                // this row's share -> the reduction buffers (natural column order)
+#pragma unroll
+                for (int e = 0; e < RS::EPT; e += 4) {
+                    *reinterpret_cast<float4*>(redq + row * Cf::RED + part * RS::EPT + e) =
+                        make_float4(xq[e], xq[e + 1], xq[e + 2], xq[e + 3]);
+                    *reinterpret_cast<float4*>(redk + row * Cf::RED + part * RS::EPT + e) =
+                        make_float4(xk[e], xk[e + 1], xk[e + 2], xk[e + 3]);
+                }
+                if (part == 0) {
+                    reds[2 * row] = fsub(gs, fmul(b, fmul(dlt, u)));       // dalpha term
+                    reds[2 * row + 1] = fmul(dlt, fsub(vi, fmul(a, u)));   // dbeta term
+                    dv[(((int64_t)seq0 + sb + t) * H + h) * DV + grow] = fmul(b, dlt);
+                }
+                // G <- alpha G - alpha beta ddelta k
+#pragma unroll
+                for (int m = 0; m < L; ++m) G[m] = ffma2(ng, kp[m], fmul2(aa, G[m]));
+                __syncthreads();
+                // the tile's row sums, rows in ascending order
+                const int64_t trow = ((int64_t)seq0 + sb + t) * H + h;
+                for (int col = tid; col < 2 * DK; col += blockDim.x) {
+                    const float* src = col < DK ? redq + col : redk + (col - DK);
+                    float s = src[0];
+                    for (int i = 1; i < RT; ++i) s = fadd(s, src[i * Cf::RED]);
+                    float* dst = col < DK ? pq : pk;
+                    dst[((int64_t)r * T_total * H + trow) * DK + (col % DK)] = s;
+                }
+                if (tid < 2) {
+                    float s = reds[tid];
+                    for (int i = 1; i < RT; ++i) s = fadd(s, reds[2 * i + tid]);
+                    (tid == 0 ? pa : pb)[(int64_t)r * T_total * H + trow] = s;
+                }
+                __syncthreads();
+            }
+        }
+    }
+    store_row_pairs<DK>(dstate + ((int64_t)nh * DV + grow) * DK + part * RS::EPT, G);
+}
+
+// dq, dk, dalpha, dbeta = the sum of the NT tiles' partials, tile 0 first.
+template <int DK, int NT>
+__global__ void k_bwd_reduce(const float* __restrict__ pq, const float* __restrict__ pk, const float* __restrict__ pa,
+                             const float* __restrict__ pb, const int32_t* __restrict__ err, int64_t TH,
+                             float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ da,
+                             float* __restrict__ db)
+{
+    if (__ldg(err)) return;
+    const int64_t nvec = TH * DK;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec + TH; i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nvec) {
+            float sq = pq[i], sk = pk[i];
+#pragma unroll
+            for (int r = 1; r < NT; ++r) {
+                sq = fadd(sq, pq[r * nvec + i]);
+                sk = fadd(sk, pk[r * nvec + i]);
+            }
+            dq[i] = sq;
+            dk[i] = sk;
+        } else {
+            const int64_t j = i - nvec;
+            float sa = pa[j], sb = pb[j];
+#pragma unroll
+            for (int r = 1; r < NT; ++r) {
+                sa = fadd(sa, pa[r * TH + j]);
+                sb = fadd(sb, pb[r * TH + j]);
+            }
+            da[j] = sa;
+            db[j] = sb;
+        }
+    }
+}
+
+}  // namespace gdn

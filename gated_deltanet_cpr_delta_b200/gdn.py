@@ -24,7 +24,8 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 #: exported symbols of include/gdn_cpr.h
 SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
            "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed",
-           "gdn_cpr_forward_noalloc", "gdn_contract_text", "gdn_contract_identity", "gdn_sha256_hex")
+           "gdn_cpr_forward_noalloc", "gdn_contract_text", "gdn_contract_identity", "gdn_sha256_hex",
+           "gdn_cpr_backward_workspace_size", "gdn_cpr_backward")
 
 #: gdn_identity_kind_t
 ID_SEMANTIC, ID_NUMERICAL_POLICY, ID_DEPLOYMENT = 0, 1, 2
@@ -84,6 +85,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_cpr_forward_noalloc.restype = ctypes.c_int
     lib.gdn_cpr_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
                                             ctypes.c_int, P, P, ctypes.POINTER(CacheStruct), P]
+    lib.gdn_cpr_backward_workspace_size.restype = sz
+    lib.gdn_cpr_backward_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+    lib.gdn_cpr_backward.restype = ctypes.c_int
+    lib.gdn_cpr_backward.argtypes = [P, P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
+                                     P, P, P, P, P, P, P, sz, P]
     _lib = lib
     return lib
 
@@ -220,6 +226,40 @@ def gdn_cpr_forward(q, k, v, alpha, beta, cu_seqlens, C: int, *, cu_seqlens_host
         st = lib.gdn_cpr_forward_timed(*args, _event_array(events, 6))
     _check(st, "gdn_cpr_forward")
     return o, chunk_states
+
+
+def gdn_cpr_backward_workspace_size(total_tokens: int, num_seqs: int, H: int, d_k: int, d_v: int, C: int) -> int:
+    return int(load_library().gdn_cpr_backward_workspace_size(total_tokens, num_seqs, H, d_k, d_v, C))
+
+
+def gdn_cpr_backward(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, C: int, *, cu_seqlens_host=None,
+                     workspace=None, grads=None):
+    """CPR backward: gradients of sum(dO * o) for the forward of the same inputs.
+
+    q, k, v, alpha, beta, cu_seqlens: as given to :func:`gdn_cpr_forward`;
+    dO [T,H,d_v] in q's dtype; chunk_states: that forward's chunk states.
+    Returns (dq, dk, dv, dalpha, dbeta, dstate_in), all fp32.  ``grads``: an
+    optional tuple of those six tensors to write into."""
+    lib = load_library()
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu().tolist()
+    cu_h = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    N = len(cu_seqlens_host) - 1
+    dev = k.device
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = (torch.empty(T, H, dk, **f32), torch.empty(T, H, dk, **f32), torch.empty(T, H, dv, **f32),
+                 torch.empty(T, H, **f32), torch.empty(T, H, **f32), torch.empty(N, H, dv, dk, **f32))
+    if workspace is None:
+        workspace = torch.empty(lib.gdn_cpr_backward_workspace_size(T, N, H, dk, dv, C), dtype=torch.uint8,
+                                device=dev)
+    st = lib.gdn_cpr_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(dO), _ptr(chunk_states),
+                              _ptr(cu_seqlens), cu_h, N, T, H, dk, dv, C, _dt(q.dtype),
+                              *[_ptr(g) for g in grads], _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(st, "gdn_cpr_backward")
+    return grads
 
 
 def gdn_decode_step(q, k, v, alpha, beta, cache: Dict[str, torch.Tensor], C: int, *, out_dtype=None, o=None,

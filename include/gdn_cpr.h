@@ -186,6 +186,49 @@ gdn_status_t gdn_cpr_forward(const void* q, const void* k, const void* v,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Device workspace, in bytes, that gdn_cpr_backward needs for a batch of
+ * total_tokens tokens in num_seqs sequences.  It holds the tables, the
+ * recomputation checkpoints (one state row tile per 8 tokens of a chunk for
+ * every (sequence, head, row tile)) and the per-row-tile partial sums of
+ * dq, dk, dalpha and dbeta.  Returns 0 for invalid sizes.
+ */
+size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H,
+                                       int32_t d_k, int32_t d_v, int32_t C);
+
+/*
+ * CPR backward (trainer): the gradients of L = sum_t dO_t . o_t for the layer
+ * of gdn_cpr_forward, with the gated delta rule
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t
+ * (IsoExec summary page, section "Chunkwise-Parallel Recurrent (CPR) Gated
+ * DeltaNet"; commentary blog, section 10), differentiated in reverse token
+ * order.  Per chunk, the states are recomputed from the boundary state the
+ * forward stored, with the forward's per-token arithmetic.
+ * Inputs:
+ *   q, k, v, alpha, beta, cu_seqlens, cu_seqlens_host, num_seqs, total_tokens,
+ *     H, d_k, d_v, C, in_dtype: as given to gdn_cpr_forward.
+ *   dO [T_total,H,d_v] in in_dtype: the gradient of the loss for o.
+ *   chunk_states: the forward's chunk_states output for these inputs.
+ * Outputs (fp32, device, caller-owned, every element written):
+ *   dq, dk [T_total,H,d_k]; dv [T_total,H,d_v]; dalpha, dbeta [T_total,H];
+ *   dstate_in [num_seqs,H,d_v,d_k]: the gradient for the forward's state_in.
+ * The result is deterministic: the row tiles' contributions are added in a
+ * fixed order, with no atomics.
+ *   workspace: at least gdn_cpr_backward_workspace_size(...) bytes of device
+ *     memory, 256-byte aligned, not shared with a concurrent call.
+ * Errors: as gdn_cpr_forward.  If the device copy of cu_seqlens disagrees
+ * with the host copy, the kernels write nothing.
+ */
+gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta, const void* dO,
+                              const float* chunk_states,
+                              const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                              int32_t num_seqs, int64_t total_tokens, int32_t H,
+                              int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
+                              float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
+                              float* dstate_in, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * One decode step: one new token for each of num_seqs sequences.
  *   q, k [num_seqs,H,d_k], v [num_seqs,H,d_v] in in_dtype; alpha, beta [num_seqs,H] fp32
  *   cache: updated in place (see gdn_cache_t).  For each (sequence, head):

@@ -92,3 +92,38 @@ def test_decode_rejects_bad_arguments(lib):
     cs2 = gdn.CacheStruct(*([1 << 20] * 6 + [0]))
     bad = dict(ok, cache=ctypes.byref(cs2))
     assert lib.gdn_decode_step(*bad.values()) == 1
+
+
+def _bwd(lib, **kw):
+    P = ctypes.c_void_p
+    cu = kw.get("cu", [0, 32])
+    cu_h = (ctypes.c_int32 * len(cu))(*cu)
+    fake = P(1 << 20)  # never dereferenced: validation fails first
+    args = dict(q=fake, k=fake, v=fake, alpha=fake, beta=fake, dO=fake, states=fake, cu=fake, cu_host=cu_h,
+                N=len(cu) - 1, T=cu[-1], H=2, dk=16, dv=16, C=16, idt=0, dq=fake, dk_=fake, dv_=fake, da=fake,
+                db=fake, ds=fake, ws=fake, wsb=1 << 30, stream=None)
+    args.update({k: v for k, v in kw.items() if k != "cu"})
+    return lib.gdn_cpr_backward(*args.values())
+
+
+def test_backward_rejects_bad_arguments(lib):
+    assert _bwd(lib, dk=24, dv=24) == 2                  # unsupported head dim
+    assert _bwd(lib, C=48) == 2                          # unsupported chunk
+    assert _bwd(lib, idt=7) == 1                         # bad dtype
+    assert _bwd(lib, cu=[0, 40, 32], T=32) == 1          # decreasing cu_seqlens
+    assert _bwd(lib, cu=[0, 32], T=33) == 1              # total mismatch
+    assert _bwd(lib, dO=ctypes.c_void_p((1 << 20) + 4)) == 1   # misaligned
+    assert _bwd(lib, states=None) == 1
+    assert _bwd(lib, ds=None) == 1
+    assert _bwd(lib, dq=None) == 1
+    assert _bwd(lib, wsb=16) == 4                        # workspace too small
+    assert _bwd(lib, ws=None) == 4
+    assert _bwd(lib, H=0) == 1
+
+
+def test_backward_workspace_size_grows_with_tokens():
+    a = gdn.gdn_cpr_backward_workspace_size(1024, 2, 4, 128, 128, 64)
+    b = gdn.gdn_cpr_backward_workspace_size(2048, 2, 4, 128, 128, 64)
+    # at least the per-tile partial sums of dq and dk for the extra tokens
+    assert b - a >= 1024 * 4 * 4 * 128 * 4 * 2
+    assert gdn.gdn_cpr_backward_workspace_size(-1, 2, 4, 64, 64, 16) == 0
