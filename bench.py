@@ -7,8 +7,9 @@ precompute, boundary chain, intra-chunk recurrence, output store) of the
 prefill workload, B=4 sequences x T=4096 tokens, H=16 heads, d_k=d_v=128,
 C=64, bf16 q/k/v, fp32 gates and state.  Inputs are synthetic, from the
 device recipe of gated_deltanet_cpr_delta_b200.synth.  The line also
-reports decode tokens/s for the decode workload: 64 sequences x 32 heads,
-prefilled to 2048 tokens, then 256 decode steps.
+reports decode tokens/s for the decode workload (64 sequences x 32 heads,
+prefilled to 2048 tokens, then 256 decode steps) and trainer fwd+bwd tokens/s
+(B=2 x 8192 tokens, 32 heads, forward then gdn_cpr_backward).
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own sequences
 (weak scaling, no data-path collective).  Timing is CUDA events on the
@@ -38,6 +39,8 @@ UNIT = "tokens/s"
 WORKLOAD = dict(name="prefill B=4 H=16 T=4096 d_k=d_v=128 C=64 bf16", seed=1, B=4, H=16, T=4096, D=128, C=64)
 DECODE = dict(name="decode 64 seqs H=32 d=128 C=64: prefill 2048, then 256 steps", seed=2, N=64, H=32, D=128,
               C=64, Lp=2048, steps=256)
+TRAIN = dict(name="trainer fwd+bwd B=2 H=32 T=8192 d_k=d_v=128 C=64 bf16, dO ~ N(0,1) bf16", seed=4, B=2, H=32,
+             T=8192, D=128, C=64)
 
 # FP32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (fma) x 1.965 GHz (max SM clock)
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -66,6 +69,14 @@ def forward_flops(tokens_heads: int, full_tokens_heads: int, dk: int, dv: int, C
 # the buffer (k, v, alpha, beta), gates and position.
 def decode_tok_bytes(dk: int, dv: int, esz: int, out_esz: int):
     return 8 * dk * dv + (2 * dk + dv) * esz + dv * out_esz + (dk + dv) * esz + 8 + 8 + 8
+
+
+# Algorithmic work of the backward per (token, head), fma = 2 flops: the state
+# recompute (u = S k, S <- alpha S + delta k^T: 3 dk*dv), G += dO q^T,
+# ddelta = G k, <G, S_{t-1}>, dq = S_t^T dO, dk = G^T delta - ab S^T ddelta
+# (2), G <- alpha G - ab ddelta k^T (2): 11 dk*dv fmas.
+def backward_flops(tokens_heads: int, dk: int, dv: int):
+    return 22 * dk * dv * tokens_heads
 
 
 # DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
@@ -342,6 +353,60 @@ def bench_decode(rank: int, world: int, warmup: int):
                          "bytes_per_launch": tb}}
 
 
+def bench_trainer(rank: int, world: int, warmup: int, steps: int):
+    """Trainer step: CPR forward + backward (gdn_cpr_backward) of the trainer
+    workload on this rank's sequences; L2 flushed before every timed step."""
+    import torch
+    from gated_deltanet_cpr_delta_b200 import gdn, synth
+    Tr = TRAIN
+    B, H, T, D, C = Tr["B"], Tr["H"], Tr["T"], Tr["D"], Tr["C"]
+    d = synth.make_batch_device(Tr["seed"], [T] * B, H, D, D, "bf16", seq_ids=rank_sequence_ids(rank, B))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(Tr["seed"] * 1_000_003 + 999 + rank)
+    dO = torch.randn(B * T, H, D, device="cuda", generator=g).to(torch.bfloat16)
+    o = torch.empty(B * T, H, D, dtype=torch.bfloat16, device="cuda")
+    st = torch.empty(gdn.gdn_num_chunk_states(d["cu_host"], C), H, D, D, dtype=torch.float32, device="cuda")
+    ws = torch.empty(gdn.gdn_cpr_workspace_size(B * T, B, H, D, D, C), dtype=torch.uint8, device="cuda")
+    wsb = torch.empty(gdn.gdn_cpr_backward_workspace_size(B * T, B, H, D, D, C), dtype=torch.uint8, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    grads = (torch.empty(B * T, H, D, **f32), torch.empty(B * T, H, D, **f32), torch.empty(B * T, H, D, **f32),
+             torch.empty(B * T, H, **f32), torch.empty(B * T, H, **f32), torch.empty(B, H, D, D, **f32))
+
+    def step(fe=None, be=None):
+        gdn.gdn_cpr_forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["cu_seqlens"], C,
+                            cu_seqlens_host=d["cu_host"], o=o, chunk_states=st, workspace=ws, events=fe)
+        gdn.gdn_cpr_backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], dO, st, d["cu_seqlens"], C,
+                             cu_seqlens_host=d["cu_host"], workspace=wsb, grads=grads, events=be)
+
+    for _ in range(max(warmup, 3)):
+        step()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for e in fev + bev:
+        for x in e:
+            x.record()
+    barrier(world)
+    for s in range(steps):
+        flush.zero_()
+        step(fev[s], bev[s])
+    barrier(world)
+    fwd_ms = [e[0].elapsed_time(e[5]) for e in fev]
+    bwd_ms = [e[0].elapsed_time(e[3]) for e in bev]
+    tot = max_over_ranks(sum(f + b for f, b in zip(fwd_ms, bwd_ms)), world)
+    kern = {n: sum(e[i].elapsed_time(e[i + 1]) for e in bev) / steps
+            for i, n in enumerate(("k_tables + k_bwd_scan", "k_bwd_chunk", "k_bwd_reduce"))}
+    fl = backward_flops(B * T * H, D, D)
+    tf = fl / (kern["k_bwd_chunk"] / 1e3) / 1e12
+    return {"workload": Tr["name"], "value": B * T * world / (tot / steps / 1e3), "unit": UNIT,
+            "ms_per_step": tot / steps, "fwd_ms": sum(fwd_ms) / steps, "bwd_ms": sum(bwd_ms) / steps,
+            "bwd_kernels_ms": kern,
+            "roofline": {"kernel": "k_bwd_chunk (per-chunk backward)", "bound": "alu", "achieved": tf,
+                         "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tf / FP32_PEAK_TFLOPS,
+                         "traffic": None, "flops_per_launch": fl,
+                         "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}}
+
+
 def run_native(args):
     import torch
     from gated_deltanet_cpr_delta_b200 import gdn, synth
@@ -449,6 +514,7 @@ def run_native(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / K
 
     dec = bench_decode(rank, world, args.warmup) if not args.no_decode else None
+    trainer = bench_trainer(rank, world, args.warmup, min(K, 5)) if not args.no_trainer else None
 
     peaks, peak_src = load_peaks()
     flops = forward_flops(B * T * H, B * (T // C) * C * H, D, D, C)
@@ -493,6 +559,7 @@ def run_native(args):
         "clocks": clocks.summary(),
         "parity": parity,
         "decode": dec,
+        "trainer": trainer,
         "peaks": {"hbm_gbs": peaks.get("hbm_gbs"), "source": peak_src},
         "kernel_source_sha": sha,
         "contract": {"id": gdn.gdn_contract_id(),
@@ -520,6 +587,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-trainer", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

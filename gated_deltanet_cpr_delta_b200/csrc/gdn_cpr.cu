@@ -272,19 +272,23 @@ gdn_status_t launch_decode(const DecArgs& a)
     return GDN_OK;
 }
 
-// Backward workspace: [err | cto | fco | so | ...] as the forward's tables,
-// then the checkpoints of every (sequence, head, row tile) CTA and the
-// per-tile partial sums of dq, dk (fp32 [NT][T][H][d_k]) and dalpha, dbeta.
+// Backward workspace: the forward's tables (err, cto, fco, so, ...), then the
+// boundary adjoints Y_c (one d_v x d_k state per chunk-state slot), the
+// checkpoints of the resident CTAs of k_bwd_chunk (at most kBwdMaxCtas), and
+// the per-row-tile partial sums of dq, dk (fp32 [NT][T][H][d_k]) and
+// dalpha, dbeta ([NT][T][H]).
+constexpr int64_t kBwdMaxCtas = 148 * 8;
+
 struct BwdWorkspace {
-    Workspace t;  // tables only (err, tok_next, cto, fco, so, ...)
-    float *scratch, *pq, *pk, *pa, *pb;
+    Workspace t;  // tables only
+    float *ybuf, *scratch, *pq, *pk, *pa, *pb;
     size_t bytes;
 };
 
 BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C)
 {
     BwdWorkspace w{};
-    const int32_t RT = dv < 32 ? dv : 32, NT = dv / RT, SUB = C < 8 ? C : 8;
+    const int32_t RT = dv < 32 ? dv : 32, NT = dv / RT, SUB = C < 8 ? C : 8;  // as gdn::BwdCfg
     const Workspace tables = carve(nullptr, 0, N, H, dk, dv, C);  // the tables part alone
     size_t off = tables.bytes;
     auto take = [&](size_t n) {
@@ -292,7 +296,11 @@ BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, 
         off = align_up(off + n);
         return o;
     };
-    const size_t o_sc = take(sizeof(float) * (size_t)N * H * NT * (C / SUB) * RT * dk);
+    const int64_t max_states = T / C + N;           // >= sum_n (floor(L_n / C) + 1)
+    const int64_t ntasks = (T / C + N) * H * NT;    // >= chunk tasks x heads x row tiles
+    const int64_t ctas = std::min<int64_t>(std::max<int64_t>(ntasks, 1), kBwdMaxCtas);
+    const size_t o_y = take(sizeof(float) * (size_t)max_states * H * dv * dk);
+    const size_t o_sc = take(sizeof(float) * (size_t)ctas * (C / SUB) * RT * dk);
     const size_t o_pq = take(sizeof(float) * (size_t)NT * T * H * dk);
     const size_t o_pk = take(sizeof(float) * (size_t)NT * T * H * dk);
     const size_t o_pa = take(sizeof(float) * (size_t)NT * T * H);
@@ -301,6 +309,7 @@ BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, 
     char* b = static_cast<char*>(base);
     if (b != nullptr) {
         w.t = carve(base, 0, N, H, dk, dv, C);
+        w.ybuf = reinterpret_cast<float*>(b + o_y);
         w.scratch = reinterpret_cast<float*>(b + o_sc);
         w.pq = reinterpret_cast<float*>(b + o_pq);
         w.pk = reinterpret_cast<float*>(b + o_pk);
@@ -321,21 +330,40 @@ struct BwdArgs {
     int64_t T_total;
     BwdWorkspace ws;
     cudaStream_t stream;
+    void* const* events;  // optional: 4 events around the kernels
 };
 
 template <int D, int C>
 gdn_status_t launch_backward(const BwdArgs& a)
 {
     using BC = gdn::BwdCfg<D, D, C>;
+    using SC = gdn::ScanCfg<D, D, C>;
+    mark(a.events, 0, a.stream);
     gdn::k_tables<<<1, 1024, 0, a.stream>>>(a.cu, a.N, C, a.T_total, a.tot.tasks, a.tot.full, a.tot.states,
                                              a.tot.hash, a.ws.t.cto, a.ws.t.fco, a.ws.t.so, a.ws.t.err, nullptr,
                                              nullptr, 0, nullptr, nullptr, 0);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-    if (set_smem(gdn::k_bwd_rows<D, D, C>, BC::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
-    gdn::k_bwd_rows<D, D, C><<<(unsigned)((int64_t)a.N * a.H * BC::NT), BC::THREADS, BC::SMEM, a.stream>>>(
-        a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.cu, a.ws.t.so, a.ws.t.err, a.N, a.H, a.T_total,
-        a.in_bf16, a.dv, a.dstate, a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.scratch);
+    if (set_smem(gdn::k_bwd_scan<D, D, C>, SC::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
+    gdn::k_bwd_scan<D, D, C><<<(unsigned)((int64_t)a.N * a.H * SC::NT), SC::THREADS, SC::SMEM, a.stream>>>(
+        a.q, a.k, a.alpha, a.beta, a.dO, a.cu, a.ws.t.so, a.ws.t.err, a.H, a.in_bf16, a.ws.ybuf, a.dstate);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    mark(a.events, 1, a.stream);
+    const int64_t ntasks = a.tot.tasks * a.H * BC::NT;
+    if (ntasks > 0) {
+        if (set_smem(gdn::k_bwd_chunk<D, D, C>, BC::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
+        int dev = 0, sms = 0, occ = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gdn::k_bwd_chunk<D, D, C>, BC::THREADS, BC::SMEM) !=
+                cudaSuccess)
+            return GDN_ERR_CUDA;
+        const int64_t grid = std::min<int64_t>({ntasks, (int64_t)sms * std::max(occ, 1), kBwdMaxCtas});
+        gdn::k_bwd_chunk<D, D, C><<<(unsigned)grid, BC::THREADS, BC::SMEM, a.stream>>>(
+            a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.ws.ybuf, a.cu, a.ws.t.cto, a.ws.t.so, a.ws.t.err, a.N,
+            a.H, a.T_total, ntasks, a.in_bf16, a.dv, a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.scratch);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    mark(a.events, 2, a.stream);
     const int64_t TH = a.T_total * a.H;
     if (TH > 0) {
         const unsigned grid = (unsigned)std::min<int64_t>((TH * (D + 1) + 255) / 256, 148 * 16);
@@ -343,6 +371,7 @@ gdn_status_t launch_backward(const BwdArgs& a)
                                                                a.dq, a.dk, a.dalpha, a.dbeta);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
+    mark(a.events, 3, a.stream);
     return GDN_OK;
 }
 
@@ -462,12 +491,13 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
     return carve_bwd(nullptr, total_tokens, num_seqs, H, d_k, d_v, C).bytes;
 }
 
-gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const float* alpha, const float* beta,
-                              const void* dO, const float* chunk_states, const int32_t* cu_seqlens,
-                              const int32_t* cu_seqlens_host, int32_t num_seqs, int64_t total_tokens, int32_t H,
-                              int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype, float* dq, float* dk,
-                              float* dv, float* dalpha, float* dbeta, float* dstate_in, void* workspace,
-                              size_t workspace_bytes, void* stream)
+gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v, const float* alpha,
+                                    const float* beta, const void* dO, const float* chunk_states,
+                                    const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int32_t num_seqs,
+                                    int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v, int32_t C,
+                                    gdn_dtype_t in_dtype, float* dq, float* dk, float* dv, float* dalpha,
+                                    float* dbeta, float* dstate_in, void* workspace, size_t workspace_bytes,
+                                    void* stream, void* const* events)
 {
     if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0)
         return GDN_ERR_INVALID_ARG;
@@ -487,7 +517,10 @@ gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const
     const BwdWorkspace need = carve_bwd(nullptr, total_tokens, num_seqs, H, d_k, d_v, C);
     if (workspace == nullptr || workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return GDN_ERR_INVALID_ARG;
-    if (num_seqs == 0) return GDN_OK;
+    if (num_seqs == 0) {
+        for (int i = 0; i < 4; ++i) mark(events, i, static_cast<cudaStream_t>(stream));
+        return GDN_OK;
+    }
     BwdArgs a;
     a.q = q; a.k = k; a.v = v; a.dO = dO; a.alpha = alpha; a.beta = beta; a.states = chunk_states;
     a.cu = cu_seqlens; a.N = num_seqs; a.H = H; a.in_bf16 = in_dtype == GDN_BF16;
@@ -495,7 +528,20 @@ gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const
     a.tot = tot; a.T_total = total_tokens;
     a.ws = carve_bwd(workspace, total_tokens, num_seqs, H, d_k, d_v, C);
     a.stream = static_cast<cudaStream_t>(stream);
+    a.events = events;
     GDN_DISPATCH(launch_backward, d_k, C, a)
+}
+
+gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const float* alpha, const float* beta,
+                              const void* dO, const float* chunk_states, const int32_t* cu_seqlens,
+                              const int32_t* cu_seqlens_host, int32_t num_seqs, int64_t total_tokens, int32_t H,
+                              int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype, float* dq, float* dk,
+                              float* dv, float* dalpha, float* dbeta, float* dstate_in, void* workspace,
+                              size_t workspace_bytes, void* stream)
+{
+    return gdn_cpr_backward_timed(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, cu_seqlens_host, num_seqs,
+                                  total_tokens, H, d_k, d_v, C, in_dtype, dq, dk, dv, dalpha, dbeta, dstate_in,
+                                  workspace, workspace_bytes, stream, nullptr);
 }
 
 gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, const float* alpha,

@@ -13,15 +13,16 @@
 //     dk_t     = G^T delta - alpha_t beta_t S_{t-1}^T ddelta
 //     G       <- alpha_t G - alpha_t beta_t ddelta k_t^T      (= dL/dS_{t-1})
 //
-// Every row i of S and G evolves on its own; only dq, dk, dalpha and dbeta sum
-// over rows.  k_bwd_rows runs one (sequence, head, tile of RT rows) per CTA,
-// serial over the sequence from its last token back: per chunk (from the
-// forward's boundary state) it recomputes the states with the forward's P_tok
-// arithmetic, keeping one checkpoint per SUB tokens (global scratch, L2
-// resident), and for each token recomputes S_{t-1} from the nearest
-// checkpoint.  The tile's row sums of the dq / dk / dalpha / dbeta terms go to
-// per-tile partial buffers; k_bwd_reduce adds the tiles in a fixed order, so
-// the gradients are deterministic.  Everything is fp32.
+// The backward keeps the forward's CPR split.  The G recursion does not need
+// the forward states, so one light serial pass (k_bwd_scan) carries G from
+// the last token to the first and stores it at every chunk boundary.  Then
+// every chunk is independent: k_bwd_chunk starts from the boundary G after the
+// chunk, recomputes the chunk's states from the forward's boundary state
+// (one checkpoint per SUB tokens, kept in an L2-resident per-CTA scratch) and
+// runs the per-token backward above.  Every row i of S and G evolves on its
+// own, so both kernels split d_v into row tiles; dq, dk, dalpha and dbeta sum
+// over rows, and the tiles' sums are added in a fixed order by k_bwd_reduce,
+// so the gradients are deterministic.  Everything is fp32.
 #pragma once
 
 #include "k_ptok.cuh"
@@ -103,17 +104,203 @@ __device__ __forceinline__ void load_pairs_slot(f2x (&p)[DK / kLeaves], const fl
     }
 }
 
-// Backward of one (sequence, head, row tile).  Outputs: dv rows (direct),
-// dstate_in rows (direct), and the tile's partial sums of dq, dk (per token,
-// [NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).
+// Serial pass over one (sequence, head, row tile): G from the last token to
+// the first, without the gradient outputs.  After the chunk starting at token
+// c*C it holds Y_c = dL/dS(c*C) through the tokens >= c*C; Y_c (c >= 1) goes
+// to ybuf at the chunk-state slot so[n] + c, Y_0 = dL/dstate_in to dstate.
+// Tokens are staged raw (bf16 or fp32) by cp.async in blocks of BLK, NBUF
+// blocks in flight; each lane widens its own slice.  The lane's EPT columns
+// are held as pairs of adjacent columns.  (Widening a bf16 block once into an
+// fp32 buffer measured slower: the extra pass and barrier sit on the serial
+// path.)
+template <int DK, int DV, int C>
+struct ScanCfg {
+    static constexpr int RT = DV < 32 ? DV : 32;
+    static constexpr int NT = DV / RT;
+    static constexpr int TPR = 4;
+    static constexpr int EPT = DK / TPR;
+    static constexpr int NP = EPT / 2;
+    static constexpr int THREADS = RT * TPR;
+    static constexpr int BLK = 16;
+    static constexpr int NBUF = 3;
+    static_assert(C % BLK == 0, "chunks are whole blocks");
+    template <int ES>
+    struct L {
+        static constexpr int PAD = EPT * ES >= 16 ? 16 : 0;   // keeps the 4 lanes' slices in distinct banks
+        static constexpr int PSB = EPT * ES + PAD;            // bytes between the lanes' slices
+        static constexpr int ROWB = TPR * PSB;                // one q or k row
+        static constexpr int DOB = RT * ES;                   // this tile's dO row
+        static constexpr int GOFF = 2 * ROWB + DOB;           // alpha, beta
+        static constexpr int TOKB = (GOFF + 8 + 15) / 16 * 16;
+        static constexpr int STAGE = BLK * TOKB;
+    };
+    static constexpr size_t SMEM = (size_t)NBUF * L<4>::STAGE;
+};
+
+template <int ES, int NP>
+__device__ __forceinline__ void widen_pairs(f2x (&p)[NP], const unsigned char* s)
+{
+    if constexpr (ES == 2) {
+        static_assert(NP % 2 == 0, "");
+#pragma unroll
+        for (int m = 0; m < NP; m += 2) {
+            const uint2 w = *reinterpret_cast<const uint2*>(s + 2 * 2 * m);
+            p[m] = pk2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+            p[m + 1] = pk2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < NP; m += 2) {
+            const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(s + 4 * 2 * m);
+            p[m] = x.x;
+            p[m + 1] = x.y;
+        }
+    }
+}
+
+template <int DK, int DV, int C, int ES>
+__device__ __forceinline__ void bwd_scan_body(const void* q, const void* k, const float* alpha, const float* beta,
+                                              const void* dO, int seq0, int Ln, int64_t slot0, int h, int H, int r,
+                                              float* ybuf, float* dstate_row, unsigned char* sm)
+{
+    using Cf = ScanCfg<DK, DV, C>;
+    using Lt = typename Cf::template L<ES>;
+    constexpr int NP = Cf::NP, EPT = Cf::EPT, RT = Cf::RT, BLK = Cf::BLK, NBUF = Cf::NBUF;
+    constexpr int QCH = DK * ES / 16;  // 16-byte pieces of a q / k row
+    constexpr int DCH = RT * ES / 16;  // of this tile's dO row
+    const int tid = threadIdx.x;
+    const int row = tid / Cf::TPR, part = tid % Cf::TPR;
+    const int grow = r * RT + row;
+    const char* qb = static_cast<const char*>(q);
+    const char* kb = static_cast<const char*>(k);
+    const char* db = static_cast<const char*>(dO);
+    const int nblk = (Ln + BLK - 1) / BLK;
+
+    auto issue = [&](int i) {
+        if (i < nblk) {
+            unsigned char* st = sm + (i % NBUF) * Lt::STAGE;
+            const int t0 = (nblk - 1 - i) * BLK, len = min(BLK, Ln - t0);
+            for (int e = tid; e < len * (2 * QCH + DCH + 2); e += blockDim.x) {
+                const int t = e / (2 * QCH + DCH + 2), w = e % (2 * QCH + DCH + 2);
+                const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+                unsigned char* d = st + t * Lt::TOKB;
+                if (w < 2 * QCH) {
+                    const int j = w % QCH;
+                    const int byte = j * 16;
+                    const int dst = Lt::PAD ? (byte / (EPT * ES)) * Lt::PSB + byte % (EPT * ES) : byte;
+                    cp_async16(d + (w < QCH ? 0 : Lt::ROWB) + dst, (w < QCH ? qb : kb) + trow * DK * ES + byte);
+                } else if (w < 2 * QCH + DCH) {
+                    const int j = w - 2 * QCH;
+                    cp_async16(d + 2 * Lt::ROWB + j * 16, db + (trow * DV + r * RT) * ES + j * 16);
+                } else {
+                    cp_async4(d + Lt::GOFF + 4 * (w - 2 * QCH - DCH), (w == 2 * QCH + DCH ? alpha : beta) + trow);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+
+    f2x G[NP];
+#pragma unroll
+    for (int m = 0; m < NP; ++m) G[m] = pk2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < NBUF - 1; ++i) issue(i);
+    for (int i = 0; i < nblk; ++i) {
+        cp_async_wait_n<NBUF - 2>();
+        __syncthreads();
+        issue(i + NBUF - 1);
+        const unsigned char* st = sm + (i % NBUF) * Lt::STAGE;
+        const int t0 = (nblk - 1 - i) * BLK, len = min(BLK, Ln - t0);
+        for (int t = len - 1; t >= 0; --t) {
+            const unsigned char* tk = st + t * Lt::TOKB;
+            f2x qp[NP], kp[NP];
+            widen_pairs<ES, NP>(qp, tk + part * Lt::PSB);
+            widen_pairs<ES, NP>(kp, tk + Lt::ROWB + part * Lt::PSB);
+            float doi;
+            if constexpr (ES == 2)
+                doi = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(tk + 2 * Lt::ROWB)[row] << 16);
+            else
+                doi = reinterpret_cast<const float*>(tk + 2 * Lt::ROWB)[row];
+            const float a = *reinterpret_cast<const float*>(tk + Lt::GOFF);
+            const float b = *reinterpret_cast<const float*>(tk + Lt::GOFF + 4);
+            const f2x oo = pk2(doi, doi);
+#pragma unroll
+            for (int m = 0; m < NP; ++m) G[m] = ffma2(oo, qp[m], G[m]);
+            f2x acc0 = fmul2(G[0], kp[0]), acc1 = fmul2(G[1], kp[1]);
+#pragma unroll
+            for (int m = 2; m < NP; m += 2) {
+                acc0 = ffma2(G[m], kp[m], acc0);
+                acc1 = ffma2(G[m + 1], kp[m + 1], acc1);
+            }
+            float l0, l1, l2, l3;
+            up2(acc0, l0, l1);
+            up2(acc1, l2, l3);
+            const float dlt = tree_4lanes(fadd(l0, l2), fadd(l1, l3));
+            const float ng = -fmul(fmul(a, b), dlt);
+            const f2x aa = pk2(a, a), nn = pk2(ng, ng);
+#pragma unroll
+            for (int m = 0; m < NP; ++m) G[m] = ffma2(nn, kp[m], fmul2(aa, G[m]));
+            const int tg = t0 + t;
+            if (tg % C == 0) {
+                float* dst = tg == 0 ? dstate_row : ybuf + (((slot0 + tg / C) * H + h) * DV + grow) * (int64_t)DK;
+#pragma unroll
+                for (int m = 0; m < NP; m += 2) {
+                    float x0, x1, x2, x3;
+                    up2(G[m], x0, x1);
+                    up2(G[m + 1], x2, x3);
+                    *reinterpret_cast<float4*>(dst + part * EPT + 2 * m) = make_float4(x0, x1, x2, x3);
+                }
+            }
+        }
+    }
+    cp_async_wait_all();
+    if (Ln == 0) {  // no tokens: dL/dstate_in = 0
+#pragma unroll
+        for (int m = 0; m < NP; m += 2)
+            *reinterpret_cast<float4*>(dstate_row + part * EPT + 2 * m) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(ScanCfg<DK, DV, C>::THREADS)
+k_bwd_scan(const void* __restrict__ q, const void* __restrict__ k, const float* __restrict__ alpha,
+           const float* __restrict__ beta, const void* __restrict__ dO, const int32_t* __restrict__ cu,
+           const int32_t* __restrict__ so, const int32_t* __restrict__ err, int H, int in_bf16,
+           float* __restrict__ ybuf, float* __restrict__ dstate)
+{
+    using Cf = ScanCfg<DK, DV, C>;
+    if (__ldg(err)) return;
+    extern __shared__ float4 smem_f4[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(smem_f4);
+    const int r = blockIdx.x % Cf::NT;
+    const int nh = blockIdx.x / Cf::NT;
+    const int h = nh % H, n = nh / H;
+    const int seq0 = __ldg(cu + n);
+    const int Ln = __ldg(cu + n + 1) - seq0;
+    const int64_t slot0 = __ldg(so + n);
+    const int row = threadIdx.x / Cf::TPR;
+    float* dstate_row = dstate + ((int64_t)nh * DV + r * Cf::RT + row) * DK;
+    if (in_bf16)
+        bwd_scan_body<DK, DV, C, 2>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, ybuf, dstate_row, sm);
+    else
+        bwd_scan_body<DK, DV, C, 4>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, ybuf, dstate_row, sm);
+}
+
+// Backward of the chunks: one (chunk, head, row tile) task at a time, CTAs
+// looping over the tasks (a persistent grid, so that the checkpoint scratch
+// is per resident CTA and stays in L2).  A task starts from G = Y_{c+1}
+// (zero after the last chunk), recomputes the chunk's states from its
+// boundary state and writes dv rows, and the tile's row sums of dq, dk
+// ([NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(BwdCfg<DK, DV, C>::THREADS)
-k_bwd_rows(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
-           const float* __restrict__ alpha, const float* __restrict__ beta, const void* __restrict__ dO,
-           const float* __restrict__ states, const int32_t* __restrict__ cu, const int32_t* __restrict__ so,
-           const int32_t* __restrict__ err, int N, int H, int64_t T_total, int in_bf16,
-           float* __restrict__ dv, float* __restrict__ dstate, float* __restrict__ pq, float* __restrict__ pk,
-           float* __restrict__ pa, float* __restrict__ pb, float* __restrict__ scratch)
+k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+            const float* __restrict__ alpha, const float* __restrict__ beta, const void* __restrict__ dO,
+            const float* __restrict__ states, const float* __restrict__ ybuf, const int32_t* __restrict__ cu,
+            const int32_t* __restrict__ cto, const int32_t* __restrict__ so, const int32_t* __restrict__ err,
+            int N, int H, int64_t T_total, int64_t ntasks, int in_bf16, float* __restrict__ dv,
+            float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pa, float* __restrict__ pb,
+            float* __restrict__ scratch)
 {
     using Cf = BwdCfg<DK, DV, C>;
     using RS = typename Cf::RS;
@@ -125,62 +312,70 @@ k_bwd_rows(const void* __restrict__ q, const void* __restrict__ k, const void* _
     float* redq = sm + Cf::RQ_OFF;
     float* redk = sm + Cf::RK_OFF;
     float* reds = sm + Cf::RS_OFF;
-
-    const int r = blockIdx.x % NT;
-    const int nh = blockIdx.x / NT;
-    const int h = nh % H, n = nh / H;
     const int tid = threadIdx.x;
     const int row = tid / RS::TPR, part = tid % RS::TPR;
-    const int grow = r * RT + row;
-    const int seq0 = __ldg(cu + n);
-    const int Ln = __ldg(cu + n + 1) - seq0;
-    const int64_t slot0 = __ldg(so + n);
     float* ck = scratch + (int64_t)blockIdx.x * Cf::SCRATCH;  // this CTA's checkpoints
 
-    // stage tokens [t0, t0 + len) of the sequence: k, q into the slot layout,
-    // this tile's v and dO rows, the gates
-    auto stage = [&](int t0, int len) {
-        constexpr int G8 = (2 * DK) / 8;
-        for (int e = tid; e < len * G8; e += blockDim.x) {
-            const int t = e / G8, el = (e % G8) * 8;
-            float x[8];
-            const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
-            load8(el < DK ? k : q, trow * DK + (el % DK), in_bf16, x);
-            float* d = tok + t * TOKF + (el >= DK ? KS : 0);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) d[RS::slot((el % DK) + m)] = x[m];
-        }
-        for (int e = tid; e < len * (2 * RT / 8); e += blockDim.x) {
-            const int t = e / (2 * RT / 8), el = (e % (2 * RT / 8)) * 8;
-            float x[8];
-            const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
-            load8(el < RT ? v : dO, trow * DV + r * RT + (el % RT), in_bf16, x);
-            float* d = tok + t * TOKF + 2 * KS + (el >= RT ? RT : 0) + (el % RT);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) d[m] = x[m];
-        }
-        for (int t = tid; t < len; t += blockDim.x) {
-            const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
-            tok[t * TOKF + 2 * KS + 2 * RT] = __ldg(alpha + trow);
-            tok[t * TOKF + 2 * KS + 2 * RT + 1] = __ldg(beta + trow);
-        }
-    };
-    auto step = [&](f2x (&Sp)[L], int t) {  // forward step with staged token t
-        const float* tt = tok + t * TOKF;
-        float d;
-        ptok_advance<DK>(Sp, tt + part * RS::PS, tt[2 * KS + row], tt[2 * KS + 2 * RT], tt[2 * KS + 2 * RT + 1], &d);
-    };
+    for (int64_t task = blockIdx.x; task < ntasks; task += gridDim.x) {
+        const int r = (int)(task % NT);
+        const int h = (int)((task / NT) % H);
+        const int ct = (int)(task / ((int64_t)NT * H));
+        const int n = find_seq(cto, N, ct);
+        const int c = ct - __ldg(cto + n);
+        const int grow = r * RT + row;
+        const int seq0 = __ldg(cu + n);
+        const int Ln = __ldg(cu + n + 1) - seq0;
+        const int64_t slot0 = __ldg(so + n);
+        const int nchunks = (Ln + C - 1) / C;
 
-    f2x G[L];
+        // stage tokens [t0, t0 + len) of the sequence: k, q into the slot layout,
+        // this tile's v and dO rows, the gates
+        auto stage = [&](int t0, int len) {
+            constexpr int G8 = (2 * DK) / 8;
+            for (int e = tid; e < len * G8; e += blockDim.x) {
+                const int t = e / G8, el = (e % G8) * 8;
+                float x[8];
+                const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+                load8(el < DK ? k : q, trow * DK + (el % DK), in_bf16, x);
+                float* d = tok + t * TOKF + (el >= DK ? KS : 0);
 #pragma unroll
-    for (int m = 0; m < L; ++m) G[m] = pk2(0.f, 0.f);
-    const int nchunks = (Ln + C - 1) / C;
-    for (int c = nchunks - 1; c >= 0; --c) {
+                for (int m = 0; m < 8; ++m) d[RS::slot((el % DK) + m)] = x[m];
+            }
+            for (int e = tid; e < len * (2 * RT / 8); e += blockDim.x) {
+                const int t = e / (2 * RT / 8), el = (e % (2 * RT / 8)) * 8;
+                float x[8];
+                const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+                load8(el < RT ? v : dO, trow * DV + r * RT + (el % RT), in_bf16, x);
+                float* d = tok + t * TOKF + 2 * KS + (el >= RT ? RT : 0) + (el % RT);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) d[m] = x[m];
+            }
+            for (int t = tid; t < len; t += blockDim.x) {
+                const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
+                tok[t * TOKF + 2 * KS + 2 * RT] = __ldg(alpha + trow);
+                tok[t * TOKF + 2 * KS + 2 * RT + 1] = __ldg(beta + trow);
+            }
+        };
+        auto step = [&](f2x (&Sp)[L], int t) {  // forward step with staged token t
+            const float* tt = tok + t * TOKF;
+            float d;
+            ptok_advance<DK>(Sp, tt + part * RS::PS, tt[2 * KS + row], tt[2 * KS + 2 * RT], tt[2 * KS + 2 * RT + 1],
+                             &d);
+        };
+
+        f2x G[L];
+        if (c + 1 < nchunks) {
+            load_row_pairs<DK>(G, ybuf + (((slot0 + c + 1) * H + h) * DV + grow) * DK + part * RS::EPT);
+        } else {
+#pragma unroll
+            for (int m = 0; m < L; ++m) G[m] = pk2(0.f, 0.f);
+        }
+        const float* S0 = states + (((slot0 + c) * H + h) * DV + grow) * DK + part * RS::EPT;
         const int cb = c * C, clen = min(C, Ln - cb);
         const int nsub = (clen + SUB - 1) / SUB;
         // checkpoints: the state at cb + j*SUB, j = 1..nsub-1 (j = 0 is the chunk state)
         f2x Sp[L];
-        load_row_pairs<DK>(Sp, states + (((slot0 + c) * H + h) * DV + grow) * DK + part * RS::EPT);
+        load_row_pairs<DK>(Sp, S0);
         for (int j = 1; j < nsub; ++j) {
             __syncthreads();
             stage(cb + (j - 1) * SUB, SUB);
@@ -196,7 +391,7 @@ k_bwd_rows(const void* __restrict__ q, const void* __restrict__ k, const void* _
             __syncthreads();
             for (int t = slen - 1; t >= 0; --t) {
                 // S_{t-1}: from the sub-chunk's checkpoint, forward over its first t tokens
-                if (j == 0) load_row_pairs<DK>(Sp, states + (((slot0 + c) * H + h) * DV + grow) * DK + part * RS::EPT);
+                if (j == 0) load_row_pairs<DK>(Sp, S0);
                 else load_row_pairs<DK>(Sp, ck + ((int64_t)(j - 1) * RT + row) * DK + part * RS::EPT);
                 for (int m = 0; m < t; ++m) step(Sp, m);
                 const float* tt = tok + t * TOKF;
@@ -259,7 +454,6 @@ k_bwd_rows(const void* __restrict__ q, const void* __restrict__ k, const void* _
             }
         }
     }
-    store_row_pairs<DK>(dstate + ((int64_t)nh * DV + grow) * DK + part * RS::EPT, G);
 }
 
 // dq, dk, dalpha, dbeta = the sum of the NT tiles' partials, tile 0 first.

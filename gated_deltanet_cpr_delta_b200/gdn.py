@@ -25,7 +25,7 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
            "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed",
            "gdn_cpr_forward_noalloc", "gdn_contract_text", "gdn_contract_identity", "gdn_sha256_hex",
-           "gdn_cpr_backward_workspace_size", "gdn_cpr_backward")
+           "gdn_cpr_backward_workspace_size", "gdn_cpr_backward", "gdn_cpr_backward_timed")
 
 #: gdn_identity_kind_t
 ID_SEMANTIC, ID_NUMERICAL_POLICY, ID_DEPLOYMENT = 0, 1, 2
@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_cpr_backward.restype = ctypes.c_int
     lib.gdn_cpr_backward.argtypes = [P, P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
                                      P, P, P, P, P, P, P, sz, P]
+    lib.gdn_cpr_backward_timed.restype = ctypes.c_int
+    lib.gdn_cpr_backward_timed.argtypes = lib.gdn_cpr_backward.argtypes + [P]
     _lib = lib
     return lib
 
@@ -233,13 +235,14 @@ def gdn_cpr_backward_workspace_size(total_tokens: int, num_seqs: int, H: int, d_
 
 
 def gdn_cpr_backward(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, C: int, *, cu_seqlens_host=None,
-                     workspace=None, grads=None):
+                     workspace=None, grads=None, events=None):
     """CPR backward: gradients of sum(dO * o) for the forward of the same inputs.
 
     q, k, v, alpha, beta, cu_seqlens: as given to :func:`gdn_cpr_forward`;
     dO [T,H,d_v] in q's dtype; chunk_states: that forward's chunk states.
     Returns (dq, dk, dv, dalpha, dbeta, dstate_in), all fp32.  ``grads``: an
-    optional tuple of those six tensors to write into."""
+    optional tuple of those six tensors to write into.  ``events``: optional
+    4 torch.cuda.Events recorded around the kernels (gdn_cpr_backward_timed)."""
     lib = load_library()
     T, H, dk = k.shape
     dv = v.shape[2]
@@ -255,9 +258,13 @@ def gdn_cpr_backward(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, C: int,
     if workspace is None:
         workspace = torch.empty(lib.gdn_cpr_backward_workspace_size(T, N, H, dk, dv, C), dtype=torch.uint8,
                                 device=dev)
-    st = lib.gdn_cpr_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(dO), _ptr(chunk_states),
-                              _ptr(cu_seqlens), cu_h, N, T, H, dk, dv, C, _dt(q.dtype),
-                              *[_ptr(g) for g in grads], _ptr(workspace), workspace.numel(), _stream(dev))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(dO), _ptr(chunk_states),
+            _ptr(cu_seqlens), cu_h, N, T, H, dk, dv, C, _dt(q.dtype),
+            *[_ptr(g) for g in grads], _ptr(workspace), workspace.numel(), _stream(dev))
+    if events is None:
+        st = lib.gdn_cpr_backward(*args)
+    else:
+        st = lib.gdn_cpr_backward_timed(*args, _event_array(events, 4))
     _check(st, "gdn_cpr_backward")
     return grads
 

@@ -201,8 +201,9 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
  *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t
  * (IsoExec summary page, section "Chunkwise-Parallel Recurrent (CPR) Gated
  * DeltaNet"; commentary blog, section 10), differentiated in reverse token
- * order.  Per chunk, the states are recomputed from the boundary state the
- * forward stored, with the forward's per-token arithmetic.
+ * order.  A serial scan carries dL/dS back to every chunk boundary; then the
+ * chunks run in parallel, each recomputing its states from the boundary state
+ * the forward stored, with the forward's per-token arithmetic.
  * Inputs:
  *   q, k, v, alpha, beta, cu_seqlens, cu_seqlens_host, num_seqs, total_tokens,
  *     H, d_k, d_v, C, in_dtype: as given to gdn_cpr_forward.
@@ -227,6 +228,21 @@ gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v,
                               float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
                               float* dstate_in, void* workspace, size_t workspace_bytes,
                               void* stream);
+
+/*
+ * gdn_cpr_backward with events: events (host array of 4 cudaEvent_t, or NULL)
+ * are recorded on the stream before the boundary-adjoint scan, after it,
+ * after the per-chunk kernel and after the tile reduction.
+ */
+gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
+                                    const float* alpha, const float* beta, const void* dO,
+                                    const float* chunk_states,
+                                    const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                    int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                    int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
+                                    float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
+                                    float* dstate_in, void* workspace, size_t workspace_bytes,
+                                    void* stream, void* const* events);
 
 /*
  * One decode step: one new token for each of num_seqs sequences.
