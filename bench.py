@@ -220,10 +220,17 @@ def cpu_baseline(budget_s: float = 10.0):
         if secs >= budget_s or T_s >= W["T"]:
             break
         T_s = min(W["T"], max(T_s * 2, int(T_s * budget_s / max(secs, 1e-3) * 1.1)))
+    reps = 1
+    if secs < budget_s:  # the whole workload is shorter than the budget: repeat it
+        reps = max(1, int(budget_s / max(secs, 1e-3)))
+        secs, toks = 0.0, 0
+        for _ in range(reps):
+            s_, t_ = oracle_sample(W["seed"], W["B"], W["H"], W["D"], W["C"], T_s)
+            secs, toks = secs + s_, toks + t_
     return {"value": toks / secs, "unit": UNIT, "cores": int(os.environ["OMP_NUM_THREADS"]), "kind": "oracle",
             "sample": f"fp64 recurrence (oracle/recurrent_fp64.c, OpenMP over (sequence, head)) on the first "
-                      f"{T_s} tokens of all {W['B']} sequences x {W['H']} heads of the prefill workload; "
-                      f"{secs:.1f} s"}
+                      f"{T_s} tokens of all {W['B']} sequences x {W['H']} heads of the prefill workload, "
+                      f"{reps} run(s); {secs:.1f} s"}
 
 
 def workload_config(world: int) -> dict:
