@@ -494,8 +494,11 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
     const HalfSync hs{2 + half};
     __shared__ int qslot[2], go[2];
     const int ntask = __ldg(cumc + maxc);
+    // Thread 0 of a half claims its next queue slot one task ahead, so the
+    // atomic's round trip overlaps the current task.
+    int next = tid == 0 ? atomicAdd(tok_next, 1) : 0;
     for (;;) {
-        if (tid == 0) qslot[half] = atomicAdd(tok_next, 1);
+        if (tid == 0) qslot[half] = next;
         hs();
         const int qi = qslot[half];
         if (qi >= ntask * H) break;
@@ -507,9 +510,11 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
         }
         const int c = lo, n = __ldg(order + t - __ldg(cumc + c));
         if (tid == 0) {  // one thread waits and decides for the half
+            next = atomicAdd(tok_next, 1);
+            // The acquire load orders this half's later state loads after the
+            // chain's release (through the barrier below): no fence needed.
             const bool ready = wait_at_least(progress + (int64_t)n * H + h, c + 1);
             if (!ready) atomicExch(err, 3);
-            __threadfence();
             go[half] = ready && *verr == 0;
         }
         hs();
