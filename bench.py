@@ -83,16 +83,19 @@ def backward_flops(tokens_heads: int, dk: int, dv: int):
 # dram__bytes_write.sum), keyed by kernel and by the sha256 of the sources that
 # kernel is compiled from; a changed source drops the figure (reported null).
 NCU_TRAFFIC = {
-    # profiles/k_chain_tok_prefill_B4_H16_T4096_d128_C64.md: 789,860,352 read + 328,601,344 written
-    ("k_chain_tok", "3a93de98f50d6c17"): 1118461696,
+    # profiles/k_chain_tok_prefill_B4_H16_T4096_d128_C64.md: 789,160,960 read + 329,176,320 written
+    ("k_chain_tok", "5a5969a3fe1e58ea"): 1118337280,
     # profiles/k_dec_tok_decode_N64_H32_d128_C64.md: 135,935,744 read + 77,555,200 written
     ("k_dec_tok", "51b392a62fe51a33"): 213490944,
+    # profiles/k_bwd_trainer_B2_H32_T8192_d128_C64.md: 1,658,930,688 read + 3,126,013,184 written
+    ("k_bwd_chunk", "0eecb72f0ac7c812"): 4784943872,
 }
 
 KERNEL_SOURCES = {
     "k_tok": ("schedule.cuh", "k_ptok.cuh"),
     "k_chain_tok": ("schedule.cuh", "k_ptok.cuh", "k_tc.cuh", "k_pchunk.cuh"),
     "k_dec_tok": ("schedule.cuh", "k_ptok.cuh", "k_decode.cuh"),
+    "k_bwd_chunk": ("schedule.cuh", "k_ptok.cuh", "k_bwd.cuh"),
 }
 
 
@@ -410,7 +413,8 @@ def bench_trainer(rank: int, world: int, warmup: int, steps: int):
             "bwd_kernels_ms": kern,
             "roofline": {"kernel": "k_bwd_chunk (per-chunk backward)", "bound": "alu", "achieved": tf,
                          "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tf / FP32_PEAK_TFLOPS,
-                         "traffic": None, "flops_per_launch": fl,
+                         "traffic": NCU_TRAFFIC.get(("k_bwd_chunk", kernel_source_sha("k_bwd_chunk"))),
+                         "flops_per_launch": fl,
                          "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}}
 
 
