@@ -363,12 +363,18 @@ def bench_decode(rank: int, world: int, warmup: int):
                          "bytes_per_launch": tb}}
 
 
-def bench_trainer(rank: int, world: int, warmup: int, steps: int):
+def bench_trainer(rank: int, world: int, warmup: int, steps: int, shape=None):
     """Trainer step: CPR forward + backward (gdn_cpr_backward) of the trainer
-    workload on this rank's sequences; L2 flushed before every timed step."""
+    workload on this rank's sequences; L2 flushed before every timed step.
+    ``shape`` (B, H, T) replaces the workload's sizes (for profiling a smaller
+    case of the same kernels)."""
     import torch
     from gated_deltanet_cpr_delta_b200 import gdn, synth
-    Tr = TRAIN
+    Tr = dict(TRAIN)
+    if shape is not None:
+        Tr.update(B=shape[0], H=shape[1], T=shape[2],
+                  name=f"trainer fwd+bwd B={shape[0]} H={shape[1]} T={shape[2]} d_k=d_v=128 C=64 bf16, "
+                       f"dO ~ N(0,1) bf16")
     B, H, T, D, C = Tr["B"], Tr["H"], Tr["T"], Tr["D"], Tr["C"]
     d = synth.make_batch_device(Tr["seed"], [T] * B, H, D, D, "bf16", seq_ids=rank_sequence_ids(rank, B))
     g = torch.Generator(device="cuda")
@@ -525,7 +531,8 @@ def run_native(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / K
 
     dec = bench_decode(rank, world, args.warmup) if not args.no_decode else None
-    trainer = bench_trainer(rank, world, args.warmup, min(K, 5)) if not args.no_trainer else None
+    tshape = tuple(int(x) for x in args.trainer_shape.split(",")) if args.trainer_shape else None
+    trainer = bench_trainer(rank, world, args.warmup, min(K, 5), tshape) if not args.no_trainer else None
 
     peaks, peak_src = load_peaks()
     flops = forward_flops(B * T * H, B * (T // C) * C * H, D, D, C)
@@ -599,6 +606,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-trainer", action="store_true")
+    ap.add_argument("--trainer-shape", default=None,
+                    help="B,H,T of the trainer section (default: the trainer workload; for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

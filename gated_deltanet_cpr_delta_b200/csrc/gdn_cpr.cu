@@ -288,7 +288,7 @@ struct BwdWorkspace {
 BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C)
 {
     BwdWorkspace w{};
-    const int32_t RT = dv < 32 ? dv : 32, NT = dv / RT, SUB = C < 8 ? C : 8;  // as gdn::BwdCfg
+    const int32_t RT = dv < 64 ? dv : 64, NT = dv / RT, SUB = C < 8 ? C : 8;  // as gdn::BwdCfg
     const Workspace tables = carve(nullptr, 0, N, H, dk, dv, C);  // the tables part alone
     size_t off = tables.bytes;
     auto take = [&](size_t n) {

@@ -32,51 +32,29 @@ namespace gdn {
 template <int DK, int DV, int C>
 struct BwdCfg {
     using RS = RowSplit<DK>;
-    static constexpr int RT = DV < 32 ? DV : 32;  // rows per CTA
+    static constexpr int RHO = 2;                 // rows per lane (k, q reads and row sums serve both)
+    static constexpr int RT = DV < 64 ? DV : 64;  // rows per CTA
     static constexpr int NT = DV / RT;            // row tiles per head
-    static constexpr int THREADS = RT * RS::TPR;
+    static constexpr int NG = RT / RHO;           // row groups (4 lanes each)
+    static constexpr int THREADS = NG * RS::TPR;
     static constexpr int SUB = C < 8 ? C : 8;     // tokens per checkpoint
     static constexpr int NCK = C / SUB;           // checkpoints per chunk
     // staged floats per token: k, q (slots), v, dO rows, gates; a multiple of 4 (16-byte rows)
     static constexpr int TOKF = ((2 * RS::KS + 2 * RT + 2) + 3) / 4 * 4;
     static constexpr int RED = DK + 4;            // reduction buffer row stride
-    // smem: SUB staged tokens | dq rows | dk rows | [RT][2] scalars
+    // smem: SUB staged tokens | dq rows | dk rows | [NG][2] scalars | the current checkpoint (lane-private rows)
     static constexpr int TOK_OFF = 0;
     static constexpr int RQ_OFF = TOK_OFF + SUB * TOKF;
-    static constexpr int RK_OFF = RQ_OFF + RT * RED;
-    static constexpr int RS_OFF = RK_OFF + RT * RED;
-    static constexpr size_t SMEM = sizeof(float) * (size_t)(RS_OFF + 2 * RT);
+    static constexpr int RK_OFF = RQ_OFF + NG * RED;
+    static constexpr int RS_OFF = RK_OFF + NG * RED;
+    static constexpr int CK_OFF = (RS_OFF + 2 * NG + 3) / 4 * 4;
+    // a lane's RHO checkpoint slices, CKS floats apart (the 4-float pad puts
+    // 8 consecutive lanes' 16-byte reads in distinct banks)
+    static constexpr int CKS = RHO * RS::EPT + 4;
+    static constexpr size_t SMEM = sizeof(float) * (size_t)(CK_OFF + THREADS * CKS);
     static constexpr int64_t SCRATCH = (int64_t)NCK * RT * DK;  // floats of checkpoints per CTA
+    static_assert(THREADS % 32 == 0, "whole warps (the tree shuffles use full masks)");
 };
-
-// One forward P_tok step on this lane's share of a row: the u tree, delta and
-// the update, with exactly the forward's operations (ptok_step without the
-// output tree).  Returns u; *d_out = delta.
-template <int DK>
-__device__ __forceinline__ float ptok_advance(f2x (&Rp)[DK / kLeaves], const float* kt, float v_i, float a, float b,
-                                              float* d_out)
-{
-    constexpr int L = DK / kLeaves;
-    f2x kp[L];
-#pragma unroll
-    for (int m = 0; m < L; m += 2) {
-        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(kt + 2 * m);
-        kp[m] = x.x;
-        kp[m + 1] = x.y;
-    }
-    f2x acc = fmul2(Rp[0], kp[0]);
-#pragma unroll
-    for (int m = 1; m < L; ++m) acc = ffma2(Rp[m], kp[m], acc);
-    float la, lb;
-    up2(acc, la, lb);
-    const float u = tree_4lanes(la, lb);
-    const float d = fmul(b, fsub(v_i, fmul(a, u)));
-    const f2x aa = pk2(a, a), dd = pk2(d, d);
-#pragma unroll
-    for (int m = 0; m < L; ++m) Rp[m] = ffma2(dd, kp[m], fmul2(aa, Rp[m]));
-    *d_out = d;
-    return u;
-}
 
 // Dot product of two lane shares of rows over all DK columns (leaf chains,
 // then the 4-lane tree), every lane of the row getting the sum.
@@ -286,12 +264,48 @@ k_bwd_scan(const void* __restrict__ q, const void* __restrict__ k, const float* 
         bwd_scan_body<DK, DV, C, 4>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, ybuf, dstate_row, sm);
 }
 
+// One forward P_tok step (the forward's operations) on RHO rows of this lane
+// that share the staged k_t.
+template <int DK, int RHO>
+__device__ __forceinline__ void adv_rows(f2x (&Sp)[RHO][DK / kLeaves], const float* kt, const float* vrow, float a,
+                                         float b)
+{
+    constexpr int L = DK / kLeaves;
+    f2x kp[L];
+    load_pairs_slot<DK>(kp, kt);
+    const f2x aa = pk2(a, a);
+#pragma unroll
+    for (int r = 0; r < RHO; ++r) {
+        const float u = row_dot<DK>(Sp[r], kp);
+        const float d = fmul(b, fsub(vrow[r], fmul(a, u)));
+        const f2x dd = pk2(d, d);
+#pragma unroll
+        for (int m = 0; m < L; ++m) Sp[r][m] = ffma2(dd, kp[m], fmul2(aa, Sp[r][m]));
+    }
+}
+
+// Stores 2*G4 floats of a lane's natural-order slice: elements m0..m0+G4-1
+// from lo[], L+m0.. from hi[].
+template <int G4>
+__device__ __forceinline__ void st_group(float* dst, int m0, int L, const float* lo, const float* hi)
+{
+    if constexpr (G4 == 4) {
+        *reinterpret_cast<float4*>(dst + m0) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<float4*>(dst + L + m0) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+    } else {
+        *reinterpret_cast<float2*>(dst + m0) = make_float2(lo[0], lo[1]);
+        *reinterpret_cast<float2*>(dst + L + m0) = make_float2(hi[0], hi[1]);
+    }
+}
+
 // Backward of the chunks: one (chunk, head, row tile) task at a time, CTAs
 // looping over the tasks (a persistent grid, so that the checkpoint scratch
-// is per resident CTA and stays in L2).  A task starts from G = Y_{c+1}
-// (zero after the last chunk), recomputes the chunk's states from its
-// boundary state and writes dv rows, and the tile's row sums of dq, dk
-// ([NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).
+// is per resident CTA and stays in L2).  Each lane holds RHO rows (a quarter
+// of each row's columns), so one read of a staged k or q serves RHO rows and
+// the lane adds its rows' dq / dk terms before they go to shared memory.  A
+// task starts from G = Y_{c+1} (zero after the last chunk), recomputes the
+// chunk's states from its boundary state and writes dv rows, and the tile's
+// row sums of dq, dk ([NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(BwdCfg<DK, DV, C>::THREADS)
 k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
@@ -305,6 +319,9 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
     using Cf = BwdCfg<DK, DV, C>;
     using RS = typename Cf::RS;
     constexpr int L = RS::L, KS = RS::KS, RT = Cf::RT, SUB = Cf::SUB, TOKF = Cf::TOKF, NT = Cf::NT;
+    constexpr int RHO = Cf::RHO, NG = Cf::NG, EPT = RS::EPT;
+    constexpr int G4 = L % 4 == 0 ? 4 : 2;
+    static_assert(L % G4 == 0, "");
     if (__ldg(err)) return;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
@@ -313,20 +330,22 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
     float* redk = sm + Cf::RK_OFF;
     float* reds = sm + Cf::RS_OFF;
     const int tid = threadIdx.x;
-    const int row = tid / RS::TPR, part = tid % RS::TPR;
-    float* ck = scratch + (int64_t)blockIdx.x * Cf::SCRATCH;  // this CTA's checkpoints
+    const int gi = tid / RS::TPR, part = tid % RS::TPR;
+    const int lrow0 = gi * RHO;  // this lane's first row in the tile
+    float* ckl = sm + Cf::CK_OFF + tid * Cf::CKS;  // lane-private copy of the current checkpoint
+    float* ck = scratch + (int64_t)blockIdx.x * Cf::SCRATCH;   // this CTA's checkpoints
 
     for (int64_t task = blockIdx.x; task < ntasks; task += gridDim.x) {
-        const int r = (int)(task % NT);
+        const int rt = (int)(task % NT);
         const int h = (int)((task / NT) % H);
         const int ct = (int)(task / ((int64_t)NT * H));
         const int n = find_seq(cto, N, ct);
         const int c = ct - __ldg(cto + n);
-        const int grow = r * RT + row;
         const int seq0 = __ldg(cu + n);
         const int Ln = __ldg(cu + n + 1) - seq0;
         const int64_t slot0 = __ldg(so + n);
         const int nchunks = (Ln + C - 1) / C;
+        const int grow0 = rt * RT + lrow0;  // this lane's first row in the head
 
         // stage tokens [t0, t0 + len) of the sequence: k, q into the slot layout,
         // this tile's v and dO rows, the gates
@@ -345,7 +364,7 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
                 const int t = e / (2 * RT / 8), el = (e % (2 * RT / 8)) * 8;
                 float x[8];
                 const int64_t trow = ((int64_t)seq0 + t0 + t) * H + h;
-                load8(el < RT ? v : dO, trow * DV + r * RT + (el % RT), in_bf16, x);
+                load8(el < RT ? v : dO, trow * DV + rt * RT + (el % RT), in_bf16, x);
                 float* d = tok + t * TOKF + 2 * KS + (el >= RT ? RT : 0) + (el % RT);
 #pragma unroll
                 for (int m = 0; m < 8; ++m) d[m] = x[m];
@@ -356,99 +375,138 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
                 tok[t * TOKF + 2 * KS + 2 * RT + 1] = __ldg(beta + trow);
             }
         };
-        auto step = [&](f2x (&Sp)[L], int t) {  // forward step with staged token t
+        auto step = [&](f2x (&Sp)[RHO][L], int t) {  // forward step with staged token t
             const float* tt = tok + t * TOKF;
-            float d;
-            ptok_advance<DK>(Sp, tt + part * RS::PS, tt[2 * KS + row], tt[2 * KS + 2 * RT], tt[2 * KS + 2 * RT + 1],
-                             &d);
+            adv_rows<DK, RHO>(Sp, tt + part * RS::PS, tt + 2 * KS + lrow0, tt[2 * KS + 2 * RT],
+                              tt[2 * KS + 2 * RT + 1]);
         };
 
-        f2x G[L];
-        if (c + 1 < nchunks) {
-            load_row_pairs<DK>(G, ybuf + (((slot0 + c + 1) * H + h) * DV + grow) * DK + part * RS::EPT);
-        } else {
+        f2x G[RHO][L];
 #pragma unroll
-            for (int m = 0; m < L; ++m) G[m] = pk2(0.f, 0.f);
+        for (int r = 0; r < RHO; ++r) {
+            if (c + 1 < nchunks) {
+                load_row_pairs<DK>(G[r], ybuf + (((slot0 + c + 1) * H + h) * DV + grow0 + r) * DK + part * EPT);
+            } else {
+#pragma unroll
+                for (int m = 0; m < L; ++m) G[r][m] = pk2(0.f, 0.f);
+            }
         }
-        const float* S0 = states + (((slot0 + c) * H + h) * DV + grow) * DK + part * RS::EPT;
+        const float* S0 = states + (((slot0 + c) * H + h) * DV + grow0) * DK + part * EPT;
         const int cb = c * C, clen = min(C, Ln - cb);
         const int nsub = (clen + SUB - 1) / SUB;
         // checkpoints: the state at cb + j*SUB, j = 1..nsub-1 (j = 0 is the chunk state)
-        f2x Sp[L];
-        load_row_pairs<DK>(Sp, S0);
+        f2x Sp[RHO][L];
+#pragma unroll
+        for (int r = 0; r < RHO; ++r) load_row_pairs<DK>(Sp[r], S0 + r * DK);
         for (int j = 1; j < nsub; ++j) {
             __syncthreads();
             stage(cb + (j - 1) * SUB, SUB);
             __syncthreads();
             for (int t = 0; t < SUB; ++t) step(Sp, t);
-            store_row_pairs<DK>(ck + ((int64_t)(j - 1) * RT + row) * DK + part * RS::EPT, Sp);
+#pragma unroll
+            for (int r = 0; r < RHO; ++r)
+                store_row_pairs<DK>(ck + ((int64_t)(j - 1) * RT + lrow0 + r) * DK + part * EPT, Sp[r]);
         }
         // backward over the sub-chunks, last first
         for (int j = nsub - 1; j >= 0; --j) {
             const int sb = cb + j * SUB, slen = min(SUB, clen - j * SUB);
             __syncthreads();
             stage(sb, slen);
+            // the sub-chunk's checkpoint into this lane's private shared rows (read back once per token)
+#pragma unroll
+            for (int r = 0; r < RHO; ++r) {
+                const float* src = j == 0 ? S0 + r * DK : ck + ((int64_t)(j - 1) * RT + lrow0 + r) * DK + part * EPT;
+#pragma unroll
+                for (int e = 0; e < EPT; e += 4)
+                    *reinterpret_cast<float4*>(ckl + r * EPT + e) = *reinterpret_cast<const float4*>(src + e);
+            }
             __syncthreads();
             for (int t = slen - 1; t >= 0; --t) {
                 // S_{t-1}: from the sub-chunk's checkpoint, forward over its first t tokens
-                if (j == 0) load_row_pairs<DK>(Sp, S0);
-                else load_row_pairs<DK>(Sp, ck + ((int64_t)(j - 1) * RT + row) * DK + part * RS::EPT);
+#pragma unroll
+                for (int r = 0; r < RHO; ++r) load_row_pairs<DK>(Sp[r], ckl + r * EPT);
                 for (int m = 0; m < t; ++m) step(Sp, m);
                 const float* tt = tok + t * TOKF;
                 const float a = tt[2 * KS + 2 * RT], b = tt[2 * KS + 2 * RT + 1];
-                const float vi = tt[2 * KS + row], doi = tt[2 * KS + RT + row];
-                f2x kp[L], qp[L];
-                load_pairs_slot<DK>(kp, tt + part * RS::PS);
-                load_pairs_slot<DK>(qp, tt + KS + part * RS::PS);
-                const float u = row_dot<DK>(Sp, kp);
-                const float de = fmul(b, fsub(vi, fmul(a, u)));
-                const f2x aa = pk2(a, a), dd = pk2(de, de), oo = pk2(doi, doi);
-                // G += dO_i q ; the dq and dk row terms ; dot products
-#pragma unroll
-                for (int m = 0; m < L; ++m) G[m] = ffma2(oo, qp[m], G[m]);
-                const float dlt = row_dot<DK>(G, kp);   // ddelta_i
-                const float gs = row_dot<DK>(G, Sp);    // <G_i, S_{t-1,i}>
+                const f2x aa = pk2(a, a);
                 const float ab = fmul(a, b);
-                const f2x ng = pk2(-fmul(ab, dlt), -fmul(ab, dlt));
-                float xq[RS::EPT], xk[RS::EPT];
+                f2x kp[L];
+                load_pairs_slot<DK>(kp, tt + part * RS::PS);
+                float u[RHO], de[RHO], dlt[RHO], vi[RHO], doi[RHO];
+                {
+                    f2x qp[L];
+                    load_pairs_slot<DK>(qp, tt + KS + part * RS::PS);
 #pragma unroll
-                for (int m = 0; m < L; ++m) {
-                    const f2x st = ffma2(dd, kp[m], fmul2(aa, Sp[m]));                 // S_t
-                    const f2x gq = fmul2(oo, st);                                      // dO_i S_t
-                    const f2x gk = ffma2(ng, Sp[m], fmul2(dd, G[m]));                  // G delta - ab ddelta S_{t-1}
-                    up2(gq, xq[m], xq[L + m]);
-                    up2(gk, xk[m], xk[L + m]);
+                    for (int r = 0; r < RHO; ++r) {
+                        vi[r] = tt[2 * KS + lrow0 + r];
+                        doi[r] = tt[2 * KS + RT + lrow0 + r];
+                        const f2x oo = pk2(doi[r], doi[r]);
+#pragma unroll
+                        for (int m = 0; m < L; ++m) G[r][m] = ffma2(oo, qp[m], G[r][m]);  // G += dO_i q
+                    }
                 }
-                // this row's share -> the reduction buffers (natural column order)
+                float ta = 0.f, tb = 0.f;  // this lane's rows' dalpha and dbeta terms
 #pragma unroll
-                for (int e = 0; e < RS::EPT; e += 4) {
-                    *reinterpret_cast<float4*>(redq + row * Cf::RED + part * RS::EPT + e) =
-                        make_float4(xq[e], xq[e + 1], xq[e + 2], xq[e + 3]);
-                    *reinterpret_cast<float4*>(redk + row * Cf::RED + part * RS::EPT + e) =
-                        make_float4(xk[e], xk[e + 1], xk[e + 2], xk[e + 3]);
+                for (int r = 0; r < RHO; ++r) {
+                    u[r] = row_dot<DK>(Sp[r], kp);
+                    de[r] = fmul(b, fsub(vi[r], fmul(a, u[r])));
+                    dlt[r] = row_dot<DK>(G[r], kp);        // ddelta_i
+                    const float gs = row_dot<DK>(G[r], Sp[r]);  // <G_i, S_{t-1,i}>
+                    ta = fadd(ta, fsub(gs, fmul(b, fmul(dlt[r], u[r]))));
+                    tb = fadd(tb, fmul(dlt[r], fsub(vi[r], fmul(a, u[r]))));
+                }
+                // the lane's rows' dq terms (dO_i S_t) and dk terms (G delta - ab ddelta S_{t-1}),
+                // added over its rows, to the reduction buffers in natural column order
+#pragma unroll
+                for (int m0 = 0; m0 < L; m0 += G4) {
+                    float ql[G4], qh[G4], kl[G4], kh[G4];
+#pragma unroll
+                    for (int mm = 0; mm < G4; ++mm) {
+                        const int m = m0 + mm;
+                        f2x sq = pk2(0.f, 0.f), sk = pk2(0.f, 0.f);
+#pragma unroll
+                        for (int r = 0; r < RHO; ++r) {
+                            const f2x dd = pk2(de[r], de[r]);
+                            const f2x st = ffma2(dd, kp[m], fmul2(aa, Sp[r][m]));   // S_t
+                            sq = ffma2(pk2(doi[r], doi[r]), st, sq);
+                            const float nb = -fmul(ab, dlt[r]);
+                            sk = ffma2(pk2(nb, nb), Sp[r][m], ffma2(dd, G[r][m], sk));
+                        }
+                        up2(sq, ql[mm], qh[mm]);
+                        up2(sk, kl[mm], kh[mm]);
+                    }
+                    st_group<G4>(redq + gi * Cf::RED + part * EPT, m0, L, ql, qh);
+                    st_group<G4>(redk + gi * Cf::RED + part * EPT, m0, L, kl, kh);
                 }
                 if (part == 0) {
-                    reds[2 * row] = fsub(gs, fmul(b, fmul(dlt, u)));       // dalpha term
-                    reds[2 * row + 1] = fmul(dlt, fsub(vi, fmul(a, u)));   // dbeta term
-                    dv[(((int64_t)seq0 + sb + t) * H + h) * DV + grow] = fmul(b, dlt);
+                    reds[2 * gi] = ta;
+                    reds[2 * gi + 1] = tb;
+#pragma unroll
+                    for (int r = 0; r < RHO; ++r)
+                        dv[(((int64_t)seq0 + sb + t) * H + h) * DV + grow0 + r] = fmul(b, dlt[r]);
                 }
                 // G <- alpha G - alpha beta ddelta k
 #pragma unroll
-                for (int m = 0; m < L; ++m) G[m] = ffma2(ng, kp[m], fmul2(aa, G[m]));
+                for (int r = 0; r < RHO; ++r) {
+                    const float nb = -fmul(ab, dlt[r]);
+                    const f2x ng = pk2(nb, nb);
+#pragma unroll
+                    for (int m = 0; m < L; ++m) G[r][m] = ffma2(ng, kp[m], fmul2(aa, G[r][m]));
+                }
                 __syncthreads();
-                // the tile's row sums, rows in ascending order
+                // the tile's row-group sums, groups in ascending order
                 const int64_t trow = ((int64_t)seq0 + sb + t) * H + h;
                 for (int col = tid; col < 2 * DK; col += blockDim.x) {
                     const float* src = col < DK ? redq + col : redk + (col - DK);
                     float s = src[0];
-                    for (int i = 1; i < RT; ++i) s = fadd(s, src[i * Cf::RED]);
+                    for (int i = 1; i < NG; ++i) s = fadd(s, src[i * Cf::RED]);
                     float* dst = col < DK ? pq : pk;
-                    dst[((int64_t)r * T_total * H + trow) * DK + (col % DK)] = s;
+                    dst[((int64_t)rt * T_total * H + trow) * DK + (col % DK)] = s;
                 }
                 if (tid < 2) {
                     float s = reds[tid];
-                    for (int i = 1; i < RT; ++i) s = fadd(s, reds[2 * i + tid]);
-                    (tid == 0 ? pa : pb)[(int64_t)r * T_total * H + trow] = s;
+                    for (int i = 1; i < NG; ++i) s = fadd(s, reds[2 * i + tid]);
+                    (tid == 0 ? pa : pb)[(int64_t)rt * T_total * H + trow] = s;
                 }
                 __syncthreads();
             }
