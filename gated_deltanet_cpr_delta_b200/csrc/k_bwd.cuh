@@ -56,17 +56,27 @@ struct BwdCfg {
     static_assert(THREADS % 32 == 0, "whole warps (the tree shuffles use full masks)");
 };
 
-// Dot product of two lane shares of rows over all DK columns (leaf chains,
-// then the 4-lane tree), every lane of the row getting the sum.
+// Dot product of two lane shares of rows over all DK columns, every lane of
+// the row getting the sum: up to 4 independent partial chains (the backward
+// has no bitwise contract, so the order is free), then the 4-lane tree.
 template <int DK>
 __device__ __forceinline__ float row_dot(const f2x (&x)[DK / kLeaves], const f2x (&y)[DK / kLeaves])
 {
     constexpr int L = DK / kLeaves;
-    f2x acc = fmul2(x[0], y[0]);
+    constexpr int NA = L < 4 ? L : 4;
+    f2x acc[NA];
 #pragma unroll
-    for (int m = 1; m < L; ++m) acc = ffma2(x[m], y[m], acc);
-    float la, lb;
-    up2(acc, la, lb);
+    for (int j = 0; j < NA; ++j) acc[j] = fmul2(x[j], y[j]);
+#pragma unroll
+    for (int m = NA; m < L; ++m) acc[m % NA] = ffma2(x[m], y[m], acc[m % NA]);
+    float la = 0.f, lb = 0.f;
+#pragma unroll
+    for (int j = 0; j < NA; ++j) {
+        float a, b;
+        up2(acc[j], a, b);
+        la = j == 0 ? a : fadd(la, a);
+        lb = j == 0 ? b : fadd(lb, b);
+    }
     return tree_4lanes(la, lb);
 }
 
