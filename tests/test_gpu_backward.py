@@ -128,3 +128,21 @@ def test_backward_trainer_size_sampled_head_vs_oracle():
                          np.array([0, T], np.int32), C)
     got = [x[sl, h:h + 1].cpu().numpy() for x in grads[:5]] + [grads[5][n:n + 1, h:h + 1].cpu().numpy()]
     check(got, ref, "trainer sample")
+
+
+def test_backward_gate_extremes_vs_oracle():
+    """alpha = 0 (a reset), alpha = 1, beta = 0 (no write) and beta = 1 at
+    scattered tokens, in fp32; the gradient formulas hold at these values."""
+    C, d = 32, 64
+    b = synth.make_batch(77, [3 * C + 7, C, 5], 2, d, d, "f32")
+    rng = np.random.default_rng(8)
+    T = b.q.shape[0]
+    for arr, vals in ((b.alpha, (0.0, 1.0)), (b.beta, (0.0, 1.0))):
+        for val in vals:
+            idx = rng.choice(T, size=T // 8, replace=False)
+            arr[idx, rng.integers(0, 2, size=idx.size)] = val
+    S0 = (rng.standard_normal((3, 2, d, d)) * 0.2).astype(np.float32)
+    dO = _dO(12, T, 2, d, "f32")
+    got = run(b, C, S0, dO)
+    ref = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, C, S0)
+    check(got, ref, "gate extremes")
