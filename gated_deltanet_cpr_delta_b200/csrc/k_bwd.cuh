@@ -48,10 +48,15 @@ struct BwdCfg {
     static constexpr int RK_OFF = RQ_OFF + NG * RED;
     static constexpr int RS_OFF = RK_OFF + NG * RED;
     static constexpr int CK_OFF = (RS_OFF + 2 * NG + 3) / 4 * 4;
-    // a lane's RHO checkpoint slices, CKS floats apart (the 4-float pad puts
-    // 8 consecutive lanes' 16-byte reads in distinct banks)
-    static constexpr int CKS = RHO * RS::EPT + 4;
-    static constexpr size_t SMEM = sizeof(float) * (size_t)(CK_OFF + THREADS * CKS);
+    // two lane-private state slots (the sub-chunk's checkpoint and its
+    // midpoint): a lane's RHO row slices, CKS floats, its 16-byte pieces
+    // XOR-swizzled by the lane index so that 8 consecutive lanes reading the
+    // same piece hit distinct banks
+    static constexpr int CKS = RHO * RS::EPT;
+    static constexpr int CK_PIECES = CKS / 4;
+    static constexpr int CK_SWZ = (CK_PIECES < 8 ? CK_PIECES : 8) - 1;
+    static constexpr int MID = SUB / 2;           // tokens from the checkpoint to the midpoint slot
+    static constexpr size_t SMEM = sizeof(float) * (size_t)(CK_OFF + 2 * THREADS * CKS);
     static constexpr int64_t SCRATCH = (int64_t)NCK * RT * DK;  // floats of checkpoints per CTA
     static_assert(THREADS % 32 == 0, "whole warps (the tree shuffles use full masks)");
 };
@@ -308,6 +313,40 @@ __device__ __forceinline__ void st_group(float* dst, int m0, int L, const float*
     }
 }
 
+// A lane's RHO rows (natural column order) to / from its swizzled slot.
+template <int DK, int RHO, int SWZ>
+__device__ __forceinline__ void slot_store(float* slot, int sw, const f2x (&Sp)[RHO][DK / kLeaves])
+{
+    constexpr int L = DK / kLeaves, EPT = 2 * L;
+#pragma unroll
+    for (int r = 0; r < RHO; ++r) {
+        float t[EPT];
+#pragma unroll
+        for (int m = 0; m < L; ++m) up2(Sp[r][m], t[m], t[L + m]);
+#pragma unroll
+        for (int e = 0; e < EPT; e += 4)
+            *reinterpret_cast<float4*>(slot + 4 * (((r * EPT + e) >> 2) ^ (sw & SWZ))) =
+                make_float4(t[e], t[e + 1], t[e + 2], t[e + 3]);
+    }
+}
+
+template <int DK, int RHO, int SWZ>
+__device__ __forceinline__ void slot_load(f2x (&Sp)[RHO][DK / kLeaves], const float* slot, int sw)
+{
+    constexpr int L = DK / kLeaves, EPT = 2 * L;
+#pragma unroll
+    for (int r = 0; r < RHO; ++r) {
+        float t[EPT];
+#pragma unroll
+        for (int e = 0; e < EPT; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(slot + 4 * (((r * EPT + e) >> 2) ^ (sw & SWZ)));
+            t[e] = x.x; t[e + 1] = x.y; t[e + 2] = x.z; t[e + 3] = x.w;
+        }
+#pragma unroll
+        for (int m = 0; m < L; ++m) Sp[r][m] = pk2(t[m], t[L + m]);
+    }
+}
+
 // Backward of the chunks: one (chunk, head, row tile) task at a time, CTAs
 // looping over the tasks (a persistent grid, so that the checkpoint scratch
 // is per resident CTA and stays in L2).  Each lane holds RHO rows (a quarter
@@ -342,7 +381,8 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
     const int tid = threadIdx.x;
     const int gi = tid / RS::TPR, part = tid % RS::TPR;
     const int lrow0 = gi * RHO;  // this lane's first row in the tile
-    float* ckl = sm + Cf::CK_OFF + tid * Cf::CKS;  // lane-private copy of the current checkpoint
+    float* slotA = sm + Cf::CK_OFF + tid * Cf::CKS;                 // the sub-chunk's checkpoint
+    float* slotB = sm + Cf::CK_OFF + (Cf::THREADS + tid) * Cf::CKS;  // the state MID tokens later
     float* ck = scratch + (int64_t)blockIdx.x * Cf::SCRATCH;   // this CTA's checkpoints
 
     for (int64_t task = blockIdx.x; task < ntasks; task += gridDim.x) {
@@ -422,20 +462,24 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
             const int sb = cb + j * SUB, slen = min(SUB, clen - j * SUB);
             __syncthreads();
             stage(sb, slen);
-            // the sub-chunk's checkpoint into this lane's private shared rows (read back once per token)
+            // the sub-chunk's checkpoint into this lane's slot A, and the state
+            // MID tokens later into slot B (read back once per token)
 #pragma unroll
             for (int r = 0; r < RHO; ++r) {
                 const float* src = j == 0 ? S0 + r * DK : ck + ((int64_t)(j - 1) * RT + lrow0 + r) * DK + part * EPT;
-#pragma unroll
-                for (int e = 0; e < EPT; e += 4)
-                    *reinterpret_cast<float4*>(ckl + r * EPT + e) = *reinterpret_cast<const float4*>(src + e);
+                load_row_pairs<DK>(Sp[r], src);
             }
+            slot_store<DK, RHO, Cf::CK_SWZ>(slotA, tid, Sp);
             __syncthreads();
+            if (slen > Cf::MID) {
+                for (int m = 0; m < Cf::MID; ++m) step(Sp, m);
+                slot_store<DK, RHO, Cf::CK_SWZ>(slotB, tid, Sp);
+            }
             for (int t = slen - 1; t >= 0; --t) {
-                // S_{t-1}: from the sub-chunk's checkpoint, forward over its first t tokens
-#pragma unroll
-                for (int r = 0; r < RHO; ++r) load_row_pairs<DK>(Sp[r], ckl + r * EPT);
-                for (int m = 0; m < t; ++m) step(Sp, m);
+                // S_{t-1}: from the nearer of the two slots, forward over the tokens in between
+                const bool fromB = t >= Cf::MID;
+                slot_load<DK, RHO, Cf::CK_SWZ>(Sp, fromB ? slotB : slotA, tid);
+                for (int m = fromB ? Cf::MID : 0; m < t; ++m) step(Sp, m);
                 const float* tt = tok + t * TOKF;
                 const float a = tt[2 * KS + 2 * RT], b = tt[2 * KS + 2 * RT + 1];
                 const f2x aa = pk2(a, a);
