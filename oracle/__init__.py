@@ -37,7 +37,7 @@ def _load():
         lib.oracle_recurrent_fp64.restype = ctypes.c_int
         lib.oracle_recurrent_fp64.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P]
         lib.oracle_adjoint_fp64.restype = ctypes.c_int
-        lib.oracle_adjoint_fp64.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
+        lib.oracle_adjoint_fp64.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
         lib.sched_forward.restype = ctypes.c_int
         lib.sched_forward.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
                                       P, P, P, P, P, P, P, P, P]
@@ -86,8 +86,9 @@ def recurrent(q, k, v, alpha, beta, cu_seqlens, C, state_in=None):
     return dict(o=o, states=states, final=final)
 
 
-def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None):
-    """fp64 gradient of L = sum_t dO_t . o_t through the recurrence
+def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=None):
+    """fp64 gradient of L = sum_t dO_t . o_t (+ <dstate_out, final state> per
+    sequence and head, when given) through the recurrence
     (oracle/adjoint_fp64.c).  Returns dict(dq, dk, dv, dalpha, dbeta,
     dstate_in [N,H,dv,dk])."""
     lib = _load()
@@ -98,9 +99,10 @@ def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None):
     dv = v.shape[2]
     N = cu.shape[0] - 1
     s_in = _c(state_in, np.float64)
+    s_out = _c(dstate_out, np.float64)
     out = dict(dq=np.zeros((T, H, dk)), dk=np.zeros((T, H, dk)), dv=np.zeros((T, H, dv)),
                dalpha=np.zeros((T, H)), dbeta=np.zeros((T, H)), dstate_in=np.zeros((N, H, dv, dk)))
-    rc = lib.oracle_adjoint_fp64(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s_in), _p(dO), _p(cu), N, H, dk, dv, C,
+    rc = lib.oracle_adjoint_fp64(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s_in), _p(s_out), _p(dO), _p(cu), N, H, dk, dv, C,
                                  _p(out["dq"]), _p(out["dk"]), _p(out["dv"]), _p(out["dalpha"]), _p(out["dbeta"]),
                                  _p(out["dstate_in"]))
     if rc:

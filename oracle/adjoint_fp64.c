@@ -20,13 +20,16 @@
  *     dk_t    = G^T delta - alpha_t beta_t S_{t-1}^T ddelta
  *     G      <- alpha_t G - alpha_t beta_t ddelta k_t^T     (= dL/dS_{t-1})
  *
- * and dstate_in = G after the first token.  The forward states come from a
- * first fp64 pass that keeps every C-th state; each C-token span is then
- * recomputed (C states) before its backward sweep.
+ * and dstate_in = G after the first token.  dstate_out (NULL = zeros) is
+ * dL/dS of each sequence's final state, from a loss term outside the outputs
+ * (a later part of the sequence, split off at that state): G starts from it
+ * at the last token.  The forward states come from a first fp64 pass that
+ * keeps every C-th state; each C-token span is then recomputed (C states)
+ * before its backward sweep.
  *
  * Layouts (fp64, row-major): q, k, dq, dk [T, H, d_k]; v, dO, dv [T, H, d_v];
- * alpha, beta, dalpha, dbeta [T, H]; state_in, dstate_in [N, H, d_v, d_k]
- * (state_in NULL = zeros).  cu_seqlens [N+1] int32.
+ * alpha, beta, dalpha, dbeta [T, H]; state_in, dstate_out, dstate_in
+ * [N, H, d_v, d_k] (state_in NULL = zeros).  cu_seqlens [N+1] int32.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -43,7 +46,7 @@ static void step_fwd(double* S, const double* k, const double* v, double a, doub
 }
 
 int oracle_adjoint_fp64(const double* q, const double* k, const double* v, const double* alpha,
-                        const double* beta, const double* state_in, const double* dO,
+                        const double* beta, const double* state_in, const double* dstate_out, const double* dO,
                         const int32_t* cu_seqlens, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C,
                         double* dq, double* dkk, double* dvv, double* dalpha, double* dbeta, double* dstate_in)
 {
@@ -70,6 +73,7 @@ int oracle_adjoint_fp64(const double* q, const double* k, const double* v, const
                 bad = 1;
                 continue;
             }
+            if (dstate_out) memcpy(G, dstate_out + ((int64_t)n * H + h) * SZ, sizeof(double) * (size_t)SZ);
             double* S = ck;
             if (state_in) memcpy(S, state_in + ((int64_t)n * H + h) * SZ, sizeof(double) * (size_t)SZ);
             else memset(S, 0, sizeof(double) * (size_t)SZ);

@@ -9,6 +9,9 @@ L = sum_t dO_t . o_t through the gated delta rule.
 * A closed form: with alpha = 1 and beta = 0 the state never changes, so
   dq_t = S_0^T dO_t, dS_0 = sum_t dO_t q_t^T, dv = dk = 0 and
   dalpha_t = <sum_{t' >= t} dO_t' q_t'^T, S_0>.
+* A gradient W for each final state (dstate_out) adds <W, S_final> to the
+  loss: the complex-step check includes that term, and in the closed form
+  W adds to dS_0 and to every G.
 """
 import numpy as np
 import pytest
@@ -17,8 +20,9 @@ import oracle
 from gated_deltanet_cpr_delta_b200 import synth
 
 
-def _loss_complex(q, k, v, alpha, beta, S0, dO, cu):
-    """sum_t dO_t . o_t with the recurrence S_t = a S (I - b k k^T) + b v k^T, complex128."""
+def _loss_complex(q, k, v, alpha, beta, S0, dO, cu, W=None):
+    """sum_t dO_t . o_t (+ sum <W, S_final>) with the recurrence
+    S_t = a S (I - b k k^T) + b v k^T, complex128."""
     L = 0.0 + 0.0j
     H = k.shape[1]
     for n in range(len(cu) - 1):
@@ -29,27 +33,31 @@ def _loss_complex(q, k, v, alpha, beta, S0, dO, cu):
                 M = np.eye(len(kt), dtype=np.complex128) - beta[t, h] * np.outer(kt, kt)
                 S = alpha[t, h] * (S @ M) + beta[t, h] * np.outer(vt, kt)
                 L += dO[t, h] @ (S @ qt)
+            if W is not None:
+                L += np.sum(W[n, h] * S)
     return L
 
 
-@pytest.mark.parametrize("C", [2, 4])
-def test_adjoint_matches_complex_step_derivatives(C):
+@pytest.mark.parametrize("C,with_w", [(2, False), (4, False), (4, True)])
+def test_adjoint_matches_complex_step_derivatives(C, with_w):
     rng = np.random.default_rng(5)
     lens, H, dk, dv = [7, 4], 1, 3, 2
     b = synth.make_batch(21, lens, H, dk, dv, "f32")
     T = int(b.cu_seqlens[-1])
     S0 = rng.standard_normal((2, H, dv, dk))
     dO = rng.standard_normal((T, H, dv))
+    W = rng.standard_normal((2, H, dv, dk)) if with_w else None
     ins = dict(q=b.q.astype(np.float64), k=b.k.astype(np.float64), v=b.v.astype(np.float64),
                alpha=b.alpha.astype(np.float64), beta=b.beta.astype(np.float64), S0=S0)
-    g = oracle.adjoint(ins["q"], ins["k"], ins["v"], ins["alpha"], ins["beta"], dO, b.cu_seqlens, C, state_in=S0)
+    g = oracle.adjoint(ins["q"], ins["k"], ins["v"], ins["alpha"], ins["beta"], dO, b.cu_seqlens, C, state_in=S0,
+                       dstate_out=W)
     grads = dict(q=g["dq"], k=g["dk"], v=g["dv"], alpha=g["dalpha"], beta=g["dbeta"], S0=g["dstate_in"])
     h = 1e-30
     for name, base in ins.items():
         for idx in np.ndindex(base.shape):
             x = {k_: v_.astype(np.complex128) for k_, v_ in ins.items()}
             x[name][idx] += 1j * h
-            d = _loss_complex(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], dO, b.cu_seqlens).imag / h
+            d = _loss_complex(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], dO, b.cu_seqlens, W).imag / h
             assert abs(d - grads[name][idx]) <= 1e-12 * max(1.0, abs(d)), (name, idx, d, grads[name][idx])
 
 
@@ -68,6 +76,26 @@ def test_adjoint_closed_form_with_a_frozen_state():
             Gt = dO[t:, h].T @ q[t:, h]
             assert abs(g["dalpha"][t, h] - np.sum(Gt * S0[0, h])) <= 1e-12 * max(1, abs(np.sum(Gt * S0[0, h])))
     assert np.all(g["dv"] == 0) and np.allclose(g["dk"], 0, atol=1e-14)
+
+
+def test_adjoint_closed_form_frozen_state_with_final_gradient():
+    rng = np.random.default_rng(16)
+    T, H, dk, dv = 6, 2, 4, 3
+    q, k, v = (rng.standard_normal((T, H, d)) for d in (dk, dk, dv))
+    alpha, beta = np.ones((T, H)), np.zeros((T, H))
+    S0 = rng.standard_normal((1, H, dv, dk))
+    W = rng.standard_normal((1, H, dv, dk))
+    dO = rng.standard_normal((T, H, dv))
+    g = oracle.adjoint(q, k, v, alpha, beta, dO, np.array([0, T], np.int32), 4, state_in=S0, dstate_out=W)
+    for h in range(H):
+        assert np.allclose(g["dstate_in"][0, h], dO[:, h].T @ q[:, h] + W[0, h], rtol=0, atol=1e-12)
+        for t in range(T):
+            Gt = dO[t:, h].T @ q[t:, h] + W[0, h]
+            assert abs(g["dalpha"][t, h] - np.sum(Gt * S0[0, h])) <= 1e-12 * max(1, abs(np.sum(Gt * S0[0, h])))
+    # an empty sequence passes the final-state gradient straight through
+    e = oracle.adjoint(q[:0], k[:0], v[:0], alpha[:0], beta[:0], dO[:0], np.array([0, 0], np.int32), 4,
+                       dstate_out=W)
+    assert np.array_equal(e["dstate_in"], W)
 
 
 def test_adjoint_is_independent_of_the_checkpoint_span():
