@@ -321,7 +321,7 @@ BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, 
 
 struct BwdArgs {
     const void *q, *k, *v, *dO;
-    const float *alpha, *beta, *states;
+    const float *alpha, *beta, *states, *dstate_out;
     const int32_t* cu;
     int32_t N, H;
     int in_bf16;
@@ -345,7 +345,8 @@ gdn_status_t launch_backward(const BwdArgs& a)
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     if (set_smem(gdn::k_bwd_scan<D, D, C>, SC::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
     gdn::k_bwd_scan<D, D, C><<<(unsigned)((int64_t)a.N * a.H * SC::NT), SC::THREADS, SC::SMEM, a.stream>>>(
-        a.q, a.k, a.alpha, a.beta, a.dO, a.cu, a.ws.t.so, a.ws.t.err, a.H, a.in_bf16, a.ws.ybuf, a.dstate);
+        a.q, a.k, a.alpha, a.beta, a.dO, a.cu, a.ws.t.so, a.ws.t.err, a.H, a.in_bf16, a.dstate_out, a.ws.ybuf,
+        a.dstate);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     const int64_t ntasks = a.tot.tasks * a.H * BC::NT;
@@ -359,7 +360,8 @@ gdn_status_t launch_backward(const BwdArgs& a)
             return GDN_ERR_CUDA;
         const int64_t grid = std::min<int64_t>({ntasks, (int64_t)sms * std::max(occ, 1), kBwdMaxCtas});
         gdn::k_bwd_chunk<D, D, C><<<(unsigned)grid, BC::THREADS, BC::SMEM, a.stream>>>(
-            a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.ws.ybuf, a.cu, a.ws.t.cto, a.ws.t.so, a.ws.t.err, a.N,
+            a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.ws.ybuf, a.dstate_out, a.cu, a.ws.t.cto, a.ws.t.so,
+            a.ws.t.err, a.N,
             a.H, a.T_total, ntasks, a.in_bf16, a.dv, a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.scratch);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
@@ -493,7 +495,7 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
 
 gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v, const float* alpha,
                                     const float* beta, const void* dO, const float* chunk_states,
-                                    const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int32_t num_seqs,
+                                    const float* dstate_out, const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int32_t num_seqs,
                                     int64_t total_tokens, int32_t H, int32_t d_k, int32_t d_v, int32_t C,
                                     gdn_dtype_t in_dtype, float* dq, float* dk, float* dv, float* dalpha,
                                     float* dbeta, float* dstate_in, void* workspace, size_t workspace_bytes,
@@ -506,7 +508,8 @@ gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
     SeqTotals tot;
     if (!seq_totals(cu_seqlens_host, num_seqs, total_tokens, C, &tot)) return GDN_ERR_INVALID_ARG;
     if (cu_seqlens == nullptr || chunk_states == nullptr || dstate_in == nullptr) return GDN_ERR_INVALID_ARG;
-    if (!aligned16(chunk_states) || !aligned16(dstate_in)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(chunk_states) || !aligned16(dstate_in) || (dstate_out && !aligned16(dstate_out)))
+        return GDN_ERR_INVALID_ARG;
     if (total_tokens > 0) {
         if (!q || !k || !v || !alpha || !beta || !dO || !dq || !dk || !dv || !dalpha || !dbeta)
             return GDN_ERR_INVALID_ARG;
@@ -523,6 +526,7 @@ gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
     }
     BwdArgs a;
     a.q = q; a.k = k; a.v = v; a.dO = dO; a.alpha = alpha; a.beta = beta; a.states = chunk_states;
+    a.dstate_out = dstate_out;
     a.cu = cu_seqlens; a.N = num_seqs; a.H = H; a.in_bf16 = in_dtype == GDN_BF16;
     a.dq = dq; a.dk = dk; a.dv = dv; a.dalpha = dalpha; a.dbeta = dbeta; a.dstate = dstate_in;
     a.tot = tot; a.T_total = total_tokens;
@@ -533,15 +537,16 @@ gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
 }
 
 gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const float* alpha, const float* beta,
-                              const void* dO, const float* chunk_states, const int32_t* cu_seqlens,
+                              const void* dO, const float* chunk_states, const float* dstate_out,
+                              const int32_t* cu_seqlens,
                               const int32_t* cu_seqlens_host, int32_t num_seqs, int64_t total_tokens, int32_t H,
                               int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype, float* dq, float* dk,
                               float* dv, float* dalpha, float* dbeta, float* dstate_in, void* workspace,
                               size_t workspace_bytes, void* stream)
 {
-    return gdn_cpr_backward_timed(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, cu_seqlens_host, num_seqs,
-                                  total_tokens, H, d_k, d_v, C, in_dtype, dq, dk, dv, dalpha, dbeta, dstate_in,
-                                  workspace, workspace_bytes, stream, nullptr);
+    return gdn_cpr_backward_timed(q, k, v, alpha, beta, dO, chunk_states, dstate_out, cu_seqlens, cu_seqlens_host,
+                                  num_seqs, total_tokens, H, d_k, d_v, C, in_dtype, dq, dk, dv, dalpha, dbeta,
+                                  dstate_in, workspace, workspace_bytes, stream, nullptr);
 }
 
 gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, const float* alpha,

@@ -97,8 +97,9 @@ __device__ __forceinline__ void load_pairs_slot(f2x (&p)[DK / kLeaves], const fl
     }
 }
 
-// Serial pass over one (sequence, head, row tile): G from the last token to
-// the first, without the gradient outputs.  After the chunk starting at token
+// Serial pass over one (sequence, head, row tile): G from the last token
+// (starting from the final state's gradient, or zero) to the first, without
+// the gradient outputs.  After the chunk starting at token
 // c*C it holds Y_c = dL/dS(c*C) through the tokens >= c*C; Y_c (c >= 1) goes
 // to ybuf at the chunk-state slot so[n] + c, Y_0 = dL/dstate_in to dstate.
 // Tokens are staged raw (bf16 or fp32) by cp.async in blocks of BLK, NBUF
@@ -154,7 +155,8 @@ __device__ __forceinline__ void widen_pairs(f2x (&p)[NP], const unsigned char* s
 template <int DK, int DV, int C, int ES>
 __device__ __forceinline__ void bwd_scan_body(const void* q, const void* k, const float* alpha, const float* beta,
                                               const void* dO, int seq0, int Ln, int64_t slot0, int h, int H, int r,
-                                              float* ybuf, float* dstate_row, unsigned char* sm)
+                                              const float* gfinal_row, float* ybuf, float* dstate_row,
+                                              unsigned char* sm)
 {
     using Cf = ScanCfg<DK, DV, C>;
     using Lt = typename Cf::template L<ES>;
@@ -193,9 +195,19 @@ __device__ __forceinline__ void bwd_scan_body(const void* q, const void* k, cons
         cp_async_commit();
     };
 
+    // G starts from the final state's gradient (zero without one)
     f2x G[NP];
+    if (gfinal_row != nullptr) {
 #pragma unroll
-    for (int m = 0; m < NP; ++m) G[m] = pk2(0.f, 0.f);
+        for (int m = 0; m < NP; m += 2) {
+            const float4 x = *reinterpret_cast<const float4*>(gfinal_row + part * EPT + 2 * m);
+            G[m] = pk2(x.x, x.y);
+            G[m + 1] = pk2(x.z, x.w);
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < NP; ++m) G[m] = pk2(0.f, 0.f);
+    }
 #pragma unroll
     for (int i = 0; i < NBUF - 1; ++i) issue(i);
     for (int i = 0; i < nblk; ++i) {
@@ -247,10 +259,14 @@ __device__ __forceinline__ void bwd_scan_body(const void* q, const void* k, cons
         }
     }
     cp_async_wait_all();
-    if (Ln == 0) {  // no tokens: dL/dstate_in = 0
+    if (Ln == 0) {  // no tokens: dL/dstate_in is the final state's gradient
 #pragma unroll
-        for (int m = 0; m < NP; m += 2)
-            *reinterpret_cast<float4*>(dstate_row + part * EPT + 2 * m) = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int m = 0; m < NP; m += 2) {
+            float x0, x1, x2, x3;
+            up2(G[m], x0, x1);
+            up2(G[m + 1], x2, x3);
+            *reinterpret_cast<float4*>(dstate_row + part * EPT + 2 * m) = make_float4(x0, x1, x2, x3);
+        }
     }
 }
 
@@ -259,7 +275,7 @@ __global__ void __launch_bounds__(ScanCfg<DK, DV, C>::THREADS)
 k_bwd_scan(const void* __restrict__ q, const void* __restrict__ k, const float* __restrict__ alpha,
            const float* __restrict__ beta, const void* __restrict__ dO, const int32_t* __restrict__ cu,
            const int32_t* __restrict__ so, const int32_t* __restrict__ err, int H, int in_bf16,
-           float* __restrict__ ybuf, float* __restrict__ dstate)
+           const float* __restrict__ dstate_out, float* __restrict__ ybuf, float* __restrict__ dstate)
 {
     using Cf = ScanCfg<DK, DV, C>;
     if (__ldg(err)) return;
@@ -272,11 +288,15 @@ k_bwd_scan(const void* __restrict__ q, const void* __restrict__ k, const float* 
     const int Ln = __ldg(cu + n + 1) - seq0;
     const int64_t slot0 = __ldg(so + n);
     const int row = threadIdx.x / Cf::TPR;
-    float* dstate_row = dstate + ((int64_t)nh * DV + r * Cf::RT + row) * DK;
+    const int64_t roff = ((int64_t)nh * DV + r * Cf::RT + row) * DK;
+    float* dstate_row = dstate + roff;
+    const float* gfinal_row = dstate_out != nullptr ? dstate_out + roff : nullptr;
     if (in_bf16)
-        bwd_scan_body<DK, DV, C, 2>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, ybuf, dstate_row, sm);
+        bwd_scan_body<DK, DV, C, 2>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, gfinal_row, ybuf, dstate_row,
+                                    sm);
     else
-        bwd_scan_body<DK, DV, C, 4>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, ybuf, dstate_row, sm);
+        bwd_scan_body<DK, DV, C, 4>(q, k, alpha, beta, dO, seq0, Ln, slot0, h, H, r, gfinal_row, ybuf, dstate_row,
+                                    sm);
 }
 
 // One forward P_tok step (the forward's operations) on RHO rows of this lane
@@ -354,12 +374,14 @@ __device__ __forceinline__ void slot_load(f2x (&Sp)[RHO][DK / kLeaves], const fl
 // the lane adds its rows' dq / dk terms before they go to shared memory.  A
 // task starts from G = Y_{c+1} (zero after the last chunk), recomputes the
 // chunk's states from its boundary state and writes dv rows, and the tile's
-// row sums of dq, dk ([NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).
+// row sums of dq, dk ([NT][T][H][DK]) and dalpha, dbeta ([NT][T][H]).  The
+// last chunk of a sequence starts from the final state's gradient when given.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(BwdCfg<DK, DV, C>::THREADS)
 k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
             const float* __restrict__ alpha, const float* __restrict__ beta, const void* __restrict__ dO,
-            const float* __restrict__ states, const float* __restrict__ ybuf, const int32_t* __restrict__ cu,
+            const float* __restrict__ states, const float* __restrict__ ybuf,
+            const float* __restrict__ dstate_out, const int32_t* __restrict__ cu,
             const int32_t* __restrict__ cto, const int32_t* __restrict__ so, const int32_t* __restrict__ err,
             int N, int H, int64_t T_total, int64_t ntasks, int in_bf16, float* __restrict__ dv,
             float* __restrict__ pq, float* __restrict__ pk, float* __restrict__ pa, float* __restrict__ pb,
@@ -436,6 +458,8 @@ k_bwd_chunk(const void* __restrict__ q, const void* __restrict__ k, const void* 
         for (int r = 0; r < RHO; ++r) {
             if (c + 1 < nchunks) {
                 load_row_pairs<DK>(G[r], ybuf + (((slot0 + c + 1) * H + h) * DV + grow0 + r) * DK + part * EPT);
+            } else if (dstate_out != nullptr) {  // the last chunk starts from the final state's gradient
+                load_row_pairs<DK>(G[r], dstate_out + (((int64_t)n * H + h) * DV + grow0 + r) * DK + part * EPT);
             } else {
 #pragma unroll
                 for (int m = 0; m < L; ++m) G[r][m] = pk2(0.f, 0.f);

@@ -88,7 +88,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_cpr_backward_workspace_size.restype = sz
     lib.gdn_cpr_backward_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
     lib.gdn_cpr_backward.restype = ctypes.c_int
-    lib.gdn_cpr_backward.argtypes = [P, P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
+    lib.gdn_cpr_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
                                      P, P, P, P, P, P, P, sz, P]
     lib.gdn_cpr_backward_timed.restype = ctypes.c_int
     lib.gdn_cpr_backward_timed.argtypes = lib.gdn_cpr_backward.argtypes + [P]
@@ -235,11 +235,13 @@ def gdn_cpr_backward_workspace_size(total_tokens: int, num_seqs: int, H: int, d_
 
 
 def gdn_cpr_backward(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, C: int, *, cu_seqlens_host=None,
-                     workspace=None, grads=None, events=None):
+                     dstate_out=None, workspace=None, grads=None, events=None):
     """CPR backward: gradients of sum(dO * o) for the forward of the same inputs.
 
     q, k, v, alpha, beta, cu_seqlens: as given to :func:`gdn_cpr_forward`;
-    dO [T,H,d_v] in q's dtype; chunk_states: that forward's chunk states.
+    dO [T,H,d_v] in q's dtype; chunk_states: that forward's chunk states;
+    dstate_out [N,H,d_v,d_k] fp32 or None: the loss gradient for each
+    sequence's final state (a later part's dstate_in, when a sequence is split).
     Returns (dq, dk, dv, dalpha, dbeta, dstate_in), all fp32.  ``grads``: an
     optional tuple of those six tensors to write into.  ``events``: optional
     4 torch.cuda.Events recorded around the kernels (gdn_cpr_backward_timed)."""
@@ -258,7 +260,7 @@ def gdn_cpr_backward(q, k, v, alpha, beta, dO, chunk_states, cu_seqlens, C: int,
     if workspace is None:
         workspace = torch.empty(lib.gdn_cpr_backward_workspace_size(T, N, H, dk, dv, C), dtype=torch.uint8,
                                 device=dev)
-    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(dO), _ptr(chunk_states),
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(dO), _ptr(chunk_states), _ptr(dstate_out),
             _ptr(cu_seqlens), cu_h, N, T, H, dk, dv, C, _dt(q.dtype),
             *[_ptr(g) for g in grads], _ptr(workspace), workspace.numel(), _stream(dev))
     if events is None:

@@ -209,6 +209,11 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
  *     H, d_k, d_v, C, in_dtype: as given to gdn_cpr_forward.
  *   dO [T_total,H,d_v] in in_dtype: the gradient of the loss for o.
  *   chunk_states: the forward's chunk_states output for these inputs.
+ *   dstate_out [num_seqs,H,d_v,d_k] fp32, or NULL for zeros: the gradient of
+ *     the loss for each sequence's final state (the state after its last
+ *     token).  A sequence split at a chunk boundary runs its later part's
+ *     backward first and passes that call's dstate_in here to the earlier
+ *     part: the result equals the unsplit backward bit for bit.
  * Outputs (fp32, device, caller-owned, every element written):
  *   dq, dk [T_total,H,d_k]; dv [T_total,H,d_v]; dalpha, dbeta [T_total,H];
  *   dstate_in [num_seqs,H,d_v,d_k]: the gradient for the forward's state_in.
@@ -221,7 +226,7 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
  */
 gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v,
                               const float* alpha, const float* beta, const void* dO,
-                              const float* chunk_states,
+                              const float* chunk_states, const float* dstate_out,
                               const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                               int32_t num_seqs, int64_t total_tokens, int32_t H,
                               int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
@@ -236,7 +241,7 @@ gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v,
  */
 gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, const void* dO,
-                                    const float* chunk_states,
+                                    const float* chunk_states, const float* dstate_out,
                                     const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                                     int32_t num_seqs, int64_t total_tokens, int32_t H,
                                     int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,

@@ -99,7 +99,7 @@ def _bwd(lib, **kw):
     cu = kw.get("cu", [0, 32])
     cu_h = (ctypes.c_int32 * len(cu))(*cu)
     fake = P(1 << 20)  # never dereferenced: validation fails first
-    args = dict(q=fake, k=fake, v=fake, alpha=fake, beta=fake, dO=fake, states=fake, cu=fake, cu_host=cu_h,
+    args = dict(q=fake, k=fake, v=fake, alpha=fake, beta=fake, dO=fake, states=fake, ds_out=None, cu=fake, cu_host=cu_h,
                 N=len(cu) - 1, T=cu[-1], H=2, dk=16, dv=16, C=16, idt=0, dq=fake, dk_=fake, dv_=fake, da=fake,
                 db=fake, ds=fake, ws=fake, wsb=1 << 30, stream=None)
     args.update({k: v for k, v in kw.items() if k != "cu"})
@@ -115,6 +115,7 @@ def test_backward_rejects_bad_arguments(lib):
     assert _bwd(lib, dO=ctypes.c_void_p((1 << 20) + 4)) == 1   # misaligned
     assert _bwd(lib, states=None) == 1
     assert _bwd(lib, ds=None) == 1
+    assert _bwd(lib, ds_out=ctypes.c_void_p((1 << 20) + 8)) == 1   # misaligned final-state gradient
     assert _bwd(lib, dq=None) == 1
     assert _bwd(lib, wsb=16) == 4                        # workspace too small
     assert _bwd(lib, ws=None) == 4

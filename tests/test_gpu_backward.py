@@ -146,3 +146,62 @@ def test_backward_gate_extremes_vs_oracle():
     got = run(b, C, S0, dO)
     ref = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, C, S0)
     check(got, ref, "gate extremes")
+
+
+def test_backward_final_state_gradient_vs_oracle():
+    """dstate_out (the loss gradient for each sequence's final state) against
+    the oracle; an empty sequence passes it straight to dstate_in."""
+    C, d, H = 32, 64, 2
+    lens = [2 * C + 5, 0, C]
+    b = synth.make_batch(91, lens, H, d, d, "bf16")
+    rng = np.random.default_rng(19)
+    S0 = (rng.standard_normal((3, H, d, d)) * 0.2).astype(np.float32)
+    W = (rng.standard_normal((3, H, d, d)) * 0.1).astype(np.float32)
+    dO = _dO(13, b.q.shape[0], H, d, "bf16")
+    dd = to_device(b)
+    _, st = gdn.gdn_cpr_forward(dd["q"], dd["k"], dd["v"], dd["alpha"], dd["beta"], dd["cu_seqlens"], C,
+                                cu_seqlens_host=dd["cu_host"], state_in=torch.from_numpy(S0).to(DEV),
+                                out_dtype=torch.float32)
+    g = gdn.gdn_cpr_backward(dd["q"], dd["k"], dd["v"], dd["alpha"], dd["beta"],
+                             torch.from_numpy(dO).to(DEV).to(torch.bfloat16), st, dd["cu_seqlens"], C,
+                             cu_seqlens_host=dd["cu_host"], dstate_out=torch.from_numpy(W).to(DEV))
+    torch.cuda.synchronize()
+    got = [x.cpu().numpy() for x in g]
+    ref = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, C, S0, dstate_out=W)
+    check(got, ref, "dstate_out")
+    assert np.array_equal(bits(got[5][1]), bits(W[1]))
+
+
+def test_backward_split_at_chunk_boundary_equals_unsplit_bitwise():
+    """A sequence split at a chunk boundary: the later part's backward first,
+    its dstate_in as the earlier part's dstate_out.  Every gradient equals the
+    unsplit backward bit for bit (the trainer's bf16 shape)."""
+    C, d, H = 64, 128, 2
+    L, s = 5 * C + 9, 3 * C
+    b = synth.make_batch(93, [L], H, d, d, "bf16")
+    dd = to_device(b)
+    rng = np.random.default_rng(23)
+    S0 = torch.from_numpy((rng.standard_normal((1, H, d, d)) * 0.2).astype(np.float32)).to(DEV)
+    W = torch.from_numpy((rng.standard_normal((1, H, d, d)) * 0.1).astype(np.float32)).to(DEV)
+    dO = torch.from_numpy(_dO(17, L, H, d, "bf16")).to(DEV).to(torch.bfloat16)
+    x = {n: dd[n] for n in ("q", "k", "v", "alpha", "beta")}
+
+    def fwd_bwd(sl, state_in, dstate_out):
+        part = {n: t[sl].contiguous() for n, t in x.items()}
+        n_tok = part["q"].shape[0]
+        cu = torch.tensor([0, n_tok], dtype=torch.int32, device=DEV)
+        _, st = gdn.gdn_cpr_forward(part["q"], part["k"], part["v"], part["alpha"], part["beta"], cu, C,
+                                    cu_seqlens_host=[0, n_tok], state_in=state_in)
+        g = gdn.gdn_cpr_backward(part["q"], part["k"], part["v"], part["alpha"], part["beta"], dO[sl].contiguous(),
+                                 st, cu, C, cu_seqlens_host=[0, n_tok], dstate_out=dstate_out)
+        return st, g
+
+    st_full, g_full = fwd_bwd(slice(0, L), S0, W)
+    st1, _ = fwd_bwd(slice(0, s), S0, None)                 # the earlier part's forward: its last state
+    _, g2 = fwd_bwd(slice(s, L), st1[-1:].contiguous(), W)  # the later part, from that state
+    _, g1 = fwd_bwd(slice(0, s), S0, g2[5])                 # the earlier part, with the later part's dstate_in
+    torch.cuda.synchronize()
+    for i in range(5):
+        assert np.array_equal(bits(g1[i]), bits(g_full[i][:s])), i
+        assert np.array_equal(bits(g2[i]), bits(g_full[i][s:])), i
+    assert np.array_equal(bits(g1[5]), bits(g_full[5]))
