@@ -18,8 +18,8 @@
 // the last token to the first and stores it at every chunk boundary.  Then
 // every chunk is independent: k_bwd_chunk starts from the boundary G after the
 // chunk, recomputes the chunk's states from the forward's boundary state
-// (one checkpoint per SUB tokens, kept in an L2-resident per-CTA scratch) and
-// runs the per-token backward above.  Every row i of S and G evolves on its
+// (one checkpoint per SUB tokens in a per-CTA global scratch, the current one
+// and its midpoint in shared memory) and runs the per-token backward above.  Every row i of S and G evolves on its
 // own, so both kernels split d_v into row tiles; dq, dk, dalpha and dbeta sum
 // over rows, and the tiles' sums are added in a fixed order by k_bwd_reduce,
 // so the gradients are deterministic.  Everything is fp32.
