@@ -23,6 +23,7 @@ import numpy as np
 
 from . import build as _build
 from . import chunkwise as _chunkwise
+from . import chunkwise_adjoint as _chunkwise_adjoint
 
 _lib = None
 
@@ -108,6 +109,11 @@ def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=N
     if rc:
         raise RuntimeError(f"oracle_adjoint_fp64 failed ({rc})")
     return out
+
+
+def adjoint_chunkwise(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=None):
+    """Independent fp64 chunkwise form of the adjoint (see :mod:`oracle.chunkwise_adjoint`)."""
+    return _chunkwise_adjoint.adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in, dstate_out)
 
 
 def chunkwise(q, k, v, alpha, beta, cu_seqlens, C, state_in=None):

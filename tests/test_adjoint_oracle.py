@@ -12,6 +12,9 @@ L = sum_t dO_t . o_t through the gated delta rule.
 * A gradient W for each final state (dstate_out) adds <W, S_final> to the
   loss: the complex-step check includes that term, and in the closed form
   W adds to dS_0 and to every G.
+* Two independent forms agree: the token-by-token reverse sweep and the
+  chunkwise form (oracle/chunkwise_adjoint.py: triangular solves and dense
+  chunk products, no division by a gate), including alpha = 0 tokens.
 """
 import numpy as np
 import pytest
@@ -105,3 +108,21 @@ def test_adjoint_is_independent_of_the_checkpoint_span():
     c = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, 16)
     for key in a:
         assert np.allclose(a[key], c[key], rtol=1e-12, atol=1e-12), key
+
+
+@pytest.mark.parametrize("C,lens,dt", [(4, [7, 4, 0], "f32"), (16, [37, 16, 5], "bf16"), (8, [20, 9], "f32")])
+def test_chunkwise_adjoint_agrees_with_the_token_sweep(C, lens, dt):
+    b = synth.make_batch(31, lens, 2, 8, 6, dt)
+    rng = np.random.default_rng(C)
+    T = b.q.shape[0]
+    b.alpha[rng.choice(T, size=3, replace=False), 0] = 0.0   # resets
+    b.beta[rng.choice(T, size=2, replace=False), 1] = 0.0
+    b.beta[rng.choice(T, size=2, replace=False), 0] = 1.0
+    S0 = rng.standard_normal((len(lens), 2, 6, 8)) * 0.3
+    W = rng.standard_normal((len(lens), 2, 6, 8)) * 0.2
+    dO = rng.standard_normal((T, 2, 6))
+    r = oracle.adjoint(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, C, S0, dstate_out=W)
+    c = oracle.adjoint_chunkwise(b.q, b.k, b.v, b.alpha, b.beta, dO, b.cu_seqlens, C, S0, dstate_out=W)
+    for key in r:
+        scale = max(np.max(np.abs(r[key])), 1e-12)
+        assert np.max(np.abs(r[key] - c[key])) <= 1e-11 * scale, key
