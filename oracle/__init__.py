@@ -111,9 +111,11 @@ def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=N
     return out
 
 
-def adjoint_chunkwise(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=None):
-    """Independent fp64 chunkwise form of the adjoint (see :mod:`oracle.chunkwise_adjoint`)."""
-    return _chunkwise_adjoint.adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in, dstate_out)
+def adjoint_chunkwise(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=None,
+                      dtype=np.float64):
+    """Independent chunkwise form of the adjoint (see :mod:`oracle.chunkwise_adjoint`),
+    fp64 unless ``dtype`` says otherwise."""
+    return _chunkwise_adjoint.adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in, dstate_out, dtype)
 
 
 def chunkwise(q, k, v, alpha, beta, cu_seqlens, C, state_in=None):

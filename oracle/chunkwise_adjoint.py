@@ -42,7 +42,7 @@ from scipy.linalg import solve_triangular
 def _decays(a: np.ndarray) -> np.ndarray:
     """D[t, s] = prod_{r=s+1..t} a_r for 0 <= s <= t <= n (tokens 1..n), 0 elsewhere."""
     n = a.shape[0]
-    D = np.zeros((n + 1, n + 1))
+    D = np.zeros((n + 1, n + 1), dtype=a.dtype)
     for s in range(n + 1):
         D[s, s] = 1.0
         for t in range(s + 1, n + 1):
@@ -50,37 +50,39 @@ def _decays(a: np.ndarray) -> np.ndarray:
     return D
 
 
-def chunk_backward(S0, Y, q, k, v, a, b, dO):
+def chunk_backward(S0, Y, q, k, v, a, b, dO, dtype=np.float64):
     """One chunk (n tokens, arrays [n, d]) from start state S0 [dv, dk] and end
     gradient Y [dv, dk].  Returns (dq, dk, dv, dalpha, dbeta, gradient at the
-    chunk start, end state)."""
+    chunk start, end state).  ``dtype`` is the arithmetic type (float64; a
+    float32 evaluation measures the form's rounding for an fp32 kernel)."""
+    S0, Y, q, k, v, a, b, dO = (np.asarray(x, dtype) for x in (S0, Y, q, k, v, a, b, dO))
     n = q.shape[0]
-    D = _decays(a)
+    D = _decays(a).astype(dtype)
     Dt = D[1:, 1:]                 # D[t, s], t, s = 1..n
     g = D[1:, 0]                   # D[t, 0]
     gp = D[:-1, 0]                 # D[t-1, 0]
     Dp = D[:-1, 1:]                # Dp[t, r] = D[t-1, r] (nonzero for r < t)
     dn = D[n, 1:]                  # D[n, t]
     KK, KQ = k @ k.T, k @ q.T
-    lower = np.tril(np.ones((n, n)), -1)
+    lower = np.tril(np.ones((n, n), dtype), -1)
     A = b[:, None] * Dt * KK * lower
-    Delta = solve_triangular(np.eye(n) + A, b[:, None] * (v - g[:, None] * (k @ S0.T)), lower=True,
-                             unit_diagonal=True)
+    Delta = solve_triangular(np.eye(n, dtype=dtype) + A, b[:, None] * (v - g[:, None] * (k @ S0.T)), lower=True,
+                             unit_diagonal=True).astype(dtype)
     U = gp[:, None] * (k @ S0.T) + (Dp * KK.T * lower) @ Delta           # u_t = S_{t-1} k_t
     S_end = D[n, 0] * S0 + (dn[:, None] * Delta).T @ k
     # backward substitution for ddelta
-    M = Dt.T * KQ * np.triu(np.ones((n, n)))                              # M[t, s] = D[s, t] (k_t . q_s), s >= t
+    M = Dt.T * KQ * np.triu(np.ones((n, n), dtype))                       # M[t, s] = D[s, t] (k_t . q_s), s >= t
     rhs = dn[:, None] * (k @ Y.T) + M @ dO
-    Dd = solve_triangular(np.eye(n) + A.T, rhs, lower=False, unit_diagonal=True)
+    Dd = solve_triangular(np.eye(n, dtype=dtype) + A.T, rhs, lower=False, unit_diagonal=True).astype(dtype)
     dv = b[:, None] * Dd
     dbeta = np.sum(Dd * (v - a[:, None] * U), axis=1)
     DoDel = dO @ Delta.T                                                  # [t, r] = dO_t . delta_r
-    incl = np.tril(np.ones((n, n)))
+    incl = np.tril(np.ones((n, n), dtype))
     dq = g[:, None] * (dO @ S0) + (Dt * DoDel * incl) @ k
     DelDo = DoDel.T                                                       # [t, s] = delta_t . dO_s
     DelDd = Delta @ Dd.T                                                  # [t, s] = delta_t . ddelta_s
-    upper_incl = np.triu(np.ones((n, n)))
-    upper = np.triu(np.ones((n, n)), 1)
+    upper_incl = np.triu(np.ones((n, n), dtype))
+    upper = np.triu(np.ones((n, n), dtype), 1)
     dk = (dn[:, None] * (Delta @ Y) + (Dt.T * DelDo * upper_incl) @ q
           - (Dt.T * DelDd * upper * b[None, :]) @ k
           - (a * b)[:, None] * (gp[:, None] * (Dd @ S0) + (Dp * DelDd.T * lower) @ k))
@@ -91,7 +93,7 @@ def chunk_backward(S0, Y, q, k, v, a, b, dO):
     cv = np.sum((Delta @ Y) * k, axis=1)        # delta_r^T Y k_r
     E1 = DelDo * KQ                             # (delta_r . dO_s)(k_r . q_s)
     E2 = DelDd * KK                             # (delta_r . ddelta_s)(k_r . k_s)
-    dalpha = np.zeros(n)
+    dalpha = np.zeros(n, dtype)
     for t in range(n):
         w_ge = Dt[t:, t]                                      # D[s, t] for s >= t
         w_gt = Dt[t + 1:, t] * b[t + 1:]                      # D[s, t] beta_s for s > t
@@ -104,9 +106,10 @@ def chunk_backward(S0, Y, q, k, v, a, b, dO):
     return dq, dk, dv, dalpha, dbeta, G0, S_end
 
 
-def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=None):
-    """fp64 gradient of sum dO . o (+ <dstate_out, final state>) per sequence
-    and head, chunk by chunk.  Same layouts and results as oracle.adjoint."""
+def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=None, dtype=np.float64):
+    """Gradient of sum dO . o (+ <dstate_out, final state>) per sequence and
+    head, chunk by chunk, in ``dtype`` arithmetic (fp64 by default).  Same
+    layouts and results as oracle.adjoint."""
     q, k, v, dO = (np.asarray(x, np.float64) for x in (q, k, v, dO))
     alpha, beta = np.asarray(alpha, np.float64), np.asarray(beta, np.float64)
     cu = np.asarray(cu_seqlens)
@@ -124,11 +127,11 @@ def adjoint(q, k, v, alpha, beta, dO, cu_seqlens, C, state_in=None, dstate_out=N
             for s0, s1 in spans:          # forward: the state at every chunk start
                 starts.append(S)
                 *_, S = chunk_backward(S, np.zeros((dv_, dk_)), q[s0:s1, h], k[s0:s1, h], v[s0:s1, h],
-                                       alpha[s0:s1, h], beta[s0:s1, h], dO[s0:s1, h])
+                                       alpha[s0:s1, h], beta[s0:s1, h], dO[s0:s1, h], dtype)
             Y = np.zeros((dv_, dk_)) if dstate_out is None else np.asarray(dstate_out, np.float64)[n, h].copy()
             for (s0, s1), S0 in reversed(list(zip(spans, starts))):
                 dq, dkk, dvv, da, db, Y, _ = chunk_backward(S0, Y, q[s0:s1, h], k[s0:s1, h], v[s0:s1, h],
-                                                            alpha[s0:s1, h], beta[s0:s1, h], dO[s0:s1, h])
+                                                            alpha[s0:s1, h], beta[s0:s1, h], dO[s0:s1, h], dtype)
                 out["dq"][s0:s1, h], out["dk"][s0:s1, h], out["dv"][s0:s1, h] = dq, dkk, dvv
                 out["dalpha"][s0:s1, h], out["dbeta"][s0:s1, h] = da, db
             out["dstate_in"][n, h] = Y
