@@ -88,7 +88,7 @@ NCU_TRAFFIC = {
     # profiles/k_dec_tok_decode_N64_H32_d128_C64.md: 135,935,744 read + 77,555,200 written
     ("k_dec_tok", "51b392a62fe51a33"): 213490944,
     # profiles/k_bwd_trainer_B2_H32_T8192_d128_C64.md: 2,963,502,592 read + 4,436,340,736 written
-    ("k_bwd_chunk", "19f547b7f0a0907e"): 7399843328,
+    ("k_bwd_chunk", "86633ff16a2874d1"): 7399843328,
 }
 
 KERNEL_SOURCES = {

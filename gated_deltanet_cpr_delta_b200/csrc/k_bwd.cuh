@@ -42,7 +42,7 @@ struct BwdCfg {
     // staged floats per token: k, q (slots), v, dO rows, gates; a multiple of 4 (16-byte rows)
     static constexpr int TOKF = ((2 * RS::KS + 2 * RT + 2) + 3) / 4 * 4;
     static constexpr int RED = DK + 4;            // reduction buffer row stride
-    // smem: SUB staged tokens | dq rows | dk rows | [NG][2] scalars | the current checkpoint (lane-private rows)
+    // smem: SUB staged tokens | dq rows | dk rows | [NG][2] scalars | two lane-private state slots
     static constexpr int TOK_OFF = 0;
     static constexpr int RQ_OFF = TOK_OFF + SUB * TOKF;
     static constexpr int RK_OFF = RQ_OFF + NG * RED;
@@ -99,9 +99,9 @@ __device__ __forceinline__ void load_pairs_slot(f2x (&p)[DK / kLeaves], const fl
 
 // Serial pass over one (sequence, head, row tile): G from the last token
 // (starting from the final state's gradient, or zero) to the first, without
-// the gradient outputs.  After the chunk starting at token
-// c*C it holds Y_c = dL/dS(c*C) through the tokens >= c*C; Y_c (c >= 1) goes
-// to ybuf at the chunk-state slot so[n] + c, Y_0 = dL/dstate_in to dstate.
+// the gradient outputs.  After the chunk starting at token c*C it holds
+// Y_c = dL/dS(c*C) through the tokens >= c*C; Y_c (c >= 1) goes to ybuf at
+// the chunk-state slot so[n] + c, Y_0 = dL/dstate_in to dstate.
 // Tokens are staged raw (bf16 or fp32) by cp.async in blocks of BLK, NBUF
 // blocks in flight; each lane widens its own slice.  The lane's EPT columns
 // are held as pairs of adjacent columns.  (Widening a bf16 block once into an
