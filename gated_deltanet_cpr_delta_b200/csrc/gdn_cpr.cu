@@ -517,6 +517,8 @@ gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
             !aligned16(dv))
             return GDN_ERR_INVALID_ARG;
     }
+    // grids of (sequence, head, row tile) and (chunk, head, row tile) index with 32-bit integers
+    if ((int64_t)num_seqs * H * d_v > INT32_MAX || tot.tasks * H > INT32_MAX) return GDN_ERR_INVALID_ARG;
     const BwdWorkspace need = carve_bwd(nullptr, total_tokens, num_seqs, H, d_k, d_v, C);
     if (workspace == nullptr || workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return GDN_ERR_INVALID_ARG;
