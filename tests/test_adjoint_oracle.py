@@ -142,3 +142,30 @@ def test_chunkwise_adjoint_in_fp32_is_well_inside_the_backward_tolerance():
     for key in r:
         scale = max(np.max(np.abs(r[key])), 1e-12)
         assert np.max(np.abs(r[key] - c[key].astype(np.float64))) <= 2e-6 * scale, key
+
+
+def test_backward_chain_step_is_the_forward_chain_transposed():
+    """The chunk-start gradient of the chunkwise adjoint equals
+    gamma_n Y - (Y Kt^T) W + F_c with W = T diag(D[.,0] beta) K,
+    Kt = diag(D[n,.]) K and F_c from the chunk's own inputs; and the end
+    state equals gamma_n S0 - (S0 W^T) Kt + U0^T Kt (the forward's update)."""
+    from oracle import chunkwise_adjoint as ca
+    rng = np.random.default_rng(41)
+    n, dk, dv = 12, 8, 6
+    q, k = rng.standard_normal((n, dk)), rng.standard_normal((n, dk))
+    v, dO = rng.standard_normal((n, dv)), rng.standard_normal((n, dv))
+    a, b = rng.uniform(0.3, 1.0, n), rng.uniform(0.0, 1.0, n)
+    a[4] = 0.0
+    S0, Y = rng.standard_normal((dv, dk)), rng.standard_normal((dv, dk))
+    *_, G0, S_end = ca.chunk_backward(S0, Y, q, k, v, a, b, dO)
+    D = ca._decays(a)
+    g, dn, gn = D[1:, 0], D[n, 1:], D[n, 0]
+    A = b[:, None] * D[1:, 1:] * (k @ k.T) * np.tril(np.ones((n, n)), -1)
+    T = np.linalg.inv(np.eye(n) + A)
+    W = T @ ((g * b)[:, None] * k)
+    U0 = T @ (b[:, None] * v)
+    Kt = dn[:, None] * k
+    M = D[1:, 1:].T * (k @ q.T) * np.triu(np.ones((n, n)))
+    F = dO.T @ (g[:, None] * q) - (T.T @ M @ dO).T @ ((g * b)[:, None] * k)
+    assert np.allclose(G0, gn * Y - (Y @ Kt.T) @ W + F, rtol=0, atol=1e-12)
+    assert np.allclose(S_end, gn * S0 - (S0 @ W.T) @ Kt + U0.T @ Kt, rtol=0, atol=1e-12)
