@@ -5,7 +5,6 @@ import ctypes
 import os
 import re
 
-import numpy as np
 import pytest
 
 from gated_deltanet_cpr_delta_b200 import build, gdn
