@@ -147,8 +147,9 @@ def test_chunkwise_adjoint_in_fp32_is_well_inside_the_backward_tolerance():
 def test_backward_chain_step_is_the_forward_chain_transposed():
     """The chunk-start gradient of the chunkwise adjoint equals
     gamma_n Y - (Y Kt^T) W + F_c with W = T diag(D[.,0] beta) K,
-    Kt = diag(D[n,.]) K and F_c from the chunk's own inputs; and the end
-    state equals gamma_n S0 - (S0 W^T) Kt + U0^T Kt (the forward's update)."""
+    Kt = diag(D[n,.]) K and F_c from the chunk's own inputs; the end state
+    equals gamma_n S0 - (S0 W^T) Kt + U0^T Kt (the forward's update); and W,
+    U0 are what the forward's chunk-local forward substitution produces."""
     from oracle import chunkwise_adjoint as ca
     rng = np.random.default_rng(41)
     n, dk, dv = 12, 8, 6
@@ -169,6 +170,14 @@ def test_backward_chain_step_is_the_forward_chain_transposed():
     F = dO.T @ (g[:, None] * q) - (T.T @ M @ dO).T @ ((g * b)[:, None] * k)
     assert np.allclose(G0, gn * Y - (Y @ Kt.T) @ W + F, rtol=0, atol=1e-12)
     assert np.allclose(S_end, gn * S0 - (S0 @ W.T) @ Kt + U0.T @ Kt, rtol=0, atol=1e-12)
+    # W and U0 are the forward's chunk-local precompute, by its forward substitution:
+    # w_t = beta_t (D[t,0] k_t - sum_{s<t} D[t,s] (k_s . k_t) w_s), u0_t likewise with v_t
+    w, u0 = np.zeros((n, dk)), np.zeros((n, dv))
+    for t in range(n):
+        c = D[t + 1, 1:t + 1] * (k[:t] @ k[t])
+        w[t] = b[t] * (D[t + 1, 0] * k[t] - c @ w[:t])
+        u0[t] = b[t] * (v[t] - c @ u0[:t])
+    assert np.allclose(w, W, rtol=0, atol=1e-12) and np.allclose(u0, U0, rtol=0, atol=1e-12)
 
 
 def test_adjoint_forms_agree_on_random_shapes():
