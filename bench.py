@@ -280,8 +280,9 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- native
 def parity_gate(d, o, st, C):
-    """Sequence 0, head 0: bitwise vs the fp32 schedule model, and the max
-    error vs the fp64 oracle (bench refuses to report a speed without it)."""
+    """Sequence 0, head 0 of the first forward: bitwise vs the fp32 schedule
+    model, and the max error vs the fp64 oracle.  Runs in the CPU-baseline
+    leg (rank 0, one GPU), the one part of the native arm that runs the oracle."""
     import numpy as np
     import torch
     import oracle
@@ -441,7 +442,10 @@ def run_native(args):
                                                   workspace=ws, events=events)
     fwd()
     torch.cuda.synchronize()
-    parity = parity_gate(d, o, st, C) if rank == 0 else None
+    # sequence 0, head 0 of this first forward; the CPU-baseline leg checks it against the oracle
+    L0 = d["cu_host"][1]
+    par_o, par_st = o[:L0, 0:1].clone(), st[:L0 // C + 1, 0:1].clone()
+    parity = None
 
     for _ in range(args.warmup):
         fwd()
@@ -588,6 +592,7 @@ def run_native(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
+        line["parity"] = parity_gate(d, par_o, par_st, C)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
