@@ -9,12 +9,18 @@ C=64, bf16 q/k/v, fp32 gates and state.  Inputs are synthetic, from the
 device recipe of gated_deltanet_cpr_delta_b200.synth.  The line also
 reports decode tokens/s for the decode workload (64 sequences x 32 heads,
 prefilled to 2048 tokens, then 256 decode steps) and trainer fwd+bwd tokens/s
-(B=2 x 8192 tokens, 32 heads, forward then gdn_cpr_backward).
+(B=2 x 8192 tokens, 32 heads, forward then gdn_cpr_backward) and varlen
+tokens/s (32 packed sequences of 128..8192 tokens, 32 heads).
 
 With N > 1 (torchrun, one rank per GPU) every rank runs its own sequences
 (weak scaling, no data-path collective).  Timing is CUDA events on the
 launching stream, the max over ranks.  L2 is flushed (a 256 MiB write)
 before every timed step.  Rank 0 prints one JSON line.
+
+Rank 0 checks the first forward against the oracle (the parity gate) before
+it prints: if the gate fails, the line carries "value": null and the
+process exits 1.  It also times the oracle on the host cores (cpu_baseline;
+--no-cpu-baseline skips only that timing).
 
 --impl reference times the CPU oracle (fp64 recurrence, OpenMP) on the host
 cores, on a bounded sample of the same workload.
@@ -41,6 +47,8 @@ DECODE = dict(name="decode 64 seqs H=32 d=128 C=64: prefill 2048, then 256 steps
               C=64, Lp=2048, steps=256)
 TRAIN = dict(name="trainer fwd+bwd B=2 H=32 T=8192 d_k=d_v=128 C=64 bf16, dO ~ N(0,1) bf16", seed=4, B=2, H=32,
              T=8192, D=128, C=64)
+VARLEN = dict(name="varlen 32 seqs L~U[128,8192] H=32 d_k=d_v=128 C=64 bf16", seed=3, N=32, H=32, D=128, C=64,
+              lo=128, hi=8192)
 
 # FP32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flop (fma) x 1.965 GHz (max SM clock)
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -83,12 +91,9 @@ def backward_flops(tokens_heads: int, dk: int, dv: int):
 # dram__bytes_write.sum), keyed by kernel and by the sha256 of the sources that
 # kernel is compiled from; a changed source drops the figure (reported null).
 NCU_TRAFFIC = {
-    # profiles/k_chain_tok_prefill_B4_H16_T4096_d128_C64.md: 789,160,960 read + 329,176,320 written
-    ("k_chain_tok", "5a5969a3fe1e58ea"): 1118337280,
-    # profiles/k_dec_tok_decode_N64_H32_d128_C64.md: 135,935,744 read + 77,555,200 written
-    ("k_dec_tok", "51b392a62fe51a33"): 213490944,
-    # profiles/k_bwd_trainer_B2_H32_T8192_d128_C64.md: 2,963,502,592 read + 4,436,340,736 written
-    ("k_bwd_chunk", "86633ff16a2874d1"): 7399843328,
+    ("k_chain_tok", "5a5969a3fe1e58ea"): 789160960 + 329176320,
+    ("k_dec_tok", "51b392a62fe51a33"): 135935744 + 77555200,
+    ("k_bwd_chunk", "86633ff16a2874d1"): 2963502592 + 4436340736,
 }
 
 KERNEL_SOURCES = {
@@ -105,6 +110,27 @@ def kernel_source_sha(kernel: str = "k_tok"):
         with open(os.path.join(ROOT, "gated_deltanet_cpr_delta_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def measure_fp32_peak():
+    """Sustained FP32 fma rate of this GPU (TFLOP/s), scalar and packed, from
+    the probe kernels of libgdn_probe.so (run before the timed regions)."""
+    import ctypes
+    import torch
+    path = os.path.join(ROOT, "gated_deltanet_cpr_delta_b200", "libgdn_probe.so")
+    lib = ctypes.CDLL(path)
+    lib.gdn_probe_fp32_tflops.restype = ctypes.c_int
+    lib.gdn_probe_fp32_tflops.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
+    sink = torch.zeros(148 * 64, dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    out = {}
+    for name, packed in (("ffma", 0), ("ffma2", 1)):
+        t = ctypes.c_double(0.0)
+        if lib.gdn_probe_fp32_tflops(packed, 20, ctypes.c_void_p(sink.data_ptr()), ctypes.byref(t), stream) != 0:
+            raise RuntimeError("FP32 peak probe failed")
+        out[name] = t.value
+    return out
 
 
 class ClockSampler:
@@ -425,12 +451,50 @@ def bench_trainer(rank: int, world: int, warmup: int, steps: int, shape=None):
                          "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}}
 
 
+def bench_varlen(rank: int, world: int, warmup: int, steps: int):
+    """Varlen workload: 32 packed sequences (lengths from the seeded draw in
+    [128, 8192]), H=32; CPR forward tokens/s with L2 flushed before each step."""
+    import torch
+    from gated_deltanet_cpr_delta_b200 import gdn, synth
+    V = VARLEN
+    lens = synth.varlen_lengths(V["seed"], V["N"], V["lo"], V["hi"])
+    H, D, C = V["H"], V["D"], V["C"]
+    d = synth.make_batch_device(V["seed"], lens, H, D, D, "bf16", seq_ids=rank_sequence_ids(rank, V["N"]))
+    T = sum(lens)
+    o = torch.empty(T, H, D, dtype=torch.bfloat16, device="cuda")
+    st = torch.empty(gdn.gdn_num_chunk_states(d["cu_host"], C), H, D, D, dtype=torch.float32, device="cuda")
+    ws = torch.empty(gdn.gdn_cpr_workspace_size(T, len(lens), H, D, D, C), dtype=torch.uint8, device="cuda")
+    fwd = lambda ev=None: gdn.gdn_cpr_forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["cu_seqlens"], C,
+                                              cu_seqlens_host=d["cu_host"], o=o, chunk_states=st, workspace=ws,
+                                              events=ev)
+    for _ in range(max(warmup, 3)):
+        fwd()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for e in kev:
+        for x in e:
+            x.record()
+    barrier(world)
+    for s_ in range(steps):
+        flush.zero_()
+        fwd(kev[s_])
+    barrier(world)
+    ms = [e[0].elapsed_time(e[5]) for e in kev]
+    total = max_over_ranks(sum(ms), world)
+    full = sum((L // C) * C for L in lens)
+    fl = forward_flops(T * H, full * H, D, D, C)
+    return {"workload": V["name"], "tokens": T, "value": T * world * steps / (total / 1e3), "unit": UNIT,
+            "ms_per_step": total / steps, "flops_per_step": sum(fl.values()),
+            "frac_fp32_peak": sum(fl.values()) / (total / steps / 1e3) / 1e12 / FP32_PEAK_TFLOPS}
+
+
 def run_native(args):
     import torch
     from gated_deltanet_cpr_delta_b200 import gdn, synth
 
     rank, world, local = dist_setup(args.gpus)
     gdn.load_library()
+    fp32_meas = measure_fp32_peak()
     W = WORKLOAD
     B, H, T, D, C = W["B"], W["H"], W["T"], W["D"], W["C"]
     d = synth.make_batch_device(W["seed"], [T] * B, H, D, D, "bf16", seq_ids=rank_sequence_ids(rank, B))
@@ -537,6 +601,7 @@ def run_native(args):
     dec = bench_decode(rank, world, args.warmup) if not args.no_decode else None
     tshape = tuple(int(x) for x in args.trainer_shape.split(",")) if args.trainer_shape else None
     trainer = bench_trainer(rank, world, args.warmup, min(K, 5), tshape) if not args.no_trainer else None
+    varlen = bench_varlen(rank, world, args.warmup, min(K, 5)) if not args.no_varlen else None
 
     peaks, peak_src = load_peaks()
     flops = forward_flops(B * T * H, B * (T // C) * C * H, D, D, C)
@@ -558,6 +623,7 @@ def run_native(args):
         kernels["k_" + n]["tflops"] = flops[n] / (kern_ms["k_" + n] / 1e3) / 1e12 if kern_ms["k_" + n] > 0 else 0
         kernels["k_" + n]["frac_fp32_peak"] = kernels["k_" + n]["tflops"] / FP32_PEAK_TFLOPS
     total_flops = sum(flops.values())
+    flops_tok_only = 7 * D * D * B * T * H
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -568,10 +634,16 @@ def run_native(args):
                      "bound": "alu", "achieved": tok_tf,
                      "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tok_tf / FP32_PEAK_TFLOPS,
                      "traffic": traffic, "flops_per_launch": main_flops,
-                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"},
+                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                     "peak_measured": fp32_meas["ffma"], "frac_measured": tok_tf / fp32_meas["ffma"]},
         "forward_roofline": {"flops_per_step": total_flops,
                              "achieved_tflops": total_flops / (ms_step / 1e3) / 1e12 / world,
-                             "frac": total_flops / (ms_step / 1e3) / 1e12 / world / FP32_PEAK_TFLOPS},
+                             "frac": total_flops / (ms_step / 1e3) / 1e12 / world / FP32_PEAK_TFLOPS,
+                             "frac_measured": total_flops / (ms_step / 1e3) / 1e12 / world / fp32_meas["ffma"],
+                             "recurrence_only_flops": flops_tok_only,
+                             "recurrence_only_frac": flops_tok_only / (ms_step / 1e3) / 1e12 / world /
+                             FP32_PEAK_TFLOPS,
+                             "peak": FP32_PEAK_TFLOPS, "peak_measured": fp32_meas["ffma"]},
         "kernels": kernels,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
@@ -582,7 +654,12 @@ def run_native(args):
         "parity": parity,
         "decode": dec,
         "trainer": trainer,
-        "peaks": {"hbm_gbs": peaks.get("hbm_gbs"), "source": peak_src},
+        "varlen": varlen,
+        "peaks": {"hbm_gbs": peaks.get("hbm_gbs"), "source": peak_src,
+                  "fp32_tflops_derived": FP32_PEAK_TFLOPS,
+                  "fp32_tflops_measured": fp32_meas,
+                  "fp32_measured_by": "libgdn_probe.so: 8 independent fma chains per thread, 8 CTAs x 256 "
+                                      "threads per SM, 20 launches, timed in this run before the forward"},
         "kernel_source_sha": sha,
         "contract": {"id": gdn.gdn_contract_id(),
                      "numerical_policy": gdn.gdn_contract_identity(gdn.ID_NUMERICAL_POLICY, D, D, C, gdn.GDN_BF16,
@@ -590,16 +667,24 @@ def run_native(args):
                      "deployment": gdn.gdn_contract_identity(gdn.ID_DEPLOYMENT, D, D, C, gdn.GDN_BF16,
                                                              gdn.GDN_BF16)},
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+    # The oracle leg, on rank 0 only: the parity gate on the first forward's
+    # snapshot (always), and the oracle's own timing (one GPU, unless skipped).
+    rc = 0
+    if rank == 0:
         line["parity"] = parity_gate(d, par_o, par_st, C)
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        if not line["parity"]["ok"]:
+            line["value"] = None  # no speed is reported for a result that failed its parity check
+            line["parity_failed"] = True
+            rc = 1
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line))
-    return 0
+    return rc
 
 
 def main():
@@ -611,6 +696,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-trainer", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--trainer-shape", default=None,
                     help="B,H,T of the trainer section (default: the trainer workload; for profiling)")
     args = ap.parse_args()

@@ -1,7 +1,9 @@
-"""Build the CUDA library libgdn_cpr.so in-tree for sm_100a with nvcc.
+"""Build the CUDA libraries in-tree for sm_100a with nvcc.
 
     python -m gated_deltanet_cpr_delta_b200.build [--force] [--verbose]
 
+libgdn_cpr.so is the layer (the C ABI of include/gdn_cpr.h).  libgdn_probe.so
+is a measurement helper for the benchmark (the FP32 fma rate of the device).
 `--verbose` adds ``-Xptxas -v`` (registers, spills, shared memory per kernel).
 """
 from __future__ import annotations
@@ -16,6 +18,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgdn_cpr.so")
+PROBE_LIB = os.path.join(PKG, "libgdn_probe.so")
+PROBE_SOURCES = ["probe_fp32.cu"]
 SOURCES = ["gdn_cpr.cu", "identity.cu"]
 DEPS = ["gdn_cpr.cu", "identity.cu", "kernels.cuh", "schedule.cuh", "k_tables.cuh", "k_ptok.cuh", "k_tc.cuh",
         "k_pchunk.cuh", "k_decode.cuh", "k_bwd.cuh"]
@@ -53,25 +57,30 @@ def flags(verbose: bool = False):
     return f
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str, deps) -> bool:
+    if not os.path.exists(lib):
         return False
-    m = os.path.getmtime(LIB)
-    srcs = [os.path.join(CSRC, s) for s in DEPS] + HEADERS + [os.path.abspath(__file__)]
+    m = os.path.getmtime(lib)
+    srcs = [os.path.join(CSRC, s) for s in deps] + HEADERS + [os.path.abspath(__file__)]
     return all(os.path.getmtime(s) <= m for s in srcs)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not verbose and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc_path(), *flags(verbose), *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
+def _nvcc(lib: str, sources, verbose: bool):
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), *flags(verbose), *[os.path.join(CSRC, s) for s in sources], "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if force or verbose or not up_to_date(LIB, DEPS):
+        _nvcc(LIB, SOURCES, verbose)
+    if force or verbose or not up_to_date(PROBE_LIB, PROBE_SOURCES):
+        _nvcc(PROBE_LIB, PROBE_SOURCES, verbose)
     return LIB
 
 

@@ -3,6 +3,7 @@
 // Validates arguments on the host, carves the caller's workspace and enqueues
 // the kernels of kernels.cuh on the caller's stream.  It allocates no device
 // memory and never synchronises.  Its only global mutable state is the
+// failure-detection test setting (gdn_test_fault_injection) and the
 // per-device address cache of gdn_cpr_forward_noalloc (end of file).
 #include "gdn_cpr.h"
 #include "kernels.cuh"
@@ -10,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -18,6 +20,12 @@ namespace {
 using gdn::ChunkCfg;
 
 constexpr size_t kAlign = 256;
+
+// Failure-detection test setting (gdn_test_fault_injection): 0 = off; 1 = the
+// fused forward kernel withholds its boundary-state publications and bounds
+// each wait for one by g_fault_wait clocks.
+std::atomic<int32_t> g_fault_mode{0};
+std::atomic<int64_t> g_fault_wait{gdn::kWaitLimit};
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -188,8 +196,12 @@ gdn_status_t launch_forward(const FwdArgs& a)
         float* states = a.states;
         void* o = a.o;
         float* cacheR = a.cache ? a.cache->R : nullptr;
+        const int32_t mode = g_fault_mode.load();
+        int withhold = mode == 1 ? 1 : 0;
+        long long wait_limit = mode == 1 ? (long long)g_fault_wait.load() : gdn::kWaitLimit;
         void* args[] = {&q, &k, &v, &alpha, &beta, &state_in, &cu, &fco, &so, &err, &N, &H, &in_bf16, &out_bf16,
-                        &w, &u, &dC, &states, &o, &cacheR, &progress, &tok_next, &order, &cumc, &maxc};
+                        &w, &u, &dC, &states, &o, &cacheR, &progress, &tok_next, &order, &cumc, &maxc,
+                        &withhold, &wait_limit};
         if (cudaLaunchCooperativeKernel((const void*)gdn::k_chain_tok<D, D, C>, dim3((unsigned)sms), dim3(256), args,
                                         fsm, a.stream) != cudaSuccess ||
             cudaGetLastError() != cudaSuccess)
@@ -257,7 +269,7 @@ gdn_status_t launch_decode(const DecArgs& a)
     mark(a.events, 0, a.stream);
     gdn::k_dec_tok<D, D, C><<<tgrid, DC::THREADS, DC::SMEM, a.stream>>>(
         a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, a.o,
-        (int)items);
+        (int)items, c.status);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
@@ -266,7 +278,7 @@ gdn_status_t launch_decode(const DecArgs& a)
     const int64_t min_grid = (NH + 1023) / 1024;
     const unsigned rgrid = (unsigned)std::max<int64_t>(std::min<int64_t>(NH, sms), min_grid);
     gdn::k_dec_resync<D, D, C><<<rgrid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
-        (int)NH, a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos);
+        (int)NH, a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, c.status);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 2, a.stream);
     return GDN_OK;
@@ -408,8 +420,23 @@ const char* gdn_status_string(gdn_status_t s)
         case GDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
         case GDN_ERR_CUDA: return "CUDA launch failed";
         case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+        case GDN_ERR_TIMEOUT: return "a bounded device wait ran out (outputs incomplete)";
+        case GDN_ERR_DEVICE_INPUT: return "device input disagrees with the host copy or is out of range";
     }
     return "unknown status";
+}
+
+gdn_status_t gdn_test_fault_injection(int32_t mode, int64_t wait_clocks)
+{
+    if (mode == 0) {
+        g_fault_mode.store(0);
+        g_fault_wait.store(gdn::kWaitLimit);
+        return GDN_OK;
+    }
+    if (mode != 1 || wait_clocks < 1 || wait_clocks > gdn::kWaitLimit) return GDN_ERR_INVALID_ARG;
+    g_fault_wait.store(wait_clocks);
+    g_fault_mode.store(1);
+    return GDN_OK;
 }
 
 int64_t gdn_num_chunk_states(const int32_t* cu_seqlens_host, int32_t num_seqs, int32_t C)
@@ -468,7 +495,8 @@ gdn_status_t gdn_cpr_forward_timed(const void* q, const void* k, const void* v, 
     a.ws = carve(workspace, total_tokens / C, num_seqs, H, d_k, d_v, C);
     a.stream = static_cast<cudaStream_t>(stream);
     a.events = events;
-    if (num_seqs == 0) {
+    if (num_seqs == 0) {  // no kernel runs: only the device status word is reset
+        if (cudaMemsetAsync(a.ws.err, 0, sizeof(int32_t), a.stream) != cudaSuccess) return GDN_ERR_CUDA;
         for (int i = 0; i < 6; ++i) mark(events, i, a.stream);
         return GDN_OK;
     }
@@ -522,7 +550,9 @@ gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
     const BwdWorkspace need = carve_bwd(nullptr, total_tokens, num_seqs, H, d_k, d_v, C);
     if (workspace == nullptr || workspace_bytes < need.bytes) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return GDN_ERR_INVALID_ARG;
-    if (num_seqs == 0) {
+    if (num_seqs == 0) {  // no kernel runs: only the device status word is reset
+        if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return GDN_ERR_CUDA;
         for (int i = 0; i < 4; ++i) mark(events, i, static_cast<cudaStream_t>(stream));
         return GDN_OK;
     }
@@ -620,6 +650,24 @@ gdn_status_t noalloc_scratch(void** out)
 }
 
 }  // namespace
+
+// The device status word is the workspace's first 4 bytes (carve: err), for
+// the forward and the backward alike.
+extern "C" gdn_status_t gdn_read_device_status(const void* workspace, int32_t* status_out, void* stream)
+{
+    if (status_out == nullptr) return GDN_ERR_INVALID_ARG;
+    const void* ws = workspace;
+    if (ws == nullptr) {
+        void* p = nullptr;
+        const gdn_status_t st = noalloc_scratch(&p);
+        if (st != GDN_OK) return st;
+        ws = p;
+    }
+    if (cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDefault, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return GDN_ERR_CUDA;
+    return GDN_OK;
+}
 
 extern "C" gdn_status_t gdn_cpr_forward_noalloc(const void* q, const void* k, const void* v, const float* alpha,
                                                 const float* beta, const float* state_in,

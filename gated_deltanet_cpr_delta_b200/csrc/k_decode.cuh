@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(DecCfg<DK, DV>::THREADS)
 k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
           const float* __restrict__ alpha, const float* __restrict__ beta, int in_bf16, int out_bf16,
           float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos, void* __restrict__ o,
-          int nitems)
+          int nitems, int32_t* status)
 {
     using Cf = DecCfg<DK, DV>;
     using RS = typename Cf::RS;
@@ -131,6 +131,7 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
         load_row_pairs<DK>(Rp, rslot(st));
         __syncthreads();  // the widened token is complete
         const bool valid = p >= 0 && p < C;  // an invalid position writes nothing
+        if (!valid && t == 0) record_error(status, GDN_ERR_DEVICE_INPUT);
         if (valid) {
             const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
             store_row_pairs<DK>(rslot(st), Rp);
@@ -176,12 +177,13 @@ struct ResyncSmem {
 // pos <- 0.  P_chunk runs the same device functions as the prefill
 // (chunk_prep, then the tcgen05 boundary step).  Persistent: CTA b handles
 // (sequence, head) pairs b, b + grid, ...  A pos outside [0, C) is left
-// unchanged.  If an MMA completion wait times out, the pairs this CTA had
-// still to resync get pos = -1 and are not written.
+// unchanged (k_dec_tok has recorded it).  If an MMA completion wait times
+// out, the pairs this CTA had still to resync get pos = -1, are not written,
+// and GDN_ERR_TIMEOUT goes to *status (when non-null).
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256, 1)
 k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
-             const float* bbuf, int32_t* pos)
+             const float* bbuf, int32_t* pos, int32_t* status)
 {
     using Sm = ResyncSmem<DK, DV, C>;
     using PL = PrepLayout<DK, DV, C>;
@@ -257,6 +259,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
         if (threadIdx.x == 0) pos[nh] = 0;
     }
     for (int r = it + threadIdx.x; r < nt; r += blockDim.x) pos[todo[r]] = -1;  // after a timeout
+    if (it < nt && threadIdx.x == 0) record_error(status, GDN_ERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x < 32) {

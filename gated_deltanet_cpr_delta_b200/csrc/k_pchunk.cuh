@@ -303,19 +303,20 @@ struct ChainSmem {
 // chunk's k^T (loaded into registers one chunk ahead) and start the next
 // chunk's w and k loads; during phase 2 they convert the next chunk's w into
 // the split operands and start its u0 and decay copies.  An MMA completion
-// wait that times out sets *err = 2 and ends the CTA; the kernels after it
-// then write nothing.
+// wait that times out records GDN_ERR_TIMEOUT in *err and ends the CTA; the
+// kernels after it then write nothing.
 //
 // progress (when non-null) publishes, for the pair, how many of its chunk
 // states are in global memory: after state c is written (and fenced),
-// progress[nh] = c + 1, with release semantics.
+// progress[nh] = c + 1, with release semantics.  With withhold != 0 nothing is
+// published (the failure-detection test hook).
 template <int DK, int DV, int C>
 __device__ __forceinline__ void chain_run(const void* __restrict__ k, const float* __restrict__ state_in,
                                           const int32_t* __restrict__ cu, const int32_t* __restrict__ fco,
                                           const int32_t* __restrict__ so, int32_t* err, int H, int in_bf16,
                                           const float* __restrict__ w_ws, const float* __restrict__ u_ws,
                                           const float* __restrict__ dC_ws, float* states, int nh,
-                                          int32_t* progress, float* sm)
+                                          int32_t* progress, int withhold, float* sm)
 {
     using Cf = ChunkCfg<DK, DV, C>;
     using Sm = ChainSmem<DK, DV, C>;
@@ -341,7 +342,7 @@ __device__ __forceinline__ void chain_run(const void* __restrict__ k, const floa
     auto state_dst = [&](int c) { return states + ((slot0 + c) * H + h) * (int64_t)DV * DK; };
     auto movers_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NP) : "memory"); };
     auto publish = [&](int count) {  // after a fence and a barrier over the writers
-        if (progress != nullptr) st_release_gpu(progress + nh, count);
+        if (progress != nullptr && !withhold) st_release_gpu(progress + nh, count);
     };
 
     auto fetch_w = [&](int c, int tid, int nthr) {  // raw w of chunk c -> wraw
@@ -427,7 +428,7 @@ __device__ __forceinline__ void chain_run(const void* __restrict__ k, const floa
         tc_store_rows<DK, DV>(Klo, state_dst(nfull), nullptr, pt, NP);
         __threadfence();
     }
-    if (!ok && threadIdx.x == 0) atomicExch(err, 2);
+    if (!ok && threadIdx.x == 0) record_error(err, GDN_ERR_TIMEOUT);
     cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -448,7 +449,7 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
     if (*reinterpret_cast<volatile int32_t*>(err)) return;
     extern __shared__ float4 smem_f4[];
     chain_run<DK, DV, C>(k, state_in, cu, fco, so, err, H, in_bf16, w_ws, u_ws, dC_ws, states, blockIdx.x, nullptr,
-                         reinterpret_cast<float*>(smem_f4));
+                         0, reinterpret_cast<float*>(smem_f4));
 }
 
 // ------------------------------------------------------------------ fused chain + P_tok
@@ -467,7 +468,10 @@ struct FusedSmem {
 // sequence order[t - cumc[c]], the sequences sorted by chunk count), two
 // tasks per CTA at a time (one per 128-thread half), each after its boundary
 // state is published.  Every CTA is resident (cooperative launch), and chains
-// wait on nothing, so every wait ends; a wait that exceeds ~1 s sets *err = 3.
+// wait on nothing, so every wait ends.  A wait gives up after wait_limit
+// clocks (kWaitLimit, about a second, in normal operation), records
+// GDN_ERR_TIMEOUT in *err and ends its half; withhold != 0 (the test hook)
+// makes the chains publish nothing, so every wait runs out.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256, 1)
 k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
@@ -476,7 +480,7 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
             int32_t* err, int N, int H, int in_bf16, int out_bf16, const float* __restrict__ w_ws,
             const float* __restrict__ u_ws, const float* __restrict__ dC_ws, float* states, void* __restrict__ o,
             float* __restrict__ cacheR, int32_t* progress, int32_t* tok_next, const int32_t* __restrict__ order,
-            const int32_t* __restrict__ cumc, int maxc)
+            const int32_t* __restrict__ cumc, int maxc, int withhold, long long wait_limit)
 {
     using Fs = FusedSmem<DK, DV, C>;
     static_assert(Fs::OK, "d_v = 128: two 128-thread P_tok tasks per CTA");
@@ -486,7 +490,7 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
     float* sm = reinterpret_cast<float*>(smem_f4);
     if ((int)blockIdx.x < N * H) {
         chain_run<DK, DV, C>(k, state_in, cu, fco, so, err, H, in_bf16, w_ws, u_ws, dC_ws, states, blockIdx.x,
-                             progress, sm);
+                             progress, withhold, sm);
         __syncthreads();
     }
     const int half = threadIdx.x >> 7, tid = threadIdx.x & 127;
@@ -513,8 +517,8 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
             next = atomicAdd(tok_next, 1);
             // The acquire load orders this half's later state loads after the
             // chain's release (through the barrier below): no fence needed.
-            const bool ready = wait_at_least(progress + (int64_t)n * H + h, c + 1);
-            if (!ready) atomicExch(err, 3);
+            const bool ready = wait_at_least(progress + (int64_t)n * H + h, c + 1, wait_limit);
+            if (!ready) record_error(err, GDN_ERR_TIMEOUT);
             go[half] = ready && *verr == 0;
         }
         hs();

@@ -22,9 +22,10 @@ __host__ __device__ inline uint64_t cu_entry_hash(int n, int32_t value)
 //   cto[n] = sum_{m<n} ceil(L_m/C)      (chunk tasks of k_tok)
 //   fco[n] = sum_{m<n} floor(L_m/C)     (full chunks: k_prep / k_chain)
 //   so[n]  = sum_{m<n} (floor(L_m/C)+1) (chunk-state slots)
-// and the totals at index N.  err[0] = 1 if the device cu_seqlens is invalid
-// or disagrees with the host copy (totals or hash); every later kernel then
-// exits without writing.
+// and the totals at index N.  err[0], the call's device status word, becomes
+// GDN_ERR_DEVICE_INPUT if the device cu_seqlens is invalid or disagrees with
+// the host copy (totals or hash), else GDN_OK; every later kernel exits
+// without writing while it is not GDN_OK.
 // With order != NULL, also the tables of the fused chain + P_tok kernel
 // (nt_n = ceil(L_n/C) chunk tasks of sequence n, maxc = max nt_n):
 //   order[r]  sequences by nt_n descending (ties by n)
@@ -93,7 +94,7 @@ __global__ void k_tables(const int32_t* __restrict__ cu, int N, int C, int64_t T
         const bool ok = !bad_any && cu[0] == 0 && (int64_t)cu[N] == T_total &&
                         tot[0] == want_tasks && tot[1] == want_full && tot[2] == want_states &&
                         hsum == want_hash;
-        err[0] = ok ? 0 : 1;
+        err[0] = ok ? (int32_t)GDN_OK : (int32_t)GDN_ERR_DEVICE_INPUT;
     }
     if (order != nullptr) {
         auto nt = [&](int m) { return (max(0, cu[m + 1] - cu[m]) + C - 1) / C; };

@@ -13,6 +13,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gdn_cpr.h"
+
 namespace gdn {
 
 constexpr unsigned kFullMask = 0xffffffffu;
@@ -187,15 +189,24 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p)
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// Waits until *p >= v; false after ~2^31 clocks (about a second).
-__device__ __forceinline__ bool wait_at_least(const int32_t* p, int32_t v)
+// The bound of every wait on another CTA's progress: 2^31 clocks, about a second.
+constexpr long long kWaitLimit = 1ll << 31;
+
+// Waits until *p >= v; false once `limit` clocks have passed.
+__device__ __forceinline__ bool wait_at_least(const int32_t* p, int32_t v, long long limit)
 {
     const long long t0 = clock64();
     while (ld_acquire_gpu(p) < v) {
-        if (clock64() - t0 > (1ll << 31)) return false;
+        if (clock64() - t0 > limit) return false;
         __nanosleep(256);
     }
     return true;
+}
+
+// The device status word: keeps the first error recorded (a gdn_status_t).
+__device__ __forceinline__ void record_error(int32_t* status, int32_t code)
+{
+    if (status != nullptr) atomicCAS(status, (int32_t)GDN_OK, code);
 }
 
 // All but the N most recently committed groups have landed.

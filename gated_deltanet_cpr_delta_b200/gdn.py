@@ -18,14 +18,17 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_cpr.so")
 
 GDN_F32, GDN_BF16 = 0, 1
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_WORKSPACE = 0, 1, 2, 3, 4
+GDN_ERR_TIMEOUT, GDN_ERR_DEVICE_INPUT = 5, 6
 _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
-           4: "GDN_ERR_WORKSPACE"}
+           4: "GDN_ERR_WORKSPACE", 5: "GDN_ERR_TIMEOUT", 6: "GDN_ERR_DEVICE_INPUT"}
 
 #: exported symbols of include/gdn_cpr.h
 SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
            "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed",
            "gdn_cpr_forward_noalloc", "gdn_contract_text", "gdn_contract_identity", "gdn_sha256_hex",
-           "gdn_cpr_backward_workspace_size", "gdn_cpr_backward", "gdn_cpr_backward_timed")
+           "gdn_cpr_backward_workspace_size", "gdn_cpr_backward", "gdn_cpr_backward_timed",
+           "gdn_read_device_status", "gdn_test_fault_injection")
 
 #: gdn_identity_kind_t
 ID_SEMANTIC, ID_NUMERICAL_POLICY, ID_DEPLOYMENT = 0, 1, 2
@@ -43,7 +46,7 @@ class GdnError(RuntimeError):
 class CacheStruct(ctypes.Structure):
     _fields_ = [("S_b", ctypes.c_void_p), ("R", ctypes.c_void_p), ("kbuf", ctypes.c_void_p),
                 ("vbuf", ctypes.c_void_p), ("abuf", ctypes.c_void_p), ("bbuf", ctypes.c_void_p),
-                ("pos", ctypes.c_void_p)]
+                ("pos", ctypes.c_void_p), ("status", ctypes.c_void_p)]
 
 
 _lib = None
@@ -92,6 +95,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                      P, P, P, P, P, P, P, sz, P]
     lib.gdn_cpr_backward_timed.restype = ctypes.c_int
     lib.gdn_cpr_backward_timed.argtypes = lib.gdn_cpr_backward.argtypes + [P]
+    lib.gdn_read_device_status.restype = ctypes.c_int
+    lib.gdn_read_device_status.argtypes = [P, P, P]
+    lib.gdn_test_fault_injection.restype = ctypes.c_int
+    lib.gdn_test_fault_injection.argtypes = [i32, i64]
     _lib = lib
     return lib
 
@@ -174,17 +181,38 @@ def gdn_cpr_workspace_size(total_tokens: int, num_seqs: int, H: int, d_k: int, d
 def new_cache(N: int, H: int, d_k: int, d_v: int, C: int, dtype: torch.dtype, device="cuda",
               state: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
     """Allocate a decode cache (gdn_cache_t layout).  With ``state`` [N,H,d_v,d_k]
-    it starts at a chunk boundary with that state, otherwise at zero."""
+    it starts at a chunk boundary with that state, otherwise at zero.  ``status``
+    is the decode step's device status word (one int32, starts at GDN_OK)."""
     S = torch.zeros(N, H, d_v, d_k, dtype=torch.float32, device=device) if state is None else state.clone()
     return dict(S_b=S, R=S.clone(), kbuf=torch.zeros(N, H, C, d_k, dtype=dtype, device=device),
                 vbuf=torch.zeros(N, H, C, d_v, dtype=dtype, device=device),
                 abuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
                 bbuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
-                pos=torch.zeros(N, H, dtype=torch.int32, device=device))
+                pos=torch.zeros(N, H, dtype=torch.int32, device=device),
+                status=torch.zeros(1, dtype=torch.int32, device=device))
 
 
 def _cache_struct(c: Dict[str, torch.Tensor]) -> CacheStruct:
-    return CacheStruct(*[c[n].data_ptr() for n in ("S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos")])
+    st = c.get("status")
+    return CacheStruct(*[c[n].data_ptr() for n in ("S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos")],
+                       st.data_ptr() if st is not None else None)
+
+
+def read_device_status(workspace: Optional[torch.Tensor] = None, device=None) -> int:
+    """The device status word of the last forward / backward that used
+    ``workspace`` (None: the no-allocation forward's fixed array), read after
+    the current stream has run that call (this synchronises the stream)."""
+    dev = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
+    out = torch.empty(1, dtype=torch.int32, device=dev)
+    _check(load_library().gdn_read_device_status(_ptr(workspace), _ptr(out), _stream(dev)),
+           "gdn_read_device_status")
+    return int(out.item())
+
+
+def set_fault_injection(mode: int, wait_clocks: int = 1 << 31) -> None:
+    """Failure-detection hook (process-wide; mode 0 = off): see
+    gdn_test_fault_injection in include/gdn_cpr.h."""
+    _check(load_library().gdn_test_fault_injection(mode, wait_clocks), "gdn_test_fault_injection")
 
 
 def gdn_cpr_forward(q, k, v, alpha, beta, cu_seqlens, C: int, *, cu_seqlens_host=None, state_in=None,

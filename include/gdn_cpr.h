@@ -21,10 +21,11 @@
  *
  * Conventions common to every call:
  *  - All tensors are caller-owned device memory unless marked "host".
- *    The library never allocates device memory and keeps no global mutable
- *    state.  It never synchronises the device.  The one exception is
- *    gdn_cpr_forward_noalloc (end of this file): it uses a fixed device array
- *    inside the library and caches that array's address per device.
+ *    The library never allocates device memory and never synchronises the
+ *    device.  It keeps global mutable state in two places only:
+ *    gdn_cpr_forward_noalloc (end of this file) uses a fixed device array
+ *    inside the library and caches that array's address per device, and
+ *    gdn_test_fault_injection holds a process-wide test setting.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
  *    The call returns once the kernels are enqueued.
  *  - Layouts are row-major and densely packed:
@@ -35,9 +36,19 @@
  *  - Supported shapes: d_k == d_v in {16, 32, 64, 128}; C in {16, 32, 64}.
  *    Any other shape returns GDN_ERR_UNSUPPORTED.
  *  - Inputs must be finite.  The results for NaN or Inf inputs are unspecified.
- *  - Errors are reported by the return code only: no exceptions, no exit,
- *    and no device trap or assert.  Invalid arguments are caught on the host
- *    before anything is enqueued.
+ *  - Errors are reported through status codes only: no exceptions, no exit,
+ *    and no device trap or assert.  There are two places:
+ *      1. The return code.  Invalid arguments and failed launches are caught on
+ *         the host before or while the kernels are enqueued.
+ *      2. The device status word.  Two errors can only be seen on the GPU
+ *         while the kernels run: a device cu_seqlens that disagrees with the
+ *         host copy (GDN_ERR_DEVICE_INPUT), and a bounded wait that ran out
+ *         (GDN_ERR_TIMEOUT).  The kernels record the first such error in a
+ *         status word.  For gdn_cpr_forward and gdn_cpr_backward that word
+ *         sits in the workspace; gdn_read_device_status copies it out.  For
+ *         gdn_decode_step it is gdn_cache_t.status.  A call whose return code
+ *         is GDN_OK can still have failed on the device: read the status word
+ *         after the stream has run the call.
  */
 #ifndef GDN_CPR_H
 #define GDN_CPR_H
@@ -54,7 +65,10 @@ typedef enum {
     GDN_ERR_INVALID_ARG = 1,   /* NULL/misaligned pointer, bad size, bad cu_seqlens */
     GDN_ERR_UNSUPPORTED = 2,   /* (d_k, d_v, C, dtype) not compiled in */
     GDN_ERR_CUDA = 3,          /* a CUDA launch or attribute call failed */
-    GDN_ERR_WORKSPACE = 4      /* workspace NULL or smaller than gdn_cpr_workspace_size() */
+    GDN_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than gdn_cpr_workspace_size() */
+    GDN_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out; the outputs are incomplete */
+    GDN_ERR_DEVICE_INPUT = 6   /* device: cu_seqlens on the device disagrees with the host copy, or a
+                                  decode position outside [0, C); nothing was written for it */
 } gdn_status_t;
 
 typedef enum {
@@ -71,6 +85,14 @@ typedef enum {
  *   vbuf [N, H, C, d_v]  in_dtype
  *   abuf [N, H, C] fp32, bbuf [N, H, C] fp32   ... their gates
  *   pos  [N, H] int32            tokens since the last boundary, 0 <= pos < C
+ *   status  one int32, or NULL   the decode step's device status word: the
+ *                                kernels store the first error they detect
+ *                                (GDN_ERR_DEVICE_INPUT for a pos outside [0, C),
+ *                                GDN_ERR_TIMEOUT for a resync whose tensor-core
+ *                                wait ran out; that pair's pos becomes -1).
+ *                                The library never clears it: the caller sets
+ *                                it to GDN_OK (0) and reads it back.  NULL: not
+ *                                recorded.  gdn_cpr_forward ignores it.
  * A fresh cache for an initial state S_0 is S_b = R = S_0 with pos = 0.  The
  * buffer contents do not matter while pos == 0.
  */
@@ -82,6 +104,7 @@ typedef struct {
     float*   abuf;
     float*   bbuf;
     int32_t* pos;
+    int32_t* status;
 } gdn_cache_t;
 
 /* Name of the arithmetic schedule every kernel executes (static string). */
@@ -133,6 +156,41 @@ gdn_status_t gdn_sha256_hex(const void* data, size_t n, char* out_hex);
 const char* gdn_status_string(gdn_status_t status);
 
 /*
+ * Device status of the last gdn_cpr_forward or gdn_cpr_backward call that used
+ * `workspace` (NULL: the fixed array of gdn_cpr_forward_noalloc on the current
+ * device).  The call enqueues on `stream` one 4-byte copy of the workspace's
+ * status word into *status_out, which may be host or device memory.  Once the
+ * stream has run it (cudaStreamSynchronize), *status_out holds a gdn_status_t:
+ *   GDN_OK               the kernels detected nothing;
+ *   GDN_ERR_DEVICE_INPUT the device cu_seqlens disagreed with the host copy;
+ *                        the kernels wrote no output;
+ *   GDN_ERR_TIMEOUT      a bounded device wait ran out (about a second of GPU
+ *                        clocks); some outputs were not written.
+ * Every forward and backward call resets the word at its start, on the
+ * stream, so the copy must be enqueued after the call it reports on and
+ * before the next call that uses the same workspace.  Returns
+ * GDN_ERR_INVALID_ARG for status_out == NULL and GDN_ERR_CUDA if the copy
+ * cannot be enqueued.  Host-side errors are not recorded here: they are the
+ * return codes of the calls themselves.
+ */
+gdn_status_t gdn_read_device_status(const void* workspace, int32_t* status_out, void* stream);
+
+/*
+ * Failure-detection hook, for tests of the status reporting.  It is
+ * process-wide and off by default.
+ *   mode 0: normal operation (wait_clocks is ignored);
+ *   mode 1: every later gdn_cpr_forward call that runs the fused chain +
+ *           intra-chunk kernel (d_v = 128 and fewer (sequence, head) pairs
+ *           than SMs) withholds the publication of its boundary states.  Each
+ *           intra-chunk task then waits for a state that never arrives.  The
+ *           wait gives up after wait_clocks GPU clocks (1 .. 2^31), the task
+ *           records GDN_ERR_TIMEOUT and ends, and the call's outputs are
+ *           incomplete.  Nothing on the GPU faults or hangs.
+ * Returns GDN_ERR_INVALID_ARG for another mode or a wait_clocks out of range.
+ */
+gdn_status_t gdn_test_fault_injection(int32_t mode, int64_t wait_clocks);
+
+/*
  * Number of chunk states the forward writes.  That is
  * sum_n (floor(L_n / C) + 1), with L_n = cu_seqlens_host[n+1] - cu_seqlens_host[n].
  * cu_seqlens_host is host memory with num_seqs + 1 entries.  Returns -1 if
@@ -159,8 +217,9 @@ size_t gdn_cpr_workspace_size(int64_t total_tokens, int32_t num_seqs, int32_t H,
  *     launch grids and is validated on the host: cu[0] == 0, non-decreasing,
  *     cu[num_seqs] == total_tokens.  The kernels check the device copy against
  *     the host copy: chunk totals and a 64-bit position-sensitive hash of
- *     the values.  If the two copies disagree, the kernels write nothing, and
- *     the outputs keep their previous contents.
+ *     the values.  If the two copies disagree, the kernels write nothing, the
+ *     outputs keep their previous contents, and the workspace's device status
+ *     word becomes GDN_ERR_DEVICE_INPUT (gdn_read_device_status).
  *   Chunks are aligned to each sequence's own token 0, so results do not
  *   depend on batch composition or packing.
  * Outputs:
@@ -222,7 +281,8 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
  *   workspace: at least gdn_cpr_backward_workspace_size(...) bytes of device
  *     memory, 256-byte aligned, not shared with a concurrent call.
  * Errors: as gdn_cpr_forward.  If the device copy of cu_seqlens disagrees
- * with the host copy, the kernels write nothing.
+ * with the host copy, the kernels write nothing and the workspace's device
+ * status word becomes GDN_ERR_DEVICE_INPUT (gdn_read_device_status).
  */
 gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v,
                               const float* alpha, const float* beta, const void* dO,
@@ -263,7 +323,10 @@ gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
  * of L tokens followed by m decode steps gives bit-identical o and cache to a
  * prefill of L + m tokens.
  * A pos outside [0, C) is not written through.  That (sequence, head) is left
- * unchanged and its o is unspecified.
+ * unchanged, its o is unspecified, and cache->status (when non-NULL) records
+ * GDN_ERR_DEVICE_INPUT.  A resync whose tensor-core completion wait runs out
+ * (about a second of GPU clocks) records GDN_ERR_TIMEOUT and sets the pos of
+ * the pairs it had not finished to -1.
  */
 gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v,
                              const float* alpha, const float* beta,

@@ -32,6 +32,26 @@ def test_contract_id(lib):
     assert lib.gdn_status_string(4) == b"workspace missing or too small"
 
 
+def test_every_status_code_has_a_name(lib):
+    hdr = open(os.path.join(ROOT, "include", "gdn_cpr.h")).read()
+    codes = {int(v): n for n, v in re.findall(r"^\s*(GDN_(?:OK|ERR_\w+))\s*=\s*(\d+)", hdr, flags=re.M)}
+    assert codes == {v: k for v, k in gdn._STATUS.items()}
+    assert codes[5] == "GDN_ERR_TIMEOUT" and codes[6] == "GDN_ERR_DEVICE_INPUT"
+    names = {c: lib.gdn_status_string(c) for c in codes}
+    assert all(n != b"unknown status" for n in names.values())
+    assert len(set(names.values())) == len(names)
+    assert lib.gdn_status_string(99) == b"unknown status"
+
+
+def test_fault_injection_and_status_read_validate_on_the_host(lib):
+    # host-side argument checks only: nothing is enqueued, so no GPU is needed
+    assert lib.gdn_test_fault_injection(2, 1000) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_test_fault_injection(1, 0) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_test_fault_injection(1, (1 << 31) + 1) == gdn.GDN_ERR_INVALID_ARG
+    assert lib.gdn_test_fault_injection(0, 0) == gdn.GDN_OK
+    assert lib.gdn_read_device_status(None, None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
 def test_num_chunk_states(lib):
     assert gdn.gdn_num_chunk_states([0, 64, 100, 100], 16) == 5 + 3 + 1
     assert gdn.gdn_num_chunk_states([0], 16) == 0
