@@ -178,7 +178,7 @@ gdn_status_t launch_forward(const FwdArgs& a)
     if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     if (a.tot.full > 0) {
-        constexpr size_t sm = gdn::PrepSmem<D, D, C>::BYTES;
+        const size_t sm = gdn::PrepCfg<D, D, C>::bytes(a.in_bf16);
         if (set_smem(gdn::k_prep<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
         gdn::k_prep<D, D, C><<<(unsigned)(a.tot.full * a.H), Cf::THREADS, sm, a.stream>>>(
             a.k, a.v, a.alpha, a.beta, a.cu, a.ws.fco, a.ws.err, a.N, a.H, a.in_bf16, a.ws.w, a.ws.u, a.ws.dC);
@@ -410,7 +410,7 @@ gdn_status_t launch_backward(const BwdArgs& a)
 
 extern "C" {
 
-const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v3/NL8/prep-mma-tf32x3/chain-tcgen05-tf32x3"; }
+const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v4/NL8/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3"; }
 
 const char* gdn_status_string(gdn_status_t s)
 {

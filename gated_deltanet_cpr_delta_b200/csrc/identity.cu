@@ -152,10 +152,13 @@ const char* kPolicy =
     "P_chunk part 1: decays D[s][s] = 1, D[t][s] = D[t-1][s]*alpha_t;\n"
     "  Gram G[t][s] = k_t.k_s (s < t) by mma.sync.m16n8k8 tf32, fp32 accumulate, K blocks of 8 ascending:\n"
     "  bf16 inputs: four accumulators by K block mod 4, G = (a0+a1)+(a2+a3); else G = (lo.hi + hi.lo) + hi.hi;\n"
-    "  c[t][s] = D[t][s]*G[t][s];\n"
-    "  forward substitution for u0 (init v_t) and w (init D[t][0]*k_t) in blocks of 16 tokens:\n"
-    "  acc = init + ((lo.hi + hi.lo) + hi.hi) of (-c) x over earlier blocks (mma.sync tf32),\n"
-    "  then acc = fma(-c[t][s], x_s, acc) for s in the block ascending; x_t = beta_t*acc\n"
+    "  A[t][s] = beta_t*(D[t][s]*G[t][s]) (s < t); T = (I + A)^-1 in blocks of 16 tokens:\n"
+    "  diagonal blocks by substitution, T[i][i] = 1, T[t][i] = fma chain over s = i..t-1 ascending of\n"
+    "  (-A[t][s])*T[s][i] from 0; block (i, j < i) by distance i - j ascending: M = A[i][j..i-1] T[j..i-1][j],\n"
+    "  T[i][j] = -(T[i][i] M), both by mma.sync.m16n8k8 tf32 split products (lo.hi + hi.lo) + hi.hi;\n"
+    "  gamma_t = beta_t*D[t][0]; u0 = (T diag(beta)) V, w = (T diag(gamma)) K by mma.sync.m16n8k8 tf32,\n"
+    "  row block r over K blocks 0..2r+1 ascending: bf16 inputs (V, K exact) lo.V + hi.V,\n"
+    "  else (lo.hi + hi.lo) + hi.hi\n"
     "P_chunk part 2: tcgen05.mma kind::tf32, M = 128, A in tensor memory, B K-major in shared memory,\n"
     "  fp32 accumulate, K blocks of 8 ascending, one accumulator per split product;\n"
     "  E = (S_lo.w_hi + S_hi.w_lo) + S_hi.w_hi, with S_hi.[w_lo; w_hi] one instruction of N = 2C;\n"

@@ -150,26 +150,27 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
 
 template <int DK, int DV, int C>
 struct ResyncSmem {
-    using Cf = ChunkCfg<DK, DV, C>;
-    using PL = PrepLayout<DK, DV, C>;
+    using P = PrepCfg<DK, DV, C>;
     using T = TcCfg<DK, DV, C>;
-    static constexpr int KX_OFF = 0;                                 // [C][KXS] k, then w
-    static constexpr int VX_OFF = KX_OFF + C * PL::KXS;              // [C][VXS] v, then u0
-    static constexpr int WLO_OFF = VX_OFF + C * PL::VXS;             // canonical w lo, then w hi ...
-    static constexpr int CC_OFF = WLO_OFF + T::W_FLOATS;             // ... in the [C][CCS] c of chunk_prep
-    static constexpr int DM_OFF = CC_OFF + C * PL::CCS;              // decays / staging
-    static constexpr int D0_OFF = DM_OFF + ((PL::DM + 3) / 4) * 4;   // D[t][0]
-    static constexpr int AB_OFF = D0_OFF + C + 4;
-    static constexpr int DC_OFF = AB_OFF + 2 * C;
-    static constexpr int KLO_OFF = DC_OFF + Cf::DCS;                 // canonical k^T lo | hi, then S' staging
-    static constexpr int KHI_OFF = KLO_OFF + T::K_FLOATS;
-    static constexpr int BAR_OFF = KLO_OFF + T::K_REGION;            // mbarrier (8 bytes) + TMEM base
+    static constexpr int WXS = DK + 4;                               // row stride of w
+    static constexpr int WX_OFF = 0;                                 // [C][WXS] w, from chunk_prep
+    static constexpr int US_OFF = WX_OFF + C * WXS;                  // [C][DV] u0
+    static constexpr int DC_OFF = US_OFF + C * DV;                   // [C+4] D[C][.]
+    // one region holds chunk_prep's raw rows and scratch, then (once w is
+    // split) the canonical w lo | hi and k^T lo | hi operands (k^T's region
+    // also stages S' after phase 2)
+    static constexpr int R1_OFF = ((DC_OFF + C + 4 + 31) / 32) * 32;  // 128-byte aligned
+    static constexpr int PREP_FL = (int)((P::bytes(0) + 3) / 4);
+    static constexpr int TC_FL = 2 * T::W_FLOATS + T::K_REGION;
+    static constexpr int R1_FL = PREP_FL > TC_FL ? PREP_FL : TC_FL;
+    static constexpr int WLO_OFF = R1_OFF;
+    static constexpr int KLO_OFF = R1_OFF + 2 * T::W_FLOATS;
+    static constexpr int BAR_OFF = R1_OFF + ((R1_FL + 3) / 4) * 4;   // mbarrier (8 bytes) + TMEM base
     // at least 120 KB, so that one CTA fits per SM: each allocates all 512 TMEM columns
     static constexpr size_t USED = sizeof(float) * (BAR_OFF + 4);
     static constexpr size_t BYTES = USED > 120 * 1024 ? USED : 120 * 1024;
     static_assert(BYTES <= 232448, "fits the 227 KB of shared memory a CTA can have");
-    static_assert(D0_OFF - CC_OFF >= T::W_FLOATS, "w hi fits in the c / decay scratch");
-    static_assert(BAR_OFF % 2 == 0 && DC_OFF % 4 == 0 && KLO_OFF % 4 == 0, "alignment");
+    static_assert(R1_OFF % 4 == 0 && US_OFF % 4 == 0 && KLO_OFF % 4 == 0 && BAR_OFF % 2 == 0, "alignment");
 };
 
 // Advances pos after k_dec_tok appended a token at slot pos, and resyncs
@@ -186,22 +187,17 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
              const float* bbuf, int32_t* pos, int32_t* status)
 {
     using Sm = ResyncSmem<DK, DV, C>;
-    using PL = PrepLayout<DK, DV, C>;
     using T = TcCfg<DK, DV, C>;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
-    float* kx = sm + Sm::KX_OFF;
-    float* vx = sm + Sm::VX_OFF;
-    float* cc = sm + Sm::CC_OFF;
-    float* dm = sm + Sm::DM_OFF;
-    float* d0 = sm + Sm::D0_OFF;
-    float* as = sm + Sm::AB_OFF;
-    float* bs = as + C;
+    float* wx = sm + Sm::WX_OFF;
+    float* us = sm + Sm::US_OFF;
     float* dCs = sm + Sm::DC_OFF;
+    unsigned char* r1 = reinterpret_cast<unsigned char*>(sm + Sm::R1_OFF);
     float* Wlo = sm + Sm::WLO_OFF;
-    float* Whi = cc;  // == Wlo + C * DK
-    float* Khi = sm + Sm::KHI_OFF;
+    float* Whi = Wlo + T::W_FLOATS;
     float* Klo = sm + Sm::KLO_OFF;
+    float* Khi = Klo + T::K_FLOATS;
     uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Sm::BAR_OFF);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Sm::BAR_OFF + 2);
 
@@ -238,22 +234,19 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
     for (; it < nt; ++it) {
         const int nh = todo[it];
         // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
-        stage_rows<DK>(kx, PL::KXS, kbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
-        stage_rows<DV>(vx, PL::VXS, vbuf, (int64_t)nh * C, C, 1, 0, in_bf16, IdxIdentity());
-        tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
-        for (int t = threadIdx.x; t < C; t += blockDim.x) {
-            as[t] = abuf[(int64_t)nh * C + t];
-            bs[t] = bbuf[(int64_t)nh * C + t];
-        }
+        prep_stage<DK, DV, C>(r1, kbuf, vbuf, abuf, bbuf, (int64_t)nh * C, 1, 0, in_bf16);
+        cp_async_commit();
+        cp_async_wait_all();
         __syncthreads();
-        chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, kx, PL::KXS, vx, PL::VXS, dCs);
-        tc_stage_w<DK, DV, C>(kx, PL::KXS, Whi, Wlo, threadIdx.x, blockDim.x);
+        chunk_prep<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, us, DV, wx, Sm::WXS, dCs);
+        tc_stage_w<DK, DV, C>(wx, Sm::WXS, Whi, Wlo, threadIdx.x, blockDim.x);
+        tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
         float* Sg = S_b + (int64_t)nh * DV * DK;
         tc_load_state<DK, DV, C>(SR, th, Sg, nullptr);
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (!tc_step<DK, DV, C>(SR, th, tbase, mbar, parity, Wlo, Klo, vx, PL::VXS, dCs, in_bf16, Sg,
+        if (!tc_step<DK, DV, C>(SR, th, tbase, mbar, parity, Wlo, Klo, us, DV, dCs, in_bf16, Sg,
                                 R + (int64_t)nh * DV * DK))
             break;
         if (threadIdx.x == 0) pos[nh] = 0;

@@ -1,6 +1,8 @@
-// k_pchunk.cuh -- chunk-boundary update P_chunk: k_prep, k_chain, k_cache_fill (sm_100a).
+// k_pchunk.cuh -- chunk-boundary update P_chunk part 2: k_chain, the fused chain + P_tok kernel,
+// k_cache_fill (sm_100a).  Part 1 (the chunk-local precompute) is in k_prep.cuh.
 #pragma once
 
+#include "k_prep.cuh"
 #include "k_ptok.cuh"
 #include "k_tc.cuh"
 
@@ -17,264 +19,6 @@ struct ChunkCfg {
     static constexpr int NTB = DV / RTB;
     static constexpr int THREADS = 256;
 };
-
-// P_chunk part 1 for one chunk, by one CTA (>= 128 threads), on the tensor
-// cores where the work is a dense contraction:
-//   D[s][s] = 1, D[t][s] = D[t-1][s] * alpha_t                     (fp32 chains)
-//   G[t][s] = k_t . k_s for s < t: mma tf32 over 8-wide blocks of d_k,
-//             ascending, k = k_hi + k_lo (k_lo = 0 and skipped when every k
-//             is exactly tf32, i.e. bf16 inputs):  G += k_lo*k_hi, k_hi*k_lo, k_hi*k_hi
-//   c[t][s] = D[t][s] * G[t][s]
-//   forward substitution for the columns x = u0 (init v_t) and w (init
-//   D[t][0] * k_t), in blocks of 16 tokens: for block b, acc_t = init_t;
-//   acc_t += sum over 8-token blocks of s < 16b (ascending) of the mma
-//   products (-c)_lo*x_hi, (-c)_hi*x_lo, (-c)_hi*x_hi; then, for s in
-//   [16b, t) ascending, acc_t = fma(-c[t][s], x_s, acc_t); x_t = beta_t * acc_t.
-// kx [C][DK+8] holds k on entry and w on exit; vx [C][DV+8] holds v on entry
-// and u0 on exit (row strides chosen so the mma fragment reads are
-// conflict-free); as, bs [C] gates; cc [C][C+4], dm, d0 are smem scratch.
-// Also writes w -> wout[t*ldw + j], u0 -> uout[t*ldu + i], D[C][s] -> dCout[s]
-// (any address space; uout may be vx itself).
-template <int DK, int DV, int C>
-struct PrepLayout {
-    static constexpr int KXS = DK + 8, VXS = DV + 8, CCS = C + 4;
-    static constexpr int NCOL = DV + DK;
-    static constexpr int STS = NCOL + 8;  // staging row stride: conflict-free fragment stores
-    static constexpr int DM = ((C + 1) * (C + 1) > 16 * STS ? (C + 1) * (C + 1) : 16 * STS);
-};
-
-template <int DK, int DV, int C>
-__device__ __forceinline__ void chunk_prep(float* kx, float* vx, const float* as, const float* bs, float* cc, float* dm,
-                                           float* d0, int k_exact, float* wout, int ldw, float* uout, int ldu,
-                                           float* dCout)
-{
-    using PL = PrepLayout<DK, DV, C>;
-    constexpr int KXS = PL::KXS, VXS = PL::VXS, CCS = PL::CCS, C1 = C + 1, NCOL = PL::NCOL, STS = PL::STS;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
-    const int nwarps = blockDim.x >> 5;
-    // decay products: column s is the chain D[t][s] = D[t-1][s] * alpha_t, t = s+1..C
-    for (int s = threadIdx.x; s <= C; s += blockDim.x) {
-        float d = 1.0f;
-        dm[s * C1 + s] = d;
-#pragma unroll
-        for (int t4i = 0; t4i < C; t4i += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(as + t4i);
-            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = t4i + e + 1;
-                if (t > s) {
-                    d = fmul(d, av[e]);
-                    dm[t * C1 + s] = d;
-                }
-            }
-        }
-    }
-    __syncthreads();
-    // Gram on the tensor cores: the (m16, n8) tiles of the lower triangle,
-    // spread over the warps; each tile's chain runs over d_k in 8-wide blocks
-    constexpr int MT = C / 16, NTILE = MT * (MT + 1);  // tile (m, q) with q <= 2m+1
-    for (int tile = warp; tile < NTILE; tile += nwarps) {
-        int m = 0;
-        while ((m + 1) * (m + 2) <= tile) ++m;
-        const int q = tile - m * (m + 1);
-        const int r0 = m * 16, n0 = q * 8;
-        float acc[4][4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
-#pragma unroll 4
-        for (int kb = 0; kb < DK / 8; ++kb) {
-            const int k0 = kb * 8;
-            const float a0 = kx[(r0 + g) * KXS + k0 + t4], a1 = kx[(r0 + g + 8) * KXS + k0 + t4];
-            const float a2 = kx[(r0 + g) * KXS + k0 + t4 + 4], a3 = kx[(r0 + g + 8) * KXS + k0 + t4 + 4];
-            const float b0 = kx[(n0 + g) * KXS + k0 + t4], b1 = kx[(n0 + g) * KXS + k0 + t4 + 4];
-            if (k_exact) {
-                const uint32_t ah[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
-                                        __float_as_uint(a3)};
-                const uint32_t bh[2] = {__float_as_uint(b0), __float_as_uint(b1)};
-                mma_tf32(acc[kb & 3], ah, bh);
-            } else {
-                uint32_t ah[4], al[4], bh[2], bl[2];
-                tf32_split(a0, ah[0], al[0]); tf32_split(a1, ah[1], al[1]);
-                tf32_split(a2, ah[2], al[2]); tf32_split(a3, ah[3], al[3]);
-                tf32_split(b0, bh[0], bl[0]); tf32_split(b1, bh[1], bl[1]);
-                mma_tf32(acc[0], al, bh);
-                mma_tf32(acc[1], ah, bl);
-                mma_tf32(acc[2], ah, bh);
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int tau = r0 + g + (c >> 1) * 8, sig = n0 + 2 * t4 + (c & 1);
-            const float G = k_exact ? fadd(fadd(acc[0][c], acc[1][c]), fadd(acc[2][c], acc[3][c]))
-                                    : fadd(fadd(acc[0][c], acc[1][c]), acc[2][c]);
-            if (sig < tau) cc[tau * CCS + sig] = fmul(dm[(tau + 1) * C1 + (sig + 1)], G);
-        }
-    }
-    for (int t = threadIdx.x; t < C; t += blockDim.x) d0[t] = dm[(t + 1) * C1];  // D[t][0], t = 1..C
-    if (dCout != nullptr)
-        for (int s = threadIdx.x; s <= C; s += blockDim.x) dCout[s] = dm[C * C1 + s];
-    __syncthreads();
-    float* stage = dm;  // [16][STS]: the block's accumulators
-    for (int b = 0; b < C / 16; ++b) {
-        const int t0 = 16 * b;
-        // init + tensor-core part: warp w owns column tiles w, w + nw, ... (each
-        // tile all u0 or all w columns); its tiles share the split c fragment
-        {
-            constexpr int NTW = (NCOL / 8 + 7) / 8;  // tiles per warp with 8 warps
-            float init[NTW][4], plh[NTW][4], phl[NTW][4], phh[NTW][4];
-            const float* xb[NTW];
-            int xs[NTW];
-#pragma unroll
-            for (int q = 0; q < NTW; ++q) {
-                const int nt = warp + nwarps * q;
-                const int n0 = nt * 8;
-                const bool is_u = n0 < DV;
-                xb[q] = is_u ? vx + n0 : kx + (n0 - DV);
-                xs[q] = is_u ? VXS : KXS;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    plh[q][c] = phl[q][c] = phh[q][c] = 0.f;
-                    const int tau = t0 + g + (c >> 1) * 8, cl = 2 * t4 + (c & 1);
-                    init[q][c] = nt >= NCOL / 8 ? 0.f
-                                 : is_u ? xb[q][tau * xs[q] + cl] : fmul(d0[tau], xb[q][tau * xs[q] + cl]);
-                }
-            }
-            for (int kb = 0; kb < 2 * b; ++kb) {
-                const int s0 = kb * 8;
-                uint32_t ah[4], al[4];
-                tf32_split(-cc[(t0 + g) * CCS + s0 + t4], ah[0], al[0]);
-                tf32_split(-cc[(t0 + g + 8) * CCS + s0 + t4], ah[1], al[1]);
-                tf32_split(-cc[(t0 + g) * CCS + s0 + t4 + 4], ah[2], al[2]);
-                tf32_split(-cc[(t0 + g + 8) * CCS + s0 + t4 + 4], ah[3], al[3]);
-#pragma unroll
-                for (int q = 0; q < NTW; ++q) {
-                    if (warp + nwarps * q < NCOL / 8) {
-                        uint32_t bh[2], bl[2];
-                        tf32_split(xb[q][(s0 + t4) * xs[q] + g], bh[0], bl[0]);
-                        tf32_split(xb[q][(s0 + t4 + 4) * xs[q] + g], bh[1], bl[1]);
-                        mma_tf32(plh[q], al, bh);
-                        mma_tf32(phl[q], ah, bl);
-                        mma_tf32(phh[q], ah, bh);
-                    }
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < NTW; ++q) {
-                const int nt = warp + nwarps * q;
-                if (nt < NCOL / 8) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float acc = b == 0 ? init[q][c]
-                                                 : fadd(init[q][c], fadd(fadd(plh[q][c], phl[q][c]), phh[q][c]));
-                        stage[(g + (c >> 1) * 8) * STS + nt * 8 + 2 * t4 + (c & 1)] = acc;
-                    }
-                }
-            }
-        }
-        __syncthreads();
-        // in-block part: one column per thread, sequential over the block's 16 tokens
-        for (int col = threadIdx.x; col < NCOL; col += blockDim.x) {
-            float xb[16];
-#pragma unroll
-            for (int tr = 0; tr < 16; ++tr) {
-                float acc = stage[tr * STS + col];
-#pragma unroll
-                for (int sr = 0; sr < tr; ++sr) acc = ffma(-cc[(t0 + tr) * CCS + t0 + sr], xb[sr], acc);
-                xb[tr] = fmul(bs[t0 + tr], acc);
-            }
-#pragma unroll
-            for (int tr = 0; tr < 16; ++tr) {
-                const int tau = t0 + tr;
-                if (col < DV) {
-                    vx[tau * VXS + col] = xb[tr];
-                    uout[tau * ldu + col] = xb[tr];
-                } else {
-                    kx[tau * KXS + (col - DV)] = xb[tr];
-                    wout[tau * ldw + (col - DV)] = xb[tr];
-                }
-            }
-        }
-        __syncthreads();
-    }
-}
-
-template <int DK, int DV, int C>
-struct PrepSmem {
-    using PL = PrepLayout<DK, DV, C>;
-    static constexpr int KX_OFF = 0;
-    static constexpr int VX_OFF = KX_OFF + C * PL::KXS;
-    static constexpr int CC_OFF = VX_OFF + C * PL::VXS;
-    static constexpr int DM_OFF = CC_OFF + C * PL::CCS;
-    static constexpr int D0_OFF = DM_OFF + ((PL::DM + 3) / 4) * 4;
-    static constexpr int AB_OFF = D0_OFF + C + 4;
-    static constexpr size_t BYTES = sizeof(float) * (AB_OFF + 2 * C);
-};
-
-// P_chunk part 1 for every full chunk: one CTA per (full chunk, head).
-template <int DK, int DV, int C>
-__global__ void __launch_bounds__(256)
-k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
-       const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ fco,
-       const int32_t* __restrict__ err, int N, int H, int in_bf16,
-       float* __restrict__ w_ws, float* __restrict__ u_ws, float* __restrict__ dC_ws)
-{
-    using Cf = ChunkCfg<DK, DV, C>;
-    using Sm = PrepSmem<DK, DV, C>;
-    using PL = PrepLayout<DK, DV, C>;
-    if (__ldg(err)) return;
-    extern __shared__ float4 smem_f4[];
-    float* sm = reinterpret_cast<float*>(smem_f4);
-    float* kx = sm + Sm::KX_OFF;
-    float* vx = sm + Sm::VX_OFF;
-    float* cc = sm + Sm::CC_OFF;
-    float* dm = sm + Sm::DM_OFF;
-    float* d0 = sm + Sm::D0_OFF;
-    float* as = sm + Sm::AB_OFF;
-    float* bs = as + C;
-
-    const int task = blockIdx.x;
-    const int h = task % H, g = task / H;
-    const int n = find_seq(fco, N, g);
-    const int64_t tok0 = (int64_t)__ldg(cu + n) + (int64_t)(g - __ldg(fco + n)) * C;
-    for (int t = threadIdx.x; t < C; t += blockDim.x) {
-        cp_async4(as + t, alpha + (tok0 + t) * H + h);
-        cp_async4(bs + t, beta + (tok0 + t) * H + h);
-    }
-    if (in_bf16) {
-        // raw bf16 rows [k | v] of the chunk land in the c / decay buffers
-        // (unused until the Gram), all copies in flight at once; then widen
-        static_assert(Sm::DM_OFF + ((PL::DM + 3) / 4) * 4 - Sm::CC_OFF >= C * (DK + DV) / 2, "raw staging fits");
-        unsigned char* raw = reinterpret_cast<unsigned char*>(cc);
-        constexpr int PK = DK / 8, PV = DV / 8;  // 16-byte pieces per row
-        for (int e = threadIdx.x; e < C * (PK + PV); e += blockDim.x) {
-            const int t = e / (PK + PV), pc = e % (PK + PV);
-            const int64_t row = (tok0 + t) * H + h;
-            const uint16_t* src = pc < PK ? reinterpret_cast<const uint16_t*>(k) + row * DK + pc * 8
-                                          : reinterpret_cast<const uint16_t*>(v) + row * DV + (pc - PK) * 8;
-            cp_async16(raw + (size_t)e * 16, src);
-        }
-        cp_async_commit();
-        cp_async_wait_all();
-        __syncthreads();
-        for (int e = threadIdx.x; e < C * (PK + PV); e += blockDim.x) {
-            const int t = e / (PK + PV), pc = e % (PK + PV);
-            float x[8];
-            lds8_raw(raw + (size_t)e * 16, 0, 1, x);
-            float* d = pc < PK ? kx + t * PL::KXS + pc * 8 : vx + t * PL::VXS + (pc - PK) * 8;
-            *reinterpret_cast<float4*>(d) = make_float4(x[0], x[1], x[2], x[3]);
-            *reinterpret_cast<float4*>(d + 4) = make_float4(x[4], x[5], x[6], x[7]);
-        }
-    } else {
-        stage_rows<DK>(kx, PL::KXS, k, tok0, C, H, h, in_bf16, IdxIdentity());
-        stage_rows<DV>(vx, PL::VXS, v, tok0, C, H, h, in_bf16, IdxIdentity());
-        cp_async_commit();
-        cp_async_wait_all();
-    }
-    __syncthreads();
-    chunk_prep<DK, DV, C>(kx, vx, as, bs, cc, dm, d0, in_bf16, w_ws + (int64_t)task * C * DK, DK,
-                          u_ws + (int64_t)task * C * DV, DV, dC_ws + (int64_t)task * Cf::DCS);
-}
 
 template <int DK, int DV, int C>
 struct ChainSmem {

@@ -18,6 +18,7 @@
 
 #include "k_tables.cuh"
 #include "k_ptok.cuh"
+#include "k_prep.cuh"
 #include "k_pchunk.cuh"
 #include "k_decode.cuh"
 #include "k_bwd.cuh"
