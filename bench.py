@@ -318,7 +318,7 @@ def parity_gate(d, o, st, C):
     cu = np.array([0, L], np.int32)
     ns = L // C + 1
     st_h = st[:ns, 0:1].contiguous().cpu().numpy()
-    mo, _ = oracle.schedule_tok_from_states(q, k, v, a, b, st_h, cu, C)
+    mo, _, _ = oracle.schedule_tok_from_states(q, k, v, a, b, st_h, cu, C)
     r = oracle.recurrent(q, k, v, a, b, cu, C)
     got = o[:L, 0:1].contiguous().cpu()
     bits_o = np.array_equal(got.view(torch.int16).numpy().view(np.uint16), oracle.to_bf16_bits(mo))

@@ -8,7 +8,9 @@
 #include "gdn_cpr.h"
 #include "kernels.cuh"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <atomic>
@@ -121,6 +123,40 @@ Workspace carve(void* base, int64_t max_full, int32_t N, int32_t H, int32_t dk, 
     return ws;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library does not link libcuda itself).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// Tensor map of a [T, H, D] token tensor for TMA boxes of D x 1 x `box`
+// tokens (one head, consecutive tokens).  The base is 16-byte aligned (checked
+// by the callers), and every stride is a multiple of 16 bytes.
+bool token_map(CUtensorMap* map, const void* base, int64_t T, int32_t H, int32_t D, int bf16, int box)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr || base == nullptr || T <= 0) return false;
+    const cuuint64_t esz = bf16 ? 2 : 4;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)H * D * esz};
+    const cuuint32_t boxd[3] = {(cuuint32_t)D, 1u, (cuuint32_t)box};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+               const_cast<void*>(base), dims, strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename K>
 cudaError_t set_smem(K* kernel, size_t bytes)
 {
@@ -185,9 +221,17 @@ gdn_status_t launch_forward(const FwdArgs& a)
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 2, a.stream);
+    // TMA descriptors of q, k, v for the intra-chunk kernels (boxes of SC tokens of one head)
+    CUtensorMap tmq, tmk, tmv;
+    if (a.tot.tasks > 0 &&
+        (!token_map(&tmq, a.q, a.T_total, a.H, D, a.in_bf16, TC::SC) ||
+         !token_map(&tmk, a.k, a.T_total, a.H, D, a.in_bf16, TC::SC) ||
+         !token_map(&tmv, a.v, a.T_total, a.H, D, a.in_bf16, TC::SC)))
+        return GDN_ERR_CUDA;
+    float* cacheRs = a.cache ? a.cache->rscale : nullptr;
     if constexpr (gdn::FusedSmem<D, D, C>::OK) if (fused) {
         mark(a.events, 3, a.stream);  // the chain has no separate time: it runs inside the next kernel
-        const void *q = a.q, *k = a.k, *v = a.v;
+        const void* k = a.k;
         const float *alpha = a.alpha, *beta = a.beta, *state_in = a.state_in;
         const int32_t *cu = a.cu, *fco = a.ws.fco, *so = a.ws.so, *order = a.ws.order, *cumc = a.ws.cumc;
         int32_t *err = a.ws.err, *progress = a.ws.progress, *tok_next = a.ws.tok_next;
@@ -199,9 +243,9 @@ gdn_status_t launch_forward(const FwdArgs& a)
         const int32_t mode = g_fault_mode.load();
         int withhold = mode == 1 ? 1 : 0;
         long long wait_limit = mode == 1 ? (long long)g_fault_wait.load() : gdn::kWaitLimit;
-        void* args[] = {&q, &k, &v, &alpha, &beta, &state_in, &cu, &fco, &so, &err, &N, &H, &in_bf16, &out_bf16,
-                        &w, &u, &dC, &states, &o, &cacheR, &progress, &tok_next, &order, &cumc, &maxc,
-                        &withhold, &wait_limit};
+        void* args[] = {&tmq, &tmk, &tmv, &k, &alpha, &beta, &state_in, &cu, &fco, &so, &err, &N, &H, &in_bf16,
+                        &out_bf16, &w, &u, &dC, &states, &o, &cacheR, &cacheRs, &progress, &tok_next, &order,
+                        &cumc, &maxc, &withhold, &wait_limit};
         if (cudaLaunchCooperativeKernel((const void*)gdn::k_chain_tok<D, D, C>, dim3((unsigned)sms), dim3(256), args,
                                         fsm, a.stream) != cudaSuccess ||
             cudaGetLastError() != cudaSuccess)
@@ -220,15 +264,16 @@ gdn_status_t launch_forward(const FwdArgs& a)
         constexpr size_t sm = TC::SMEM;
         if (set_smem(gdn::k_tok<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
         gdn::k_tok<D, D, C><<<(unsigned)(a.tot.tasks * a.H), TC::THREADS, sm, a.stream>>>(
-            a.q, a.k, a.v, a.alpha, a.beta, a.cu, a.ws.cto, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.out_bf16,
-            a.states, a.o, a.cache ? a.cache->R : nullptr);
+            tmq, tmk, tmv, a.alpha, a.beta, a.cu, a.ws.cto, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.out_bf16,
+            a.states, a.o, a.cache ? a.cache->R : nullptr, cacheRs);
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 4, a.stream);
     if (a.cache != nullptr && a.N > 0) {
         const gdn_cache_t& c = *a.cache;
         gdn::k_cache_fill<D, D, C><<<(unsigned)((int64_t)a.N * a.H), 256, 0, a.stream>>>(
-            a.k, a.v, a.alpha, a.beta, a.cu, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.states, c.S_b, c.R, c.kbuf,
+            a.k, a.v, a.alpha, a.beta, a.cu, a.ws.so, a.ws.err, a.N, a.H, a.in_bf16, a.states, c.S_b, c.R, c.rscale,
+            c.kbuf,
             c.vbuf, c.abuf, c.bbuf, c.pos);
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     }
@@ -268,7 +313,8 @@ gdn_status_t launch_decode(const DecArgs& a)
     const unsigned tgrid = (unsigned)std::min<int64_t>(items, (int64_t)sms * per_sm);
     mark(a.events, 0, a.stream);
     gdn::k_dec_tok<D, D, C><<<tgrid, DC::THREADS, DC::SMEM, a.stream>>>(
-        a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, a.o,
+        a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.rscale, c.kbuf, c.vbuf, c.abuf, c.bbuf,
+        c.pos, a.o,
         (int)items, c.status);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
@@ -278,7 +324,7 @@ gdn_status_t launch_decode(const DecArgs& a)
     const int64_t min_grid = (NH + 1023) / 1024;
     const unsigned rgrid = (unsigned)std::max<int64_t>(std::min<int64_t>(NH, sms), min_grid);
     gdn::k_dec_resync<D, D, C><<<rgrid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
-        (int)NH, a.in_bf16, c.S_b, c.R, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, c.status);
+        (int)NH, a.in_bf16, c.S_b, c.R, c.rscale, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, c.status);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 2, a.stream);
     return GDN_OK;
@@ -410,7 +456,7 @@ gdn_status_t launch_backward(const BwdArgs& a)
 
 extern "C" {
 
-const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v4/NL8/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3"; }
+const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v5/NL8/ptok-scaled/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3"; }
 
 const char* gdn_status_string(gdn_status_t s)
 {
@@ -477,7 +523,8 @@ gdn_status_t gdn_cpr_forward_timed(const void* q, const void* k, const void* v, 
     }
     if (cache_out != nullptr) {
         const gdn_cache_t& c = *cache_out;
-        if (!c.S_b || !c.R || !c.kbuf || !c.vbuf || !c.abuf || !c.bbuf || !c.pos) return GDN_ERR_INVALID_ARG;
+        if (!c.S_b || !c.R || !c.rscale || !c.kbuf || !c.vbuf || !c.abuf || !c.bbuf || !c.pos)
+            return GDN_ERR_INVALID_ARG;
         if (!aligned16(c.S_b) || !aligned16(c.R) || !aligned16(c.kbuf) || !aligned16(c.vbuf))
             return GDN_ERR_INVALID_ARG;
         if (total_tokens > 0 && (!k || !v || !alpha || !beta)) return GDN_ERR_INVALID_ARG;
@@ -597,7 +644,7 @@ gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, 
     }
     const gdn_cache_t& c = *cache;
     if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
-    if (!c.S_b || !c.R || !c.kbuf || !c.vbuf || !c.abuf || !c.bbuf || !c.pos) return GDN_ERR_INVALID_ARG;
+    if (!c.S_b || !c.R || !c.rscale || !c.kbuf || !c.vbuf || !c.abuf || !c.bbuf || !c.pos) return GDN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(c.S_b) || !aligned16(c.R) ||
         !aligned16(c.kbuf) || !aligned16(c.vbuf))
         return GDN_ERR_INVALID_ARG;

@@ -137,7 +137,7 @@ const char* kSemantic =
     "chunking: boundaries every C tokens from each sequence's own token 0\n"
     "composition: boundary states by the chunk update P_chunk; every output by the per-token recurrence P_tok\n"
     "  started at its chunk's boundary state; decode runs P_tok and after C buffered tokens sets\n"
-    "  S_b <- P_chunk(S_b, buffer), R <- S_b\n"
+    "  S_b <- P_chunk(S_b, buffer), and the running state <- S_b\n"
     "inputs: q, k [T][H][d_k], v [T][H][d_v] in in_dtype (bf16 widened exactly); alpha, beta [T][H] fp32; no q scaling\n"
     "outputs: o [T][H][d_v] in out_dtype; chunk states at positions 0, C, ..., floor(L/C)*C\n";
 
@@ -146,8 +146,10 @@ const char* kPolicy =
     "fp32 operations: IEEE binary32, round to nearest even, subnormals kept, no contraction\n"
     "tree(x, y): 8 leaves of d_k/8 contiguous elements; leaf = x[0]*y[0], then fma ascending;\n"
     "  result ((l0+l1)+(l2+l3))+((l4+l5)+(l6+l7))\n"
-    "P_tok per row i: u = tree(R_i, k); delta = beta*(v_i - alpha*u); R_ij = fma(delta, k_j, alpha*R_ij);\n"
-    "  o_i = tree(R_i, q)\n"
+    "P_tok on a running state c*R (c = 1, R = the boundary state at a chunk start), per token:\n"
+    "  kq = tree(k, q); cn = alpha*c; per row i, over R before the token: dk = tree(R_i, k), dq = tree(R_i, q),\n"
+    "  d = beta*(v_i - cn*dk); if cn >= 2^-64: dt = d*rcp.rn(cn), R_ij = fma(dt, k_j, R_ij),\n"
+    "  o_i = cn*fma(dt, kq, dq), c = cn; else (fold): R_ij = fma(d, k_j, cn*R_ij), o_i = fma(d, kq, cn*dq), c = 1\n"
     "split of an fp32 operand x: hi = cvt.rna.tf32(x), lo = cvt.rna.tf32(x - hi); k has no lo part for bf16 inputs\n"
     "P_chunk part 1: decays D[s][s] = 1, D[t][s] = D[t-1][s]*alpha_t;\n"
     "  Gram G[t][s] = k_t.k_s (s < t) by mma.sync.m16n8k8 tf32, fp32 accumulate, K blocks of 8 ascending:\n"

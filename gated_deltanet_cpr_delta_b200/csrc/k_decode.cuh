@@ -7,9 +7,11 @@
 namespace gdn {
 
 // ------------------------------------------------------------------ decode
-// One decode token per (sequence, head): P_tok on the running state R, and
-// the token appended to the buffer at slot pos (pos itself is advanced by
-// k_dec_resync, which runs next).  Work item = (sequence-head, row tile).
+// One decode token per (sequence, head): P_tok on the running state
+// rscale * R (the prefill's per-token step: tok_step_row), and the token
+// appended to the buffer at slot pos (pos and rscale themselves are advanced
+// by k_dec_resync, which runs next, so that every row tile of the pair reads
+// the same old scale).  Work item = (sequence-head, row tile).
 // Persistent: CTA b takes items b, b + grid, ...  Each item's state rows and
 // raw token stream into shared memory by cp.async, DecCfg::S - 1 items ahead
 // of the one being computed, so several items' loads are in flight per CTA
@@ -36,8 +38,8 @@ template <int DK, int DV, int C>
 __global__ void __launch_bounds__(DecCfg<DK, DV>::THREADS)
 k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
           const float* __restrict__ alpha, const float* __restrict__ beta, int in_bf16, int out_bf16,
-          float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos, void* __restrict__ o,
-          int nitems, int32_t* status)
+          float* R, const float* rscale, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos,
+          void* __restrict__ o, int nitems, int32_t* status)
 {
     using Cf = DecCfg<DK, DV>;
     using RS = typename Cf::RS;
@@ -76,6 +78,7 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
             if (t == 0) cp_async4(gates, alpha + nh);
             if (t == 1) cp_async4(gates + 1, beta + nh);
             if (t == 2) cp_async4(gates + 2, pos + nh);
+            if (t == 3) cp_async4(gates + 3, rscale + nh);
         }
         cp_async_commit();
     };
@@ -91,7 +94,7 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
         const int nh = it / Cf::NT, r = it % Cf::NT;
         const unsigned char* rw = raw(st);
         const float* gates = reinterpret_cast<const float*>(rw + 16 * (2 * kp + vp));
-        const float a = gates[0], b = gates[1];
+        const float a = gates[0], b = gates[1], cs = gates[3];
         const int p = __float_as_int(gates[2]);
         if (t < 2 * kp + vp) {  // widen the raw token
             const uint4 pc = *reinterpret_cast<const uint4*>(rw + 16 * t);
@@ -133,7 +136,12 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
         const bool valid = p >= 0 && p < C;  // an invalid position writes nothing
         if (!valid && t == 0) record_error(status, GDN_ERR_DEVICE_INPUT);
         if (valid) {
-            const float ot = ptok_step<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], a, b);
+            const float cn = fmul(a, cs);
+            const bool fold = !(cn >= kFoldTau);
+            const float rc = fold ? 1.0f : __frcp_rn(cn);
+            const float kq = tok_kq<DK>(ks + part * RS::PS, qs + part * RS::PS);
+            const float ot = tok_step_row<DK>(Rp, ks + part * RS::PS, qs + part * RS::PS, vs[row], b, kq, cn, rc,
+                                              fold);
             store_row_pairs<DK>(rslot(st), Rp);
             if (part == 0) store1(o, (int64_t)nh * DV + r * Cf::RT + row, out_bf16, ot);
         }
@@ -173,9 +181,10 @@ struct ResyncSmem {
     static_assert(R1_OFF % 4 == 0 && US_OFF % 4 == 0 && KLO_OFF % 4 == 0 && BAR_OFF % 2 == 0, "alignment");
 };
 
-// Advances pos after k_dec_tok appended a token at slot pos, and resyncs
-// where that token completed a chunk: S_b <- P_chunk(S_b, buffer), R <- S_b,
-// pos <- 0.  P_chunk runs the same device functions as the prefill
+// Advances pos and the running scale after k_dec_tok appended a token at slot
+// pos (rscale <- alpha * rscale, or 1 where that product falls below the fold
+// threshold, as k_dec_tok computed it), and resyncs where the token completed a
+// chunk: S_b <- P_chunk(S_b, buffer), R <- S_b, rscale <- 1, pos <- 0.  P_chunk runs the same device functions as the prefill
 // (chunk_prep, then the tcgen05 boundary step).  Persistent: CTA b handles
 // (sequence, head) pairs b, b + grid, ...  A pos outside [0, C) is left
 // unchanged (k_dec_tok has recorded it).  If an MMA completion wait times
@@ -183,8 +192,8 @@ struct ResyncSmem {
 // and GDN_ERR_TIMEOUT goes to *status (when non-null).
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256, 1)
-k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const void* vbuf, const float* abuf,
-             const float* bbuf, int32_t* pos, int32_t* status)
+k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const void* kbuf, const void* vbuf,
+             const float* abuf, const float* bbuf, int32_t* pos, int32_t* status)
 {
     using Sm = ResyncSmem<DK, DV, C>;
     using T = TcCfg<DK, DV, C>;
@@ -212,7 +221,10 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, const void* kbuf, const 
         if (p < 0 || p >= C) continue;          // invalid: left unchanged
         if (p + 1 < C) {
             pos[nh] = p + 1;
+            const float cn = fmul(abuf[(int64_t)nh * C + p], rscale[nh]);
+            rscale[nh] = cn >= kFoldTau ? cn : 1.0f;
         } else {
+            rscale[nh] = 1.0f;
             const int slot = atomicAdd(&ntodo, 1);
             if (slot < 1024) todo[slot] = nh;   // the host sizes the grid so that a CTA has <= 1024 pairs
         }

@@ -199,7 +199,7 @@ k_chain(const void* __restrict__ k, const float* __restrict__ state_in, const in
 // ------------------------------------------------------------------ fused chain + P_tok
 template <int DK, int DV, int C>
 struct FusedSmem {
-    static constexpr size_t TOK = ((TokCfg<DK, DV, C>::SMEM + 15) / 16) * 16;  // one P_tok task
+    static constexpr size_t TOK = ((TokCfg<DK, DV, C>::SMEM + 127) / 128) * 128;  // one P_tok task, 128-byte aligned
     static constexpr size_t BYTES = ChainSmem<DK, DV, C>::BYTES > 2 * TOK ? ChainSmem<DK, DV, C>::BYTES : 2 * TOK;
     static constexpr bool OK = TokCfg<DK, DV, C>::THREADS == 128;  // two P_tok tasks per 256-thread CTA
 };
@@ -218,20 +218,22 @@ struct FusedSmem {
 // makes the chains publish nothing, so every wait runs out.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256, 1)
-k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+k_chain_tok(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const __grid_constant__ CUtensorMap tm_v, const void* __restrict__ k,
             const float* __restrict__ alpha, const float* __restrict__ beta, const float* __restrict__ state_in,
             const int32_t* __restrict__ cu, const int32_t* __restrict__ fco, const int32_t* __restrict__ so,
             int32_t* err, int N, int H, int in_bf16, int out_bf16, const float* __restrict__ w_ws,
             const float* __restrict__ u_ws, const float* __restrict__ dC_ws, float* states, void* __restrict__ o,
-            float* __restrict__ cacheR, int32_t* progress, int32_t* tok_next, const int32_t* __restrict__ order,
-            const int32_t* __restrict__ cumc, int maxc, int withhold, long long wait_limit)
+            float* __restrict__ cacheR, float* __restrict__ cacheRs, int32_t* progress, int32_t* tok_next,
+            const int32_t* __restrict__ order, const int32_t* __restrict__ cumc, int maxc, int withhold,
+            long long wait_limit)
 {
     using Fs = FusedSmem<DK, DV, C>;
     static_assert(Fs::OK, "d_v = 128: two 128-thread P_tok tasks per CTA");
     volatile int32_t* verr = err;
     if (*verr) return;
-    extern __shared__ float4 smem_f4[];
-    float* sm = reinterpret_cast<float*>(smem_f4);
+    extern __shared__ __align__(128) float4 smem_a128[];  // TMA boxes need 128-byte alignment
+    float* sm = reinterpret_cast<float*>(smem_a128);
     if ((int)blockIdx.x < N * H) {
         chain_run<DK, DV, C>(k, state_in, cu, fco, so, err, H, in_bf16, w_ws, u_ws, dC_ws, states, blockIdx.x,
                              progress, withhold, sm);
@@ -240,6 +242,9 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
     const int half = threadIdx.x >> 7, tid = threadIdx.x & 127;
     float* tsm = sm + half * (Fs::TOK / 4);
     const HalfSync hs{2 + half};
+    tok_context_init<DK, DV, C>(tsm, tid);
+    hs();
+    uint32_t phase = 0;
     __shared__ int qslot[2], go[2];
     const int ntask = __ldg(cumc + maxc);
     // Thread 0 of a half claims its next queue slot one task ahead, so the
@@ -268,18 +273,21 @@ k_chain_tok(const void* __restrict__ q, const void* __restrict__ k, const void* 
         hs();
         if (!go[half]) break;
         const int seq0 = __ldg(cu + n);
-        tok_task<DK, DV, C, true>(q, k, v, alpha, beta, n, c, h, H, seq0, __ldg(cu + n + 1) - seq0,
-                                  (int64_t)__ldg(so + n) + c, in_bf16, out_bf16, states, o, cacheR, tsm, tid, hs);
+        if (!tok_task<DK, DV, C, true>(TokMaps{&tm_q, &tm_k, &tm_v}, alpha, beta, n, c, h, H, seq0,
+                                       __ldg(cu + n + 1) - seq0, (int64_t)__ldg(so + n) + c, in_bf16, out_bf16,
+                                       states, o, cacheR, cacheRs, tsm, tid, hs, phase, err))
+            break;
     }
 }
 
-// Decode cache for a continuation: one CTA per (sequence, head).
+// Decode cache for a continuation: one CTA per (sequence, head).  The running
+// state of a partial last chunk (R, rscale) comes from the intra-chunk kernel.
 template <int DK, int DV, int C>
 __global__ void __launch_bounds__(256)
 k_cache_fill(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
              const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ so,
              const int32_t* __restrict__ err, int N, int H, int in_bf16, const float* __restrict__ states,
-             float* S_b, float* R, void* kbuf, void* vbuf, float* abuf, float* bbuf, int32_t* pos)
+             float* S_b, float* R, float* rscale, void* kbuf, void* vbuf, float* abuf, float* bbuf, int32_t* pos)
 {
     if (__ldg(err)) return;
     const int nh = blockIdx.x;
@@ -315,7 +323,10 @@ k_cache_fill(const void* __restrict__ k, const void* __restrict__ v, const float
         abuf[(int64_t)nh * C + s] = __ldg(alpha + tok * H + h);
         bbuf[(int64_t)nh * C + s] = __ldg(beta + tok * H + h);
     }
-    if (threadIdx.x == 0) pos[nh] = p;
+    if (threadIdx.x == 0) {
+        pos[nh] = p;
+        if (p == 0) rscale[nh] = 1.0f;  // otherwise the intra-chunk kernel wrote the running scale
+    }
 }
 
 }  // namespace gdn

@@ -121,7 +121,7 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, int bf16, float* u
                                            float* dCout)
 {
     using P = PrepCfg<DK, DV, C>;
-    constexpr int MS = P::MS, SS = P::SS, NB = P::NB, NCOL = P::NCOL;
+    constexpr int MS = P::MS, SS = P::SS, NB = P::NB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const int nwarps = blockDim.x >> 5;
     const int krb = P::krb(bf16), vrb = P::vrb(bf16);

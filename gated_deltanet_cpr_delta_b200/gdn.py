@@ -44,9 +44,9 @@ class GdnError(RuntimeError):
 
 
 class CacheStruct(ctypes.Structure):
-    _fields_ = [("S_b", ctypes.c_void_p), ("R", ctypes.c_void_p), ("kbuf", ctypes.c_void_p),
-                ("vbuf", ctypes.c_void_p), ("abuf", ctypes.c_void_p), ("bbuf", ctypes.c_void_p),
-                ("pos", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+    _fields_ = [("S_b", ctypes.c_void_p), ("R", ctypes.c_void_p), ("rscale", ctypes.c_void_p),
+                ("kbuf", ctypes.c_void_p), ("vbuf", ctypes.c_void_p), ("abuf", ctypes.c_void_p),
+                ("bbuf", ctypes.c_void_p), ("pos", ctypes.c_void_p), ("status", ctypes.c_void_p)]
 
 
 _lib = None
@@ -181,10 +181,12 @@ def gdn_cpr_workspace_size(total_tokens: int, num_seqs: int, H: int, d_k: int, d
 def new_cache(N: int, H: int, d_k: int, d_v: int, C: int, dtype: torch.dtype, device="cuda",
               state: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
     """Allocate a decode cache (gdn_cache_t layout).  With ``state`` [N,H,d_v,d_k]
-    it starts at a chunk boundary with that state, otherwise at zero.  ``status``
-    is the decode step's device status word (one int32, starts at GDN_OK)."""
+    it starts at a chunk boundary with that state, otherwise at zero.  The
+    running state is ``rscale * R``.  ``status`` is the decode step's device
+    status word (one int32, starts at GDN_OK)."""
     S = torch.zeros(N, H, d_v, d_k, dtype=torch.float32, device=device) if state is None else state.clone()
-    return dict(S_b=S, R=S.clone(), kbuf=torch.zeros(N, H, C, d_k, dtype=dtype, device=device),
+    return dict(S_b=S, R=S.clone(), rscale=torch.ones(N, H, dtype=torch.float32, device=device),
+                kbuf=torch.zeros(N, H, C, d_k, dtype=dtype, device=device),
                 vbuf=torch.zeros(N, H, C, d_v, dtype=dtype, device=device),
                 abuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
                 bbuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
@@ -194,7 +196,7 @@ def new_cache(N: int, H: int, d_k: int, d_v: int, C: int, dtype: torch.dtype, de
 
 def _cache_struct(c: Dict[str, torch.Tensor]) -> CacheStruct:
     st = c.get("status")
-    return CacheStruct(*[c[n].data_ptr() for n in ("S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos")],
+    return CacheStruct(*[c[n].data_ptr() for n in ("S_b", "R", "rscale", "kbuf", "vbuf", "abuf", "bbuf", "pos")],
                        st.data_ptr() if st is not None else None)
 
 

@@ -80,7 +80,12 @@ typedef enum {
  * Decode cache of N sequences.  It is the complete resumable state of a CPR
  * layer at any token position.  All fields are caller-owned device memory.
  *   S_b  [N, H, d_v, d_k] fp32   the last chunk-boundary state (position floor(p/C)*C)
- *   R    [N, H, d_v, d_k] fp32   the running per-token state (== S_b when pos == 0)
+ *   R    [N, H, d_v, d_k] fp32   the running per-token state divided by rscale
+ *   rscale [N, H] fp32           the running state's scale: the running state is
+ *                                rscale * R.  The per-token step keeps the decay
+ *                                in this scale and folds it into R when it would
+ *                                fall below 2^-64 (R == S_b and rscale == 1 when
+ *                                pos == 0)
  *   kbuf [N, H, C, d_k]  in_dtype  the tokens since the last boundary ...
  *   vbuf [N, H, C, d_v]  in_dtype
  *   abuf [N, H, C] fp32, bbuf [N, H, C] fp32   ... their gates
@@ -93,12 +98,13 @@ typedef enum {
  *                                The library never clears it: the caller sets
  *                                it to GDN_OK (0) and reads it back.  NULL: not
  *                                recorded.  gdn_cpr_forward ignores it.
- * A fresh cache for an initial state S_0 is S_b = R = S_0 with pos = 0.  The
- * buffer contents do not matter while pos == 0.
+ * A fresh cache for an initial state S_0 is S_b = R = S_0 with rscale = 1 and
+ * pos = 0.  The buffer contents do not matter while pos == 0.
  */
 typedef struct {
     float*   S_b;
     float*   R;
+    float*   rscale;
     void*    kbuf;
     void*    vbuf;
     float*   abuf;
@@ -387,10 +393,17 @@ gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v,
  *    GDN_NOALLOC_SCRATCH_BYTES.  At d_k = d_v = 128 and C = 64 that is about
  *    65,000 (token, head) pairs, for example 4,000 tokens with 16 heads.  Larger
  *    batches return GDN_ERR_WORKSPACE before anything is enqueued.
- *  - Every device that loads the library holds the array until the process exits.
+ *  - Every device that uses the library holds the array until the process
+ *    exits.  CUDA loads modules lazily by default, so the array is committed on
+ *    a device at the first call there (unless CUDA_MODULE_LOADING=EAGER): a
+ *    caller that reserves the whole device for its own pool makes one call
+ *    first.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it.  Make
- *    that first call before any stream capture begins.
+ *    (cudaGetSymbolAddress, with that device current) and caches it per device
+ *    ordinal for the life of the process.  Make that first call before any
+ *    stream capture begins.  The cache does not survive cudaDeviceReset (the
+ *    module is reloaded at another address): do not use this entry point after
+ *    a device reset in the same process.
  *  - All calls on a device share the one array, and it keeps the last call's
  *    contents; no part of it needs to start at zero.  Calls whose work
  *    overlaps on the GPU (different streams, or different host threads)

@@ -41,9 +41,9 @@ def _load():
         lib.oracle_adjoint_fp64.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
         lib.sched_forward.restype = ctypes.c_int
         lib.sched_forward.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
-                                      P, P, P, P, P, P, P, P, P]
+                                      P, P, P, P, P, P, P, P, P, P]
         lib.sched_decode_step.restype = ctypes.c_int
-        lib.sched_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P,
+        lib.sched_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P,
                                           i32, i32, i32, i32, i32, P]
         lib.sched_f32_to_bf16.restype = None
         lib.sched_f32_to_bf16.argtypes = [P, P, ctypes.c_int64]
@@ -126,7 +126,8 @@ def chunkwise(q, k, v, alpha, beta, cu_seqlens, C, state_in=None):
 def schedule_forward(q, k, v, alpha, beta, cu_seqlens, C, state_in=None, with_cache=False):
     """fp32 schedule model of the CPR forward.  Inputs must be fp32-valued
     (bf16 inputs widened exactly).  Returns dict(o (fp32, before the output
-    cast), states, and with_cache: S_b, R, kbuf, vbuf, abuf, bbuf, pos)."""
+    cast), states, and with_cache: S_b, R, kbuf, vbuf, abuf, bbuf, pos, rscale),
+    the running state being rscale * R."""
     lib = _load()
     q, k, v = _c(q, np.float32), _c(k, np.float32), _c(v, np.float32)
     alpha, beta = _c(alpha, np.float32), _c(beta, np.float32)
@@ -138,13 +139,13 @@ def schedule_forward(q, k, v, alpha, beta, cu_seqlens, C, state_in=None, with_ca
     o = np.zeros((T, H, dv), np.float32)
     states = np.zeros((num_chunk_states(cu, C), H, dv, dk), np.float32)
     out = dict(o=o, states=states)
-    cache = [None] * 7
+    cache = [None] * 8
     if with_cache:
         cache = [np.zeros((N, H, dv, dk), np.float32), np.zeros((N, H, dv, dk), np.float32),
                  np.zeros((N, H, C, dk), np.float32), np.zeros((N, H, C, dv), np.float32),
                  np.zeros((N, H, C), np.float32), np.zeros((N, H, C), np.float32),
-                 np.zeros((N, H), np.int32)]
-        out.update(zip(["S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos"], cache))
+                 np.zeros((N, H), np.int32), np.zeros((N, H), np.float32)]
+        out.update(zip(["S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos", "rscale"], cache))
     rc = lib.sched_forward(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(s_in), _p(cu),
                            N, H, dk, dv, C, _p(o), _p(states), *[_p(a) for a in cache])
     if rc:
@@ -163,7 +164,7 @@ def schedule_decode_step(cache, q, k, v, alpha, beta, C):
     dv = v.shape[2]
     o = np.zeros((N, H, dv), np.float32)
     rc = lib.sched_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
-                               *[_p(cache[n]) for n in ["S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos"]],
+                               *[_p(cache[n]) for n in ["S_b", "R", "kbuf", "vbuf", "abuf", "bbuf", "pos", "rscale"]],
                                N, H, dk, dv, C, _p(o))
     if rc:
         raise RuntimeError(f"sched_decode_step failed ({rc})")
@@ -182,12 +183,13 @@ def to_bf16_bits(x):
 def schedule_tok_from_states(q, k, v, alpha, beta, states, cu_seqlens, C):
     """fp32 schedule model of P_tok, started from the given boundary states
     (chunk_states layout).  Returns (o [T,H,dv] fp32 before the output cast,
-    R_final [N,H,dv,dk])."""
+    R_final [N,H,dv,dk], Rs_final [N,H]): the running state Rs * R after each
+    sequence's last token."""
     lib = _load()
     if not hasattr(lib, "_tok_states_ready"):
         P, i32 = ctypes.c_void_p, ctypes.c_int32
         lib.sched_tok_from_states.restype = ctypes.c_int
-        lib.sched_tok_from_states.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P]
+        lib.sched_tok_from_states.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P]
         lib._tok_states_ready = True
     q, k, v = _c(q, np.float32), _c(k, np.float32), _c(v, np.float32)
     alpha, beta = _c(alpha, np.float32), _c(beta, np.float32)
@@ -198,8 +200,9 @@ def schedule_tok_from_states(q, k, v, alpha, beta, states, cu_seqlens, C):
     N = cu.shape[0] - 1
     o = np.zeros((T, H, dv), np.float32)
     Rf = np.zeros((N, H, dv, dk), np.float32)
+    Rs = np.zeros((N, H), np.float32)
     rc = lib.sched_tok_from_states(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(states), _p(cu),
-                                   N, H, dk, dv, C, _p(o), _p(Rf))
+                                   N, H, dk, dv, C, _p(o), _p(Rf), _p(Rs))
     if rc:
         raise RuntimeError(f"sched_tok_from_states failed ({rc})")
-    return o, Rf
+    return o, Rf, Rs

@@ -103,12 +103,16 @@ class Fp32Schedule:
     """The fp32 CPR schedule, replayed with exact rationals and an explicit
     binary32 rounding after every operation (tiny inputs only).
 
-    ``mul(a,b) = rn32(a*b)``, ``add``/``sub`` likewise, and
-    ``fma(a,b,c) = rn32(a*b + c)`` (one rounding).  The schedule is the one
-    stated in the design notes: NL = 8 contiguous leaves over d_k, each an
-    ascending fused multiply-add chain started by a plain product, combined
-    by the fixed tree ((0+1)+(2+3))+((4+5)+(6+7)).
+    ``mul(a,b) = rn32(a*b)``, ``add``/``sub`` likewise, ``rcp(a) = rn32(1/a)``
+    and ``fma(a,b,c) = rn32(a*b + c)`` (one rounding).  The reduction tree has
+    NL = 8 contiguous leaves over d_k, each an ascending fused multiply-add
+    chain started by a plain product, combined by the fixed tree
+    ((0+1)+(2+3))+((4+5)+(6+7)).  The per-token step keeps its running state
+    as a scale times a matrix (see :meth:`p_tok`).
     """
+
+    #: a decay whose new scale would fall below this is folded into the matrix
+    FOLD_TAU = Fraction(1, 2 ** 64)
 
     NL = 8
 
@@ -141,16 +145,36 @@ class Fp32Schedule:
         add = self.add
         return add(add(add(p[0], p[1]), add(p[2], p[3])), add(add(p[4], p[5]), add(p[6], p[7])))
 
-    def p_tok(self, R: Mat, k, v, q, a, b):
-        """One per-token step on the running state R (returns new R and o)."""
+    @staticmethod
+    def rcp(a):
+        return rn32(1 / F(a))
+
+    def p_tok(self, R: Mat, c, k, v, q, a, b):
+        """One per-token step on the running state c * R; returns (R, c, o).
+
+        With cn = a*c: if cn >= 2^-64 the decay stays in the scale (c <- cn)
+        and row i gets dt = (b*(v_i - cn*tree(R_i, k))) * rcp(cn),
+        R_ij <- fma(dt, k_j, R_ij), o_i = cn * fma(dt, tree(k, q), tree(R_i, q));
+        otherwise it is folded into R (c <- 1): d = b*(v_i - cn*tree(R_i, k)),
+        R_ij <- fma(d, k_j, cn*R_ij), o_i = fma(d, tree(k, q), cn*tree(R_i, q)).
+        The trees over R are taken before the update."""
+        kq = self.tree(k, q)
+        cn = self.mul(a, c)
+        fold = not (cn >= self.FOLD_TAU)
+        rc = None if fold else self.rcp(cn)
         R2, o = [], []
         for i, Ri in enumerate(R):
-            u = self.tree(Ri, k)
-            d = self.mul(b, self.sub(v[i], self.mul(a, u)))
-            row = [self.fma(d, k[j], self.mul(a, Ri[j])) for j in range(len(Ri))]
-            R2.append(row)
-            o.append(self.tree(row, q))
-        return R2, o
+            dk = self.tree(Ri, k)
+            dq = self.tree(Ri, q)
+            d = self.mul(b, self.sub(v[i], self.mul(cn, dk)))
+            if not fold:
+                dt = self.mul(d, rc)
+                R2.append([self.fma(dt, k[j], Ri[j]) for j in range(len(Ri))])
+                o.append(self.mul(cn, self.fma(dt, kq, dq)))
+            else:
+                R2.append([self.fma(d, k[j], self.mul(cn, Ri[j])) for j in range(len(Ri))])
+                o.append(self.fma(d, kq, self.mul(cn, dq)))
+        return R2, (Fraction(1) if fold else cn), o
 
     def p_chunk(self, S: Mat, ks, vs, al, be):
         """Chunk-boundary update of S over the C tokens ks/vs/al/be."""
@@ -205,9 +229,9 @@ class Fp32Schedule:
         outs = []
         for c0 in range(0, T, C):
             n = min(C, T - c0)
-            R = B
+            R, c = B, Fraction(1)
             for t in range(c0, c0 + n):
-                R, o = self.p_tok(R, k[t], v[t], q[t], alpha[t], beta[t])
+                R, c, o = self.p_tok(R, c, k[t], v[t], q[t], alpha[t], beta[t])
                 outs.append(o)
             if n == C:
                 B = self.p_chunk(B, k[c0:c0 + C], v[c0:c0 + C], alpha[c0:c0 + C], beta[c0:c0 + C])

@@ -3,8 +3,8 @@
  *
  * Scalar CPU model, in IEEE fp32, of the arithmetic schedule that the CUDA
  * kernels are required to execute bit for bit.  It is written from the
- * schedule's text (the "Arithmetic schedule" section of the design notes),
- * not from the kernels, and it shares no code with them.  Only tests/,
+ * schedule stated below, not from the kernels, and it shares no code with
+ * them.  Only tests/,
  * __graft_entry__.smoke() and bench.py's cpu_baseline leg may load it.
  *
  * Every floating-point operation below is one IEEE-754 binary32 operation
@@ -23,9 +23,17 @@
  * Schedule (NL = 8 leaves, L = d_k / 8):
  *   tree(x, y): leaf l = x[lL]*y[lL], then fma(x[lL+m], y[lL+m], .) for
  *               m = 1..L-1; result ((p0+p1)+(p2+p3)) + ((p4+p5)+(p6+p7)).
- *   P_tok(R; k, v, q, a, b), every row i:
- *               u = tree(R_i, k); d = b * (v_i - a * u);
- *               R_ij = fma(d, k_j, a * R_ij); o_i = tree(R_i, q).
+ *   P_tok on a running state kept as c * Rt (a scale c and a matrix Rt;
+ *               c = 1 and Rt = the boundary state at a chunk's start), one
+ *               token (k, v, q, a, b):
+ *               kq = tree(k, q); cn = a * c;
+ *               for every row i: dk = tree(Rt_i, k), dq = tree(Rt_i, q)
+ *               (over Rt before the token), d = b * (v_i - cn * dk);
+ *               if cn >= 2^-64:  dt = d * (1 / cn) (the reciprocal rounded),
+ *                                Rt_ij = fma(dt, k_j, Rt_ij),
+ *                                o_i = cn * fma(dt, kq, dq);   c = cn
+ *               else (a fold):   Rt_ij = fma(d, k_j, cn * Rt_ij),
+ *                                o_i = fma(d, kq, cn * dq);    c = 1.
  *   P_chunk(S; k_1..C, v_1..C, a_1..C, b_1..C):
  *               D[s][s] = 1, D[t][s] = D[t-1][s] * a_t          (t > s)
  *               c[t][s] = D[t][s] * tree(k_s, k_t)              (s < t)
@@ -37,9 +45,9 @@
  *               S'_ij   = chain_{t=1..C} fma(e_t[i], k_t[j], .)
  *                         starting from D[C][0] * S_ij
  *   Composition: B_0 = state_in, B_{n+1} = P_chunk(B_n, chunk n); the
- *   outputs of chunk n come from P_tok steps started at B_n.  Decode runs
- *   P_tok on a running state R and, once C tokens are buffered, sets
- *   S_b = P_chunk(S_b, buffer), R = S_b.
+ *   outputs of chunk n come from P_tok steps started at (c = 1, Rt = B_n).
+ *   Decode runs P_tok on a running state (c, Rt) and, once C tokens are
+ *   buffered, sets S_b = P_chunk(S_b, buffer), Rt = S_b, c = 1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -60,22 +68,40 @@ static float tree32(const float* x, const float* y, int dk)
     return ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
 }
 
-/* One P_tok step on a d_v x d_k running state R (in place); writes o[d_v]. */
-static void p_tok(float* R, const float* k, const float* v, const float* q,
+/* The scale below which a decay is folded into the matrix (2^-64). */
+#define FOLD_TAU 0x1p-64f
+
+/* One P_tok step on a running state c * Rt (Rt d_v x d_k and *c updated in
+ * place); writes o[d_v]. */
+static void p_tok(float* R, float* c, const float* k, const float* v, const float* q,
                   float a, float b, int dk, int dv, float* o)
 {
+    const float kq = tree32(k, q, dk);
+    const float cn = a * *c;
+    const int fold = !(cn >= FOLD_TAU);
+    const float rc = fold ? 1.0f : 1.0f / cn;
     for (int i = 0; i < dv; ++i) {
         float* Ri = R + (int64_t)i * dk;
-        const float u = tree32(Ri, k, dk);
-        const float au = a * u;
-        const float r = v[i] - au;
+        const float dkv = tree32(Ri, k, dk);
+        const float dqv = tree32(Ri, q, dk);
+        const float cu = cn * dkv;
+        const float r = v[i] - cu;
         const float d = b * r;
-        for (int j = 0; j < dk; ++j) {
-            const float aR = a * Ri[j];
-            Ri[j] = fmaf(d, k[j], aR);
+        if (!fold) {
+            const float dt = d * rc;
+            const float t = fmaf(dt, kq, dqv);
+            o[i] = cn * t;
+            for (int j = 0; j < dk; ++j) Ri[j] = fmaf(dt, k[j], Ri[j]);
+        } else {
+            const float cdq = cn * dqv;
+            o[i] = fmaf(d, kq, cdq);
+            for (int j = 0; j < dk; ++j) {
+                const float cR = cn * Ri[j];
+                Ri[j] = fmaf(d, k[j], cR);
+            }
         }
-        o[i] = tree32(Ri, q, dk);
     }
+    *c = fold ? 1.0f : cn;
 }
 
 /*
@@ -160,14 +186,15 @@ void sched_f32_to_bf16(const float* x, uint16_t* y, int64_t n)
  * CPR forward (prefill / trainer forward) under the schedule.
  * Layouts as the fp64 oracle, in fp32.  Also fills the decode cache for a
  * continuation when the cache pointers are non-NULL: S_b, R [N,H,dv,dk],
- * kbuf [N,H,C,dk], vbuf [N,H,C,dv], abuf/bbuf [N,H,C], pos [N,H].
+ * kbuf [N,H,C,dk], vbuf [N,H,C,dv], abuf/bbuf [N,H,C], pos [N,H], and
+ * Rs_out [N,H] the running state's scale (the running state is Rs * R).
  */
 int sched_forward(const float* q, const float* k, const float* v,
                   const float* alpha, const float* beta, const float* state_in,
                   const int32_t* cu_seqlens, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C,
                   float* o, float* states,
                   float* S_b, float* R_out, float* kbuf, float* vbuf, float* abuf, float* bbuf,
-                  int32_t* pos)
+                  int32_t* pos, float* Rs_out)
 {
     if (N < 0 || H <= 0 || dk <= 0 || dk % NL || dv <= 0 || C <= 0) return 1;
     int64_t* soff = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N + 1));
@@ -192,12 +219,14 @@ int sched_forward(const float* q, const float* k, const float* v,
             memcpy(states + (slot * H + h) * SZ, B, sizeof(float) * (size_t)SZ);
             const int32_t t0 = cu_seqlens[n], L = cu_seqlens[n + 1] - t0;
             memcpy(R, B, sizeof(float) * (size_t)SZ);
+            float rs = 1.0f;
             for (int32_t c0 = 0; c0 < L; c0 += C) {
                 const int32_t len = (L - c0 < C) ? (L - c0) : C;
                 memcpy(R, B, sizeof(float) * (size_t)SZ);
+                rs = 1.0f;
                 for (int32_t t = 0; t < len; ++t) {
                     const int64_t tok = (int64_t)(t0 + c0 + t) * H + h;
-                    p_tok(R, k + tok * dk, v + tok * dv, q + tok * dk, alpha[tok], beta[tok],
+                    p_tok(R, &rs, k + tok * dk, v + tok * dv, q + tok * dk, alpha[tok], beta[tok],
                           dk, dv, o + tok * dv);
                 }
                 if (len == C) {
@@ -212,6 +241,7 @@ int sched_forward(const float* q, const float* k, const float* v,
             const int64_t nh = (int64_t)n * H + h;
             if (S_b) memcpy(S_b + nh * SZ, B, sizeof(float) * (size_t)SZ);
             if (R_out) memcpy(R_out + nh * SZ, p ? R : B, sizeof(float) * (size_t)SZ);
+            if (Rs_out) Rs_out[nh] = p ? rs : 1.0f;
             if (pos) pos[nh] = p;
             for (int32_t s = 0; s < p; ++s) {
                 const int64_t tok = (int64_t)(t0 + L - p + s) * H + h;
@@ -234,7 +264,7 @@ int sched_forward(const float* q, const float* k, const float* v,
 int sched_decode_step(const float* q, const float* k, const float* v,
                       const float* alpha, const float* beta,
                       float* S_b, float* R, float* kbuf, float* vbuf, float* abuf, float* bbuf,
-                      int32_t* pos, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C, float* o)
+                      int32_t* pos, float* Rs, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C, float* o)
 {
     if (N < 0 || H <= 0 || dk <= 0 || dk % NL || dv <= 0 || C <= 0) return 1;
     const int64_t SZ = (int64_t)dv * dk;
@@ -245,7 +275,7 @@ int sched_decode_step(const float* q, const float* k, const float* v,
             const int64_t nh = (int64_t)n * H + h;
             int32_t p = pos[nh];
             if (p < 0 || p >= C) { bad = 1; continue; }
-            p_tok(R + nh * SZ, k + nh * dk, v + nh * dv, q + nh * dk, alpha[nh], beta[nh],
+            p_tok(R + nh * SZ, Rs + nh, k + nh * dk, v + nh * dv, q + nh * dk, alpha[nh], beta[nh],
                   dk, dv, o + nh * dv);
             memcpy(kbuf + (nh * C + p) * dk, k + nh * dk, sizeof(float) * (size_t)dk);
             memcpy(vbuf + (nh * C + p) * dv, v + nh * dv, sizeof(float) * (size_t)dv);
@@ -256,6 +286,7 @@ int sched_decode_step(const float* q, const float* k, const float* v,
                 if (p_chunk(S_b + nh * SZ, kbuf + nh * C * dk, dk, vbuf + nh * C * dv, dv,
                             abuf + nh * C, bbuf + nh * C, 1, dk, dv, C)) { bad = 1; continue; }
                 memcpy(R + nh * SZ, S_b + nh * SZ, sizeof(float) * (size_t)SZ);
+                Rs[nh] = 1.0f;
                 p = 0;
             }
             pos[nh] = p;
@@ -267,14 +298,15 @@ int sched_decode_step(const float* q, const float* k, const float* v,
 /*
  * P_tok over every chunk, started from GIVEN boundary states (layout of the
  * forward's chunk_states).  o [T,H,dv] fp32 before the output cast; R_final
- * [N,H,dv,dk]: the running state after each sequence's last token (the
- * boundary state itself when L % C == 0).  This isolates the per-token
- * schedule from how the boundary states were produced.
+ * [N,H,dv,dk] and Rs_final [N,H]: the running state (Rs * R) after each
+ * sequence's last token (the boundary state itself, scale 1, when
+ * L % C == 0).  This isolates the per-token schedule from how the boundary
+ * states were produced.
  */
 int sched_tok_from_states(const float* q, const float* k, const float* v,
                           const float* alpha, const float* beta, const float* states,
                           const int32_t* cu_seqlens, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C,
-                          float* o, float* R_final)
+                          float* o, float* R_final, float* Rs_final)
 {
     if (N < 0 || H <= 0 || dk <= 0 || dk % NL || dv <= 0 || C <= 0) return 1;
     int64_t* soff = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N + 1));
@@ -294,21 +326,25 @@ int sched_tok_from_states(const float* q, const float* k, const float* v,
             if (!R) { bad = 1; continue; }
             const int32_t t0 = cu_seqlens[n], L = cu_seqlens[n + 1] - t0;
             memcpy(R, states + (soff[n] * H + h) * SZ, sizeof(float) * (size_t)SZ);
+            float rs = 1.0f;
             for (int32_t c0 = 0; c0 < L; c0 += C) {
                 memcpy(R, states + ((soff[n] + c0 / C) * H + h) * SZ, sizeof(float) * (size_t)SZ);
+                rs = 1.0f;
                 const int32_t len = (L - c0 < C) ? (L - c0) : C;
                 for (int32_t t = 0; t < len; ++t) {
                     const int64_t tok = (int64_t)(t0 + c0 + t) * H + h;
-                    p_tok(R, k + tok * dk, v + tok * dv, q + tok * dk, alpha[tok], beta[tok], dk, dv, o + tok * dv);
+                    p_tok(R, &rs, k + tok * dk, v + tok * dv, q + tok * dk, alpha[tok], beta[tok], dk, dv,
+                          o + tok * dv);
                 }
             }
+            const int64_t nh = (int64_t)n * H + h;
             if (R_final) {
-                const int64_t nh = (int64_t)n * H + h;
                 if (L % C == 0)
                     memcpy(R_final + nh * SZ, states + ((soff[n] + L / C) * H + h) * SZ, sizeof(float) * (size_t)SZ);
                 else
                     memcpy(R_final + nh * SZ, R, sizeof(float) * (size_t)SZ);
             }
+            if (Rs_final) Rs_final[nh] = (L % C == 0) ? 1.0f : rs;
             free(R);
         }
     }

@@ -33,7 +33,7 @@ def check_pair(d, o, st, n, h, C, state_base, bf16_out=True):
     assert np.max(np.abs(got_o - r["o"])) <= 2e-2 * np.max(np.abs(r["o"]))
     assert np.max(np.abs(got_s - r["states"])) <= 2e-2 * np.max(np.abs(r["states"]))
     # per-token schedule bit-exact against the fp32 model, started from the GPU's boundary states
-    mo, _ = oracle.schedule_tok_from_states(q, k, v, a, b, st[state_base:state_base + ns, h:h + 1].cpu().numpy(),
+    mo, _, _ = oracle.schedule_tok_from_states(q, k, v, a, b, st[state_base:state_base + ns, h:h + 1].cpu().numpy(),
                                             cu, C)
     if bf16_out:
         assert np.array_equal(bits(o[a0:a1, h:h + 1].contiguous()), oracle.to_bf16_bits(mo))

@@ -82,9 +82,10 @@ def test_forward_at_gate_extremes(d, C, dtype, lens):
     b = plant_extremes(synth.make_batch(1000 + d + C, lens, H, d, d, dtype), C, d * C)
     o, st, cache = forward(b, C, cache=True)
     st_h = st.cpu().numpy()
-    mo, mR = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st_h, b.cu_seqlens, C)
+    mo, mR, mRs = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st_h, b.cu_seqlens, C)
     assert np.array_equal(bits(o), bits(mo))
     assert np.array_equal(bits(cache["R"]), bits(mR))
+    assert np.array_equal(bits(cache["rscale"]), bits(mRs))
     r = oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)
     tol(dtype, o.cpu().numpy(), r["o"], "o")
     tol(dtype, st_h, r["states"], "states")
@@ -117,7 +118,7 @@ def test_decode_across_resyncs_at_gate_extremes(d, C, Lp, steps):
                                 cache, C, out_dtype=torch.float32)
         assert np.array_equal(bits(o), bits(fo[idx.cpu()])), s
     torch.cuda.synchronize()
-    for key in ("S_b", "R", "pos"):
+    for key in ("S_b", "R", "rscale", "pos"):
         assert torch.equal(cache[key], full_c[key]), key
     assert int(cache["status"].item()) == gdn.GDN_OK
     r = oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)

@@ -50,7 +50,7 @@ def test_tiny_workload_bitwise_prefill_vs_decode_and_oracle():
     b = synth.make_batch(cfg["seed"], [cfg["T"]] * cfg["B"], cfg["H"], cfg["dk"], cfg["dv"], cfg["dtype"])
     C = cfg["C"]
     o, st, _ = fwd(b, C)
-    mo, _ = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st.cpu().numpy(), b.cu_seqlens, C)
+    mo, _, _ = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st.cpu().numpy(), b.cu_seqlens, C)
     assert np.array_equal(bits(o), bits(mo))
     r = oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)
     tol_check("f32", o.cpu().numpy(), r["o"], "o")
@@ -64,6 +64,7 @@ def test_tiny_workload_bitwise_prefill_vs_decode_and_oracle():
     assert np.array_equal(bits(torch.cat(outs)), bits(o))
     assert np.array_equal(bits(cache["S_b"][0]), bits(st[-1]))
     assert np.array_equal(bits(cache["R"][0]), bits(st[-1]))
+    assert torch.all(cache["rscale"] == 1.0)
     assert int(cache["pos"].max()) == 0
 
 
@@ -82,9 +83,10 @@ def test_forward_vs_schedule_model_and_oracle(d, C, dtype):
     o, st, cache = fwd(b, C, torch.float32, torch.from_numpy(S0).to(DEV), cache=True)
     st_h = st.cpu().numpy()
     # P_tok bit for bit: the model's per-token schedule, started from the GPU's boundary states
-    mo, mR = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st_h, b.cu_seqlens, C)
+    mo, mR, mRs = oracle.schedule_tok_from_states(b.q, b.k, b.v, b.alpha, b.beta, st_h, b.cu_seqlens, C)
     assert np.array_equal(bits(o), bits(mo))
     assert np.array_equal(bits(cache["R"]), bits(mR))
+    assert np.array_equal(bits(cache["rscale"]), bits(mRs))
     # the first state of every sequence is state_in itself; S_b is the last boundary state
     first = np.concatenate([[0], np.cumsum([L // C + 1 for L in lens])])
     last = first[1:] - 1
@@ -131,7 +133,7 @@ def test_decode_equals_prefill_bitwise(d, C, Lp, steps):
                                 cache, C, out_dtype=torch.float32)
         assert np.array_equal(bits(o), bits(fo[idx.cpu()])), s
     torch.cuda.synchronize()
-    for key in ("S_b", "R", "pos"):
+    for key in ("S_b", "R", "rscale", "pos"):
         assert np.array_equal(bits(cache[key]) if key != "pos" else cache[key].cpu().numpy(),
                               bits(full_c[key]) if key != "pos" else full_c[key].cpu().numpy()), key
     p = int(full_c["pos"][0, 0])
@@ -179,10 +181,10 @@ def test_fused_chain_tok_path_equals_separate_kernels():
     ns = sum(L // C + 1 for L in lens)
     assert np.array_equal(bits(o), bits(o_big[:T]))
     assert np.array_equal(bits(st), bits(st_big[:ns]))
-    for key in ("S_b", "R", "pos"):
+    for key in ("S_b", "R", "rscale", "pos"):
         assert torch.equal(c[key], c_big[key][:len(lens)]), key
     # and the fused result is the model's P_tok from the GPU's states, bit for bit
-    mo, _ = oracle.schedule_tok_from_states(small.q, small.k, small.v, small.alpha, small.beta, st.cpu().numpy(),
+    mo, _, _ = oracle.schedule_tok_from_states(small.q, small.k, small.v, small.alpha, small.beta, st.cpu().numpy(),
                                             small.cu_seqlens, C)
     assert np.array_equal(bits(o), oracle.to_bf16_bits(mo))
 

@@ -42,9 +42,15 @@ def _as_frac(a):
     return [[Fraction(float(x)) for x in row] for row in a]
 
 
-@pytest.mark.parametrize("T,dk,dv,C,seed", [(5, 8, 3, 2, 0), (9, 16, 2, 4, 1), (7, 8, 4, 3, 2)])
-def test_c_model_equals_exact_rounding_replay(T, dk, dv, C, seed):
+@pytest.mark.parametrize("T,dk,dv,C,seed,folds", [(5, 8, 3, 2, 0, False), (9, 16, 2, 4, 1, False),
+                                                   (7, 8, 4, 3, 2, False), (9, 8, 3, 9, 3, True)])
+def test_c_model_equals_exact_rounding_replay(T, dk, dv, C, seed, folds):
     b = synth.make_batch(seed, [T], 1, dk, dv, "f32")
+    if folds:  # decays that push the running scale below 2^-64 (folds), and a reset
+        b.alpha[1, 0] = np.float32(2.0 ** -40)
+        b.alpha[2, 0] = np.float32(2.0 ** -30)   # scale 2^-70 -> fold
+        b.alpha[4, 0] = 0.0                      # reset -> fold
+        b.alpha[6, 0] = np.float32(3e-38)        # -> fold
     S0 = synth.bf16_values(np.random.default_rng(seed).standard_normal((1, 1, dv, dk)).astype(np.float32))
     m = oracle.schedule_forward(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C, S0)
     sch = exact.Fp32Schedule()
@@ -132,7 +138,7 @@ def test_prefill_equals_decode_bitwise(Lp, steps, C):
     for s in range(steps):
         idx = bat.cu_seqlens[:-1] + Lp + s
         assert np.array_equal(outs[s], full["o"][idx]), s
-    for key in ("S_b", "R", "pos", "kbuf", "vbuf", "abuf", "bbuf"):
+    for key in ("S_b", "R", "rscale", "pos", "kbuf", "vbuf", "abuf", "bbuf"):
         if key in ("kbuf", "vbuf", "abuf", "bbuf"):
             p = int(full["pos"][0, 0])
             assert np.array_equal(m[key][:, :, :p], full[key][:, :, :p]), key
@@ -150,12 +156,12 @@ def test_tok_from_states_reproduces_the_model_forward():
     C = 16
     bat = synth.make_batch(10, [40, 16, 5, 0, 33], 2, 16, 16, "bf16")
     m = oracle.schedule_forward(bat.q, bat.k, bat.v, bat.alpha, bat.beta, bat.cu_seqlens, C, with_cache=True)
-    o, Rf = oracle.schedule_tok_from_states(bat.q, bat.k, bat.v, bat.alpha, bat.beta, m["states"],
-                                            bat.cu_seqlens, C)
-    assert np.array_equal(o, m["o"]) and np.array_equal(Rf, m["R"])
+    o, Rf, Rs = oracle.schedule_tok_from_states(bat.q, bat.k, bat.v, bat.alpha, bat.beta, m["states"],
+                                                bat.cu_seqlens, C)
+    assert np.array_equal(o, m["o"]) and np.array_equal(Rf, m["R"]) and np.array_equal(Rs, m["rscale"])
     # and it really uses the states it is given: other states change the outputs
-    o2, _ = oracle.schedule_tok_from_states(bat.q, bat.k, bat.v, bat.alpha, bat.beta, m["states"] * 2,
-                                            bat.cu_seqlens, C)
+    o2, _, _ = oracle.schedule_tok_from_states(bat.q, bat.k, bat.v, bat.alpha, bat.beta, m["states"] * 2,
+                                               bat.cu_seqlens, C)
     assert not np.array_equal(o2, m["o"])
 
 
@@ -211,3 +217,34 @@ def test_perturbed_schedule_is_detected_but_within_tolerance():
     B = np.array([[float(x) for x in r] for r in o_b])
     assert not np.array_equal(A, B)
     assert np.max(np.abs(A - B)) <= 1e-5
+
+
+def test_scaled_state_folds_and_represents_the_state():
+    """The running state is c * R.  A decay that would take the scale below
+    2^-64 is folded into R (c returns to 1); alpha = 0 folds to an exact reset
+    (R = beta v k^T, the closed form); and c * R stays within fp32 rounding of
+    the plain recurrence's state in between."""
+    dk, dv, C = 16, 8, 64
+    b = synth.make_batch(21, [40], 1, dk, dv, "f32")
+    b.alpha[5:10, 0] = np.float32(2.0 ** -20)   # four of these reach 2^-80: one fold
+    b.alpha[20, 0] = 0.0                         # reset
+    m = oracle.schedule_forward(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C, with_cache=True)
+    R, Rs = m["R"][0, 0].astype(np.float64), float(m["rscale"][0, 0])
+    r = oracle.recurrent(b.q, b.k, b.v, b.alpha, b.beta, b.cu_seqlens, C)
+    # the running state after the last token (the 40 tokens are one partial chunk)
+    Sref = np.zeros((dv, dk))
+    for t in range(40):
+        k, v, a, bb = b.k[t, 0].astype(np.float64), b.v[t, 0].astype(np.float64), float(b.alpha[t, 0]), float(b.beta[t, 0])
+        Sref = a * (Sref - bb * np.outer(Sref @ k, k)) + bb * np.outer(v, k)
+    assert np.max(np.abs(Rs * R - Sref)) <= 1e-5 * max(1.0, np.max(np.abs(Sref)))
+    assert Rs <= 1.0 and Rs >= 2.0 ** -64
+    # the scale after the last token is the product of the decays since the last fold (the reset)
+    expect = np.float32(1.0)
+    for t in range(21, 40):
+        expect = np.float32(expect * b.alpha[t, 0])
+    assert np.float32(Rs) == expect
+    # the token after the reset sees only itself: o_20 = beta v (k . q) up to rounding
+    t = 20
+    o20 = float(b.beta[t, 0]) * b.v[t, 0].astype(np.float64) * float(b.k[t, 0].astype(np.float64) @ b.q[t, 0])
+    assert np.max(np.abs(m["o"][t, 0] - o20)) <= 1e-6
+    assert np.max(np.abs(m["o"] - r["o"])) <= 1e-5
