@@ -309,13 +309,12 @@ gdn_status_t launch_decode(const DecArgs& a)
             cudaSuccess ||
         per_sm <= 0)
         return GDN_ERR_CUDA;
-    const int64_t items = NH * DC::NT;
-    const unsigned tgrid = (unsigned)std::min<int64_t>(items, (int64_t)sms * per_sm);
+    const unsigned tgrid = (unsigned)std::min<int64_t>(NH, (int64_t)sms * per_sm);
     mark(a.events, 0, a.stream);
     gdn::k_dec_tok<D, D, C><<<tgrid, DC::THREADS, DC::SMEM, a.stream>>>(
         a.q, a.k, a.v, a.alpha, a.beta, a.in_bf16, a.out_bf16, c.R, c.rscale, c.kbuf, c.vbuf, c.abuf, c.bbuf,
         c.pos, a.o,
-        (int)items, c.status);
+        (int)NH, c.status);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
     constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
@@ -323,9 +322,25 @@ gdn_status_t launch_decode(const DecArgs& a)
     // persistent: one CTA per SM, and at most 1024 (sequence, head) pairs per CTA
     const int64_t min_grid = (NH + 1023) / 1024;
     const unsigned rgrid = (unsigned)std::max<int64_t>(std::min<int64_t>(NH, sms), min_grid);
-    gdn::k_dec_resync<D, D, C><<<rgrid, ChunkCfg<D, D, C>::THREADS, sm, a.stream>>>(
-        (int)NH, a.in_bf16, c.S_b, c.R, c.rscale, c.kbuf, c.vbuf, c.abuf, c.bbuf, c.pos, c.status);
-    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    // programmatic dependent launch: the resync grid is scheduled while the
+    // per-token step finishes and waits on the device (griddepcontrol.wait)
+    // for its results, which hides its launch latency on the many steps that
+    // have nothing to resync
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rgrid);
+    cfg.blockDim = dim3(ChunkCfg<D, D, C>::THREADS);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gdn::k_dec_resync<D, D, C>, (int)NH, a.in_bf16, c.S_b, c.R, c.rscale,
+                           (const void*)c.kbuf, (const void*)c.vbuf, (const float*)c.abuf, (const float*)c.bbuf,
+                           c.pos, c.status) != cudaSuccess ||
+        cudaGetLastError() != cudaSuccess)
+        return GDN_ERR_CUDA;
     mark(a.events, 2, a.stream);
     return GDN_OK;
 }
@@ -456,7 +471,7 @@ gdn_status_t launch_backward(const BwdArgs& a)
 
 extern "C" {
 
-const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v5/NL8/ptok-scaled/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3"; }
+const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v6/NL8/ptok-scaled/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3-1acc"; }
 
 const char* gdn_status_string(gdn_status_t s)
 {

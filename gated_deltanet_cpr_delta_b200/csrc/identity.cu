@@ -162,11 +162,12 @@ const char* kPolicy =
     "  row block r over K blocks 0..2r+1 ascending: bf16 inputs (V, K exact) lo.V + hi.V,\n"
     "  else (lo.hi + hi.lo) + hi.hi\n"
     "P_chunk part 2: tcgen05.mma kind::tf32, M = 128, A in tensor memory, B K-major in shared memory,\n"
-    "  fp32 accumulate, K blocks of 8 ascending, one accumulator per split product;\n"
-    "  E = (S_lo.w_hi + S_hi.w_lo) + S_hi.w_hi, with S_hi.[w_lo; w_hi] one instruction of N = 2C;\n"
+    "  fp32 accumulate, one accumulator per phase fed in this order: lo.hi over K blocks of 8 ascending,\n"
+    "  then hi.lo, then hi.hi;\n"
+    "  E = S_lo.w_hi ; S_hi.w_lo ; S_hi.w_hi (one accumulator);\n"
     "  e_t = D[C][t]*(u0_t - E);\n"
-    "  S' = ((D[C][0]*S + e_lo.k_hi) [+ e_hi.k_lo]) + e_hi.k_hi, the bracket absent for bf16 inputs and\n"
-    "  e_hi.[k_lo; k_hi] one instruction of N = 2 d_k otherwise\n"
+    "  P = e_lo.k_hi [; e_hi.k_lo] ; e_hi.k_hi (one accumulator), the bracket absent for bf16 inputs;\n"
+    "  S' = D[C][0]*S + P\n"
     "output store: fp32, or bf16 round to nearest even\n";
 
 int write_text(gdn_identity_kind_t kind, int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,

@@ -9,10 +9,12 @@ namespace gdn {
 // ------------------------------------------------------------------ decode
 // One decode token per (sequence, head): P_tok on the running state
 // rscale * R (the prefill's per-token step: tok_step_row), and the token
-// appended to the buffer at slot pos (pos and rscale themselves are advanced
-// by k_dec_resync, which runs next, so that every row tile of the pair reads
-// the same old scale).  Work item = (sequence-head, row tile).
-// Persistent: CTA b takes items b, b + grid, ...  Each item's state rows and
+// appended to the buffer at slot pos.  Work item = (sequence-head, row tile).
+// Persistent: CTA b takes the pairs b, b + grid, ..., each with all its row
+// tiles in a row, so that once its last tile is done the CTA advances the
+// pair's pos and rscale (every tile has read the old values by then).  A pair
+// whose buffer is now full gets pos = C: k_dec_resync, which runs next, does
+// its resync and sets pos = 0.  Each item's state rows and
 // raw token stream into shared memory by cp.async, DecCfg::S - 1 items ahead
 // of the one being computed, so several items' loads are in flight per CTA
 // without holding registers.  Each lane's slice of a row (EPT contiguous
@@ -38,8 +40,8 @@ template <int DK, int DV, int C>
 __global__ void __launch_bounds__(DecCfg<DK, DV>::THREADS)
 k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
           const float* __restrict__ alpha, const float* __restrict__ beta, int in_bf16, int out_bf16,
-          float* R, const float* rscale, void* kbuf, void* vbuf, float* abuf, float* bbuf, const int32_t* pos,
-          void* __restrict__ o, int nitems, int32_t* status)
+          float* R, float* rscale, void* kbuf, void* vbuf, float* abuf, float* bbuf, int32_t* pos,
+          void* __restrict__ o, int npairs, int32_t* status)
 {
     using Cf = DecCfg<DK, DV>;
     using RS = typename Cf::RS;
@@ -48,6 +50,9 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
     float* ks = sm + Cf::S * Cf::STAGE;
     float* qs = ks + RS::KS;
     float* vs = qs + RS::KS;
+    // the resync kernel that follows may be scheduled now; it waits for this
+    // grid's completion before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int t = threadIdx.x;
     const int row = t / RS::TPR, part = t % RS::TPR;
     const int esz = in_bf16 ? 2 : 4;
@@ -63,9 +68,11 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
     };
     auto raw = [&](int st) { return reinterpret_cast<unsigned char*>(sm + st * Cf::STAGE + Cf::RSTAGE); };
 
-    auto fetch = [&](int it, int st) {  // item it -> stage st; always commits a group
-        if (it < nitems) {
-            const int nh = it / Cf::NT, r = it % Cf::NT;
+    // this CTA's j-th item: pair blockIdx.x + (j / NT) * grid, row tile j % NT
+    auto item_pair = [&](int j) { return (int)blockIdx.x + (j / Cf::NT) * G; };
+    auto fetch = [&](int j, int st) {  // item j -> stage st; always commits a group
+        const int nh = item_pair(j), r = j % Cf::NT;
+        if (nh < npairs) {
             const float* src = R + ((int64_t)nh * DV + r * Cf::RT) * DK;
             for (int f = t; f < Cf::RT * CPR; f += Cf::THREADS) cp_async16(chunk_slot(st, f), src + 4 * f);
             unsigned char* rw = raw(st);
@@ -83,15 +90,14 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
         cp_async_commit();
     };
 
-    int it = blockIdx.x;
 #pragma unroll
-    for (int s = 0; s < Cf::S - 1; ++s) fetch(it + s * G, s);
-    for (int i = 0; it < nitems; ++i, it += G) {
-        const int st = i % Cf::S;
-        fetch(it + (Cf::S - 1) * G, (i + Cf::S - 1) % Cf::S);
+    for (int j = 0; j < Cf::S - 1; ++j) fetch(j, j);
+    for (int j = 0; item_pair(j) < npairs; ++j) {
+        const int st = j % Cf::S;
+        fetch(j + Cf::S - 1, (j + Cf::S - 1) % Cf::S);
         cp_async_wait_n<Cf::S - 1>();  // this item's copies (each thread's own) have landed
         __syncthreads();
-        const int nh = it / Cf::NT, r = it % Cf::NT;
+        const int nh = item_pair(j), r = j % Cf::NT;
         const unsigned char* rw = raw(st);
         const float* gates = reinterpret_cast<const float*>(rw + 16 * (2 * kp + vp));
         const float a = gates[0], b = gates[1], cs = gates[3];
@@ -113,10 +119,14 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
             if (t < 2 * kp) {
                 float* d = t < kp ? ks : qs;
                 const int j0 = (t < kp ? t : t - kp) * el;
-                for (int m = 0; m < el; ++m) d[RS::slot(j0 + m)] = x[m];
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    if (m < el) d[RS::slot(j0 + m)] = x[m];
             } else {
                 const int i0 = (t - 2 * kp) * el;
-                for (int m = 0; m < el; ++m) vs[i0 + m] = x[m];
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    if (m < el) vs[i0 + m] = x[m];
             }
             // append the raw token at slot p: k by tile 0, each tile its v rows
             if (p >= 0 && p < C) {
@@ -150,6 +160,15 @@ k_dec_tok(const void* __restrict__ q, const void* __restrict__ k, const void* __
             float* dst = R + ((int64_t)nh * DV + r * Cf::RT) * DK;
             for (int f = t; f < Cf::RT * CPR; f += Cf::THREADS)
                 *reinterpret_cast<float4*>(dst + 4 * f) = *reinterpret_cast<const float4*>(chunk_slot(st, f));
+            if (r == Cf::NT - 1 && t == 0) {  // the pair's last tile: advance pos and the scale
+                const float cn = fmul(a, cs);
+                if (p + 1 < C) {
+                    pos[nh] = p + 1;
+                    rscale[nh] = cn >= kFoldTau ? cn : 1.0f;
+                } else {
+                    pos[nh] = C;  // full buffer: the resync follows
+                }
+            }
         }
         __syncthreads();  // ks / qs / vs and this stage are free again
     }
@@ -181,13 +200,13 @@ struct ResyncSmem {
     static_assert(R1_OFF % 4 == 0 && US_OFF % 4 == 0 && KLO_OFF % 4 == 0 && BAR_OFF % 2 == 0, "alignment");
 };
 
-// Advances pos and the running scale after k_dec_tok appended a token at slot
-// pos (rscale <- alpha * rscale, or 1 where that product falls below the fold
-// threshold, as k_dec_tok computed it), and resyncs where the token completed a
-// chunk: S_b <- P_chunk(S_b, buffer), R <- S_b, rscale <- 1, pos <- 0.  P_chunk runs the same device functions as the prefill
+// Resyncs the pairs whose buffer k_dec_tok has just filled (pos == C):
+// S_b <- P_chunk(S_b, buffer), R <- S_b, rscale <- 1, pos <- 0.  A step with
+// no such pair costs one read of pos per pair.  P_chunk runs the same device functions as the prefill
 // (chunk_prep, then the tcgen05 boundary step).  Persistent: CTA b handles
-// (sequence, head) pairs b, b + grid, ...  A pos outside [0, C) is left
-// unchanged (k_dec_tok has recorded it).  If an MMA completion wait times
+// (sequence, head) pairs b, b + grid, ...  Other positions are left as they
+// are (k_dec_tok has advanced them, or recorded them as invalid).  If an MMA
+// completion wait times
 // out, the pairs this CTA had still to resync get pos = -1, are not written,
 // and GDN_ERR_TIMEOUT goes to *status (when non-null).
 template <int DK, int DV, int C>
@@ -210,21 +229,16 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
     uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Sm::BAR_OFF);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Sm::BAR_OFF + 2);
 
-    // this CTA's pairs are blockIdx.x + i*gridDim.x: read all their positions
-    // at once, advance the ones inside a chunk, and list the ones at a boundary
+    // launched programmatically after k_dec_tok: wait for that grid's results
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // this CTA's pairs are blockIdx.x + i*gridDim.x: list the ones k_dec_tok
+    // left at a full buffer (pos == C)
     __shared__ int todo[1024];
     __shared__ int ntodo;
     if (threadIdx.x == 0) ntodo = 0;
     __syncthreads();
     for (int nh = blockIdx.x + threadIdx.x * gridDim.x; nh < NH; nh += blockDim.x * gridDim.x) {
-        const int p = pos[nh];
-        if (p < 0 || p >= C) continue;          // invalid: left unchanged
-        if (p + 1 < C) {
-            pos[nh] = p + 1;
-            const float cn = fmul(abuf[(int64_t)nh * C + p], rscale[nh]);
-            rscale[nh] = cn >= kFoldTau ? cn : 1.0f;
-        } else {
-            rscale[nh] = 1.0f;
+        if (pos[nh] == C) {
             const int slot = atomicAdd(&ntodo, 1);
             if (slot < 1024) todo[slot] = nh;   // the host sizes the grid so that a CTA has <= 1024 pairs
         }
@@ -261,7 +275,10 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
         if (!tc_step<DK, DV, C>(SR, th, tbase, mbar, parity, Wlo, Klo, us, DV, dCs, in_bf16, Sg,
                                 R + (int64_t)nh * DV * DK))
             break;
-        if (threadIdx.x == 0) pos[nh] = 0;
+        if (threadIdx.x == 0) {
+            pos[nh] = 0;
+            rscale[nh] = 1.0f;
+        }
     }
     for (int r = it + threadIdx.x; r < nt; r += blockDim.x) pos[todo[r]] = -1;  // after a timeout
     if (it < nt && threadIdx.x == 0) record_error(status, GDN_ERR_TIMEOUT);

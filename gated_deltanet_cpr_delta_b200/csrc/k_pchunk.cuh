@@ -166,7 +166,7 @@ __device__ __forceinline__ void chain_run(const void* __restrict__ k, const floa
         }
         ok = tc_wait(mbar, parity);
         if (!ok) break;
-        tc_epilogue_S<DK, DV, C>(SR, th, d0, in_bf16, Klo);
+        tc_epilogue_S<DK, DV, C>(SR, th, d0, Klo);
     }
     if (ok && nfull > 0 && mover) {
         tc_store_rows<DK, DV>(Klo, state_dst(nfull), nullptr, pt, NP);

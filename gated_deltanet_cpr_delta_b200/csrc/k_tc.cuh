@@ -6,13 +6,13 @@
 //   phase 1   E = S w^T            A = S   (TMEM, hi/lo split), B = w   (smem)
 //   e_t[i]    = D[C][t] * (u0_t[i] - E[i][t])
 //   phase 2   P = e k              A = e   (TMEM, hi/lo split), B = k^T (smem)
-//   S'[i][j]  = ((D[C][0] * S[i][j] + P_lh) [+ P_hl]) + P_hh
-// Each fp32 operand x is split as hi = tf32_rna(x), lo = tf32_rna(x - hi), and
-// every split product (lo*hi, hi*lo, hi*hi) accumulates over the K blocks of 8
-// in ascending order in its own TMEM accumulator; the accumulators are summed in
-// the order written above.  k is exact in tf32 for bf16 inputs, so its lo
-// product is absent there.  The prefill chain and the decode resync call the
-// same device functions, so both give the same bits.
+//   S'[i][j]  = D[C][0] * S[i][j] + P[i][j]
+// Each fp32 operand x is split as hi = tf32_rna(x), lo = tf32_rna(x - hi).
+// A phase accumulates its split products in ONE TMEM accumulator, in this
+// order: lo*hi over the K blocks of 8 ascending, then hi*lo, then hi*hi.  k is
+// exact in tf32 for bf16 inputs, so its lo product is absent there.  The
+// epilogues then read one value per element.  The prefill chain and the decode
+// resync call the same device functions, so both give the same bits.
 //
 // Thread roles (256 threads): thread 0 issues the MMAs; in the epilogues warp w
 // reads TMEM lane quarter w % 4 (row i = 32 * (w % 4) + lane) and the half
@@ -97,28 +97,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* mbar)
                  : "memory");
 }
 
-// 8 consecutive TMEM columns of this thread's lane, for three column starts,
-// then wait for the loads (one asm block, so no use can move above the wait).
-__device__ __forceinline__ void tmem_ld8x3(uint32_t a0, uint32_t a1, uint32_t a2, float (&x)[8], float (&y)[8],
-                                           float (&z)[8])
+// 8 consecutive TMEM columns of this thread's lane, then wait for the load.
+__device__ __forceinline__ void tmem_ld8(uint32_t a0, float (&x)[8])
 {
-    uint32_t r[24];
+    uint32_t r[8];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%24];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%25];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16,%17,%18,%19,%20,%21,%22,%23}, [%26];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23])
-        : "r"(a0), "r"(a1), "r"(a2)
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(a0)
         : "memory");
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        x[m] = __uint_as_float(r[m]);
-        y[m] = __uint_as_float(r[8 + m]);
-        z[m] = __uint_as_float(r[16 + m]);
-    }
+    for (int m = 0; m < 8; ++m) x[m] = __uint_as_float(r[m]);
 }
 
 __device__ __forceinline__ void tmem_st8(uint32_t a, const uint32_t (&v)[8])
@@ -145,15 +135,14 @@ struct TcCfg {
     static_assert(DK % 16 == 0 && DK <= 128 && DV <= 128 && C % 16 == 0 && C <= 64, "tile shapes");
     static constexpr int THREADS = 256;
     static constexpr uint32_t TMEM_COLS = 512;
-    // TMEM columns.  Live ranges: S (phase 1 A) | D1 (phase 1 accumulators,
-    // read by the e epilogue) | e (phase 2 A) | D2 (phase 2 accumulators, read
-    // by the S' epilogue, which then writes S for the next chunk).  Products
-    // that share an operand are one MMA with the other operand stacked along N
-    // (w_lo above w_hi, k_lo above k_hi), so their accumulators are adjacent.
+    // TMEM columns.  Live ranges: S (phase 1 A) | D1 (phase 1 accumulator,
+    // read by the e epilogue) | e (phase 2 A) | D2 (phase 2 accumulator, read
+    // by the S' epilogue, which then writes S for the next chunk; D2 takes
+    // S_hi's columns, which phase 1 no longer needs).
     static constexpr uint32_t S_HI = 0, S_LO = 128;
-    static constexpr uint32_t D1_HL = 256, D1_HH = 256 + C, D1_LH = 384;   // S_hi w_lo | S_hi w_hi ; S_lo w_hi
-    static constexpr uint32_t E_HI = 448, E_LO = 0;
-    static constexpr uint32_t D2_LH = 64, D2_HL = 192, D2_HH = 192 + DK;   // e_lo k_hi ; e_hi k_lo | e_hi k_hi
+    static constexpr uint32_t D1 = 256;                  // C columns
+    static constexpr uint32_t E_HI = 320, E_LO = 384;    // C columns each
+    static constexpr uint32_t D2 = 0;                    // DK columns
     // smem operands (bytes): w [C rows][DK] and k^T [DK rows][C], K-major.
     static constexpr uint32_t LBO = 128;
     static constexpr uint32_t SBO_W = DK * 32;
@@ -167,7 +156,8 @@ struct TcCfg {
     {
         return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
     }
-    static constexpr uint32_t IDESC1 = idesc(C), IDESC1X2 = idesc(2 * C), IDESC2 = idesc(DK), IDESC2X2 = idesc(2 * DK);
+    static constexpr uint32_t IDESC1 = idesc(C), IDESC2 = idesc(DK);
+    static_assert(E_LO + C <= TMEM_COLS && D2 + DK <= S_LO, "TMEM column map");
 };
 
 // ------------------------------------------------------------- staging
@@ -274,9 +264,8 @@ __device__ __forceinline__ void tc_load_state(float (&SR)[DK / 2], const TcThrea
 // before tc_issue_phase2 the same holds for k^T (Khi/Klo).  The issuing
 // functions run on thread 0 only; the others run on every thread.
 
-// Phase 1: E = S w^T, three split products into their own accumulators.
-// Wlo and Whi are adjacent (Whi = Wlo + C * DK), so S_hi w_lo and S_hi w_hi
-// are one MMA of N = 2C.
+// Phase 1: E = S w^T, the three split products into one accumulator (Whi =
+// Wlo + C * DK).
 template <int DK, int DV, int C>
 __device__ __forceinline__ void tc_issue_phase1(uint32_t tbase, const float* Wlo, uint64_t* mbar)
 {
@@ -284,18 +273,22 @@ __device__ __forceinline__ void tc_issue_phase1(uint32_t tbase, const float* Wlo
     tc_fence_after();
     const uint32_t wl = smem_u32(Wlo), wh = wl + 4u * T::W_FLOATS;
 #pragma unroll 1
-    for (int kb = 0; kb < DK / 8; ++kb) {
-        const uint32_t acc = kb > 0;
-        mma_tf32_ts(tbase + T::D1_HL, tbase + T::S_HI + 8 * kb, smem_desc(wl + 256u * kb, T::LBO, T::SBO_W),
-                    T::IDESC1X2, acc);
-        mma_tf32_ts(tbase + T::D1_LH, tbase + T::S_LO + 8 * kb, smem_desc(wh + 256u * kb, T::LBO, T::SBO_W),
-                    T::IDESC1, acc);
-    }
+    for (int kb = 0; kb < DK / 8; ++kb)
+        mma_tf32_ts(tbase + T::D1, tbase + T::S_LO + 8 * kb, smem_desc(wh + 256u * kb, T::LBO, T::SBO_W), T::IDESC1,
+                    kb > 0);
+#pragma unroll 1
+    for (int kb = 0; kb < DK / 8; ++kb)
+        mma_tf32_ts(tbase + T::D1, tbase + T::S_HI + 8 * kb, smem_desc(wl + 256u * kb, T::LBO, T::SBO_W), T::IDESC1,
+                    1);
+#pragma unroll 1
+    for (int kb = 0; kb < DK / 8; ++kb)
+        mma_tf32_ts(tbase + T::D1, tbase + T::S_HI + 8 * kb, smem_desc(wh + 256u * kb, T::LBO, T::SBO_W), T::IDESC1,
+                    1);
     mma_commit(mbar);
 }
 
-// Phase 2: P = e k: e_lo k_hi, and e_hi k_hi (exact k) or e_hi [k_lo; k_hi]
-// as one MMA of N = 2 DK (Khi = Klo + K_FLOATS).
+// Phase 2: P = e k: e_lo k_hi, [e_hi k_lo,] e_hi k_hi into one accumulator
+// (Khi = Klo + K_FLOATS; k_lo only when k is not exact in tf32).
 template <int DK, int DV, int C>
 __device__ __forceinline__ void tc_issue_phase2(uint32_t tbase, const float* Klo, int k_exact, uint64_t* mbar)
 {
@@ -303,17 +296,19 @@ __device__ __forceinline__ void tc_issue_phase2(uint32_t tbase, const float* Klo
     tc_fence_after();
     const uint32_t kl = smem_u32(Klo), kh = kl + 4u * T::K_FLOATS;
 #pragma unroll 1
-    for (int kb = 0; kb < C / 8; ++kb) {
-        const uint32_t acc = kb > 0;
-        mma_tf32_ts(tbase + T::D2_LH, tbase + T::E_LO + 8 * kb, smem_desc(kh + 256u * kb, T::LBO, T::SBO_K),
-                    T::IDESC2, acc);
-        if (k_exact)
-            mma_tf32_ts(tbase + T::D2_HH, tbase + T::E_HI + 8 * kb, smem_desc(kh + 256u * kb, T::LBO, T::SBO_K),
-                        T::IDESC2, acc);
-        else
-            mma_tf32_ts(tbase + T::D2_HL, tbase + T::E_HI + 8 * kb, smem_desc(kl + 256u * kb, T::LBO, T::SBO_K),
-                        T::IDESC2X2, acc);
+    for (int kb = 0; kb < C / 8; ++kb)
+        mma_tf32_ts(tbase + T::D2, tbase + T::E_LO + 8 * kb, smem_desc(kh + 256u * kb, T::LBO, T::SBO_K), T::IDESC2,
+                    kb > 0);
+    if (!k_exact) {
+#pragma unroll 1
+        for (int kb = 0; kb < C / 8; ++kb)
+            mma_tf32_ts(tbase + T::D2, tbase + T::E_HI + 8 * kb, smem_desc(kl + 256u * kb, T::LBO, T::SBO_K),
+                        T::IDESC2, 1);
     }
+#pragma unroll 1
+    for (int kb = 0; kb < C / 8; ++kb)
+        mma_tf32_ts(tbase + T::D2, tbase + T::E_HI + 8 * kb, smem_desc(kh + 256u * kb, T::LBO, T::SBO_K), T::IDESC2,
+                    1);
     mma_commit(mbar);
 }
 
@@ -339,15 +334,13 @@ __device__ __forceinline__ float tc_epilogue_e(const TcThread<DK>& th, const flo
 #pragma unroll
     for (int c8 = 0; c8 < C / 16; ++c8) {
         const uint32_t col = t0 + 8 * c8;
-        float lh[8], hl[8], hh[8];
-        tmem_ld8x3(th.lane_base + T::D1_LH + col, th.lane_base + T::D1_HL + col, th.lane_base + T::D1_HH + col, lh,
-                   hl, hh);
+        float E[8];
+        tmem_ld8(th.lane_base + T::D1 + col, E);
         uint32_t eh[8], el[8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const int t = t0 + 8 * c8 + m;
-            const float E = fadd(fadd(lh[m], hl[m]), hh[m]);
-            const float e = th.row < DV ? fmul(dCs[t + 1], fsub(us[t * ldu + th.row], E)) : 0.f;
+            const float e = th.row < DV ? fmul(dCs[t + 1], fsub(us[t * ldu + th.row], E[m])) : 0.f;
             tf32_split(e, eh[m], el[m]);
         }
         tmem_st8(th.lane_base + T::E_HI + t0 + 8 * c8, eh);
@@ -360,29 +353,22 @@ __device__ __forceinline__ float tc_epilogue_e(const TcThread<DK>& th, const flo
     return d0;
 }
 
-// S' = ((d0 S + P_lh) [+ P_hl]) + P_hh on this thread's half row: into SR,
+// S' = d0 S + P on this thread's half row: into SR,
 // TMEM (as the next chunk's phase-1 operand) and the rows [DV][DK] at `stage`
 // (free smem; 16-byte chunks swizzled by row so that these row-per-thread
 // writes are conflict-free).  Ends with a barrier.
 template <int DK, int DV, int C>
-__device__ __forceinline__ void tc_epilogue_S(float (&SR)[DK / 2], const TcThread<DK>& th, float d0, int k_exact,
-                                              float* stage)
+__device__ __forceinline__ void tc_epilogue_S(float (&SR)[DK / 2], const TcThread<DK>& th, float d0, float* stage)
 {
     using T = TcCfg<DK, DV, C>;
     constexpr int NC = DK / 4, SW = (NC < 8 ? NC : 8) - 1;
     const int j0 = th.hf * (DK / 2);
 #pragma unroll
     for (int c8 = 0; c8 < DK / 16; ++c8) {
-        const uint32_t col = j0 + 8 * c8;
-        float lh[8], hl[8], hh[8];
-        tmem_ld8x3(th.lane_base + T::D2_LH + col, th.lane_base + T::D2_HL + col, th.lane_base + T::D2_HH + col, lh,
-                   hl, hh);
+        float P[8];
+        tmem_ld8(th.lane_base + T::D2 + j0 + 8 * c8, P);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            float x = fadd(fmul(d0, SR[8 * c8 + m]), lh[m]);
-            if (!k_exact) x = fadd(x, hl[m]);
-            SR[8 * c8 + m] = fadd(x, hh[m]);
-        }
+        for (int m = 0; m < 8; ++m) SR[8 * c8 + m] = fadd(fmul(d0, SR[8 * c8 + m]), P[m]);
     }
     if (th.row < DV) {
 #pragma unroll
@@ -429,7 +415,7 @@ __device__ __forceinline__ bool tc_step(float (&SR)[DK / 2], const TcThread<DK>&
     const float d0 = tc_epilogue_e<DK, DV, C>(th, us, ldu, dCs);
     if (threadIdx.x == 0) tc_issue_phase2<DK, DV, C>(tbase, Klo, k_exact, mbar);
     if (!tc_wait(mbar, parity)) return false;
-    tc_epilogue_S<DK, DV, C>(SR, th, d0, k_exact, Klo);
+    tc_epilogue_S<DK, DV, C>(SR, th, d0, Klo);
     tc_store_rows<DK, DV>(Klo, dst1, dst2, threadIdx.x, blockDim.x);
     __syncthreads();
     return true;
