@@ -87,20 +87,34 @@ def backward_flops(tokens_heads: int, dk: int, dv: int):
     return 22 * dk * dv * tokens_heads
 
 
+# Algorithmic work of k_bgrad per (chunk, head), the chunk form's dense
+# products (fma = 2 flops, one product per pair of matrices, before the 3xTF32
+# split): six d x d x C products (S0 w^T, S0 K^T, Y K^T, S0^T dO^T, S0^T Dd^T,
+# Y^T Delta^T) = 12 C d^2, and the C x C x d products ([K; Q] K^T 4, U 2, Dd 4,
+# [dO; Dd] Delta^T 4, dk 4, dq 2, and P_chunk part 1: Gram 1, u0 and w 2) =
+# 23 C^2 d.
+def bgrad_flops(chunks_heads: int, d: int, C: int):
+    return (12 * C * d * d + 23 * C * C * d) * chunks_heads
+
+
+# tf32 dense tensor-core peak from the measured (or fallback) bf16 peak and the
+# nominal tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s dense per GPU)
+TF32_PER_BF16 = 1.1 / 2.25
+
+
 # DRAM traffic per launch from ncu captures (dram__bytes_read.sum +
 # dram__bytes_write.sum), keyed by kernel and by the sha256 of the sources that
 # kernel is compiled from; a changed source drops the figure (reported null).
 NCU_TRAFFIC = {
     ("k_chain_tok", "5a5969a3fe1e58ea"): 789160960 + 329176320,
     ("k_dec_tok", "51b392a62fe51a33"): 135935744 + 77555200,
-    ("k_bwd_chunk", "86633ff16a2874d1"): 2963502592 + 4436340736,
 }
 
 KERNEL_SOURCES = {
     "k_tok": ("schedule.cuh", "k_ptok.cuh"),
     "k_chain_tok": ("schedule.cuh", "k_ptok.cuh", "k_tc.cuh", "k_pchunk.cuh"),
     "k_dec_tok": ("schedule.cuh", "k_ptok.cuh", "k_decode.cuh"),
-    "k_bwd_chunk": ("schedule.cuh", "k_ptok.cuh", "k_bwd.cuh"),
+    "k_bgrad": ("schedule.cuh", "k_ptok.cuh", "k_tc.cuh", "k_prep.cuh", "k_bgrad.cuh"),
 }
 
 
@@ -438,17 +452,20 @@ def bench_trainer(rank: int, world: int, warmup: int, steps: int, shape=None):
     bwd_ms = [e[0].elapsed_time(e[3]) for e in bev]
     tot = max_over_ranks(sum(f + b for f, b in zip(fwd_ms, bwd_ms)), world)
     kern = {n: sum(e[i].elapsed_time(e[i + 1]) for e in bev) / steps
-            for i, n in enumerate(("k_tables + k_bwd_scan", "k_bwd_chunk", "k_bwd_reduce"))}
-    fl = backward_flops(B * T * H, D, D)
-    tf = fl / (kern["k_bwd_chunk"] / 1e3) / 1e12
+            for i, n in enumerate(("k_tables + k_bwd_scan", "k_bprep", "k_bgrad"))}
+    chunks = B * ((T + C - 1) // C) * H
+    fl = bgrad_flops(chunks, D, C)
+    tf = fl / (kern["k_bgrad"] / 1e3) / 1e12
+    peaks, src = load_peaks()
+    tpk = peaks["bf16_tflops"] * TF32_PER_BF16
     return {"workload": Tr["name"], "value": B * T * world / (tot / steps / 1e3), "unit": UNIT,
             "ms_per_step": tot / steps, "fwd_ms": sum(fwd_ms) / steps, "bwd_ms": sum(bwd_ms) / steps,
             "bwd_kernels_ms": kern,
-            "roofline": {"kernel": "k_bwd_chunk (per-chunk backward)", "bound": "alu", "achieved": tf,
-                         "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": tf / FP32_PEAK_TFLOPS,
-                         "traffic": NCU_TRAFFIC.get(("k_bwd_chunk", kernel_source_sha("k_bwd_chunk"))),
+            "roofline": {"kernel": "k_bgrad (per-chunk gradients on tcgen05, 3xTF32)", "bound": "tensor",
+                         "achieved": tf, "peak": tpk, "unit": "TFLOP/s", "frac": tf / tpk,
+                         "traffic": NCU_TRAFFIC.get(("k_bgrad", kernel_source_sha("k_bgrad"))),
                          "flops_per_launch": fl,
-                         "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}}
+                         "peak_source": f"tf32 dense = bf16 dense ({src}) x 1.1/2.25 (nominal ratio)"}}
 
 
 def bench_varlen(rank: int, world: int, warmup: int, steps: int):

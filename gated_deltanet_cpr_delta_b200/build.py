@@ -22,7 +22,7 @@ PROBE_LIB = os.path.join(PKG, "libgdn_probe.so")
 PROBE_SOURCES = ["probe_fp32.cu"]
 SOURCES = ["gdn_cpr.cu", "identity.cu"]
 DEPS = ["gdn_cpr.cu", "identity.cu", "kernels.cuh", "schedule.cuh", "tma.cuh", "k_tables.cuh", "k_ptok.cuh",
-        "k_tc.cuh", "k_prep.cuh", "k_pchunk.cuh", "k_decode.cuh", "k_bwd.cuh"]
+        "k_tc.cuh", "k_prep.cuh", "k_pchunk.cuh", "k_decode.cuh", "k_bwd.cuh", "k_bgrad.cuh"]
 HEADERS = [os.path.join(ROOT, "include", "gdn_cpr.h")]
 
 

@@ -347,21 +347,20 @@ gdn_status_t launch_decode(const DecArgs& a)
 
 // Backward workspace: the forward's tables (err, cto, fco, so, ...), then the
 // boundary adjoints Y_c (one d_v x d_k state per chunk-state slot), the
-// checkpoints of the resident CTAs of k_bwd_chunk (at most kBwdMaxCtas), and
-// the per-row-tile partial sums of dq, dk (fp32 [NT][T][H][d_k]) and
-// dalpha, dbeta ([NT][T][H]).
-constexpr int64_t kBwdMaxCtas = 148 * 8;
+// chunk-local operands of every (chunk, head) task (k_bprep -> k_bgrad) and
+// the per-CTA scratch of k_bgrad (at most kBwdMaxCtas resident CTAs).
+constexpr int64_t kBwdMaxCtas = 148 * 4;
 
 struct BwdWorkspace {
     Workspace t;  // tables only
-    float *ybuf, *scratch, *pq, *pk, *pa, *pb;
+    float *ybuf, *prep, *scratch;
     size_t bytes;
 };
 
 BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, int32_t dv, int32_t C)
 {
     BwdWorkspace w{};
-    const int32_t RT = dv < 64 ? dv : 64, NT = dv / RT, SUB = C < 8 ? C : 8;  // as gdn::BwdCfg
+    (void)dk;
     const Workspace tables = carve(nullptr, 0, N, H, dk, dv, C);  // the tables part alone
     size_t off = tables.bytes;
     auto take = [&](size_t n) {
@@ -369,25 +368,19 @@ BwdWorkspace carve_bwd(void* base, int64_t T, int32_t N, int32_t H, int32_t dk, 
         off = align_up(off + n);
         return o;
     };
-    const int64_t max_states = T / C + N;           // >= sum_n (floor(L_n / C) + 1)
-    const int64_t ntasks = (T / C + N) * H * NT;    // >= chunk tasks x heads x row tiles
+    const int64_t max_states = T / C + N;   // >= sum_n (floor(L_n / C) + 1)
+    const int64_t ntasks = (T / C + N) * H;  // >= chunk tasks x heads
     const int64_t ctas = std::min<int64_t>(std::max<int64_t>(ntasks, 1), kBwdMaxCtas);
     const size_t o_y = take(sizeof(float) * (size_t)max_states * H * dv * dk);
-    const size_t o_sc = take(sizeof(float) * (size_t)ctas * (C / SUB) * RT * dk);
-    const size_t o_pq = take(sizeof(float) * (size_t)NT * T * H * dk);
-    const size_t o_pk = take(sizeof(float) * (size_t)NT * T * H * dk);
-    const size_t o_pa = take(sizeof(float) * (size_t)NT * T * H);
-    const size_t o_pb = take(sizeof(float) * (size_t)NT * T * H);
+    const size_t o_pw = take(sizeof(float) * (size_t)ntasks * (2 * C * dv + C * C + 8 * C));  // gdn::BgCfg::PW
+    const size_t o_sc = take(sizeof(float) * (size_t)ctas * 4 * C * dv);  // gdn::BgCfg::SCR (d_k = d_v)
     w.bytes = off;
     char* b = static_cast<char*>(base);
     if (b != nullptr) {
         w.t = carve(base, 0, N, H, dk, dv, C);
         w.ybuf = reinterpret_cast<float*>(b + o_y);
+        w.prep = reinterpret_cast<float*>(b + o_pw);
         w.scratch = reinterpret_cast<float*>(b + o_sc);
-        w.pq = reinterpret_cast<float*>(b + o_pq);
-        w.pk = reinterpret_cast<float*>(b + o_pk);
-        w.pa = reinterpret_cast<float*>(b + o_pa);
-        w.pb = reinterpret_cast<float*>(b + o_pb);
     }
     return w;
 }
@@ -409,7 +402,7 @@ struct BwdArgs {
 template <int D, int C>
 gdn_status_t launch_backward(const BwdArgs& a)
 {
-    using BC = gdn::BwdCfg<D, D, C>;
+    using BG = gdn::BgCfg<D, C>;
     using SC = gdn::ScanCfg<D, D, C>;
     mark(a.events, 0, a.stream);
     gdn::k_tables<<<1, 1024, 0, a.stream>>>(a.cu, a.N, C, a.T_total, a.tot.tasks, a.tot.full, a.tot.states,
@@ -422,28 +415,29 @@ gdn_status_t launch_backward(const BwdArgs& a)
         a.dstate);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
-    const int64_t ntasks = a.tot.tasks * a.H * BC::NT;
+    const int64_t ntasks = a.tot.tasks * a.H;
     if (ntasks > 0) {
-        if (set_smem(gdn::k_bwd_chunk<D, D, C>, BC::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
-        int dev = 0, sms = 0, occ = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gdn::k_bwd_chunk<D, D, C>, BC::THREADS, BC::SMEM) !=
-                cudaSuccess)
-            return GDN_ERR_CUDA;
-        const int64_t grid = std::min<int64_t>({ntasks, (int64_t)sms * std::max(occ, 1), kBwdMaxCtas});
-        gdn::k_bwd_chunk<D, D, C><<<(unsigned)grid, BC::THREADS, BC::SMEM, a.stream>>>(
-            a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.ws.ybuf, a.dstate_out, a.cu, a.ws.t.cto, a.ws.t.so,
-            a.ws.t.err, a.N,
-            a.H, a.T_total, ntasks, a.in_bf16, a.dv, a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.scratch);
+        const size_t psm = gdn::PrepCfg<D, D, C>::bytes(a.in_bf16);
+        if (set_smem(gdn::k_bprep<D, C>, psm) != cudaSuccess) return GDN_ERR_CUDA;
+        gdn::k_bprep<D, C><<<(unsigned)ntasks, 256, psm, a.stream>>>(a.k, a.v, a.alpha, a.beta, a.cu, a.ws.t.cto,
+                                                                     a.ws.t.err, a.N, a.H, a.in_bf16, a.ws.prep);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 2, a.stream);
-    const int64_t TH = a.T_total * a.H;
-    if (TH > 0) {
-        const unsigned grid = (unsigned)std::min<int64_t>((TH * (D + 1) + 255) / 256, 148 * 16);
-        gdn::k_bwd_reduce<D, BC::NT><<<grid, 256, 0, a.stream>>>(a.ws.pq, a.ws.pk, a.ws.pa, a.ws.pb, a.ws.t.err, TH,
-                                                               a.dq, a.dk, a.dalpha, a.dbeta);
+    if (ntasks > 0) {
+        if (set_smem(gdn::k_bgrad<D, C>, BG::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
+        int dev = 0, sms = 0, occ = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gdn::k_bgrad<D, C>, BG::THREADS, BG::SMEM) !=
+                cudaSuccess)
+            return GDN_ERR_CUDA;
+        // resident CTAs per SM: by shared memory and by tensor memory (512 columns per SM)
+        const int per_sm = std::max(1, std::min<int>(occ, 512 / (int)BG::TMEM_COLS));
+        const int64_t grid = std::min<int64_t>({ntasks, (int64_t)sms * per_sm, kBwdMaxCtas});
+        gdn::k_bgrad<D, C><<<(unsigned)grid, BG::THREADS, BG::SMEM, a.stream>>>(
+            a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.ws.ybuf, a.dstate_out, a.cu, a.ws.t.cto, a.ws.t.so,
+            a.ws.t.err, a.N, a.H, ntasks, a.in_bf16, a.ws.prep, a.dq, a.dk, a.dv, a.dalpha, a.dbeta, a.ws.scratch);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 3, a.stream);

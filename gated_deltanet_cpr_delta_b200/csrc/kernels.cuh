@@ -13,7 +13,7 @@
 //   k_tok       P_tok over every chunk in parallel -> o (and the running cache state)
 //   k_cache_fill decode cache for a continuation
 // Decode: k_dec_tok (P_tok + append), then k_dec_resync (P_chunk at a boundary).
-// Backward: k_bwd_scan (boundary adjoints, serial per sequence, head and row tile), k_bwd_chunk (per chunk), k_bwd_reduce.
+// Backward: k_bwd_scan (boundary adjoints, serial per sequence, head and row tile), k_bgrad (per chunk, tcgen05).
 #pragma once
 
 #include "k_tables.cuh"
@@ -22,3 +22,4 @@
 #include "k_pchunk.cuh"
 #include "k_decode.cuh"
 #include "k_bwd.cuh"
+#include "k_bgrad.cuh"
