@@ -425,19 +425,19 @@ gdn_status_t launch_backward(const BwdArgs& a)
     }
     mark(a.events, 2, a.stream);
     if (ntasks > 0) {
-        if (set_smem(gdn::k_bgrad<D, C>, BG::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
+        auto kern = a.in_bf16 ? gdn::k_bgrad<D, C, true> : gdn::k_bgrad<D, C, false>;
+        if (set_smem(kern, BG::SMEM) != cudaSuccess) return GDN_ERR_CUDA;
         int dev = 0, sms = 0, occ = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gdn::k_bgrad<D, C>, BG::THREADS, BG::SMEM) !=
-                cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, BG::THREADS, BG::SMEM) != cudaSuccess)
             return GDN_ERR_CUDA;
         // resident CTAs per SM: by shared memory and by tensor memory (512 columns per SM)
         const int per_sm = std::max(1, std::min<int>(occ, 512 / (int)BG::TMEM_COLS));
         const int64_t grid = std::min<int64_t>({ntasks, (int64_t)sms * per_sm, kBwdMaxCtas});
-        gdn::k_bgrad<D, C><<<(unsigned)grid, BG::THREADS, BG::SMEM, a.stream>>>(
+        kern<<<(unsigned)grid, BG::THREADS, BG::SMEM, a.stream>>>(
             a.q, a.k, a.v, a.alpha, a.beta, a.dO, a.states, a.ws.ybuf, a.dstate_out, a.cu, a.ws.t.cto, a.ws.t.so,
-            a.ws.t.err, a.N, a.H, ntasks, a.in_bf16, a.ws.prep, a.dq, a.dk, a.dv, a.dalpha, a.dbeta, a.ws.scratch);
+            a.ws.t.err, a.N, a.H, ntasks, a.ws.prep, a.dq, a.dk, a.dv, a.dalpha, a.dbeta, a.ws.scratch);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 3, a.stream);

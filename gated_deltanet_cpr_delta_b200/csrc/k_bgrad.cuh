@@ -47,7 +47,7 @@ namespace gdn {
 template <int D, int C>
 struct BgCfg {
     static_assert(D % 16 == 0 && D <= 128 && C % 16 == 0 && C <= 64, "tile shapes");
-    static constexpr int THREADS = 256;
+    static constexpr int THREADS = 512;
     static constexpr int BK = D > 2 * C ? D : 2 * C;  // widest K of a B operand
     static constexpr int ACOLS = 2 * BK;              // TMEM: A (hi | lo)
     static constexpr uint32_t S0C = ACOLS, S1C = ACOLS + C, S2C = ACOLS + 2 * C, S3C = ACOLS + 3 * C;  // accumulators
@@ -69,7 +69,7 @@ struct BgCfg {
     enum { VA, VB, VG, VGP, VDN, VAV, VBV, VCV, VDB, VDU, NV };
     static constexpr int V_OFF = KQ_OFF + MAT;
     static constexpr int P_OFF = V_OFF + NV * VS;  // [4 quantities][4 lane quarters][C]
-    static constexpr int YS_OFF = P_OFF + 16 * C;  // [8] warp partials of <Y, S0>, [8] the total
+    static constexpr int YS_OFF = P_OFF + 16 * C;  // [16] warp partials of <Y, S0>
     static constexpr int BAR_OFF = (YS_OFF + 16 + 3) / 4 * 4;
     static constexpr int FLOATS = BAR_OFF + 4;
     static constexpr size_t SMEM = sizeof(float) * (size_t)FLOATS;
@@ -100,26 +100,49 @@ __device__ __forceinline__ float bg_load1(const void* base, int64_t off, int bf1
                 : __ldg(reinterpret_cast<const float*>(base) + off);
 }
 
-// A operand rows in TMEM: this thread's lane row th.row, the half th.hf of the
-// K columns; f(m, k0, x) gives A[m][k0 .. k0+7].  hi goes to column chi + k,
-// lo (when lo_too) to clo + k.  Every value is fetched before the first store
-// (the stores are ordered with memory, so loads after one would wait for it).
-// Waits for its stores.
-template <int D, int K, typename F>
-__device__ __forceinline__ void bg_put_a(const TcThread<D>& th, uint32_t chi, uint32_t clo, bool lo_too, F f)
+// 512 threads: warp w reads and writes TMEM lane quarter q = w % 4 (rows
+// 32 q .. 32 q + 31, one per lane) and takes the 8-column groups g with
+// g % 4 == p = w / 4.
+constexpr int kBgThreads = 512, kBgParts = 4;
+
+struct BgThread {
+    int q, p, row;
+    uint32_t lane_base;  // TMEM address of this warp's lane quarter, column 0
+    __device__ explicit BgThread(uint32_t tbase)
+    {
+        const int w = threadIdx.x >> 5;
+        q = w & 3;
+        p = w >> 2;
+        row = 32 * q + (threadIdx.x & 31);
+        lane_base = tbase + ((uint32_t)(32 * q) << 16);
+    }
+};
+
+// A operand rows in TMEM, K columns: this thread's lane row th.row and its
+// column groups; f(m, k0, x) gives A[m][k0 .. k0+7].  hi goes to column
+// chi + k, lo (when lo_too(g) for the group g = k0 / 8) to clo + k.  Every
+// value is fetched before the first store (the stores are ordered with
+// memory, so a load after one would wait for it).  Waits for its stores.
+template <int K, typename L, typename F>
+__device__ __forceinline__ void bg_put_a(const BgThread& th, uint32_t chi, uint32_t clo, L lo_too, F f)
 {
-    constexpr int G = K / 16;  // groups of 8 columns per thread
-    float x[G][8];
+    constexpr int NG = K / 8, GPT = (NG + kBgParts - 1) / kBgParts;
+    float x[GPT][8];
 #pragma unroll
-    for (int c8 = 0; c8 < G; ++c8) f(th.row, th.hf * (K / 2) + 8 * c8, x[c8]);
+    for (int j = 0; j < GPT; ++j) {
+        const int g = th.p + kBgParts * j;
+        if (g < NG) f(th.row, 8 * g, x[j]);
+    }
 #pragma unroll
-    for (int c8 = 0; c8 < G; ++c8) {
-        const int k0 = th.hf * (K / 2) + 8 * c8;
-        uint32_t h[8], l[8];
+    for (int j = 0; j < GPT; ++j) {
+        const int g = th.p + kBgParts * j;
+        if (g < NG) {
+            uint32_t h[8], l[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) tf32_split(x[c8][m], h[m], l[m]);
-        tmem_st8(th.lane_base + chi + k0, h);
-        if (lo_too) tmem_st8(th.lane_base + clo + k0, l);
+            for (int m = 0; m < 8; ++m) tf32_split(x[j][m], h[m], l[m]);
+            tmem_st8(th.lane_base + chi + 8 * g, h);
+            if (lo_too(g)) tmem_st8(th.lane_base + clo + 8 * g, l);
+        }
     }
     tmem_wait_st();
 }
@@ -131,16 +154,16 @@ __device__ __forceinline__ void bg_put_a(const TcThread<D>& th, uint32_t chi, ui
 template <int N, int K, typename F>
 __device__ __forceinline__ void bg_put_b(float* bh, float* bl, F f)
 {
-    constexpr int KQ4 = K / 4, TOT = N * KQ4, IT = (TOT + 255) / 256;
+    constexpr int KQ4 = K / 4, TOT = N * KQ4, IT = (TOT + kBgThreads - 1) / kBgThreads;
     float4 x[IT];
 #pragma unroll
     for (int it = 0; it < IT; ++it) {
-        const int e = threadIdx.x + 256 * it;
+        const int e = threadIdx.x + kBgThreads * it;
         if (e < TOT) x[it] = f(((e >> 3) / KQ4) * 8 + (e & 7), (e >> 3) % KQ4);
     }
 #pragma unroll
     for (int it = 0; it < IT; ++it) {
-        const int e = threadIdx.x + 256 * it;
+        const int e = threadIdx.x + kBgThreads * it;
         if (e < TOT) {
             const int r8 = e & 7, c4 = (e >> 3) % KQ4, rg = (e >> 3) / KQ4;
             uint32_t h[4], l[4];
@@ -265,19 +288,21 @@ k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __r
     }
 }
 
-// The per-chunk gradients of every (chunk, head) task; persistent.
-template <int D, int C>
-__global__ void __launch_bounds__(256, 1)
+// The per-chunk gradients of every (chunk, head) task; persistent.  BF16:
+// the inputs are bf16 (else fp32), fixed at compile time so that no load
+// carries a dtype branch.
+template <int D, int C, bool BF16>
+__global__ void __launch_bounds__(kBgThreads, 1)
 k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
         const float* __restrict__ alpha, const float* __restrict__ beta, const void* __restrict__ dO,
         const float* __restrict__ states, const float* __restrict__ ybuf, const float* __restrict__ dstate_out,
         const int32_t* __restrict__ cu, const int32_t* __restrict__ cto, const int32_t* __restrict__ so,
-        int32_t* err, int N, int H, int64_t ntasks, int in_bf16, const float* __restrict__ pw,
+        int32_t* err, int N, int H, int64_t ntasks, const float* __restrict__ pw,
         float* __restrict__ dq, float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dalpha,
         float* __restrict__ dbeta, float* __restrict__ scratch)
 {
     using Cf = BgCfg<D, C>;
-    constexpr int LD = Cf::LD, BK = Cf::BK, H2 = C / 2;
+    constexpr int LD = Cf::LD, BK = Cf::BK, NG = C / 8;
     if (*reinterpret_cast<volatile const int32_t*>(err)) return;
     extern __shared__ float4 smem_f4[];
     float* sm = reinterpret_cast<float*>(smem_f4);
@@ -285,9 +310,9 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
     float* Bl = Bh + C * BK;
     float* DOD = sm + Cf::DOD_OFF;  // DOD[t][r] = dO_t . Delta_r
     float* DDD = sm + Cf::DDD_OFF;  // DDD[t][r] = Dd_t . Delta_r
-    float* N1 = sm + Cf::N1_OFF;    // N1 = T^T M
-    float* FF = sm + Cf::F_OFF;     // F[r][t] of psi
-    float* Ts = sm + Cf::T_OFF;     // T
+    float* N1 = sm + Cf::N1_OFF;    // N1 = T^T M, later Ediff
+    float* FF = sm + Cf::F_OFF;     // M, later F
+    float* Ts = sm + Cf::T_OFF;     // T, later E2b
     float* DM = sm + Cf::DM_OFF;    // D[t][s]
     float* KK = sm + Cf::KK_OFF;    // k_t . k_s
     float* KQ = sm + Cf::KQ_OFF;    // k_t . q_s
@@ -306,13 +331,17 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tslot;
-    const TcThread<D> th(tbase);
+    const BgThread th(tbase);
     uint32_t parity = 0;
     float* gD = scratch + (int64_t)blockIdx.x * Cf::SCR;  // Delta [C][D]
     float* gKS = gD + C * D;                               // KS[t][i] = (S0 k_t)_i
     float* gKY = gKS + C * D;                              // dn_t (Y k_t)_i
     float* gDd = gKY + C * D;                              // Dd [C][D]
     const uint32_t a_hi = tbase, a_lo_D = tbase + D, a_lo_2C = tbase + 2 * C, a_lo_C = tbase + C;
+    constexpr int in_bf16 = BF16 ? 1 : 0;
+    constexpr bool ex = BF16;  // k, q, v, dO exact in tf32
+    auto all_lo = [](int) { return true; };
+    auto no_lo_if_exact = [&](int) { return !ex; };
     bool ok = true;
 
     // sync, issue (thread 0) and wait for the MMAs; false after a timeout
@@ -327,18 +356,17 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         }
         return tc_wait(mbar, parity);
     };
-    // per-column sums over the 128 lanes, for the quantity slot qn: each
-    // thread passes its 8 values of columns hf*C/2 + 8 cb ..; after the
-    // barrier of finish_sums, out[t] = ((p0 + p1) + p2) + p3 over the four
-    // lane quarters
-    auto col_sum8 = [&](int qn, int cb, float (&x)[8]) {
+    // per-column sums over the 128 lanes for the quantity slot qn: a warp
+    // passes the 8 values of its column group g; after a barrier,
+    // finish_sums gives out[t] = ((p0 + p1) + p2) + p3 over the lane quarters
+    auto col_sum8 = [&](int qn, int g, float (&x)[8]) {
         const float s = bg_warp_sum8(x);
-        if ((lane & 3) == 0) part[(qn * 4 + th.q) * C + th.hf * H2 + 8 * cb + (lane >> 2)] = s;
+        if ((lane & 3) == 0) part[(qn * 4 + th.q) * C + 8 * g + (lane >> 2)] = s;
     };
     auto finish_sums = [&](int qn, float* out) {
         for (int t = tid; t < C; t += blockDim.x) {
-            const float* p = part + qn * 4 * C + t;
-            out[t] = ((p[0] + p[C]) + p[2 * C]) + p[3 * C];
+            const float* pp = part + qn * 4 * C + t;
+            out[t] = ((pp[0] + pp[C]) + pp[2 * C]) + pp[3 * C];
         }
     };
 
@@ -353,7 +381,10 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         const int nchunks = (Ln + C - 1) / C;
         const int len = min(C, Ln - c * C);
         const int64_t tok0 = (int64_t)seq0 + (int64_t)c * C;
-        auto trow = [&](int t) { return (tok0 + t) * H + h; };  // token row of [T, H, .] tensors
+        const int64_t tb = (tok0 * H + h) * D;  // element offset of the chunk's first token row
+        const int RS = H * D;                    // token row stride (elements)
+        auto tok1 = [&](const void* base, int t, int i) { return bg_load1(base, tb + (t * RS + i), in_bf16); };
+        auto trow = [&](int t) { return (tok0 + t) * H + h; };  // row of [T, H] gates
         const float* S0 = states + ((slot0 + c) * H + h) * (int64_t)D * D;
         const float* Y = c + 1 < nchunks ? ybuf + ((slot0 + c + 1) * H + h) * (int64_t)D * D
                                          : (dstate_out != nullptr ? dstate_out + ((int64_t)n * H + h) * D * D
@@ -366,7 +397,15 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         {
             const float* pT = pwt + 2 * C * D;
             const float* pv = pT + C * C;
-            for (int e = tid; e < C * C; e += blockDim.x) Ts[(e / C) * LD + e % C] = pT[e];
+            constexpr int TI = (C * C + kBgThreads - 1) / kBgThreads;
+            float tv[TI];  // every value fetched before the first store
+#pragma unroll
+            for (int j = 0; j < TI; ++j) tv[j] = tid + j * kBgThreads < C * C ? pT[tid + j * kBgThreads] : 0.f;
+#pragma unroll
+            for (int j = 0; j < TI; ++j) {
+                const int e = tid + j * kBgThreads;
+                if (e < C * C) Ts[(e / C) * LD + e % C] = tv[j];
+            }
             for (int t = tid; t < C; t += blockDim.x) {
                 va[t] = pv[t];
                 vb[t] = pv[C + t];
@@ -386,11 +425,11 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             }
         }
 
-        // ---- E = S0 w^T (A = S0)
-        bg_put_a<D, D>(th, a_hi, a_lo_D, true, [&](int m, int k0, float (&x)[8]) {
+        // ---- E = S0 w^T (A = S0), then KS = S0 K^T (B = K)
+        bg_put_a<D>(th, a_hi, a_lo_D, all_lo, [&](int m, int k0, float (&x)[8]) {
             if (m < D) {
-                const float4 x0 = __ldg(reinterpret_cast<const float4*>(S0 + (int64_t)m * D + k0));
-                const float4 x1 = __ldg(reinterpret_cast<const float4*>(S0 + (int64_t)m * D + k0 + 4));
+                const float4 x0 = __ldg(reinterpret_cast<const float4*>(S0 + m * D + k0));
+                const float4 x1 = __ldg(reinterpret_cast<const float4*>(S0 + m * D + k0 + 4));
                 x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w;
                 x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
             } else {
@@ -404,26 +443,25 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                   bg_mma(tbase + Cf::S1C, a_hi, a_lo_D, false, Bh, Bl, false, D * 32, 0, D / 8, Cf::IDESC, acc);
               })))
             break;
-        // ---- KS = S0 K^T (same A), then KY = Y K^T, then [K; Q] K^T: B = K
-        const bool ex = in_bf16 != 0;
         bg_put_b<C, D>(Bh, ex ? nullptr : Bl, [&](int r, int c4) {
-            return r < len ? bg_load4(k, trow(r) * D + 4 * c4, in_bf16) : make_float4(0.f, 0.f, 0.f, 0.f);
+            return r < len ? bg_load4(k, tb + (r * RS + 4 * c4), in_bf16) : make_float4(0.f, 0.f, 0.f, 0.f);
         });
         if (!(ok = run([&] {
                   uint32_t acc = 0;
                   bg_mma(tbase + Cf::S2C, a_hi, a_lo_D, false, Bh, Bl, ex, D * 32, 0, D / 8, Cf::IDESC, acc);
               })))
             break;
+        // ---- KY = Y K^T (A = Y; <Y, S0> on the way), then [K; Q] K^T (same B)
         {
             float ys = 0.f;
-            bg_put_a<D, D>(th, a_hi, a_lo_D, true, [&](int m, int k0, float (&x)[8]) {
+            bg_put_a<D>(th, a_hi, a_lo_D, all_lo, [&](int m, int k0, float (&x)[8]) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) x[j] = 0.f;
                 if (m < D && Y != nullptr) {
-                    const float4 y0 = __ldg(reinterpret_cast<const float4*>(Y + (int64_t)m * D + k0));
-                    const float4 y1 = __ldg(reinterpret_cast<const float4*>(Y + (int64_t)m * D + k0 + 4));
-                    const float4 s0 = __ldg(reinterpret_cast<const float4*>(S0 + (int64_t)m * D + k0));
-                    const float4 s1 = __ldg(reinterpret_cast<const float4*>(S0 + (int64_t)m * D + k0 + 4));
+                    const float4 y0 = __ldg(reinterpret_cast<const float4*>(Y + m * D + k0));
+                    const float4 y1 = __ldg(reinterpret_cast<const float4*>(Y + m * D + k0 + 4));
+                    const float4 s0 = __ldg(reinterpret_cast<const float4*>(S0 + m * D + k0));
+                    const float4 s1 = __ldg(reinterpret_cast<const float4*>(S0 + m * D + k0 + 4));
                     x[0] = y0.x; x[1] = y0.y; x[2] = y0.z; x[3] = y0.w;
                     x[4] = y1.x; x[5] = y1.y; x[6] = y1.z; x[7] = y1.w;
                     ys += ((y0.x * s0.x + y0.y * s0.y) + (y0.z * s0.z + y0.w * s0.w)) +
@@ -439,10 +477,10 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                   bg_mma(tbase + Cf::S3C, a_hi, a_lo_D, false, Bh, Bl, ex, D * 32, 0, D / 8, Cf::IDESC, acc);
               })))
             break;
-        bg_put_a<D, D>(th, a_hi, a_lo_D, !ex, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<D>(th, a_hi, a_lo_D, no_lo_if_exact, [&](int m, int k0, float (&x)[8]) {
             const int t = m % C;
             if (m < 2 * C && t < len) {
-                load8(m < C ? k : q, trow(t) * D + k0, in_bf16, x);
+                load8(m < C ? k : q, tb + (t * RS + k0), in_bf16, x);
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) x[j] = 0.f;
@@ -454,12 +492,14 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
               })))
             break;
 
-        // ---- epilogue: KK, KQ; Delta, KS, dn KY to the scratch; cv
-        const float ysum = ((ysp[0] + ysp[1]) + (ysp[2] + ysp[3])) + ((ysp[4] + ysp[5]) + (ysp[6] + ysp[7]));
+        // ---- epilogue: KK, KQ; Delta, KS, dn KY to the scratch; cv_t = Delta_t . (Y k_t)
+        float ysum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kBgThreads / 32; ++w) ysum += ysp[w];
         {
             const int m = th.row, i = th.row;
-            for (int cb = 0; cb < C / 16; ++cb) {
-                const int t0 = th.hf * H2 + 8 * cb;
+            for (int g = th.p; g < NG; g += kBgParts) {
+                const int t0 = 8 * g;
                 float x[8], E[8], KS[8], KY[8], u0r[8];  // global values fetched first, all in flight
 #pragma unroll
                 for (int j = 0; j < 8; ++j) u0r[j] = i < D ? gU[(t0 + j) * D + i] : 0.f;
@@ -485,41 +525,66 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                         cv[j] = dl * KY[j];
                     }
                 }
-                col_sum8(0, cb, cv);
+                col_sum8(0, g, cv);
             }
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         finish_sums(0, vcv);
-        // N1[t][u] = sum_{t <= s <= u} T[s][t] D[u][s] KQ[s][u]  (T^T M, upper triangle)
+        // M[s][u] = D[u][s] KQ[s][u] (u >= s) into FF, then N1 = T^T M (upper
+        // triangle), 2 x 4 outputs per thread, s over T's and M's nonzeros
         for (int e = tid; e < C * C; e += blockDim.x) {
-            const int t = e / C, u = e % C;
-            float acc = 0.f;
-            for (int s = t; s <= u; ++s) acc = fmaf(Ts[s * LD + t], DM[u * LD + s] * KQ[s * LD + u], acc);
-            N1[t * LD + u] = acc;
+            const int s_ = e / C, u = e % C;
+            FF[s_ * LD + u] = u >= s_ ? DM[u * LD + s_] * KQ[s_ * LD + u] : 0.f;
+        }
+        __syncthreads();
+        if (tid < C * C / 8) {
+            const int t0 = 2 * (tid / (C / 4)), u0 = 4 * (tid % (C / 4));
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            const int s1 = min(C - 1, u0 + 3);
+            for (int s_ = t0; s_ <= s1; ++s_) {
+                const float a0 = Ts[s_ * LD + t0], a1 = Ts[s_ * LD + t0 + 1];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float bm = FF[s_ * LD + u0 + j];
+                    acc[0][j] = fmaf(a0, bm, acc[0][j]);
+                    acc[1][j] = fmaf(a1, bm, acc[1][j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                N1[t0 * LD + u0 + j] = acc[0][j];
+                N1[(t0 + 1) * LD + u0 + j] = acc[1][j];
+            }
         }
 
         // ---- U^T = gp KS^T + Delta^T Xu^T, Xu[t][r] = D[t-1][r] KK[r][t] (r < t)
-        bg_put_a<D, C>(th, a_hi, a_lo_C, true, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<C>(th, a_hi, a_lo_C, all_lo, [&](int m, int k0, float (&x)[8]) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) x[j] = m < D ? gD[(k0 + j) * D + m] : 0.f;
         });
         {  // accumulator S0C starts as gp_t KS[i][t]; every value fetched before the first store
-            float x[C / 16][8];
+            constexpr int GPT = (NG + kBgParts - 1) / kBgParts;
+            float x[GPT][8];
 #pragma unroll
-            for (int cb = 0; cb < C / 16; ++cb)
+            for (int jg = 0; jg < GPT; ++jg) {
+                const int g = th.p + kBgParts * jg;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int t = th.hf * H2 + 8 * cb + j;
-                    x[cb][j] = th.row < D ? vgp[t] * gKS[t * D + th.row] : 0.f;
+                    const int t = 8 * g + j;
+                    x[jg][j] = (g < NG && th.row < D) ? vgp[t] * gKS[t * D + th.row] : 0.f;
                 }
+            }
 #pragma unroll
-            for (int cb = 0; cb < C / 16; ++cb) {
-                uint32_t u[8];
+            for (int jg = 0; jg < GPT; ++jg) {
+                const int g = th.p + kBgParts * jg;
+                if (g < NG) {
+                    uint32_t u[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) u[j] = __float_as_uint(x[cb][j]);
-                tmem_st8(th.lane_base + Cf::S0C + th.hf * H2 + 8 * cb, u);
+                    for (int j = 0; j < 8; ++j) u[j] = __float_as_uint(x[jg][j]);
+                    tmem_st8(th.lane_base + Cf::S0C + 8 * g, u);
+                }
             }
             tmem_wait_st();
         }
@@ -539,23 +604,24 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             break;
 
         // ---- Dd^T = [dn KY^T | dO^T] [T^T | N1]^T: K = 2C, A lo at column 2C
-        bg_put_a<D, 2*C>(th, a_hi, a_lo_2C, th.hf == 0 || !ex, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<2 * C>(th, a_hi, a_lo_2C, [&](int g) { return g < C / 8 || !ex; },
+                        [&](int m, int k0, float (&x)[8]) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int s = k0 + j;
-                x[j] = 0.f;
-                if (m < D) {
-                    if (s < C) x[j] = gKY[s * D + m];
-                    else if (s - C < len) x[j] = bg_load1(dO, trow(s - C) * D + m, in_bf16);
-                }
-            }
-        });
-        bg_put_b<C, 2*C>(Bh, Bl, [&](int t, int c4) {
+                            for (int j = 0; j < 8; ++j) {
+                                const int s_ = k0 + j;
+                                x[j] = 0.f;
+                                if (m < D) {
+                                    if (s_ < C) x[j] = gKY[s_ * D + m];
+                                    else if (s_ - C < len) x[j] = tok1(dO, s_ - C, m);
+                                }
+                            }
+                        });
+        bg_put_b<C, 2 * C>(Bh, Bl, [&](int t, int c4) {
             float x[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int s = 4 * c4 + j;
-                x[j] = s < C ? Ts[s * LD + t] : N1[t * LD + s - C];
+                const int s_ = 4 * c4 + j;
+                x[j] = s_ < C ? Ts[s_ * LD + t] : N1[t * LD + s_ - C];
             }
             return make_float4(x[0], x[1], x[2], x[3]);
         });
@@ -571,13 +637,13 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         // ---- epilogue: dv, Dd to the scratch; sums for dbeta, Dd.U, bv
         {
             const int i = th.row;
-            for (int cb = 0; cb < C / 16; ++cb) {
-                const int t0 = th.hf * H2 + 8 * cb;
+            for (int g = th.p; g < NG; g += kBgParts) {
+                const int t0 = 8 * g;
                 float U[8], Dd[8], pdb[8], pdu[8], pbv[8], vr[8], ksr[8];  // global values fetched first
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int t = t0 + j;
-                    vr[j] = (i < D && t < len) ? bg_load1(v, trow(t) * D + i, in_bf16) : 0.f;
+                    vr[j] = (i < D && t < len) ? tok1(v, t, i) : 0.f;
                     ksr[j] = i < D ? gKS[t * D + i] : 0.f;
                 }
                 tmem_ld8(th.lane_base + Cf::S0C + t0, U);
@@ -589,16 +655,16 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                     if (i < D) {
                         gDd[t * D + i] = Dd[j];
                         if (t < len) {
-                            dv[trow(t) * D + i] = vb[t] * Dd[j];
+                            dv[tb + (t * RS + i)] = vb[t] * Dd[j];
                             pdb[j] = Dd[j] * (vr[j] - va[t] * U[j]);
                         }
                         pdu[j] = Dd[j] * U[j];
                         pbv[j] = Dd[j] * ksr[j];
                     }
                 }
-                col_sum8(1, cb, pdb);
-                col_sum8(2, cb, pdu);
-                col_sum8(3, cb, pbv);
+                col_sum8(1, g, pdb);
+                col_sum8(2, g, pdu);
+                col_sum8(3, g, pbv);
             }
         }
         tc_fence_before();
@@ -609,12 +675,12 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         finish_sums(3, vbv);
 
         // ---- q1 = S0^T dO^T (A = S0^T), then av and the dq accumulator g q1
-        bg_put_a<D, D>(th, a_hi, a_lo_D, true, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<D>(th, a_hi, a_lo_D, all_lo, [&](int m, int k0, float (&x)[8]) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = m < D ? __ldg(S0 + (int64_t)(k0 + j) * D + m) : 0.f;
+            for (int j = 0; j < 8; ++j) x[j] = m < D ? __ldg(S0 + (k0 + j) * D + m) : 0.f;
         });
         bg_put_b<C, D>(Bh, ex ? nullptr : Bl, [&](int r, int c4) {
-            return r < len ? bg_load4(dO, trow(r) * D + 4 * c4, in_bf16) : make_float4(0.f, 0.f, 0.f, 0.f);
+            return r < len ? bg_load4(dO, tb + (r * RS + 4 * c4), in_bf16) : make_float4(0.f, 0.f, 0.f, 0.f);
         });
         if (!(ok = run([&] {
                   uint32_t acc = 0;
@@ -623,24 +689,20 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             break;
         {
             const int j = th.row;
-            for (int cb = 0; cb < C / 16; ++cb) {
-                const int t0 = th.hf * H2 + 8 * cb;
+            for (int g = th.p; g < NG; g += kBgParts) {
+                const int t0 = 8 * g;
                 float q1[8], pav[8], qr[8];  // global values fetched first
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t = t0 + e;
-                    qr[e] = (j < D && t < len) ? bg_load1(q, trow(t) * D + j, in_bf16) : 0.f;
-                }
                 uint32_t sc[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qr[e] = (j < D && t0 + e < len) ? tok1(q, t0 + e, j) : 0.f;
                 tmem_ld8(th.lane_base + Cf::S2C + t0, q1);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int t = t0 + e;
                     pav[e] = q1[e] * qr[e];
-                    sc[e] = __float_as_uint(vg[t] * q1[e]);
+                    sc[e] = __float_as_uint(vg[t0 + e] * q1[e]);
                 }
                 tmem_st8(th.lane_base + Cf::S2C + t0, sc);
-                col_sum8(0, cb, pav);
+                col_sum8(0, g, pav);
             }
             tmem_wait_st();
         }
@@ -658,9 +720,9 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         finish_sums(0, vav);
 
         // ---- dk += Y^T (dn Delta)^T (A = Y^T)
-        bg_put_a<D, D>(th, a_hi, a_lo_D, true, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<D>(th, a_hi, a_lo_D, all_lo, [&](int m, int k0, float (&x)[8]) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = (m < D && Y != nullptr) ? __ldg(Y + (int64_t)(k0 + j) * D + m) : 0.f;
+            for (int j = 0; j < 8; ++j) x[j] = (m < D && Y != nullptr) ? __ldg(Y + (k0 + j) * D + m) : 0.f;
         });
         bg_put_b<C, D>(Bh, Bl, [&](int t, int c4) {
             const float f = vdn[t];
@@ -674,10 +736,10 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             break;
 
         // ---- [dO; Dd] Delta^T -> DOD, DDD
-        bg_put_a<D, D>(th, a_hi, a_lo_D, true, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<D>(th, a_hi, a_lo_D, all_lo, [&](int m, int k0, float (&x)[8]) {
             const int t = m % C;
             if (m < C && t < len) {
-                load8(dO, trow(t) * D + k0, in_bf16, x);
+                load8(dO, tb + (t * RS + k0), in_bf16, x);
             } else if (m >= C && m < 2 * C) {
                 const float4 x0 = *reinterpret_cast<const float4*>(gDd + t * D + k0);
                 const float4 x1 = *reinterpret_cast<const float4*>(gDd + t * D + k0 + 4);
@@ -696,8 +758,8 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             break;
         {
             const int m = th.row;
-            for (int cb = 0; cb < C / 16; ++cb) {
-                const int t0 = th.hf * H2 + 8 * cb;
+            for (int g = th.p; g < NG; g += kBgParts) {
+                const int t0 = 8 * g;
                 float x[8];
                 tmem_ld8(th.lane_base + Cf::S0C + t0, x);
 #pragma unroll
@@ -711,54 +773,84 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         __syncthreads();
         tc_fence_after();
 
-        // ---- dalpha: F[r][t] = sum_{s>=t} D[s][t] (DOD[s][r] KQ[r][s] - [s>t] beta_s DDD[s][r] KK[r][s]), r < t;
-        // psi_t = gp_t (dn_t <Y,S0> + sum_{s>=t} D[s][t] av_s - sum_{s>t} D[s][t] beta_s bv_s)
-        //       + sum_{r<t} D[t-1][r] (dn_t cv_r + F[r][t])
+        // ---- dalpha.  With E1[r][s] = DOD[s][r] KQ[r][s] and E2b[r][s] = beta_s DDD[s][r] KK[r][s]:
+        //   F[r][t] = sum_{s>=t} E1[r][s] D[s][t] - sum_{s>t} E2b[r][s] D[s][t]
+        //           = sum_{s>=t} (E1 - E2b)[r][s] D[s][t] + E2b[r][t]
+        //   psi_t   = gp_t (dn_t <Y,S0> + sum_{s>=t} D[s][t] (av_s - beta_s bv_s) + beta_t bv_t)
+        //           + sum_{r<t} D[t-1][r] (dn_t cv_r + F[r][t])
+        float* Ed = N1;  // E1 - E2b
+        float* E2 = Ts;  // E2b
         for (int e = tid; e < C * C; e += blockDim.x) {
-            const int r = e / C, t = e % C;
-            float acc = 0.f;
-            if (r < t) {
-                for (int s = t; s < C; ++s) {
-                    float x = DOD[s * LD + r] * KQ[r * LD + s];
-                    if (s > t) x -= vb[s] * DDD[s * LD + r] * KK[r * LD + s];
-                    acc = fmaf(DM[s * LD + t], x, acc);
-                }
-            }
-            FF[r * LD + t] = acc;
+            const int r = e / C, s_ = e % C;
+            const float e2 = vb[s_] * DDD[s_ * LD + r] * KK[r * LD + s_];
+            E2[r * LD + s_] = e2;
+            Ed[r * LD + s_] = DOD[s_ * LD + r] * KQ[r * LD + s_] - e2;
         }
         __syncthreads();
-        for (int t = tid; t < len; t += blockDim.x) {
-            float a = vdn[t] * ysum;
-            for (int s = t; s < C; ++s) {
-                float x = vav[s];
-                if (s > t) x -= vb[s] * vbv[s];
-                a = fmaf(DM[s * LD + t], x, a);
+        if (tid < C * C / 8) {  // F, 2 x 4 outputs per thread
+            const int r0 = 2 * (tid / (C / 4)), t0 = 4 * (tid % (C / 4));
+            float acc[2][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc[0][j] = E2[r0 * LD + t0 + j];
+                acc[1][j] = E2[(r0 + 1) * LD + t0 + j];
             }
-            float psi = vgp[t] * a;
-            for (int r = 0; r < t; ++r) psi = fmaf(DM[(t - 1) * LD + r], vdn[t] * vcv[r] + FF[r * LD + t], psi);
-            dalpha[trow(t)] = psi - vb[t] * vdu[t];
-            dbeta[trow(t)] = vdb[t];
+            for (int s_ = t0; s_ < C; ++s_) {
+                const float e0 = Ed[r0 * LD + s_], e1 = Ed[(r0 + 1) * LD + s_];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float dm = DM[s_ * LD + t0 + j];  // zero for s < t
+                    acc[0][j] = fmaf(e0, dm, acc[0][j]);
+                    acc[1][j] = fmaf(e1, dm, acc[1][j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                FF[r0 * LD + t0 + j] = acc[0][j];
+                FF[(r0 + 1) * LD + t0 + j] = acc[1][j];
+            }
+        }
+        __syncthreads();
+        {  // psi: 8 threads per token t, each over the s and r with s, r = sub (mod 8)
+            const int t = tid >> 3, sub = tid & 7;
+            float a = 0.f, b = 0.f;
+            if (t < C) {
+                for (int s_ = t + ((sub - t) & 7); s_ < C; s_ += 8)
+                    a = fmaf(DM[s_ * LD + t], vav[s_] - vb[s_] * vbv[s_], a);
+                for (int r = sub; r < t; r += 8) b = fmaf(DM[(t - 1) * LD + r], vdn[t] * vcv[r] + FF[r * LD + t], b);
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                a += __shfl_xor_sync(0xffffffffu, a, o);
+                b += __shfl_xor_sync(0xffffffffu, b, o);
+            }
+            if (t < len && sub == 0) {
+                const float psi = vgp[t] * ((vdn[t] * ysum + a) + vb[t] * vbv[t]) + b;
+                dalpha[trow(t)] = psi - vb[t] * vdu[t];
+                dbeta[trow(t)] = vdb[t];
+            }
         }
 
         // ---- dk += [Q^T | K^T] [X1 | -X23]^T; dq += K^T Xq^T  (A = [Q^T | K^T], K = 2C)
-        bg_put_a<D, 2*C>(th, a_hi, a_lo_2C, !ex, [&](int m, int k0, float (&x)[8]) {
+        bg_put_a<2 * C>(th, a_hi, a_lo_2C, no_lo_if_exact, [&](int m, int k0, float (&x)[8]) {
+            const void* src = k0 < C ? q : k;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const int s = (k0 + j) % C;
-                x[j] = (m < D && s < len) ? bg_load1(k0 < C ? q : k, trow(s) * D + m, in_bf16) : 0.f;
+                const int s_ = (k0 + j) % C;
+                x[j] = (m < D && s_ < len) ? tok1(src, s_, m) : 0.f;
             }
         });
-        bg_put_b<C, 2*C>(Bh, Bl, [&](int t, int c4) {
+        bg_put_b<C, 2 * C>(Bh, Bl, [&](int t, int c4) {
             float x[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int s = (4 * c4 + j) % C;
+                const int s_ = (4 * c4 + j) % C;
                 if (4 * c4 < C) {  // X1[t][s] = D[s][t] DOD[s][t] (s >= t)
-                    x[j] = s >= t ? DM[s * LD + t] * DOD[s * LD + t] : 0.f;
+                    x[j] = s_ >= t ? DM[s_ * LD + t] * DOD[s_ * LD + t] : 0.f;
                 } else {           // -X23[t][s]
                     float y = 0.f;
-                    if (s > t) y = DM[s * LD + t] * vb[s] * DDD[s * LD + t];
-                    else if (s < t) y = va[t] * vb[t] * DM[(t - 1) * LD + s] * DDD[t * LD + s];
+                    if (s_ > t) y = DM[s_ * LD + t] * vb[s_] * DDD[s_ * LD + t];
+                    else if (s_ < t) y = va[t] * vb[t] * DM[(t - 1) * LD + s_] * DDD[t * LD + s_];
                     x[j] = -y;
                 }
             }
@@ -789,8 +881,8 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         // ---- dq, dk
         {
             const int j = th.row;
-            for (int cb = 0; cb < C / 16; ++cb) {
-                const int t0 = th.hf * H2 + 8 * cb;
+            for (int g = th.p; g < NG; g += kBgParts) {
+                const int t0 = 8 * g;
                 float xq[8], xk[8];
                 tmem_ld8(th.lane_base + Cf::S2C + t0, xq);
                 tmem_ld8(th.lane_base + Cf::S3C + t0, xk);
@@ -799,8 +891,8 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                     for (int e = 0; e < 8; ++e) {
                         const int t = t0 + e;
                         if (t < len) {
-                            dq[trow(t) * D + j] = xq[e];
-                            dk[trow(t) * D + j] = xk[e];
+                            dq[tb + (t * RS + j)] = xq[e];
+                            dk[tb + (t * RS + j)] = xk[e];
                         }
                     }
                 }
