@@ -55,14 +55,14 @@ struct BgCfg {
     static_assert(ACOLS + 4 * C <= 512, "TMEM columns");
     static constexpr int LD = C + 1;  // row stride of the C x C matrices
     static constexpr int MAT = C * LD;
-    // smem (floats): [B hi | B lo | DOD | DDD | N1 | F] [T | DM | KK | KQ] vectors partials
+    // smem (floats): [B hi | B lo] [T, then DOD | N1, then DDD | M, then F | DM | KK, then E2b |
+    // KQ, then E1 - E2b] vectors partials [bf16 token tiles q | k | dO]; each C x C buffer is
+    // taken over by the second matrix once the first is dead
     static constexpr int B_OFF = 0;
-    static constexpr int DOD_OFF = 2 * C * BK;
-    static constexpr int DDD_OFF = DOD_OFF + MAT;
-    static constexpr int N1_OFF = DDD_OFF + MAT;
+    static constexpr int T_OFF = 2 * C * BK;
+    static constexpr int N1_OFF = T_OFF + MAT;
     static constexpr int F_OFF = N1_OFF + MAT;
-    static constexpr int T_OFF = F_OFF + MAT;
-    static constexpr int DM_OFF = T_OFF + MAT;
+    static constexpr int DM_OFF = F_OFF + MAT;
     static constexpr int KK_OFF = DM_OFF + MAT;
     static constexpr int KQ_OFF = KK_OFF + MAT;
     static constexpr int VS = C + 4;
@@ -70,7 +70,9 @@ struct BgCfg {
     static constexpr int V_OFF = KQ_OFF + MAT;
     static constexpr int P_OFF = V_OFF + NV * VS;  // [4 quantities][4 lane quarters][C]
     static constexpr int YS_OFF = P_OFF + 16 * C;  // [16] warp partials of <Y, S0>
-    static constexpr int BAR_OFF = (YS_OFF + 16 + 3) / 4 * 4;
+    static constexpr int TILE_OFF = (YS_OFF + 16 + 3) / 4 * 4;      // 16-byte aligned
+    static constexpr int TILE_FL = 3 * C * D / 2;                   // three [C][D] bf16 tiles
+    static constexpr int BAR_OFF = TILE_OFF + TILE_FL;
     static constexpr int FLOATS = BAR_OFF + 4;
     static constexpr size_t SMEM = sizeof(float) * (size_t)FLOATS;
     static constexpr int64_t SCR = 4 * (int64_t)C * D;  // per-CTA scratch floats: Delta | KS | dn KY | Dd
@@ -308,11 +310,11 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
     float* sm = reinterpret_cast<float*>(smem_f4);
     float* Bh = sm + Cf::B_OFF;
     float* Bl = Bh + C * BK;
-    float* DOD = sm + Cf::DOD_OFF;  // DOD[t][r] = dO_t . Delta_r
-    float* DDD = sm + Cf::DDD_OFF;  // DDD[t][r] = Dd_t . Delta_r
-    float* N1 = sm + Cf::N1_OFF;    // N1 = T^T M, later Ediff
+    float* Ts = sm + Cf::T_OFF;     // T
+    float* DOD = Ts;                // then DOD[t][r] = dO_t . Delta_r
+    float* N1 = sm + Cf::N1_OFF;    // N1 = T^T M
+    float* DDD = N1;                // then DDD[t][r] = Dd_t . Delta_r
     float* FF = sm + Cf::F_OFF;     // M, later F
-    float* Ts = sm + Cf::T_OFF;     // T, later E2b
     float* DM = sm + Cf::DM_OFF;    // D[t][s]
     float* KK = sm + Cf::KK_OFF;    // k_t . k_s
     float* KQ = sm + Cf::KQ_OFF;    // k_t . q_s
@@ -323,6 +325,10 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
     float* ysp = sm + Cf::YS_OFF;
     uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Cf::BAR_OFF);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Cf::BAR_OFF + 2);
+    // bf16 inputs: the chunk's q, k, dO rows are staged once per task ([C][D] each)
+    uint16_t* tq = reinterpret_cast<uint16_t*>(sm + Cf::TILE_OFF);
+    uint16_t* tk = tq + C * D;
+    uint16_t* tdo = tk + C * D;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     if (tid == 0) mbar_init(mbar, 1);
@@ -384,6 +390,51 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         const int64_t tb = (tok0 * H + h) * D;  // element offset of the chunk's first token row
         const int RS = H * D;                    // token row stride (elements)
         auto tok1 = [&](const void* base, int t, int i) { return bg_load1(base, tb + (t * RS + i), in_bf16); };
+        // element (t, i), 4 elements (t, 4 c4 ..) and 8 elements (t, k0 ..) of q, k or dO (which = 0, 1, 2):
+        // from the staged tiles for bf16 inputs, else from global memory
+        auto tl1 = [&](int which, int t, int i) -> float {
+            if constexpr (BF16) {
+                return __uint_as_float((uint32_t)(which == 0 ? tq : which == 1 ? tk : tdo)[t * D + i] << 16);
+            } else {
+                return tok1(which == 0 ? q : which == 1 ? k : dO, t, i);
+            }
+        };
+        auto tl4 = [&](int which, int t, int c4) -> float4 {
+            if constexpr (BF16) {
+                const uint2 r = *reinterpret_cast<const uint2*>((which == 0 ? tq : which == 1 ? tk : tdo) + t * D +
+                                                                4 * c4);
+                return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                                   __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+            } else {
+                return bg_load4(which == 0 ? q : which == 1 ? k : dO, tb + (t * RS + 4 * c4), in_bf16);
+            }
+        };
+        auto tl8 = [&](int which, int t, int k0, float (&x)[8]) {
+            if constexpr (BF16) {
+                const uint4 r = *reinterpret_cast<const uint4*>((which == 0 ? tq : which == 1 ? tk : tdo) + t * D + k0);
+                const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    x[2 * m] = __uint_as_float(w[m] << 16);
+                    x[2 * m + 1] = __uint_as_float(w[m] & 0xffff0000u);
+                }
+            } else {
+                load8(which == 0 ? q : which == 1 ? k : dO, tb + (t * RS + k0), in_bf16, x);
+            }
+        };
+        if constexpr (BF16) {  // stage the tiles (rows past the chunk's end are zero); waited for before KS
+            constexpr int PR = D * 2 / 16;  // 16-byte pieces per row
+            for (int e = tid; e < 3 * C * PR; e += blockDim.x) {
+                const int which = e / (C * PR), rem = e % (C * PR), t = rem / PR, pc = rem % PR;
+                uint16_t* dst = (which == 0 ? tq : which == 1 ? tk : tdo) + t * D + 8 * pc;
+                if (t < len)
+                    cp_async16(dst, reinterpret_cast<const uint16_t*>(which == 0 ? q : which == 1 ? k : dO) +
+                                        tb + (int64_t)t * RS + 8 * pc);
+                else
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            cp_async_commit();
+        }
         auto trow = [&](int t) { return (tok0 + t) * H + h; };  // row of [T, H] gates
         const float* S0 = states + ((slot0 + c) * H + h) * (int64_t)D * D;
         const float* Y = c + 1 < nchunks ? ybuf + ((slot0 + c + 1) * H + h) * (int64_t)D * D
@@ -438,13 +489,14 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             }
         });
         bg_put_b<C, D>(Bh, Bl, [&](int r, int c4) { return *reinterpret_cast<const float4*>(gW + r * D + 4 * c4); });
+        if constexpr (BF16) cp_async_wait_all();  // the tiles, visible to all after the barrier in run
         if (!(ok = run([&] {
                   uint32_t acc = 0;
                   bg_mma(tbase + Cf::S1C, a_hi, a_lo_D, false, Bh, Bl, false, D * 32, 0, D / 8, Cf::IDESC, acc);
               })))
             break;
         bg_put_b<C, D>(Bh, ex ? nullptr : Bl, [&](int r, int c4) {
-            return r < len ? bg_load4(k, tb + (r * RS + 4 * c4), in_bf16) : make_float4(0.f, 0.f, 0.f, 0.f);
+            return r < len ? tl4(1, r, c4) : make_float4(0.f, 0.f, 0.f, 0.f);
         });
         if (!(ok = run([&] {
                   uint32_t acc = 0;
@@ -480,7 +532,7 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         bg_put_a<D>(th, a_hi, a_lo_D, no_lo_if_exact, [&](int m, int k0, float (&x)[8]) {
             const int t = m % C;
             if (m < 2 * C && t < len) {
-                load8(m < C ? k : q, tb + (t * RS + k0), in_bf16, x);
+                tl8(m < C ? 1 : 0, t, k0, x);
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) x[j] = 0.f;
@@ -612,7 +664,7 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                                 x[j] = 0.f;
                                 if (m < D) {
                                     if (s_ < C) x[j] = gKY[s_ * D + m];
-                                    else if (s_ - C < len) x[j] = tok1(dO, s_ - C, m);
+                                    else if (s_ - C < len) x[j] = tl1(2, s_ - C, m);
                                 }
                             }
                         });
@@ -680,7 +732,7 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
             for (int j = 0; j < 8; ++j) x[j] = m < D ? __ldg(S0 + (k0 + j) * D + m) : 0.f;
         });
         bg_put_b<C, D>(Bh, ex ? nullptr : Bl, [&](int r, int c4) {
-            return r < len ? bg_load4(dO, tb + (r * RS + 4 * c4), in_bf16) : make_float4(0.f, 0.f, 0.f, 0.f);
+            return r < len ? tl4(2, r, c4) : make_float4(0.f, 0.f, 0.f, 0.f);
         });
         if (!(ok = run([&] {
                   uint32_t acc = 0;
@@ -694,7 +746,7 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
                 float q1[8], pav[8], qr[8];  // global values fetched first
                 uint32_t sc[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) qr[e] = (j < D && t0 + e < len) ? tok1(q, t0 + e, j) : 0.f;
+                for (int e = 0; e < 8; ++e) qr[e] = (j < D && t0 + e < len) ? tl1(0, t0 + e, j) : 0.f;
                 tmem_ld8(th.lane_base + Cf::S2C + t0, q1);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -739,7 +791,7 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         bg_put_a<D>(th, a_hi, a_lo_D, all_lo, [&](int m, int k0, float (&x)[8]) {
             const int t = m % C;
             if (m < C && t < len) {
-                load8(dO, tb + (t * RS + k0), in_bf16, x);
+                tl8(2, t, k0, x);
             } else if (m >= C && m < 2 * C) {
                 const float4 x0 = *reinterpret_cast<const float4*>(gDd + t * D + k0);
                 const float4 x1 = *reinterpret_cast<const float4*>(gDd + t * D + k0 + 4);
@@ -778,8 +830,8 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
         //           = sum_{s>=t} (E1 - E2b)[r][s] D[s][t] + E2b[r][t]
         //   psi_t   = gp_t (dn_t <Y,S0> + sum_{s>=t} D[s][t] (av_s - beta_s bv_s) + beta_t bv_t)
         //           + sum_{r<t} D[t-1][r] (dn_t cv_r + F[r][t])
-        float* Ed = N1;  // E1 - E2b
-        float* E2 = Ts;  // E2b
+        float* Ed = KQ;  // E1 - E2b, in place over KQ (each element reads only its own KQ, KK)
+        float* E2 = KK;  // E2b, in place over KK
         for (int e = tid; e < C * C; e += blockDim.x) {
             const int r = e / C, s_ = e % C;
             const float e2 = vb[s_] * DDD[s_ * LD + r] * KK[r * LD + s_];
@@ -833,11 +885,11 @@ k_bgrad(const void* __restrict__ q, const void* __restrict__ k, const void* __re
 
         // ---- dk += [Q^T | K^T] [X1 | -X23]^T; dq += K^T Xq^T  (A = [Q^T | K^T], K = 2C)
         bg_put_a<2 * C>(th, a_hi, a_lo_2C, no_lo_if_exact, [&](int m, int k0, float (&x)[8]) {
-            const void* src = k0 < C ? q : k;
+            const int which = k0 < C ? 0 : 1;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int s_ = (k0 + j) % C;
-                x[j] = (m < D && s_ < len) ? tok1(src, s_, m) : 0.f;
+                x[j] = (m < D && s_ < len) ? tl1(which, s_, m) : 0.f;
             }
         });
         bg_put_b<C, 2 * C>(Bh, Bl, [&](int t, int c4) {
