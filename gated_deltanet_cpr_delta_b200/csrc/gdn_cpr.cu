@@ -291,6 +291,7 @@ struct DecArgs {
     void* o;
     cudaStream_t stream;
     void* const* events;  // optional: 3 events around the kernels
+    int may_resync;       // 0: the caller guarantees that no buffer fills in this step
 };
 
 template <int D, int C>
@@ -317,6 +318,10 @@ gdn_status_t launch_decode(const DecArgs& a)
         (int)NH, c.status);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     mark(a.events, 1, a.stream);
+    if (!a.may_resync) {  // no pair reaches the end of its buffer: nothing to resync
+        mark(a.events, 2, a.stream);
+        return GDN_OK;
+    }
     constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
     if (set_smem(gdn::k_dec_resync<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
     // persistent: one CTA per SM, and at most 1024 (sequence, head) pairs per CTA
@@ -637,10 +642,10 @@ gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v, const
                                   dstate_in, workspace, workspace_bytes, stream, nullptr);
 }
 
-gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, const float* alpha,
-                                   const float* beta, const gdn_cache_t* cache, int32_t num_seqs, int32_t H,
-                                   int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
-                                   gdn_dtype_t out_dtype, void* o, void* stream, void* const* events)
+gdn_status_t gdn_decode_step_ex(const void* q, const void* k, const void* v, const float* alpha,
+                                const float* beta, const gdn_cache_t* cache, int32_t num_seqs, int32_t H,
+                                int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                                void* o, int32_t may_resync, void* stream, void* const* events)
 {
     if (num_seqs < 0 || H <= 0 || d_k <= 0 || d_v <= 0 || C <= 0) return GDN_ERR_INVALID_ARG;
     if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return GDN_ERR_INVALID_ARG;
@@ -660,8 +665,17 @@ gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, 
     DecArgs a;
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.cache = cache;
     a.N = num_seqs; a.H = H; a.in_bf16 = in_dtype == GDN_BF16; a.out_bf16 = out_dtype == GDN_BF16;
-    a.o = o; a.stream = static_cast<cudaStream_t>(stream); a.events = events;
+    a.o = o; a.stream = static_cast<cudaStream_t>(stream); a.events = events; a.may_resync = may_resync != 0;
     GDN_DISPATCH(launch_decode, d_k, C, a)
+}
+
+gdn_status_t gdn_decode_step_timed(const void* q, const void* k, const void* v, const float* alpha,
+                                   const float* beta, const gdn_cache_t* cache, int32_t num_seqs, int32_t H,
+                                   int32_t d_k, int32_t d_v, int32_t C, gdn_dtype_t in_dtype,
+                                   gdn_dtype_t out_dtype, void* o, void* stream, void* const* events)
+{
+    return gdn_decode_step_ex(q, k, v, alpha, beta, cache, num_seqs, H, d_k, d_v, C, in_dtype, out_dtype, o, 1,
+                              stream, events);
 }
 
 gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const float* alpha, const float* beta,

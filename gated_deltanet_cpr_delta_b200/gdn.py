@@ -26,6 +26,7 @@ _STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "
 #: exported symbols of include/gdn_cpr.h
 SYMBOLS = ("gdn_contract_id", "gdn_status_string", "gdn_num_chunk_states", "gdn_cpr_workspace_size",
            "gdn_cpr_forward", "gdn_decode_step", "gdn_cpr_forward_timed", "gdn_decode_step_timed",
+           "gdn_decode_step_ex",
            "gdn_cpr_forward_noalloc", "gdn_contract_text", "gdn_contract_identity", "gdn_sha256_hex",
            "gdn_cpr_backward_workspace_size", "gdn_cpr_backward", "gdn_cpr_backward_timed",
            "gdn_read_device_status", "gdn_test_fault_injection")
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gdn_cpr_forward_timed.argtypes = lib.gdn_cpr_forward.argtypes + [P]
     lib.gdn_decode_step_timed.restype = ctypes.c_int
     lib.gdn_decode_step_timed.argtypes = lib.gdn_decode_step.argtypes + [P]
+    lib.gdn_decode_step_ex.restype = ctypes.c_int
+    lib.gdn_decode_step_ex.argtypes = lib.gdn_decode_step.argtypes[:-1] + [i32, P, P]
     lib.gdn_cpr_forward_noalloc.restype = ctypes.c_int
     lib.gdn_cpr_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, ctypes.c_int,
                                             ctypes.c_int, P, P, ctypes.POINTER(CacheStruct), P]
@@ -183,7 +186,9 @@ def new_cache(N: int, H: int, d_k: int, d_v: int, C: int, dtype: torch.dtype, de
     """Allocate a decode cache (gdn_cache_t layout).  With ``state`` [N,H,d_v,d_k]
     it starts at a chunk boundary with that state, otherwise at zero.  The
     running state is ``rscale * R``.  ``status`` is the decode step's device
-    status word (one int32, starts at GDN_OK)."""
+    status word (one int32, starts at GDN_OK).  ``pos_host`` is a host copy of
+    each sequence's buffer position (CPU int32 [N]): :func:`gdn_decode_step`
+    skips the resync launch on steps where no buffer can fill."""
     S = torch.zeros(N, H, d_v, d_k, dtype=torch.float32, device=device) if state is None else state.clone()
     return dict(S_b=S, R=S.clone(), rscale=torch.ones(N, H, dtype=torch.float32, device=device),
                 kbuf=torch.zeros(N, H, C, d_k, dtype=dtype, device=device),
@@ -191,7 +196,14 @@ def new_cache(N: int, H: int, d_k: int, d_v: int, C: int, dtype: torch.dtype, de
                 abuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
                 bbuf=torch.zeros(N, H, C, dtype=torch.float32, device=device),
                 pos=torch.zeros(N, H, dtype=torch.int32, device=device),
-                status=torch.zeros(1, dtype=torch.int32, device=device))
+                status=torch.zeros(1, dtype=torch.int32, device=device),
+                pos_host=torch.zeros(N, dtype=torch.int32))
+
+
+def _set_pos_host(cache: Dict[str, torch.Tensor], cu_seqlens_host, C: int):
+    """After a prefill into ``cache``: each sequence's position is L mod C."""
+    cu = [int(x) for x in cu_seqlens_host]
+    cache["pos_host"] = torch.tensor([(cu[n + 1] - cu[n]) % C for n in range(len(cu) - 1)], dtype=torch.int32)
 
 
 def _cache_struct(c: Dict[str, torch.Tensor]) -> CacheStruct:
@@ -257,6 +269,8 @@ def gdn_cpr_forward(q, k, v, alpha, beta, cu_seqlens, C: int, *, cu_seqlens_host
     else:
         st = lib.gdn_cpr_forward_timed(*args, _event_array(events, 6))
     _check(st, "gdn_cpr_forward")
+    if cache_out is not None:
+        _set_pos_host(cache_out, cu_seqlens_host, C)
     return o, chunk_states
 
 
@@ -305,7 +319,10 @@ def gdn_decode_step(q, k, v, alpha, beta, cache: Dict[str, torch.Tensor], C: int
                     events=None):
     """One decode token per sequence.  q,k [N,H,d_k], v [N,H,d_v]; alpha, beta [N,H].
     ``cache`` (from :func:`new_cache` or a forward's ``cache_out``) is updated in place.
-    ``events``: optional 3 torch.cuda.Events (calls gdn_decode_step_timed)."""
+    ``events``: optional 3 torch.cuda.Events around the two kernels.  With the
+    cache's ``pos_host`` (kept by :func:`new_cache`, the forwards and this call)
+    the resync launch is skipped on steps where no sequence's buffer fills
+    (gdn_decode_step_ex's hint); without it the resync is always launched."""
     lib = load_library()
     N, H, dk = k.shape
     dv = v.shape[2]
@@ -313,13 +330,15 @@ def gdn_decode_step(q, k, v, alpha, beta, cache: Dict[str, torch.Tensor], C: int
     if o is None:
         o = torch.empty(N, H, dv, dtype=out_dtype, device=k.device)
     cs = _cache_struct(cache)
-    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), ctypes.byref(cs), N, H, dk,
-            dv, C, _dt(q.dtype), _dt(out_dtype), _ptr(o), _stream(k.device))
-    if events is None:
-        st = lib.gdn_decode_step(*args)
-    else:
-        st = lib.gdn_decode_step_timed(*args, _event_array(events, 3))
+    ph = cache.get("pos_host")
+    may_resync = 1 if ph is None else int(bool(((ph + 1) >= C).any()))
+    st = lib.gdn_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), ctypes.byref(cs), N, H, dk,
+                                dv, C, _dt(q.dtype), _dt(out_dtype), _ptr(o), may_resync, _stream(k.device),
+                                _event_array(events, 3) if events is not None else None)
     _check(st, "gdn_decode_step")
+    if ph is not None:
+        ph += 1
+        ph[ph >= C] = 0
     return o
 
 
@@ -352,4 +371,6 @@ def gdn_cpr_forward_noalloc(q, k, v, alpha, beta, cu_seqlens, C: int, *, cu_seql
                                      _ptr(o), _ptr(chunk_states), ctypes.byref(cs) if cs is not None else None,
                                      _stream(dev))
     _check(st, "gdn_cpr_forward_noalloc")
+    if cache_out is not None:
+        _set_pos_host(cache_out, cu_seqlens_host, C)
     return o, chunk_states

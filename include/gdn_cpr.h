@@ -342,6 +342,28 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v,
                              void* o, void* stream);
 
 /*
+ * gdn_decode_step with a host-side hint and optional events.
+ *   may_resync = 0: the caller guarantees that no (sequence, head) buffer
+ *     fills in this step, i.e. every pos is below C - 1 before the call (the
+ *     positions follow from the prefill lengths: pos = L mod C after a prefill
+ *     of L tokens, then + 1 per step, wrapping to 0 at C).  Only the per-token
+ *     kernel is enqueued; the resync launch is skipped.
+ *   may_resync != 0: exactly gdn_decode_step.
+ *   events: NULL, or 3 events as for gdn_decode_step_timed (with the resync
+ *     skipped, events[1] and events[2] are recorded back to back).
+ * A wrong guarantee does not write out of bounds: a pair whose buffer filled
+ * is left at pos = C, and the next step's per-token kernel treats that as an
+ * invalid position (GDN_ERR_DEVICE_INPUT in cache->status, nothing written
+ * for it) until a call with may_resync != 0 runs its resync.
+ */
+gdn_status_t gdn_decode_step_ex(const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta,
+                                const gdn_cache_t* cache,
+                                int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v, int32_t C,
+                                gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                                void* o, int32_t may_resync, void* stream, void* const* events);
+
+/*
  * Per-kernel timing variants, for benchmarks and profilers.  These are the
  * same calls with the same launches and the same results.  In addition they
  * record caller-created CUDA events (cudaEvent_t, created on the current

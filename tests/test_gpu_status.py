@@ -110,3 +110,59 @@ def test_decode_status_records_an_invalid_position():
     torch.cuda.synchronize()
     assert int(cache["status"].item()) == gdn.GDN_ERR_DEVICE_INPUT
     assert int(cache["pos"][0, 0]) == 99 and int(cache["pos"][1, 0]) == 2
+
+
+def test_decode_resync_hint_skips_the_launch_and_a_wrong_hint_is_reported():
+    """The host hint (gdn_decode_step_ex, may_resync): the binding's pos_host
+    skips the resync launch only where no buffer fills, and the results equal
+    the always-resync path bit for bit across a boundary.  A wrong hint leaves
+    the filled pair at pos = C; the next step refuses that position
+    (GDN_ERR_DEVICE_INPUT, nothing written) and a resync brings it back."""
+    C, D, H, N = 16, 16, 2, 2
+    Lp, steps = 13, 6  # the 3rd step fills the buffers
+    b = synth.make_batch(760, [Lp + steps] * N, H, D, D, "bf16")
+    cu = b.cu_seqlens
+    sl = np.concatenate([np.arange(cu[n], cu[n] + Lp) for n in range(N)])
+    pre = synth.Batch(b.q[sl], b.k[sl], b.v[sl], b.alpha[sl], b.beta[sl], (np.arange(N + 1) * Lp).astype(np.int32),
+                      b.dtype)
+    dd = to_device(b)
+
+    def prefill():
+        d = to_device(pre)
+        c = gdn.new_cache(N, H, D, D, C, d["q"].dtype, DEV)
+        gdn.gdn_cpr_forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["cu_seqlens"], C,
+                            cu_seqlens_host=d["cu_host"], out_dtype=torch.float32, cache_out=c)
+        return c
+
+    hinted, always = prefill(), prefill()
+    assert hinted["pos_host"].tolist() == [Lp % C] * N
+    del always["pos_host"]  # no host positions: every step launches the resync
+    for s in range(steps):
+        idx = torch.from_numpy((cu[:-1] + Lp + s).astype(np.int64)).to(DEV)
+        args = (dd["q"][idx], dd["k"][idx], dd["v"][idx], dd["alpha"][idx], dd["beta"][idx])
+        o1 = gdn.gdn_decode_step(*args, hinted, C, out_dtype=torch.float32)
+        o2 = gdn.gdn_decode_step(*args, always, C, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(o1), bits(o2)), s
+    for key in ("S_b", "R", "rscale", "pos", "kbuf", "vbuf"):
+        assert torch.equal(hinted[key], always[key]), key
+    assert hinted["pos_host"].tolist() == [(Lp + steps) % C] * N
+    assert int(hinted["status"].item()) == gdn.GDN_OK
+
+    # a wrong hint: the binding believes the step cannot fill a buffer
+    wrong = prefill()
+    for s in range(2):
+        idx = torch.from_numpy((cu[:-1] + Lp + s).astype(np.int64)).to(DEV)
+        gdn.gdn_decode_step(dd["q"][idx], dd["k"][idx], dd["v"][idx], dd["alpha"][idx], dd["beta"][idx], wrong, C)
+    wrong["pos_host"][:] = 0
+    idx = torch.from_numpy((cu[:-1] + Lp + 2).astype(np.int64)).to(DEV)
+    step3 = (dd["q"][idx], dd["k"][idx], dd["v"][idx], dd["alpha"][idx], dd["beta"][idx])
+    gdn.gdn_decode_step(*step3, wrong, C)
+    torch.cuda.synchronize()
+    assert (wrong["pos"] == C).all() and int(wrong["status"].item()) == gdn.GDN_OK
+    del wrong["pos_host"]  # next step: unknown positions, the resync runs after the refused token
+    gdn.gdn_decode_step(*step3, wrong, C)
+    torch.cuda.synchronize()
+    assert int(wrong["status"].item()) == gdn.GDN_ERR_DEVICE_INPUT
+    assert torch.equal(wrong["S_b"], always["S_b"])  # the resync over the full buffer happened
+    assert (wrong["pos"] == 0).all()
