@@ -267,8 +267,9 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
  * (IsoExec summary page, section "Chunkwise-Parallel Recurrent (CPR) Gated
  * DeltaNet"; commentary blog, section 10), differentiated in reverse token
  * order.  A serial scan carries dL/dS back to every chunk boundary; then the
- * chunks run in parallel, each recomputing its states from the boundary state
- * the forward stored, with the forward's per-token arithmetic.
+ * chunks run in parallel, each from the boundary state the forward stored and
+ * the adjoint at its end, as dense products of chunk matrices on the tensor
+ * cores (tf32 with a hi/lo split of every fp32 operand).
  * Inputs:
  *   q, k, v, alpha, beta, cu_seqlens, cu_seqlens_host, num_seqs, total_tokens,
  *     H, d_k, d_v, C, in_dtype: as given to gdn_cpr_forward.
@@ -282,8 +283,8 @@ size_t gdn_cpr_backward_workspace_size(int64_t total_tokens, int32_t num_seqs, i
  * Outputs (fp32, device, caller-owned, every element written):
  *   dq, dk [T_total,H,d_k]; dv [T_total,H,d_v]; dalpha, dbeta [T_total,H];
  *   dstate_in [num_seqs,H,d_v,d_k]: the gradient for the forward's state_in.
- * The result is deterministic: the row tiles' contributions are added in a
- * fixed order, with no atomics.
+ * The result is deterministic: every sum has a fixed order and there are no
+ * atomics, so repeats give the same bits.
  *   workspace: at least gdn_cpr_backward_workspace_size(...) bytes of device
  *     memory, 256-byte aligned, not shared with a concurrent call.
  * Errors: as gdn_cpr_forward.  If the device copy of cu_seqlens disagrees
@@ -303,7 +304,7 @@ gdn_status_t gdn_cpr_backward(const void* q, const void* k, const void* v,
 /*
  * gdn_cpr_backward with events: events (host array of 4 cudaEvent_t, or NULL)
  * are recorded on the stream before the boundary-adjoint scan, after it,
- * after the per-chunk kernel and after the tile reduction.
+ * after the chunk-local precompute and after the per-chunk gradients.
  */
 gdn_status_t gdn_cpr_backward_timed(const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, const void* dO,

@@ -1,13 +1,16 @@
 """GPU parity of the CPR backward (gdn_cpr_backward, through the C ABI)
 against the fp64 adjoint oracle (oracle/adjoint_fp64.c).
 
-The loss is L = sum_t dO_t . o_t.  The kernels compute in fp32 from inputs
-that both sides read as the same values (bf16 inputs are widened exactly), so
-the only differences are fp32 rounding in the recomputed states, the adjoint
-state G and the row sums.  Bound: max|g - g*| <= 2e-4 * max(||g*||_inf, 1e-3)
-for every gradient (fp32 rounding, about 6e-8 relative per operation, grows
-with the d_k-term dot products and the few hundred steps of G in these cases;
-the bound leaves a margin of ~10x over what the arithmetic gives).
+The loss is L = sum_t dO_t . o_t.  The kernels compute in fp32-class
+arithmetic from inputs that both sides read as the same values (bf16 inputs
+are widened exactly): the boundary adjoints by a serial fp32 scan, each
+chunk's gradients by dense chunk-form products on the tensor cores with every
+fp32 operand split into two tf32 parts (lo*hi + hi*lo + hi*hi).  The only
+differences are rounding in the forward's boundary states, the adjoints and
+those products.  Bound: max|g - g*| <= 2e-4 * max(||g*||_inf, 1e-3) for every
+gradient (the chunk form evaluated in fp32 stays within 4e-7 of the fp64
+sweep on these sizes; the bound leaves a wide margin, and plain tf32 products
+would exceed it).
 Also: repeats are bit-identical (no atomics), batch composition does not change
 a sequence's gradients, and a sampled (sequence, head) at the trainer's full
 size (B=2, H=32, T=8192, d=128, C=64, bf16) matches the oracle.
