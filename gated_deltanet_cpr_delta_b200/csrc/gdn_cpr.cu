@@ -322,11 +322,27 @@ gdn_status_t launch_decode(const DecArgs& a)
         mark(a.events, 2, a.stream);
         return GDN_OK;
     }
-    constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
-    if (set_smem(gdn::k_dec_resync<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
     // persistent: one CTA per SM, and at most 1024 (sequence, head) pairs per CTA
     const int64_t min_grid = (NH + 1023) / 1024;
     const unsigned rgrid = (unsigned)std::max<int64_t>(std::min<int64_t>(NH, sms), min_grid);
+    if constexpr (2 * C <= D) {  // the resync in two kernels: P_chunk part 1 per pair, then the chain step
+        const size_t psm = gdn::PrepCfg<D, D, C>::bytes(a.in_bf16);
+        if (set_smem(gdn::k_dec_rprep<D, D, C>, psm) != cudaSuccess) return GDN_ERR_CUDA;
+        gdn::k_dec_rprep<D, D, C><<<(unsigned)NH, 256, psm, a.stream>>>(
+            (int)NH, a.in_bf16, (const void*)c.kbuf, (const void*)c.vbuf, (const float*)c.abuf,
+            (const float*)c.bbuf, c.pos, c.R);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+        constexpr size_t ssm = gdn::RstepSmem<D, D, C>::BYTES;
+        if (set_smem(gdn::k_dec_rstep<D, D, C>, ssm) != cudaSuccess) return GDN_ERR_CUDA;
+        gdn::k_dec_rstep<D, D, C><<<rgrid, 256, ssm, a.stream>>>((int)NH, a.in_bf16, c.S_b, c.R, c.rscale,
+                                                                 (const void*)c.kbuf, (const float*)c.abuf, c.pos,
+                                                                 c.status);
+        if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+        mark(a.events, 2, a.stream);
+        return GDN_OK;
+    }
+    constexpr size_t sm = gdn::ResyncSmem<D, D, C>::BYTES;
+    if (set_smem(gdn::k_dec_resync<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
     // programmatic dependent launch: the resync grid is scheduled while the
     // per-token step finishes and waits on the device (griddepcontrol.wait)
     // for its results, which hides its launch latency on the many steps that

@@ -291,4 +291,142 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
 }
 
 
+// The resync in two kernels, for 2C <= d (u0 and w of a chunk fit in one
+// d x d state): on a step where buffers fill, the running state R of those
+// pairs is dead until the resync rewrites it, so it holds their P_chunk
+// part 1 operands in between.
+//   k_dec_rprep: one CTA per pair, 3 CTAs per SM; a pair at pos == C runs
+//     chunk_prep on its buffer: u0 -> R[0 .. C*d), w -> R[C*d .. 2*C*d).
+//   k_dec_rstep: persistent, one CTA per SM; for each pair at pos == C the
+//     tcgen05 step (tc_step) from S_b with w, k^T (from the buffer), u0
+//     (staged from R into shared memory) and D[C][.] (from the buffered
+//     gates, in chunk_prep's order of products), writing S_b and R; then
+//     pos = 0, rscale = 1.
+// The device functions and their operands are the single kernel's, so the
+// results are bit for bit the same.
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256, 3)
+k_dec_rprep(int NH, int in_bf16, const void* kbuf, const void* vbuf, const float* abuf, const float* bbuf,
+            const int32_t* pos, float* R)
+{
+    static_assert(2 * C * DV <= DV * DK && DK == DV, "u0 and w fit in one state");
+    const int nh = blockIdx.x;
+    if (nh >= NH || pos[nh] != C) return;
+    extern __shared__ float4 smem_f4[];
+    unsigned char* base = reinterpret_cast<unsigned char*>(smem_f4);
+    // buffer rows are [nh][slot][D]: a [T, H=1, D] tensor starting at token nh*C
+    prep_stage<DK, DV, C>(base, kbuf, vbuf, abuf, bbuf, (int64_t)nh * C, 1, 0, in_bf16);
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    float* out = R + (int64_t)nh * DV * DK;
+    chunk_prep<DK, DV, C>(prep_bufs<DK, DV, C>(base, in_bf16), in_bf16, out, DV, out + C * DV, DK, nullptr);
+}
+
+template <int DK, int DV, int C>
+struct RstepSmem {
+    using T = TcCfg<DK, DV, C>;
+    static constexpr int WLO_OFF = 0;
+    static constexpr int KLO_OFF = WLO_OFF + 2 * T::W_FLOATS;
+    static constexpr int DC_OFF = KLO_OFF + ((T::K_REGION + 3) / 4) * 4;  // [C + 4] D[C][.]
+    static constexpr int AS_OFF = DC_OFF + ((C + 4 + 3) / 4) * 4;         // [C] the buffered alphas
+    static constexpr int US_OFF = AS_OFF + ((C + 3) / 4) * 4;             // [C][DV] u0, from R
+    static constexpr int WXS = DK + 4;                                     // row stride of w
+    static constexpr int WX_OFF = US_OFF + C * DV;                         // [C][WXS] w, from R
+    static constexpr int BAR_OFF = WX_OFF + C * WXS;
+    // at least 120 KB, so that one CTA fits per SM: each allocates all 512 TMEM columns
+    static constexpr size_t USED = sizeof(float) * (BAR_OFF + 4);
+    static constexpr size_t BYTES = USED > 120 * 1024 ? USED : 120 * 1024;
+    static_assert(BYTES <= 232448, "fits the 227 KB of shared memory a CTA can have");
+};
+
+template <int DK, int DV, int C>
+__global__ void __launch_bounds__(256, 1)
+k_dec_rstep(int NH, int in_bf16, float* S_b, float* R, float* rscale, const void* kbuf, const float* abuf,
+            int32_t* pos, int32_t* status)
+{
+    using Sm = RstepSmem<DK, DV, C>;
+    using T = TcCfg<DK, DV, C>;
+    extern __shared__ float4 smem_f4[];
+    float* sm = reinterpret_cast<float*>(smem_f4);
+    float* Wlo = sm + Sm::WLO_OFF;
+    float* Whi = Wlo + T::W_FLOATS;
+    float* Klo = sm + Sm::KLO_OFF;
+    float* Khi = Klo + T::K_FLOATS;
+    float* dCs = sm + Sm::DC_OFF;
+    float* as_ = sm + Sm::AS_OFF;
+    float* us = sm + Sm::US_OFF;
+    float* wx = sm + Sm::WX_OFF;
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + Sm::BAR_OFF);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Sm::BAR_OFF + 2);
+    // this CTA's pairs are blockIdx.x + i*gridDim.x: list the ones at a full buffer
+    __shared__ int todo[1024];
+    __shared__ int ntodo;
+    if (threadIdx.x == 0) ntodo = 0;
+    __syncthreads();
+    for (int nh = blockIdx.x + threadIdx.x * gridDim.x; nh < NH; nh += blockDim.x * gridDim.x) {
+        if (pos[nh] == C) {
+            const int slot = atomicAdd(&ntodo, 1);
+            if (slot < 1024) todo[slot] = nh;   // the host sizes the grid so that a CTA has <= 1024 pairs
+        }
+    }
+    __syncthreads();
+    const int nt = min(ntodo, 1024);
+    if (nt == 0) return;
+
+    if (threadIdx.x == 0) mbar_init(mbar, 1);
+    if (threadIdx.x < 32) tmem_alloc(tslot, T::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tslot;
+    const TcThread<DK> th(tbase);
+    uint32_t parity = 0;
+    float SR[DK / 2];
+    int it = 0;
+    for (; it < nt; ++it) {
+        const int nh = todo[it];
+        float* Rn = R + (int64_t)nh * DV * DK;  // u0 rows [C][DV], then w rows [C][DK]
+        // u0, w and the alphas to shared memory by cp.async, every copy in flight at once
+        for (int f = threadIdx.x; f < C * (DV + DK) / 4; f += blockDim.x) {
+            if (f < C * DV / 4) {
+                cp_async16(us + 4 * f, Rn + 4 * f);
+            } else {
+                const int g = f - C * DV / 4, t = g / (DK / 4), c4 = g % (DK / 4);
+                cp_async16(wx + t * Sm::WXS + 4 * c4, Rn + C * DV + t * DK + 4 * c4);
+            }
+        }
+        for (int t = threadIdx.x; t < C; t += blockDim.x) cp_async4(as_ + t, abuf + (int64_t)nh * C + t);
+        cp_async_commit();
+        tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
+        float* Sg = S_b + (int64_t)nh * DV * DK;
+        cp_async_wait_all();
+        __syncthreads();
+        tc_stage_w<DK, DV, C>(wx, Sm::WXS, Whi, Wlo, threadIdx.x, blockDim.x);
+        for (int s_ = threadIdx.x; s_ <= C; s_ += blockDim.x) {  // D[C][s], chunk_prep's order of products
+            float d = 1.0f;
+            for (int t = s_; t < C; ++t) d = fmul(d, as_[t]);
+            dCs[s_] = d;
+        }
+        tc_load_state<DK, DV, C>(SR, th, Sg, nullptr);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (!tc_step<DK, DV, C>(SR, th, tbase, mbar, parity, Wlo, Klo, us, DV, dCs, in_bf16, Sg, Rn))
+            break;
+        if (threadIdx.x == 0) {
+            pos[nh] = 0;
+            rscale[nh] = 1.0f;
+        }
+    }
+    for (int r = it + threadIdx.x; r < nt; r += blockDim.x) pos[todo[r]] = -1;  // after a timeout
+    if (it < nt && threadIdx.x == 0) record_error(status, GDN_ERR_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        tc_fence_after();
+        tmem_dealloc(tbase, T::TMEM_COLS);
+    }
+}
+
 }  // namespace gdn
