@@ -331,7 +331,8 @@ def gdn_decode_step(q, k, v, alpha, beta, cache: Dict[str, torch.Tensor], C: int
         o = torch.empty(N, H, dv, dtype=out_dtype, device=k.device)
     cs = _cache_struct(cache)
     ph = cache.get("pos_host")
-    may_resync = 1 if ph is None else int(bool(((ph + 1) >= C).any()))
+    ph = ph.numpy() if ph is not None else None  # numpy view of the CPU tensor: cheap host arithmetic
+    may_resync = 1 if ph is None else int((ph >= C - 1).any())
     st = lib.gdn_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), ctypes.byref(cs), N, H, dk,
                                 dv, C, _dt(q.dtype), _dt(out_dtype), _ptr(o), may_resync, _stream(k.device),
                                 _event_array(events, 3) if events is not None else None)
