@@ -215,9 +215,10 @@ gdn_status_t launch_forward(const FwdArgs& a)
     mark(a.events, 1, a.stream);
     if (a.tot.full > 0) {
         const size_t sm = gdn::PrepCfg<D, D, C>::bytes(a.in_bf16);
-        if (set_smem(gdn::k_prep<D, D, C>, sm) != cudaSuccess) return GDN_ERR_CUDA;
-        gdn::k_prep<D, D, C><<<(unsigned)(a.tot.full * a.H), Cf::THREADS, sm, a.stream>>>(
-            a.k, a.v, a.alpha, a.beta, a.cu, a.ws.fco, a.ws.err, a.N, a.H, a.in_bf16, a.ws.w, a.ws.u, a.ws.dC);
+        auto kern = a.in_bf16 ? gdn::k_prep<D, D, C, true> : gdn::k_prep<D, D, C, false>;
+        if (set_smem(kern, sm) != cudaSuccess) return GDN_ERR_CUDA;
+        kern<<<(unsigned)(a.tot.full * a.H), Cf::THREADS, sm, a.stream>>>(
+            a.k, a.v, a.alpha, a.beta, a.cu, a.ws.fco, a.ws.err, a.N, a.H, a.ws.w, a.ws.u, a.ws.dC);
         if ((e = cudaGetLastError()) != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 2, a.stream);
@@ -327,9 +328,10 @@ gdn_status_t launch_decode(const DecArgs& a)
     const unsigned rgrid = (unsigned)std::max<int64_t>(std::min<int64_t>(NH, sms), min_grid);
     if constexpr (2 * C <= D) {  // the resync in two kernels: P_chunk part 1 per pair, then the chain step
         const size_t psm = gdn::PrepCfg<D, D, C>::bytes(a.in_bf16);
-        if (set_smem(gdn::k_dec_rprep<D, D, C>, psm) != cudaSuccess) return GDN_ERR_CUDA;
-        gdn::k_dec_rprep<D, D, C><<<(unsigned)NH, 256, psm, a.stream>>>(
-            (int)NH, a.in_bf16, (const void*)c.kbuf, (const void*)c.vbuf, (const float*)c.abuf,
+        auto rprep = a.in_bf16 ? gdn::k_dec_rprep<D, D, C, true> : gdn::k_dec_rprep<D, D, C, false>;
+        if (set_smem(rprep, psm) != cudaSuccess) return GDN_ERR_CUDA;
+        rprep<<<(unsigned)NH, 256, psm, a.stream>>>(
+            (int)NH, (const void*)c.kbuf, (const void*)c.vbuf, (const float*)c.abuf,
             (const float*)c.bbuf, c.pos, c.R);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
         constexpr size_t ssm = gdn::RstepSmem<D, D, C>::BYTES;
@@ -439,9 +441,10 @@ gdn_status_t launch_backward(const BwdArgs& a)
     const int64_t ntasks = a.tot.tasks * a.H;
     if (ntasks > 0) {
         const size_t psm = gdn::PrepCfg<D, D, C>::bytes(a.in_bf16);
-        if (set_smem(gdn::k_bprep<D, C>, psm) != cudaSuccess) return GDN_ERR_CUDA;
-        gdn::k_bprep<D, C><<<(unsigned)ntasks, 256, psm, a.stream>>>(a.k, a.v, a.alpha, a.beta, a.cu, a.ws.t.cto,
-                                                                     a.ws.t.err, a.N, a.H, a.in_bf16, a.ws.prep);
+        auto bprep = a.in_bf16 ? gdn::k_bprep<D, C, true> : gdn::k_bprep<D, C, false>;
+        if (set_smem(bprep, psm) != cudaSuccess) return GDN_ERR_CUDA;
+        bprep<<<(unsigned)ntasks, 256, psm, a.stream>>>(a.k, a.v, a.alpha, a.beta, a.cu, a.ws.t.cto, a.ws.t.err,
+                                                        a.N, a.H, a.ws.prep);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
     }
     mark(a.events, 2, a.stream);

@@ -235,13 +235,14 @@ __device__ __forceinline__ float bg_warp_sum8(float (&x)[8])
 
 // The chunk-local operands of every (chunk, head) task, chunks of C tokens
 // padded as k_bgrad pads them: P_chunk part 1 (chunk_prep: u0, w and T) and
-// the gates, into pw + task * BgCfg::PW.  One CTA per task.
-template <int D, int C>
+// the gates, into pw + task * BgCfg::PW.  One CTA per task; BF: bf16 inputs.
+template <int D, int C, bool BF>
 __global__ void __launch_bounds__(256, 3)
 k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
         const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ cto,
-        const int32_t* err, int N, int H, int in_bf16, float* __restrict__ pw)
+        const int32_t* err, int N, int H, float* __restrict__ pw)
 {
+    constexpr int in_bf16 = BF;
     using P = PrepCfg<D, D, C>;
     if (*reinterpret_cast<volatile const int32_t*>(err)) return;
     extern __shared__ float4 smem_f4[];
@@ -274,7 +275,7 @@ k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __r
     cp_async_wait_all();
     __syncthreads();
     float* out = pw + task * BgCfg<D, C>::PW;
-    chunk_prep<D, D, C>(b, in_bf16, out, D, out + C * D, D, nullptr);
+    chunk_prep<D, D, C, BF>(b, out, D, out + C * D, D, nullptr);
     float* oT = out + 2 * C * D;
     for (int e = tid; e < C * C; e += blockDim.x) {
         const int t = e / C, s = e % C;

@@ -264,7 +264,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
-        chunk_prep<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, us, DV, wx, Sm::WXS, dCs);
+        chunk_prep_any<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, us, DV, wx, Sm::WXS, dCs);
         tc_stage_w<DK, DV, C>(wx, Sm::WXS, Whi, Wlo, threadIdx.x, blockDim.x);
         tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
         float* Sg = S_b + (int64_t)nh * DV * DK;
@@ -304,11 +304,12 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
 //     pos = 0, rscale = 1.
 // The device functions and their operands are the single kernel's, so the
 // results are bit for bit the same.
-template <int DK, int DV, int C>
+template <int DK, int DV, int C, bool BF>
 __global__ void __launch_bounds__(256, 3)
-k_dec_rprep(int NH, int in_bf16, const void* kbuf, const void* vbuf, const float* abuf, const float* bbuf,
+k_dec_rprep(int NH, const void* kbuf, const void* vbuf, const float* abuf, const float* bbuf,
             const int32_t* pos, float* R)
 {
+    constexpr int in_bf16 = BF;
     static_assert(2 * C * DV <= DV * DK && DK == DV, "u0 and w fit in one state");
     const int nh = blockIdx.x;
     if (nh >= NH || pos[nh] != C) return;
@@ -320,7 +321,7 @@ k_dec_rprep(int NH, int in_bf16, const void* kbuf, const void* vbuf, const float
     cp_async_wait_all();
     __syncthreads();
     float* out = R + (int64_t)nh * DV * DK;
-    chunk_prep<DK, DV, C>(prep_bufs<DK, DV, C>(base, in_bf16), in_bf16, out, DV, out + C * DV, DK, nullptr);
+    chunk_prep<DK, DV, C, BF>(prep_bufs<DK, DV, C>(base, in_bf16), out, DV, out + C * DV, DK, nullptr);
 }
 
 template <int DK, int DV, int C>

@@ -85,10 +85,11 @@ __device__ __forceinline__ PrepBufs prep_bufs(unsigned char* base, int bf16)
     return b;
 }
 
-__device__ __forceinline__ float ld_raw(const unsigned char* rowp, int col, int bf16)
+template <bool BF>
+__device__ __forceinline__ float ld_raw(const unsigned char* rowp, int col)
 {
-    return bf16 ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(rowp)[col] << 16)
-                : reinterpret_cast<const float*>(rowp)[col];
+    if constexpr (BF) return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(rowp)[col] << 16);
+    else return reinterpret_cast<const float*>(rowp)[col];
 }
 
 // 3xTF32 products of one m16n8 tile over k blocks [kb0, kb1): fa(kb, i) gives
@@ -112,27 +113,33 @@ __device__ __forceinline__ void mma3_tile(float (&lh)[4], float (&hl)[4], float 
 __device__ __forceinline__ float sum3(float lh, float hl, float hh) { return fadd(fadd(lh, hl), hh); }
 
 // P_chunk part 1 of one chunk by one CTA (blockDim.x >= max(C + 1, 32 * (C / 16))).
-// The caller has staged the raw k, v rows and the gates (b.as, b.bs) and
-// synchronised.  Writes u0 -> uout[t * ldu + i], w -> wout[t * ldw + j] (any
-// address space) and, when dCout is non-null, D[C][s] -> dCout[s].  Ends with
-// a barrier.
-template <int DK, int DV, int C>
-__device__ __forceinline__ void chunk_prep(const PrepBufs& b, int bf16, float* uout, int ldu, float* wout, int ldw,
+// BF: the raw rows are bf16 (else fp32).  The caller has staged the raw k, v
+// rows and the gates (b.as, b.bs) and synchronised.  Writes u0 -> uout[t * ldu
+// + i], w -> wout[t * ldw + j] (any address space) and, when dCout is
+// non-null, D[C][s] -> dCout[s].  Ends with a barrier.
+template <int DK, int DV, int C, bool BF>
+__device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int ldu, float* wout, int ldw,
                                            float* dCout)
 {
     using P = PrepCfg<DK, DV, C>;
     constexpr int MS = P::MS, SS = P::SS, NB = P::NB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const int nwarps = blockDim.x >> 5;
-    const int krb = P::krb(bf16), vrb = P::vrb(bf16);
+    constexpr int krb = P::krb(BF), vrb = P::vrb(BF);
     float* TD = b.TD;
-    // decay products: column s is the chain D[t][s] = D[t-1][s] * alpha_t
+    // decay products: column s is the chain D[t][s] = D[t-1][s] * alpha_t.  The
+    // loop over t is unrolled with s as a predicate, so the alpha loads are
+    // independent of the chain and issue ahead of it.
     for (int s = threadIdx.x; s <= C; s += blockDim.x) {
         float d = 1.0f;
         TD[s * MS + s] = d;
-        for (int t = s + 1; t <= C; ++t) {
-            d = fmul(d, b.as[t - 1]);
-            TD[t * MS + s] = d;
+#pragma unroll
+        for (int t = 1; t <= C; ++t) {
+            const float a = b.as[t - 1];
+            if (t > s) {
+                d = fmul(d, a);
+                TD[t * MS + s] = d;
+            }
         }
     }
     __syncthreads();
@@ -154,10 +161,10 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, int bf16, float* u
 #pragma unroll 4
             for (int kb = 0; kb < DK / 8; ++kb) {
                 const int k0 = kb * 8;
-                const float a0 = ld_raw(ra, k0 + t4, bf16), a1 = ld_raw(rb, k0 + t4, bf16);
-                const float a2 = ld_raw(ra, k0 + t4 + 4, bf16), a3 = ld_raw(rb, k0 + t4 + 4, bf16);
-                const float b0 = ld_raw(rn, k0 + t4, bf16), b1 = ld_raw(rn, k0 + t4 + 4, bf16);
-                if (bf16) {
+                const float a0 = ld_raw<BF>(ra, k0 + t4), a1 = ld_raw<BF>(rb, k0 + t4);
+                const float a2 = ld_raw<BF>(ra, k0 + t4 + 4), a3 = ld_raw<BF>(rb, k0 + t4 + 4);
+                const float b0 = ld_raw<BF>(rn, k0 + t4), b1 = ld_raw<BF>(rn, k0 + t4 + 4);
+                if constexpr (BF) {
                     const uint32_t ah[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
                                             __float_as_uint(a3)};
                     const uint32_t bh[2] = {__float_as_uint(b0), __float_as_uint(b1)};
@@ -175,8 +182,8 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, int bf16, float* u
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int tau = r0 + g + (c >> 1) * 8, sig = n0 + 2 * t4 + (c & 1);
-                const float G = bf16 ? fadd(fadd(acc[0][c], acc[1][c]), fadd(acc[2][c], acc[3][c]))
-                                     : fadd(fadd(acc[0][c], acc[1][c]), acc[2][c]);
+                const float G = BF ? fadd(fadd(acc[0][c], acc[1][c]), fadd(acc[2][c], acc[3][c]))
+                                   : fadd(fadd(acc[0][c], acc[1][c]), acc[2][c]);
                 if (sig < tau) b.A[tau * MS + sig] = fmul(b.bs[tau], fmul(TD[(tau + 1) * MS + (sig + 1)], G));
             }
         }
@@ -290,12 +297,12 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, int bf16, float* u
                         uint32_t bh[2], bl[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const float x = ld_raw(src + (size_t)(8 * kb + t4 + 4 * u) * rb, 8 * cb + g, bf16);
-                            if (bf16) bh[u] = __float_as_uint(x);
+                            const float x = ld_raw<BF>(src + (size_t)(8 * kb + t4 + 4 * u) * rb, 8 * cb + g);
+                            if constexpr (BF) bh[u] = __float_as_uint(x);
                             else tf32_split(x, bh[u], bl[u]);
                         }
                         mma_tf32(lh[j], al, bh);
-                        if (!bf16) mma_tf32(hl[j], ah, bl);
+                        if constexpr (!BF) mma_tf32(hl[j], ah, bl);
                         mma_tf32(hh[j], ah, bh);
                     }
                 }
@@ -311,7 +318,7 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, int bf16, float* u
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const int c = 2 * hv + e;
-                            x[e] = bf16 ? fadd(lh[j][c], hh[j][c]) : sum3(lh[j][c], hl[j][c], hh[j][c]);
+                            x[e] = BF ? fadd(lh[j][c], hh[j][c]) : sum3(lh[j][c], hl[j][c], hh[j][c]);
                         }
                         *reinterpret_cast<float2*>(out + (int64_t)t * ld + col) = make_float2(x[0], x[1]);
                     }
@@ -352,14 +359,25 @@ __device__ __forceinline__ void prep_stage(unsigned char* base, const void* k, c
     }
 }
 
-// P_chunk part 1 for every full chunk: one CTA per (full chunk, head).
+// chunk_prep with the input dtype chosen at run time (both forms inlined).
 template <int DK, int DV, int C>
+__device__ __forceinline__ void chunk_prep_any(const PrepBufs& b, int bf16, float* uout, int ldu, float* wout,
+                                               int ldw, float* dCout)
+{
+    if (bf16) chunk_prep<DK, DV, C, true>(b, uout, ldu, wout, ldw, dCout);
+    else chunk_prep<DK, DV, C, false>(b, uout, ldu, wout, ldw, dCout);
+}
+
+// P_chunk part 1 for every full chunk: one CTA per (full chunk, head).  BF:
+// bf16 inputs (else fp32), fixed at compile time.
+template <int DK, int DV, int C, bool BF>
 __global__ void __launch_bounds__(256, 3)
 k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
        const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ fco,
-       const int32_t* __restrict__ err, int N, int H, int in_bf16,
+       const int32_t* __restrict__ err, int N, int H,
        float* __restrict__ w_ws, float* __restrict__ u_ws, float* __restrict__ dC_ws)
 {
+    constexpr int in_bf16 = BF;
     if (__ldg(err)) return;
     extern __shared__ float4 smem_f4[];
     unsigned char* base = reinterpret_cast<unsigned char*>(smem_f4);
@@ -372,8 +390,8 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
     cp_async_wait_all();
     __syncthreads();
     const PrepBufs b = prep_bufs<DK, DV, C>(base, in_bf16);
-    chunk_prep<DK, DV, C>(b, in_bf16, u_ws + (int64_t)task * C * DV, DV, w_ws + (int64_t)task * C * DK, DK,
-                          dC_ws + (int64_t)task * (C + 4));
+    chunk_prep<DK, DV, C, BF>(b, u_ws + (int64_t)task * C * DV, DV, w_ws + (int64_t)task * C * DK, DK,
+                              dC_ws + (int64_t)task * (C + 4));
 }
 
 }  // namespace gdn
