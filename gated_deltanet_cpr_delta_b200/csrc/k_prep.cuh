@@ -127,6 +127,18 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
     const int nwarps = blockDim.x >> 5;
     constexpr int krb = P::krb(BF), vrb = P::vrb(BF);
     float* TD = b.TD;
+    if constexpr (BF) {
+        // Re-lay each 8-element block of the raw k rows as (0,4,1,5,2,6,3,7):
+        // 32-bit word j then holds elements j and j + 4, the pair one lane of
+        // an m16n8k8 fragment takes, so one load serves both.
+        unsigned char* kr = const_cast<unsigned char*>(b.kr);
+        for (int e = threadIdx.x; e < C * (DK / 8); e += blockDim.x) {
+            uint4* p = reinterpret_cast<uint4*>(kr + (size_t)(e / (DK / 8)) * krb + 16 * (e % (DK / 8)));
+            const uint4 x = *p;
+            *p = make_uint4(__byte_perm(x.x, x.z, 0x5410), __byte_perm(x.x, x.z, 0x7632),
+                            __byte_perm(x.y, x.w, 0x5410), __byte_perm(x.y, x.w, 0x7632));
+        }
+    }
     // decay products: column s is the chain D[t][s] = D[t-1][s] * alpha_t.  The
     // loop over t is unrolled with s as a predicate, so the alpha loads are
     // independent of the chain and issue ahead of it.
@@ -143,49 +155,64 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
         }
     }
     __syncthreads();
-    // Gram on the tensor cores, the (m16, n8) tiles of the lower triangle;
+    // Gram on the tensor cores, by 16 x 16 blocks (m, p <= m) of the lower
+    // triangle, each two (m16, n8) tiles that share the A fragment;
     // A[t][s] = beta_t * (D[t][s] * G[t][s]) (1-indexed t, s)
     {
-        constexpr int MT = C / 16, NTILE = MT * (MT + 1);  // tile (m, q) with q <= 2m+1
-        for (int tile = warp; tile < NTILE; tile += nwarps) {
+        constexpr int MT = C / 16, NBLK = MT * (MT + 1) / 2;
+        for (int blk = warp; blk < NBLK; blk += nwarps) {
             int m = 0;
-            while ((m + 1) * (m + 2) <= tile) ++m;
-            const int q = tile - m * (m + 1);
-            const int r0 = m * 16, n0 = q * 8;
+            while ((m + 1) * (m + 2) / 2 <= blk) ++m;
+            const int p = blk - m * (m + 1) / 2;
+            const int r0 = m * 16;
             const unsigned char* ra = b.kr + (size_t)(r0 + g) * krb;
             const unsigned char* rb = b.kr + (size_t)(r0 + g + 8) * krb;
-            const unsigned char* rn = b.kr + (size_t)(n0 + g) * krb;
-            float acc[4][4];
+            float acc[2][4][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[h][u][0] = acc[h][u][1] = acc[h][u][2] = acc[h][u][3] = 0.f;
 #pragma unroll 4
             for (int kb = 0; kb < DK / 8; ++kb) {
                 const int k0 = kb * 8;
-                const float a0 = ld_raw<BF>(ra, k0 + t4), a1 = ld_raw<BF>(rb, k0 + t4);
-                const float a2 = ld_raw<BF>(ra, k0 + t4 + 4), a3 = ld_raw<BF>(rb, k0 + t4 + 4);
-                const float b0 = ld_raw<BF>(rn, k0 + t4), b1 = ld_raw<BF>(rn, k0 + t4 + 4);
-                if constexpr (BF) {
-                    const uint32_t ah[4] = {__float_as_uint(a0), __float_as_uint(a1), __float_as_uint(a2),
-                                            __float_as_uint(a3)};
-                    const uint32_t bh[2] = {__float_as_uint(b0), __float_as_uint(b1)};
-                    mma_tf32(acc[kb & 3], ah, bh);
+                if constexpr (BF) {  // re-laid rows: word k0/2 + t4 holds elements k0 + t4 and k0 + t4 + 4
+                    const uint32_t xa = reinterpret_cast<const uint32_t*>(ra)[k0 / 2 + t4];
+                    const uint32_t xb = reinterpret_cast<const uint32_t*>(rb)[k0 / 2 + t4];
+                    const uint32_t ah[4] = {xa << 16, xb << 16, xa & 0xffff0000u, xb & 0xffff0000u};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t xn = reinterpret_cast<const uint32_t*>(
+                            b.kr + (size_t)(16 * p + 8 * h + g) * krb)[k0 / 2 + t4];
+                        const uint32_t bh[2] = {xn << 16, xn & 0xffff0000u};
+                        mma_tf32(acc[h][kb & 3], ah, bh);
+                    }
                 } else {
-                    uint32_t ah[4], al[4], bh[2], bl[2];
-                    tf32_split(a0, ah[0], al[0]); tf32_split(a1, ah[1], al[1]);
-                    tf32_split(a2, ah[2], al[2]); tf32_split(a3, ah[3], al[3]);
-                    tf32_split(b0, bh[0], bl[0]); tf32_split(b1, bh[1], bl[1]);
-                    mma_tf32(acc[0], al, bh);
-                    mma_tf32(acc[1], ah, bl);
-                    mma_tf32(acc[2], ah, bh);
+                    uint32_t ah[4], al[4];
+                    tf32_split(ld_raw<BF>(ra, k0 + t4), ah[0], al[0]);
+                    tf32_split(ld_raw<BF>(rb, k0 + t4), ah[1], al[1]);
+                    tf32_split(ld_raw<BF>(ra, k0 + t4 + 4), ah[2], al[2]);
+                    tf32_split(ld_raw<BF>(rb, k0 + t4 + 4), ah[3], al[3]);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const unsigned char* rn = b.kr + (size_t)(16 * p + 8 * h + g) * krb;
+                        uint32_t bh[2], bl[2];
+                        tf32_split(ld_raw<BF>(rn, k0 + t4), bh[0], bl[0]);
+                        tf32_split(ld_raw<BF>(rn, k0 + t4 + 4), bh[1], bl[1]);
+                        mma_tf32(acc[h][0], al, bh);
+                        mma_tf32(acc[h][1], ah, bl);
+                        mma_tf32(acc[h][2], ah, bh);
+                    }
                 }
             }
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int tau = r0 + g + (c >> 1) * 8, sig = n0 + 2 * t4 + (c & 1);
-                const float G = BF ? fadd(fadd(acc[0][c], acc[1][c]), fadd(acc[2][c], acc[3][c]))
-                                   : fadd(fadd(acc[0][c], acc[1][c]), acc[2][c]);
-                if (sig < tau) b.A[tau * MS + sig] = fmul(b.bs[tau], fmul(TD[(tau + 1) * MS + (sig + 1)], G));
-            }
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int tau = r0 + g + (c >> 1) * 8, sig = 16 * p + 8 * h + 2 * t4 + (c & 1);
+                    const float G = BF ? fadd(fadd(acc[h][0][c], acc[h][1][c]), fadd(acc[h][2][c], acc[h][3][c]))
+                                       : fadd(fadd(acc[h][0][c], acc[h][1][c]), acc[h][2][c]);
+                    if (sig < tau) b.A[tau * MS + sig] = fmul(b.bs[tau], fmul(TD[(tau + 1) * MS + (sig + 1)], G));
+                }
         }
     }
     for (int t = threadIdx.x; t < C; t += blockDim.x) {  // D[t][0] and gamma_t = beta_t * D[t][0], t = 1..C
@@ -273,6 +300,8 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
         const float* scale = half ? b.gam : b.bs;
         const unsigned char* src = half ? b.kr : b.vr;
         const int rb = half ? krb : vrb;
+        // column 8 cb + g of a k row sits at 8 cb + pg once the rows are re-laid
+        const int pg = (BF && half) ? 2 * (g & 3) + (g >> 2) : g;
         float* out = half ? wout : uout;
         const int ld = half ? ldw : ldu;
 #pragma unroll 1
@@ -297,7 +326,7 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
                         uint32_t bh[2], bl[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const float x = ld_raw<BF>(src + (size_t)(8 * kb + t4 + 4 * u) * rb, 8 * cb + g);
+                            const float x = ld_raw<BF>(src + (size_t)(8 * kb + t4 + 4 * u) * rb, 8 * cb + pg);
                             if constexpr (BF) bh[u] = __float_as_uint(x);
                             else tf32_split(x, bh[u], bl[u]);
                         }
