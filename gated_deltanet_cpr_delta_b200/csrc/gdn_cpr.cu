@@ -332,7 +332,7 @@ gdn_status_t launch_decode(const DecArgs& a)
         if (set_smem(rprep, psm) != cudaSuccess) return GDN_ERR_CUDA;
         rprep<<<(unsigned)NH, 256, psm, a.stream>>>(
             (int)NH, (const void*)c.kbuf, (const void*)c.vbuf, (const float*)c.abuf,
-            (const float*)c.bbuf, c.pos, c.R, c.status);
+            (const float*)c.bbuf, c.pos, c.R);
         if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
         constexpr size_t ssm = gdn::RstepSmem<D, D, C>::BYTES;
         if (set_smem(gdn::k_dec_rstep<D, D, C>, ssm) != cudaSuccess) return GDN_ERR_CUDA;
@@ -489,7 +489,7 @@ gdn_status_t launch_backward(const BwdArgs& a)
 
 extern "C" {
 
-const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v7/NL8/ptok-scaled/prep-inverse-tf32x3-products-tcgen05/chain-tcgen05-tf32x3-1acc"; }
+const char* gdn_contract_id(void) { return "gdn-cpr-schedule-v6/NL8/ptok-scaled/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3-1acc"; }
 
 const char* gdn_status_string(gdn_status_t s)
 {

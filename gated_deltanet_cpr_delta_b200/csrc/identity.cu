@@ -158,10 +158,9 @@ const char* kPolicy =
     "  diagonal blocks by substitution, T[i][i] = 1, T[t][i] = fma chain over s = i..t-1 ascending of\n"
     "  (-A[t][s])*T[s][i] from 0; block (i, j < i) by distance i - j ascending: M = A[i][j..i-1] T[j..i-1][j],\n"
     "  T[i][j] = -(T[i][i] M), both by mma.sync.m16n8k8 tf32 split products (lo.hi + hi.lo) + hi.hi;\n"
-    "  gamma_t = beta_t*D[t][0]; u0^T = V^T (T diag(beta))^T, w^T = K^T (T diag(gamma))^T by tcgen05.mma\n"
-    "  kind::tf32, M = 128 feature rows, A (V^T, K^T) in tensor memory, B K-major in shared memory, N = 16:\n"
-    "  per 16-token row block r of T one fp32 accumulator over K blocks 0..2r+1 ascending, fed\n"
-    "  V.T_lo ; V.T_hi for bf16 inputs (V, K exact), else V_hi.T_lo ; V_lo.T_hi ; V_hi.T_hi\n"
+    "  gamma_t = beta_t*D[t][0]; u0 = (T diag(beta)) V, w = (T diag(gamma)) K by mma.sync.m16n8k8 tf32,\n"
+    "  row block r over K blocks 0..2r+1 ascending: bf16 inputs (V, K exact) lo.V + hi.V,\n"
+    "  else (lo.hi + hi.lo) + hi.hi\n"
     "P_chunk part 2: tcgen05.mma kind::tf32, M = 128, A in tensor memory, B K-major in shared memory,\n"
     "  fp32 accumulate, one accumulator per phase fed in this order: lo.hi over K blocks of 8 ascending,\n"
     "  then hi.lo, then hi.hi;\n"

@@ -240,7 +240,7 @@ template <int D, int C, bool BF>
 __global__ void __launch_bounds__(256, 3)
 k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
         const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ cto,
-        int32_t* err, int N, int H, float* __restrict__ pw)
+        const int32_t* err, int N, int H, float* __restrict__ pw)
 {
     constexpr int in_bf16 = BF;
     using P = PrepCfg<D, D, C>;
@@ -275,11 +275,7 @@ k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __r
     cp_async_wait_all();
     __syncthreads();
     float* out = pw + task * BgCfg<D, C>::PW;
-    const uint32_t tbase = prep_tc_open<D, D, C, BF>(b);
-    uint32_t parity = 0;
-    if (!chunk_prep<D, D, C, BF>(b, tbase, b.mbar, parity, out, D, out + C * D, D, nullptr) && tid == 0)
-        record_error(err, GDN_ERR_TIMEOUT);
-    prep_tc_close<D, D, C, BF>(tbase);
+    chunk_prep<D, D, C, BF>(b, out, D, out + C * D, D, nullptr);
     float* oT = out + 2 * C * D;
     for (int e = tid; e < C * C; e += blockDim.x) {
         const int t = e / C, s = e % C;

@@ -264,9 +264,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
-        if (!chunk_prep_any<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, tbase, mbar, parity, us, DV, wx,
-                                       Sm::WXS, dCs))
-            break;
+        chunk_prep_any<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, us, DV, wx, Sm::WXS, dCs);
         tc_stage_w<DK, DV, C>(wx, Sm::WXS, Whi, Wlo, threadIdx.x, blockDim.x);
         tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
         float* Sg = S_b + (int64_t)nh * DV * DK;
@@ -309,7 +307,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
 template <int DK, int DV, int C, bool BF>
 __global__ void __launch_bounds__(256, 3)
 k_dec_rprep(int NH, const void* kbuf, const void* vbuf, const float* abuf, const float* bbuf,
-            int32_t* pos, float* R, int32_t* status)
+            const int32_t* pos, float* R)
 {
     constexpr int in_bf16 = BF;
     static_assert(2 * C * DV <= DV * DK && DK == DV, "u0 and w fit in one state");
@@ -323,15 +321,7 @@ k_dec_rprep(int NH, const void* kbuf, const void* vbuf, const float* abuf, const
     cp_async_wait_all();
     __syncthreads();
     float* out = R + (int64_t)nh * DV * DK;
-    const PrepBufs b = prep_bufs<DK, DV, C>(base, in_bf16);
-    const uint32_t tbase = prep_tc_open<DK, DV, C, BF>(b);
-    uint32_t parity = 0;
-    if (!chunk_prep<DK, DV, C, BF>(b, tbase, b.mbar, parity, out, DV, out + C * DV, DK, nullptr) &&
-        threadIdx.x == 0) {
-        pos[nh] = -1;  // not resynced: the step kernel skips the pair and the next token step refuses it
-        record_error(status, GDN_ERR_TIMEOUT);
-    }
-    prep_tc_close<DK, DV, C, BF>(tbase);
+    chunk_prep<DK, DV, C, BF>(prep_bufs<DK, DV, C>(base, in_bf16), out, DV, out + C * DV, DK, nullptr);
 }
 
 template <int DK, int DV, int C>

@@ -27,7 +27,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_contract_id(lib):
-    assert gdn.gdn_contract_id() == "gdn-cpr-schedule-v7/NL8/ptok-scaled/prep-inverse-tf32x3-products-tcgen05/chain-tcgen05-tf32x3-1acc"
+    assert gdn.gdn_contract_id() == "gdn-cpr-schedule-v6/NL8/ptok-scaled/prep-inverse-mma-tf32x3/chain-tcgen05-tf32x3-1acc"
     assert lib.gdn_status_string(0) == b"ok"
     assert lib.gdn_status_string(4) == b"workspace missing or too small"
 
