@@ -237,7 +237,7 @@ __device__ __forceinline__ float bg_warp_sum8(float (&x)[8])
 // padded as k_bgrad pads them: P_chunk part 1 (chunk_prep: u0, w and T) and
 // the gates, into pw + task * BgCfg::PW.  One CTA per task; BF: bf16 inputs.
 template <int D, int C, bool BF>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256, PrepCfg<D, D, C>::ctas_per_sm(BF))
 k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
         const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ cto,
         const int32_t* err, int N, int H, float* __restrict__ pw)
@@ -258,8 +258,9 @@ k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __r
     auto trow = [&](int t) { return (tok0 + t) * H + h; };
     const PrepBufs b = prep_bufs<D, D, C>(reinterpret_cast<unsigned char*>(smem_f4), in_bf16);
     const int esz = in_bf16 ? 2 : 4, pk = D * esz / 16;
-    for (int e = tid; e < C * 2 * pk; e += blockDim.x) {
-        const int t = e / (2 * pk), pc = e % (2 * pk), isv = pc >= pk, p = pc % pk;
+    const int nparts = P::v_in_a(in_bf16) ? 1 : 2;  // k rows, and v rows unless chunk_prep stages them
+    for (int e = tid; e < C * nparts * pk; e += blockDim.x) {
+        const int t = e / (nparts * pk), pc = e % (nparts * pk), isv = pc >= pk, p = pc % pk;
         unsigned char* dst = const_cast<unsigned char*>(isv ? b.vr + (size_t)t * P::vrb(in_bf16)
                                                              : b.kr + (size_t)t * P::krb(in_bf16)) + 16 * p;
         if (t < len)
@@ -275,7 +276,7 @@ k_bprep(const void* __restrict__ k, const void* __restrict__ v, const float* __r
     cp_async_wait_all();
     __syncthreads();
     float* out = pw + task * BgCfg<D, C>::PW;
-    chunk_prep<D, D, C, BF>(b, out, D, out + C * D, D, nullptr);
+    chunk_prep<D, D, C, BF>(b, VSrc{v, tok0, H, h, len}, out, D, out + C * D, D, nullptr);
     float* oT = out + 2 * C * D;
     for (int e = tid; e < C * C; e += blockDim.x) {
         const int t = e / C, s = e % C;

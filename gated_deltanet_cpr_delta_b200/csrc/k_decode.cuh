@@ -264,7 +264,8 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
-        chunk_prep_any<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, us, DV, wx, Sm::WXS, dCs);
+        chunk_prep_any<DK, DV, C>(prep_bufs<DK, DV, C>(r1, in_bf16), in_bf16, VSrc{vbuf, (int64_t)nh * C, 1, 0, C},
+                                  us, DV, wx, Sm::WXS, dCs);
         tc_stage_w<DK, DV, C>(wx, Sm::WXS, Whi, Wlo, threadIdx.x, blockDim.x);
         tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
         float* Sg = S_b + (int64_t)nh * DV * DK;
@@ -295,7 +296,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
 // d x d state): on a step where buffers fill, the running state R of those
 // pairs is dead until the resync rewrites it, so it holds their P_chunk
 // part 1 operands in between.
-//   k_dec_rprep: one CTA per pair, 3 CTAs per SM; a pair at pos == C runs
+//   k_dec_rprep: one CTA per pair, 3-4 CTAs per SM; a pair at pos == C runs
 //     chunk_prep on its buffer: u0 -> R[0 .. C*d), w -> R[C*d .. 2*C*d).
 //   k_dec_rstep: persistent, one CTA per SM; for each pair at pos == C the
 //     tcgen05 step (tc_step) from S_b with w, k^T (from the buffer), u0
@@ -305,7 +306,7 @@ k_dec_resync(int NH, int in_bf16, float* S_b, float* R, float* rscale, const voi
 // The device functions and their operands are the single kernel's, so the
 // results are bit for bit the same.
 template <int DK, int DV, int C, bool BF>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256, PrepCfg<DK, DV, C>::ctas_per_sm(BF))
 k_dec_rprep(int NH, const void* kbuf, const void* vbuf, const float* abuf, const float* bbuf,
             const int32_t* pos, float* R)
 {
@@ -321,7 +322,8 @@ k_dec_rprep(int NH, const void* kbuf, const void* vbuf, const float* abuf, const
     cp_async_wait_all();
     __syncthreads();
     float* out = R + (int64_t)nh * DV * DK;
-    chunk_prep<DK, DV, C, BF>(prep_bufs<DK, DV, C>(base, in_bf16), out, DV, out + C * DV, DK, nullptr);
+    chunk_prep<DK, DV, C, BF>(prep_bufs<DK, DV, C>(base, in_bf16), VSrc{vbuf, (int64_t)nh * C, 1, 0, C}, out, DV,
+                              out + C * DV, DK, nullptr);
 }
 
 template <int DK, int DV, int C>

@@ -35,21 +35,51 @@ template <int DK, int DV, int C>
 struct PrepCfg {
     static constexpr int NB = C / 16;          // 16-token blocks
     static constexpr int MS = C + 4;           // row stride of A, T and the decays (floats)
-    static constexpr int SS = 16 + 4;          // row stride of the 16 x 16 scratch blocks
     static constexpr int NCOL = DV + DK;       // columns of [u0 | w]
     // raw input rows, in the input dtype, padded by 16 bytes per row: the row
     // stride is 4 words mod 32, which keeps the fragment reads conflict-free
     __host__ __device__ static constexpr int krb(int bf16) { return DK * (bf16 ? 2 : 4) + 16; }
     __host__ __device__ static constexpr int vrb(int bf16) { return DV * (bf16 ? 2 : 4) + 16; }
-    // float offsets of the scratch that follows the raw rows
+    // float offsets of the scratch that follows the raw rows: A | TD | small.
+    // The off-diagonal steps of T keep their 16 x 16 intermediates M_j in A's
+    // unused upper triangle (block (j, NB-1)).
     static constexpr int A_FL = C * MS;
     static constexpr int TD_FL = (C + 1) * MS;
-    static constexpr int M_FL = (NB > 1 ? NB - 1 : 1) * 16 * SS;
     static constexpr int SMALL_FL = 5 * (C + 4);  // d0, dC, alpha, beta, gamma
-    static constexpr int SCRATCH_FL = A_FL + TD_FL + M_FL + SMALL_FL;
-    __host__ __device__ static constexpr size_t raw_bytes(int bf16) { return (size_t)C * (krb(bf16) + vrb(bf16)); }
+    static constexpr int SCRATCH_FL = A_FL + TD_FL + SMALL_FL;
+    // bf16 v rows that fit in A's region go there once A is dead (chunk_prep
+    // stages them after T is complete): v is needed only by the products
+    __host__ __device__ static constexpr bool v_in_a(int bf16) { return bf16 && C * vrb(bf16) <= 4 * A_FL; }
+    __host__ __device__ static constexpr size_t raw_bytes(int bf16)
+    {
+        return (size_t)C * krb(bf16) + (v_in_a(bf16) ? 0 : (size_t)C * vrb(bf16));
+    }
     __host__ __device__ static constexpr size_t bytes(int bf16) { return raw_bytes(bf16) + 4 * (size_t)SCRATCH_FL; }
+    // CTAs of 256 threads that the shared memory allows per SM (4 needs at most 64 registers a thread)
+    __host__ __device__ static constexpr int ctas_per_sm(int bf16) { return bytes(bf16) + 1024 <= 233472 / 4 ? 4 : 3; }
 };
+
+// Where a chunk's v rows come from: rows (tok0 + t) * H + h of a [T, H, DV]
+// tensor for t < len, zero rows after.
+struct VSrc {
+    const void* v;
+    int64_t tok0;
+    int H, h, len;
+};
+
+template <int DV, int C, bool BF>
+__device__ __forceinline__ void stage_v_rows(const VSrc& s, unsigned char* vr, int vrb, int tid, int nthr)
+{
+    constexpr int esz = BF ? 2 : 4, pv = DV * esz / 16;  // 16-byte pieces per row
+    for (int e = tid; e < C * pv; e += nthr) {
+        const int t = e / pv, pc = e % pv;
+        unsigned char* dst = vr + (size_t)t * vrb + 16 * pc;
+        if (t < s.len)
+            cp_async16(dst, reinterpret_cast<const char*>(s.v) + ((s.tok0 + t) * s.H + s.h) * DV * esz + 16 * pc);
+        else
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
 
 // The shared-memory pieces chunk_prep works on.
 struct PrepBufs {
@@ -57,7 +87,7 @@ struct PrepBufs {
     const unsigned char* vr;  // [C] raw v rows, stride vrb
     float* A;                 // [C][MS]
     float* TD;                // [C+1][MS]: decays, then T
-    float* M;                 // [NB-1][16][SS]
+    float* M;                 // M_j at M + 16 j MS, row stride MS (A's upper triangle)
     float* d0;                // [C]: D[t][0], t = 1..C
     float* dC;                // [C+1]: D[C][s]
     const float* as;          // [C] alpha
@@ -71,12 +101,12 @@ __device__ __forceinline__ PrepBufs prep_bufs(unsigned char* base, int bf16)
     using P = PrepCfg<DK, DV, C>;
     PrepBufs b;
     b.kr = base;
-    b.vr = base + (size_t)C * P::krb(bf16);
     float* f = reinterpret_cast<float*>(base + P::raw_bytes(bf16));
+    b.vr = P::v_in_a(bf16) ? reinterpret_cast<unsigned char*>(f) : base + (size_t)C * P::krb(bf16);
     b.A = f;
     b.TD = f + P::A_FL;
-    b.M = b.TD + P::TD_FL;
-    b.d0 = b.M + P::M_FL;
+    b.M = f + 16 * (P::NB - 1);
+    b.d0 = b.TD + P::TD_FL;
     b.dC = b.d0 + (C + 4);
     float* as = b.dC + (C + 4);
     b.as = as;
@@ -113,16 +143,17 @@ __device__ __forceinline__ void mma3_tile(float (&lh)[4], float (&hl)[4], float 
 __device__ __forceinline__ float sum3(float lh, float hl, float hh) { return fadd(fadd(lh, hl), hh); }
 
 // P_chunk part 1 of one chunk by one CTA (blockDim.x >= max(C + 1, 32 * (C / 16))).
-// BF: the raw rows are bf16 (else fp32).  The caller has staged the raw k, v
-// rows and the gates (b.as, b.bs) and synchronised.  Writes u0 -> uout[t * ldu
-// + i], w -> wout[t * ldw + j] (any address space) and, when dCout is
-// non-null, D[C][s] -> dCout[s].  Ends with a barrier.
+// BF: the raw rows are bf16 (else fp32).  The caller has staged the raw k
+// rows, the v rows unless PrepCfg::v_in_a (then chunk_prep stages them from
+// vs once T is complete) and the gates (b.as, b.bs), and synchronised.
+// Writes u0 -> uout[t * ldu + i], w -> wout[t * ldw + j] (any address space)
+// and, when dCout is non-null, D[C][s] -> dCout[s].  Ends with a barrier.
 template <int DK, int DV, int C, bool BF>
-__device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int ldu, float* wout, int ldw,
-                                           float* dCout)
+__device__ __forceinline__ void chunk_prep(const PrepBufs& b, const VSrc& vs, float* uout, int ldu, float* wout,
+                                           int ldw, float* dCout)
 {
     using P = PrepCfg<DK, DV, C>;
-    constexpr int MS = P::MS, SS = P::SS, NB = P::NB;
+    constexpr int MS = P::MS, NB = P::NB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
     const int nwarps = blockDim.x >> 5;
     constexpr int krb = P::krb(BF), vrb = P::vrb(BF);
@@ -251,7 +282,7 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
     for (int d = 1; d < NB; ++d) {
         const int j = warp;
         const int i = j + d;
-        float* Mj = b.M + j * 16 * SS;
+        float* Mj = b.M + j * 16 * MS;
         if (i < NB) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -264,7 +295,7 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
                           [&](int kb, int u) { return TD[(8 * kb + t4 + u * 4) * MS + n0 + g]; });
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    Mj[(g + (c >> 1) * 8) * SS + 8 * nt + 2 * t4 + (c & 1)] = sum3(lh[c], hl[c], hh[c]);
+                    Mj[(g + (c >> 1) * 8) * MS + 8 * nt + 2 * t4 + (c & 1)] = sum3(lh[c], hl[c], hh[c]);
             }
         }
         __syncwarp();
@@ -276,7 +307,7 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
                           [&](int kb, int u) {
                               return TD[(16 * i + g + (u & 1) * 8) * MS + 16 * i + 8 * kb + t4 + (u >> 1) * 4];
                           },
-                          [&](int kb, int u) { return Mj[(8 * kb + t4 + u * 4) * SS + 8 * nt + g]; });
+                          [&](int kb, int u) { return Mj[(8 * kb + t4 + u * 4) * MS + 8 * nt + g]; });
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     TD[(16 * i + g + (c >> 1) * 8) * MS + 16 * j + 8 * nt + 2 * t4 + (c & 1)] =
@@ -284,6 +315,17 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
             }
         }
         __syncthreads();
+    }
+    if constexpr (P::v_in_a(BF)) {
+        // A is dead: the v rows go to its region.  Only the u0 half (warps
+        // 0-3) reads them, so those 128 threads copy, wait and meet at a
+        // named barrier while the w half starts.
+        if (threadIdx.x < 128) {
+            stage_v_rows<DV, C, BF>(vs, const_cast<unsigned char*>(b.vr), vrb, threadIdx.x, 128);
+            cp_async_commit();
+            cp_async_wait_all();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
     }
     // [u0 | w] on the tensor cores: u0 = (T diag(beta)) V, w = (T diag(gamma)) K
     // with gamma_s = beta_s * D[s][0].  The first half of the warps takes the
@@ -358,9 +400,10 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, float* uout, int l
     __syncthreads();
 }
 
-// Stage one chunk's raw k, v rows (token rows tok0.., head h of [T, H, D]
-// tensors, or of the decode buffers with H = 1) and gates into the layout of
-// prep_bufs, by cp.async; the caller commits, waits and synchronises.
+// Stage one chunk's raw k rows, v rows (unless PrepCfg::v_in_a) and gates
+// (token rows tok0.., head h of [T, H, D] tensors, or of the decode buffers
+// with H = 1) into the layout of prep_bufs, by cp.async; the caller commits,
+// waits and synchronises.
 template <int DK, int DV, int C>
 __device__ __forceinline__ void prep_stage(unsigned char* base, const void* k, const void* v, const float* alpha,
                                            const float* beta, int64_t tok0, int H, int h, int bf16)
@@ -371,8 +414,9 @@ __device__ __forceinline__ void prep_stage(unsigned char* base, const void* k, c
     const int pk = DK * esz / 16, pv = DV * esz / 16;  // 16-byte pieces per row
     unsigned char* kr = const_cast<unsigned char*>(b.kr);
     unsigned char* vr = const_cast<unsigned char*>(b.vr);
-    for (int e = threadIdx.x; e < C * (pk + pv); e += blockDim.x) {
-        const int t = e / (pk + pv), pc = e % (pk + pv);
+    const int pvs = P::v_in_a(bf16) ? 0 : pv;  // v rows staged here unless chunk_prep stages them
+    for (int e = threadIdx.x; e < C * (pk + pvs); e += blockDim.x) {
+        const int t = e / (pk + pvs), pc = e % (pk + pvs);
         const int64_t row = (tok0 + t) * H + h;
         if (pc < pk)
             cp_async16(kr + (size_t)t * P::krb(bf16) + 16 * pc, reinterpret_cast<const char*>(k) + row * DK * esz + 16 * pc);
@@ -390,17 +434,17 @@ __device__ __forceinline__ void prep_stage(unsigned char* base, const void* k, c
 
 // chunk_prep with the input dtype chosen at run time (both forms inlined).
 template <int DK, int DV, int C>
-__device__ __forceinline__ void chunk_prep_any(const PrepBufs& b, int bf16, float* uout, int ldu, float* wout,
-                                               int ldw, float* dCout)
+__device__ __forceinline__ void chunk_prep_any(const PrepBufs& b, int bf16, const VSrc& vs, float* uout, int ldu,
+                                               float* wout, int ldw, float* dCout)
 {
-    if (bf16) chunk_prep<DK, DV, C, true>(b, uout, ldu, wout, ldw, dCout);
-    else chunk_prep<DK, DV, C, false>(b, uout, ldu, wout, ldw, dCout);
+    if (bf16) chunk_prep<DK, DV, C, true>(b, vs, uout, ldu, wout, ldw, dCout);
+    else chunk_prep<DK, DV, C, false>(b, vs, uout, ldu, wout, ldw, dCout);
 }
 
 // P_chunk part 1 for every full chunk: one CTA per (full chunk, head).  BF:
 // bf16 inputs (else fp32), fixed at compile time.
 template <int DK, int DV, int C, bool BF>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256, PrepCfg<DK, DV, C>::ctas_per_sm(BF))
 k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __restrict__ alpha,
        const float* __restrict__ beta, const int32_t* __restrict__ cu, const int32_t* __restrict__ fco,
        const int32_t* __restrict__ err, int N, int H,
@@ -419,8 +463,8 @@ k_prep(const void* __restrict__ k, const void* __restrict__ v, const float* __re
     cp_async_wait_all();
     __syncthreads();
     const PrepBufs b = prep_bufs<DK, DV, C>(base, in_bf16);
-    chunk_prep<DK, DV, C, BF>(b, u_ws + (int64_t)task * C * DV, DV, w_ws + (int64_t)task * C * DK, DK,
-                              dC_ws + (int64_t)task * (C + 4));
+    chunk_prep<DK, DV, C, BF>(b, VSrc{v, tok0, H, h, C}, u_ws + (int64_t)task * C * DV, DV,
+                              w_ws + (int64_t)task * C * DK, DK, dC_ws + (int64_t)task * (C + 4));
 }
 
 }  // namespace gdn
