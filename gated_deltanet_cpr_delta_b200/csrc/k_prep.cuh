@@ -142,7 +142,7 @@ __device__ __forceinline__ void mma3_tile(float (&lh)[4], float (&hl)[4], float 
 
 __device__ __forceinline__ float sum3(float lh, float hl, float hh) { return fadd(fadd(lh, hl), hh); }
 
-// P_chunk part 1 of one chunk by one CTA (blockDim.x >= max(C + 1, 32 * (C / 16))).
+// P_chunk part 1 of one chunk by one CTA of 256 threads.
 // BF: the raw rows are bf16 (else fp32).  The caller has staged the raw k
 // rows, the v rows unless PrepCfg::v_in_a (then chunk_prep stages them from
 // vs once T is complete) and the gates (b.as, b.bs), and synchronised.
@@ -276,16 +276,16 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, const VSrc& vs, fl
         for (int t = 0; t < 16; ++t) TD[(i0 + t) * MS + i] = t > ri ? acc[t] : (t == ri ? 1.0f : 0.0f);
     }
     __syncthreads();
-    // off-diagonal blocks, by distance d below the diagonal: warp j computes
-    // block (i = j + d, j) as  M = A[i-rows][16j, 16i) T[16j, 16i)[j-cols], then
-    // T_ij = -(T_ii M), both on the tensor cores (3xTF32)
+    // off-diagonal blocks, by distance d below the diagonal: block (i = j + d, j)
+    // is M = A[i-rows][16j, 16i) T[16j, 16i)[j-cols], then T_ij = -(T_ii M),
+    // both on the tensor cores (3xTF32).  Each 8-column half nt of the block
+    // needs only its own columns of M, so warp 2 j + nt computes it alone.
     for (int d = 1; d < NB; ++d) {
-        const int j = warp;
+        const int j = warp >> 1, nt = warp & 1;
         const int i = j + d;
         float* Mj = b.M + j * 16 * MS;
         if (i < NB) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            {
                 const int n0 = 16 * j + 8 * nt;
                 float lh[4] = {0.f, 0.f, 0.f, 0.f}, hl[4] = {0.f, 0.f, 0.f, 0.f}, hh[4] = {0.f, 0.f, 0.f, 0.f};
                 mma3_tile(lh, hl, hh, 2 * j, 2 * i,
@@ -297,11 +297,8 @@ __device__ __forceinline__ void chunk_prep(const PrepBufs& b, const VSrc& vs, fl
                 for (int c = 0; c < 4; ++c)
                     Mj[(g + (c >> 1) * 8) * MS + 8 * nt + 2 * t4 + (c & 1)] = sum3(lh[c], hl[c], hh[c]);
             }
-        }
-        __syncwarp();
-        if (i < NB) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            __syncwarp();
+            {
                 float lh[4] = {0.f, 0.f, 0.f, 0.f}, hl[4] = {0.f, 0.f, 0.f, 0.f}, hh[4] = {0.f, 0.f, 0.f, 0.f};
                 mma3_tile(lh, hl, hh, 0, 2,
                           [&](int kb, int u) {
