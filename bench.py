@@ -111,7 +111,7 @@ TF32_PER_BF16 = 1.1 / 2.25
 NCU_TRAFFIC = {
     ("k_chain_tok", "6ffe60d00cafadbf"): 787287552 + 328396544,
     ("k_dec_tok", "aa7d300e7bc460f2"): 135931904 + 75910656,
-    ("k_bgrad", "5dea3500210019e4"): 2768417792 + 2326212864,
+    ("k_bgrad", "0a3b676036fe7e31"): 2770113280 + 2330992128,
 }
 
 KERNEL_SOURCES = {
