@@ -111,11 +111,15 @@ def test_forward_vs_schedule_model_and_oracle(d, C, dtype):
     tol_check(dtype, st.cpu().numpy(), r["states"], "states")
 
 
-@pytest.mark.parametrize("d,C,Lp,steps", [(16, 16, 0, 40), (16, 16, 21, 50), (64, 32, 64, 70),
-                                          (128, 64, 130, 140), (128, 16, 16, 40)])
-def test_decode_equals_prefill_bitwise(d, C, Lp, steps):
+# 2C > d runs the resync as one kernel (k_dec_resync), 2C <= d as two (k_dec_rprep, k_dec_rstep)
+@pytest.mark.parametrize("d,C,Lp,steps,dtype", [(16, 16, 0, 40, "bf16"), (16, 16, 21, 50, "bf16"),
+                                                (64, 32, 64, 70, "bf16"), (128, 64, 130, 140, "bf16"),
+                                                (128, 16, 16, 40, "bf16"), (64, 64, 70, 140, "bf16"),
+                                                (64, 64, 70, 140, "f32"), (32, 32, 10, 80, "f32"),
+                                                (128, 64, 60, 80, "f32")])
+def test_decode_equals_prefill_bitwise(d, C, Lp, steps, dtype):
     N, H = 3, 2
-    b = synth.make_batch(200 + d, [Lp + steps] * N, H, d, d, "bf16")
+    b = synth.make_batch(200 + d, [Lp + steps] * N, H, d, d, dtype)
     full_o, full_st, full_c = fwd(b, C, torch.float32, cache=True)
     cu = b.cu_seqlens
     if Lp > 0:
@@ -124,7 +128,7 @@ def test_decode_equals_prefill_bitwise(d, C, Lp, steps):
                           (np.arange(N + 1) * Lp).astype(np.int32), b.dtype)
         _, _, cache = fwd(pre, C, torch.float32, cache=True)
     else:
-        cache = gdn.new_cache(N, H, d, d, C, torch.bfloat16, DEV)
+        cache = gdn.new_cache(N, H, d, d, C, torch.bfloat16 if dtype == "bf16" else torch.float32, DEV)
     dd = to_device(b)
     fo = full_o.cpu()
     for s in range(steps):
