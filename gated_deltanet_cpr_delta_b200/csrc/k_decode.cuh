@@ -388,20 +388,28 @@ k_dec_rstep(int NH, int in_bf16, float* S_b, float* R, float* rscale, const void
     uint32_t parity = 0;
     float SR[DK / 2];
     int it = 0;
-    for (; it < nt; ++it) {
-        const int nh = todo[it];
-        float* Rn = R + (int64_t)nh * DV * DK;  // u0 rows [C][DV], then w rows [C][DK]
-        // u0, w and the alphas to shared memory by cp.async, every copy in flight at once
-        for (int f = threadIdx.x; f < C * (DV + DK) / 4; f += blockDim.x) {
-            if (f < C * DV / 4) {
-                cp_async16(us + 4 * f, Rn + 4 * f);
-            } else {
-                const int g = f - C * DV / 4, t = g / (DK / 4), c4 = g % (DK / 4);
-                cp_async16(wx + t * Sm::WXS + 4 * c4, Rn + C * DV + t * DK + 4 * c4);
-            }
+    // u0 rows [C][DV], then w rows [C][DK], parked in the pair's R by k_dec_rprep.  The
+    // next pair's w and alphas are copied in while this pair's step runs, its u0 once
+    // the step has consumed this one's.
+    auto fetch_w = [&](int nh) {
+        const float* Rn = R + (int64_t)nh * DV * DK;
+        for (int f = threadIdx.x; f < C * DK / 4; f += blockDim.x) {
+            const int t = f / (DK / 4), c4 = f % (DK / 4);
+            cp_async16(wx + t * Sm::WXS + 4 * c4, Rn + C * DV + t * DK + 4 * c4);
         }
         for (int t = threadIdx.x; t < C; t += blockDim.x) cp_async4(as_ + t, abuf + (int64_t)nh * C + t);
         cp_async_commit();
+    };
+    auto fetch_u = [&](int nh) {
+        const float* Rn = R + (int64_t)nh * DV * DK;
+        for (int f = threadIdx.x; f < C * DV / 4; f += blockDim.x) cp_async16(us + 4 * f, Rn + 4 * f);
+        cp_async_commit();
+    };
+    fetch_w(todo[0]);
+    fetch_u(todo[0]);
+    for (; it < nt; ++it) {
+        const int nh = todo[it];
+        float* Rn = R + (int64_t)nh * DV * DK;
         tc_stage_kT<DK, DV, C>(kbuf, (int64_t)nh * C, 1, 0, in_bf16, Khi, Klo);
         float* Sg = S_b + (int64_t)nh * DV * DK;
         cp_async_wait_all();
@@ -409,20 +417,27 @@ k_dec_rstep(int NH, int in_bf16, float* S_b, float* R, float* rscale, const void
         tc_stage_w<DK, DV, C>(wx, Sm::WXS, Whi, Wlo, threadIdx.x, blockDim.x);
         for (int s_ = threadIdx.x; s_ <= C; s_ += blockDim.x) {  // D[C][s], chunk_prep's order of products
             float d = 1.0f;
-            for (int t = s_; t < C; ++t) d = fmul(d, as_[t]);
+#pragma unroll
+            for (int t = 0; t < C; ++t) {
+                const float a = as_[t];
+                if (t >= s_) d = fmul(d, a);
+            }
             dCs[s_] = d;
         }
         tc_load_state<DK, DV, C>(SR, th, Sg, nullptr);
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        __syncthreads();  // wx and as_ are consumed
+        if (it + 1 < nt) fetch_w(todo[it + 1]);
         if (!tc_step<DK, DV, C>(SR, th, tbase, mbar, parity, Wlo, Klo, us, DV, dCs, in_bf16, Sg, Rn))
             break;
         if (threadIdx.x == 0) {
             pos[nh] = 0;
             rscale[nh] = 1.0f;
         }
+        if (it + 1 < nt) fetch_u(todo[it + 1]);  // the step's epilogue has consumed us
     }
+    cp_async_wait_all();
     for (int r = it + threadIdx.x; r < nt; r += blockDim.x) pos[todo[r]] = -1;  // after a timeout
     if (it < nt && threadIdx.x == 0) record_error(status, GDN_ERR_TIMEOUT);
     tc_fence_before();
